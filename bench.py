@@ -1,0 +1,483 @@
+"""Benchmark of the paged decode-attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step is one layer's decode step of the named workload, through the
+library's C ABI: copy-on-write block copies (workloads that have them), the
+cache write of each sequence's new token, then paged decode attention.
+Inputs are seeded synthetic tensors resident in HBM; L2 is flushed (a
+256 MiB write) before every timed step, outside the step's events.
+
+Printed (rank 0, one JSON line): KV-read GB/s of the whole step (``value``),
+% of the measured HBM peak, sequences/s, the decode launch's roofline
+fraction, the end-to-end figure through the same API with host buffers, the
+fp64 CPU oracle's throughput on a bounded sample, SM clocks sampled during the
+timed region, and a few secondary workloads.
+
+N > 1 (torchrun, one process per GPU): every rank runs its own replica of the
+workload (weak scaling, no collective on the data path); timings are the max
+over ranks.  ``--impl reference`` times the CPU oracle instead (rank 0 only).
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import shutil
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "paged decode attention: achieved KV-read HBM GB/s (% of peak), seq/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def measured_hbm_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing
+# ---------------------------------------------------------------------------
+def dist_setup(n_gpus):
+    import torch
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return rank, world
+
+
+def dist_max(x: float) -> float:
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()):
+        return x
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def dist_barrier():
+    import torch.distributed as dist
+
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+
+
+def dist_done():
+    import torch.distributed as dist
+
+    if dist.is_available() and dist.is_initialized():
+        dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+        exe = shutil.which("nvidia-smi")
+        if exe is None:
+            return
+        os.makedirs(os.path.dirname(self.path), exist_ok=True)
+        self.f = open(self.path, "w")
+        self.proc = subprocess.Popen([exe, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                      "-i", str(gpu_index), "-lms", "50"], stdout=self.f,
+                                     stderr=subprocess.DEVNULL)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# workload on the device
+# ---------------------------------------------------------------------------
+class DeviceWorkload:
+    def __init__(self, name: str, seed: int, partition_size: int | None = None):
+        import torch
+
+        import paged_kv_cache_362_b200 as pa
+        from workloads import build_workload, device_values, get_config
+
+        self.pa = pa
+        self.cfg = get_config(name)
+        self.wl = build_workload(self.cfg, seed=seed)
+        self.P = self.cfg.partition_size if partition_size is None else partition_size
+        dev = torch.device("cuda")
+        v = device_values(self.wl, dev)
+        self.q, self.key, self.value = v["q"], v["key"], v["value"]
+        self.kc, self.vc = v["key_cache"], v["value_cache"]
+        wl = self.wl
+        self.bt = torch.from_numpy(wl.block_tables).to(dev)
+        self.cl = torch.from_numpy(wl.context_lens).to(dev)
+        self.slots = torch.from_numpy(wl.slot_mapping).to(dev)
+        self.pairs = torch.from_numpy(np.ascontiguousarray(wl.copy_pairs)).to(dev)
+        self.has_copy = wl.copy_pairs.shape[0] > 0
+        c = self.cfg
+        self.max_ctx = wl.max_context_len
+        self.ws = pa.make_workspace(wl.num_seqs, c.num_heads, c.num_kv_heads, c.head_dim, self.max_ctx, self.P)
+        self.out = torch.empty_like(self.q)
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.kv_bytes = wl.kv_bytes()
+        np_max = -(-self.max_ctx // self._resolved_partition())
+        self.launches_per_step = (1 if self.has_copy else 0) + 1 + 2 + (1 if np_max > 1 else 0)
+
+    def _resolved_partition(self):
+        if self.P:
+            return self.P
+        # the library's automatic choice, restated only to count launches
+        c, B = self.cfg, self.wl.num_seqs
+        P = 512
+        while P > 64 and B * c.num_kv_heads * -(-self.max_ctx // P) < 8 * 148:
+            P //= 2
+        return P
+
+    def pre(self):
+        if self.has_copy:
+            self.pa.copy_blocks(self.kc, self.vc, self.pairs, status=self.status)
+        self.pa.reshape_and_cache(self.key, self.value, self.kc, self.vc, self.slots, status=self.status)
+
+    def decode(self):
+        c = self.cfg
+        self.pa.decode(self.out, self.q, self.kc, self.vc, self.bt, self.cl, c.scale, self.max_ctx, self.ws,
+                       partition_size=self.P, status=self.status)
+
+
+def time_steps(w: DeviceWorkload, steps: int, warmup: int, flush, use_graph: bool):
+    """Per-step CUDA-event times (ms) of [pre, decode] and of decode alone."""
+    import torch
+
+    stream = torch.cuda.current_stream()
+    graph_pre = graph_dec = None
+    if use_graph:
+        for _ in range(3):
+            w.pre()
+            w.decode()
+        torch.cuda.synchronize()
+        s = torch.cuda.Stream()
+        s.wait_stream(stream)
+        with torch.cuda.stream(s):
+            graph_pre = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph_pre, stream=s):
+                w.pre()
+            graph_dec = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph_dec, stream=s):
+                w.decode()
+        stream.wait_stream(s)
+        torch.cuda.synchronize()
+
+    def run_pre():
+        graph_pre.replay() if graph_pre is not None else w.pre()
+
+    def run_dec():
+        graph_dec.replay() if graph_dec is not None else w.decode()
+
+    for _ in range(max(warmup, 3)):
+        flush()
+        run_pre()
+        run_dec()
+    torch.cuda.synchronize()
+    dist_barrier()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for e0, e1, e2 in ev:
+        flush()
+        e0.record(stream)
+        run_pre()
+        e1.record(stream)
+        run_dec()
+        e2.record(stream)
+    torch.cuda.synchronize()
+    dist_barrier()
+    step_ms = [e0.elapsed_time(e2) for e0, _, e2 in ev]
+    dec_ms = [e1.elapsed_time(e2) for _, e1, e2 in ev]
+    return step_ms, dec_ms
+
+
+def time_e2e(w: DeviceWorkload, steps: int, warmup: int, flush):
+    """The same step through the public API from pinned host buffers: H2D inputs, step, D2H output."""
+    import torch
+
+    host = {}
+    for name in ("q", "key", "value", "slots", "bt", "cl") + (("pairs",) if w.has_copy else ()):
+        t = getattr(w, name)
+        h = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+        h.copy_(t)
+        host[name] = h
+    out_h = torch.empty(w.out.shape, dtype=w.out.dtype, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_h.numel() * out_h.element_size()
+    stream = torch.cuda.current_stream()
+
+    def one():
+        for name, h in host.items():
+            getattr(w, name).copy_(h, non_blocking=True)
+        w.pre()
+        w.decode()
+        out_h.copy_(w.out, non_blocking=True)
+
+    for _ in range(max(warmup, 3)):
+        flush()
+        one()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for e0, e1 in ev:
+        flush()
+        e0.record(stream)
+        one()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in ev], h2d, d2h
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (reported baseline; also the --impl reference arm)
+# ---------------------------------------------------------------------------
+def _oracle_subproblem(name: str, seed: int, nseq: int, sample_seed: int):
+    """Host pools holding only ``nseq`` sampled sequences' blocks, values drawn on the host."""
+    from workloads import Workload, build_workload, get_config, host_values
+
+    cfg = get_config(name)
+    wl = build_workload(cfg, seed=seed)
+    rng = np.random.default_rng(sample_seed)
+    seqs = np.sort(rng.choice(wl.num_seqs, size=min(nseq, wl.num_seqs), replace=False))
+    nblk = [-(-int(wl.context_lens[b]) // 16) for b in seqs]
+    ids = sorted({int(x) for b, n in zip(seqs, nblk) for x in wl.block_tables[b, :n]})
+    remap = {o: i for i, o in enumerate(ids)}
+    bt = np.full((len(seqs), max(1, max(nblk))), -1, np.int32)
+    for i, (b, n) in enumerate(zip(seqs, nblk)):
+        bt[i, :n] = [remap[int(x)] for x in wl.block_tables[b, :n]]
+    sub = Workload(cfg=cfg, seed=sample_seed, context_lens=wl.context_lens[seqs].copy(), block_tables=bt,
+                   slot_mapping=np.zeros(0, np.int64), copy_pairs=np.zeros((0, 2), np.int64),
+                   num_blocks=max(1, len(ids)))
+    return cfg, sub, host_values(sub), wl.num_seqs
+
+
+def _oracle_run(cfg, sub, v, threads):
+    from oracle import c_oracle
+
+    c_oracle.decode(v["q"], v["key_cache"], v["value_cache"], sub.block_tables, sub.context_lens, cfg.scale,
+                    cfg.dtype, cfg.num_kv_heads, num_threads=threads)
+
+
+def oracle_sample_throughput(name: str, seed: int, budget_s: float, max_seqs: int):
+    """fp64 C oracle on a bounded sample of the workload: (KV GB/s, seq/s, threads, sample text)."""
+    cfg, sub, v, total = _oracle_subproblem(name, seed, max_seqs, seed + 7)
+    threads = os.cpu_count() or 1
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        _oracle_run(cfg, sub, v, threads)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or reps >= 50:
+            break
+    per = el / reps
+    sample = (f"{sub.num_seqs} of {total} sequences of {name} (seed {seed}), {reps} run(s), "
+              f"fp64 C oracle with OpenMP")
+    return sub.kv_bytes() / per / 1e9, sub.num_seqs / per, threads, sample, per
+
+
+def run_reference(args):
+    """The CPU oracle as the reference arm: W + K steps, each a bounded sample of the workload."""
+    threads = os.cpu_count() or 1
+    cfg, sub, v, total = _oracle_subproblem(args.workload, args.seed, 8, args.seed + 1)
+    t0 = time.perf_counter()
+    _oracle_run(cfg, sub, v, threads)
+    per8 = max(time.perf_counter() - t0, 1e-4)
+    steps, warm = args.steps, args.warmup
+    per_step_budget = args.ref_total_s / max(1, steps + warm)
+    nseq = int(max(1, min(total, 8 * per_step_budget / per8)))
+    subs = [_oracle_subproblem(args.workload, args.seed, nseq, args.seed + 100 + i) for i in range(4)]
+    for i in range(warm):
+        c, s_, v_, _ = subs[i % 4]
+        _oracle_run(c, s_, v_, threads)
+    times, kv, seqs = [], 0, 0
+    for i in range(steps):
+        c, s_, v_, _ = subs[i % 4]
+        t0 = time.perf_counter()
+        _oracle_run(c, s_, v_, threads)
+        times.append(time.perf_counter() - t0)
+        kv += s_.kv_bytes()
+        seqs += s_.num_seqs
+    el = sum(times)
+    gbs = kv / el / 1e9
+    sample = (f"each step: {nseq} of {total} sequences of {args.workload} (4 rotating seeded samples), "
+              f"fp64 C oracle with OpenMP on {threads} threads")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": steps, "warmup": warm, "ms_per_step": round(1e3 * el / steps, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": args.workload, "seed": args.seed,
+                                        "sample_seqs_per_step": nseq},
+        "seq_per_s": round(seqs / el, 3),
+        "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="churned256")
+    ap.add_argument("--partition-size", type=int, default=None)
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-graph", action="store_true", help="launch every step from the host (no CUDA graph)")
+    ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of CPU oracle timing")
+    ap.add_argument("--cpu-seqs", type=int, default=64)
+    ap.add_argument("--ref-total-s", type=float, default=90.0, help="CPU seconds the reference arm may take")
+    args = ap.parse_args()
+
+    if args.impl == "reference":
+        if int(os.environ.get("RANK", "0")) == 0:
+            run_reference(args)
+        return
+    rank, world = dist_setup(args.gpus)
+
+    import torch
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    peak, peak_kind = measured_hbm_peak()
+    flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    flush = lambda: flush_buf.zero_()
+    use_graph = not args.no_graph
+
+    w = DeviceWorkload(args.workload, args.seed + rank, args.partition_size)
+    clocks = ClockSampler(torch.cuda.current_device())
+    step_ms, dec_ms = time_steps(w, args.steps, args.warmup, flush, use_graph)
+    clk = clocks.stop()
+    torch.cuda.synchronize()
+    status = int(w.status.item())
+    if status != 0:
+        raise SystemExit(f"device status {status}: {w.pa.error_string(status)}")
+
+    ms = dist_max(float(np.mean(step_ms)))
+    dec = dist_max(float(np.mean(dec_ms)))
+    total_bytes = w.kv_bytes * world
+    value = total_bytes / (ms * 1e-3) / 1e9
+    achieved = w.kv_bytes / (dec * 1e-3) / 1e9
+
+    e2e_ms, h2d, d2h = time_e2e(w, max(50, args.steps // 10), args.warmup, flush)
+    e2e = dist_max(float(np.mean(e2e_ms)))
+
+    secondary = {}
+    if not args.no_secondary:
+        for name in ("long32k", "qwen_layer", "shared_prefix"):
+            if name == args.workload:
+                continue
+            sw = DeviceWorkload(name, args.seed + rank)
+            s_step, s_dec = time_steps(sw, max(50, args.steps // 10), args.warmup, flush, use_graph)
+            sd = dist_max(float(np.mean(s_dec)))
+            ss = dist_max(float(np.mean(s_step)))
+            secondary[name] = {
+                "decode_ms": round(sd, 5), "step_ms": round(ss, 5),
+                "decode_kv_gbs": round(sw.kv_bytes / (sd * 1e-3) / 1e9, 1),
+                "decode_frac_of_peak": round(sw.kv_bytes / (sd * 1e-3) / 1e9 / peak, 4),
+                "kv_bytes": sw.kv_bytes, "seq_per_s": round(sw.wl.num_seqs / (ss * 1e-3), 1),
+            }
+            del sw
+            torch.cuda.empty_cache()
+
+    cpu = None
+    if rank == 0 and world == 1:
+        gbs, sps, threads, sample, _ = oracle_sample_throughput(args.workload, args.seed, args.cpu_budget,
+                                                                args.cpu_seqs)
+        cpu = {"value": round(gbs, 4), "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": sample}
+
+    if rank == 0:
+        c = w.cfg
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": c.dtype, "data": "synthetic",
+            "config": {"workload": c.name, "num_seqs": w.wl.num_seqs, "num_heads": c.num_heads,
+                       "num_kv_heads": c.num_kv_heads, "head_dim": c.head_dim, "block_size": 16,
+                       "num_blocks": c.num_blocks, "mean_context": float(np.mean(w.wl.context_lens)),
+                       "max_context": w.max_ctx, "partition_size": w.P or "auto",
+                       "parallelism": f"replicas x{world}",
+                       "l2": "flushed before every timed step (256 MiB write, outside the step's events)",
+                       "cuda_graph": use_graph,
+                       "step": ("copy_blocks + " if w.has_copy else "") + "reshape_and_cache + decode"},
+            "pct_of_peak": round(100 * value / world / peak, 2),
+            "seq_per_s": round(w.wl.num_seqs * world / (ms * 1e-3), 1),
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                         "frac": round(achieved / peak, 4), "traffic": None, "kernel": "pa_decode (plan + "
+                         "partition + reduce launches)", "peak_kind": peak_kind},
+            "cpu_baseline": cpu,
+            "e2e": {"value": round(total_bytes / (e2e * 1e-3) / 1e9, 2), "unit": "GB/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e, 5)},
+            "gpu_launches": w.launches_per_step * args.steps,
+            "clocks": clk,
+            "secondary": secondary,
+        }
+        print(json.dumps(line), flush=True)
+    dist_done()
+
+
+if __name__ == "__main__":
+    main()

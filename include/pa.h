@@ -1,0 +1,170 @@
+/*
+ * pa.h -- C ABI of the B200 (sm_100a) paged KV-cache decode-attention library.
+ *
+ * What the library implements is the hot path the pages describe:
+ *   - the KV cache lives in a shared pool of fixed-size physical blocks of 16
+ *     tokens, and each request reaches its blocks through a block table that
+ *     maps logical block index -> physical block index ("PagedAttention"
+ *     digest, section "PagedAttention in one picture");
+ *   - each decoded token appends one K/V entry inside the current logical
+ *     block ("LLM Inference Visualizer", lesson 06, "How paging grows");
+ *   - attention walks the block table and gathers K and V from wherever they
+ *     live, computing exactly ordinary attention ("PagedAttention" digest,
+ *     sections "PagedAttention in one picture", "Why the attention kernel
+ *     works at all" and "Misconceptions");
+ *   - a shared block that a request must write is cloned first
+ *     (copy-on-write; "PagedAttention" digest, section "Copy-on-write: when
+ *     two requests share a prefix").
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  * All tensor arguments are DEVICE pointers owned by the caller.  Scalars
+ *    are passed by value.  Nothing is allocated, and no state is kept between
+ *    calls.
+ *  * Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *    default stream).  A return of PA_OK means the work was enqueued.
+ *  * Arguments that can be checked on the host are checked before anything is
+ *    enqueued; a failing check returns PA_ERR_INVALID_ARG or
+ *    PA_ERR_UNSUPPORTED and enqueues nothing.  A failed launch returns
+ *    PA_ERR_CUDA.
+ *  * Values that only the device sees (block ids, slots, context lengths) are
+ *    range-checked by the kernels.  A bad value is skipped -- never read or
+ *    written out of bounds -- and PA_ERR_OUT_OF_RANGE is OR-ed into
+ *    `*status` when `status` is not NULL.  `status` is a device int32 the
+ *    caller zeroes and reads back after synchronising.  Kernels never trap.
+ *  * Dtypes: q, K, V, out and the appended key/value share one element type.
+ *  * Pool layout (both key_cache and value_cache):
+ *        [num_blocks][num_kv_heads][block_size = 16][head_dim]   row-major,
+ *    so one (block, KV head) tile of 16 tokens is a contiguous run of
+ *    16 * head_dim elements.  Slot s of the pool is block s / 16, offset s % 16.
+ *  * GQA: query head h uses KV head h / (num_heads / num_kv_heads).
+ *  * Supported: block_size 16; head_dim 64 or 128; float32, float16, bfloat16.
+ */
+#ifndef PA_H_
+#define PA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t, declared here so the header needs no CUDA headers. */
+typedef struct CUstream_st* pa_stream_t;
+
+/* Host return codes; the device status word ORs the same bit values. */
+typedef enum {
+    PA_OK = 0,
+    PA_ERR_INVALID_ARG = 1,   /* null pointer, negative size, misaligned buffer, small workspace */
+    PA_ERR_UNSUPPORTED = 2,   /* valid but not implemented: block_size != 16, head_dim, dtype */
+    PA_ERR_OUT_OF_RANGE = 4,  /* device: block id, slot or context length outside its range */
+    PA_ERR_CUDA = 8,          /* a CUDA launch or query failed */
+    PA_ERR_TIMEOUT = 16       /* device: a bounded wait inside a kernel gave up */
+} pa_status;
+
+typedef enum { PA_F32 = 0, PA_F16 = 1, PA_BF16 = 2 } pa_dtype;
+
+/*
+ * pa_reshape_and_cache -- write the K/V of newly decoded tokens into the pool.
+ *
+ * For every token t < num_tokens with s = slot_mapping[t] >= 0:
+ *     key_cache  [s / 16][h][s % 16][:] = key  [t][h][:]   for all h < num_kv_heads
+ *     value_cache[s / 16][h][s % 16][:] = value[t][h][:]
+ * A negative slot is padding and writes nothing.  A slot >= num_blocks * 16
+ * writes nothing and sets PA_ERR_OUT_OF_RANGE in *status.  The copy is
+ * bit-exact.  Distinct tokens must name distinct slots (otherwise which one
+ * lands is unspecified).
+ *
+ *   key, value      [num_tokens][num_kv_heads][head_dim], contiguous, 16-byte aligned
+ *   key_cache,
+ *   value_cache     pools, layout above, 16-byte aligned
+ *   slot_mapping    int64 [num_tokens]
+ *   status          nullable device int32, OR-ed with PA_ERR_* bits
+ */
+pa_status pa_reshape_and_cache(const void* key, const void* value, void* key_cache, void* value_cache,
+                               const int64_t* slot_mapping, int64_t num_tokens, int32_t num_blocks,
+                               int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                               pa_dtype dtype, int32_t* status, pa_stream_t stream);
+
+/*
+ * pa_decode_workspace_size -- bytes of device workspace pa_decode needs.
+ *
+ * The workspace holds the work list of (sequence, partition, KV head) items
+ * and, for sequences split into several partitions, each partition's
+ * (max logit, sum of exponentials, unnormalised output) in fp32.  The result
+ * depends only on the arguments given here; pass the same values (including
+ * partition_size, 0 = automatic) to pa_decode.  Returns 0 for invalid
+ * arguments.
+ */
+size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads,
+                                int32_t head_dim, int32_t max_context_len, int32_t partition_size);
+
+/*
+ * pa_decode -- one decode step of attention through the block tables.
+ *
+ * For every sequence b < num_seqs and query head h < num_heads, with
+ * n = context_lens[b] and g = h / (num_heads / num_kv_heads):
+ *     K_i = key_cache  [block_tables[b][i / 16]][g][i % 16][:]   (i < n)
+ *     V_i = value_cache[block_tables[b][i / 16]][g][i % 16][:]
+ *     out[b][h][:] = sum_i softmax_i(scale * q[b][h][:] . K_i) V_i
+ * computed in fp32 from the stored values and rounded to the element type.
+ * n = 0 gives a zero row.  The context is split into partitions of
+ * partition_size tokens that run in parallel; a second kernel merges them.
+ * The merge is exact algebra, so the result does not depend on the split
+ * beyond fp32 rounding, and it does not depend on where blocks live.
+ *
+ *   out                 [num_seqs][num_heads][head_dim], 16-byte aligned
+ *   q                   [num_seqs][num_heads][head_dim], 16-byte aligned
+ *   key_cache,
+ *   value_cache         pools, layout above
+ *   block_tables        int32 [num_seqs][max_blocks_per_seq]; only the first
+ *                       ceil(n / 16) entries of row b are read, each must be
+ *                       in [0, num_blocks) (else PA_ERR_OUT_OF_RANGE and the
+ *                       block is skipped)
+ *   context_lens        int32 [num_seqs]; a value outside
+ *                       [0, min(max_context_len, max_blocks_per_seq * 16)] is
+ *                       clamped into that range and sets PA_ERR_OUT_OF_RANGE
+ *   max_context_len     host-side upper bound of context_lens (sizes the split)
+ *   partition_size      tokens per partition: 0 = automatic, else a multiple
+ *                       of 16 in [16, 512]
+ *   workspace           device buffer of at least pa_decode_workspace_size()
+ *                       bytes, 256-byte aligned; contents need no initialising
+ *                       and are scratch between calls.  Calls that share a
+ *                       workspace must not overlap in time.
+ */
+pa_status pa_decode(void* out, const void* q, const void* key_cache, const void* value_cache,
+                    const int32_t* block_tables, int32_t max_blocks_per_seq,
+                    const int32_t* context_lens, int32_t num_seqs, int32_t num_heads,
+                    int32_t num_kv_heads, int32_t head_dim, int32_t block_size, int32_t num_blocks,
+                    float scale, int32_t max_context_len, int32_t partition_size, void* workspace,
+                    size_t workspace_bytes, pa_dtype dtype, int32_t* status, pa_stream_t stream);
+
+/*
+ * pa_copy_blocks -- copy-on-write clone of whole blocks, in both pools.
+ *
+ * For each pair k < num_pairs with (src, dst) = (block_pairs[2k], block_pairs[2k+1]):
+ *     key_cache[dst] = key_cache[src];  value_cache[dst] = value_cache[src]
+ * (all num_kv_heads * 16 * head_dim elements; bit-exact).  A pair with an id
+ * outside [0, num_blocks) is skipped and sets PA_ERR_OUT_OF_RANGE.  No dst
+ * may repeat and no dst may also be a src in the same call (that would be a
+ * write/write or read/write race); the result is then unspecified.
+ *
+ *   block_pairs   int64 [num_pairs][2], device
+ */
+pa_status pa_copy_blocks(void* key_cache, void* value_cache, const int64_t* block_pairs,
+                         int32_t num_pairs, int32_t num_blocks, int32_t num_kv_heads,
+                         int32_t head_dim, int32_t block_size, pa_dtype dtype, int32_t* status,
+                         pa_stream_t stream);
+
+/* Static, human-readable name of a status code (or of the lowest bit set). */
+const char* pa_get_error_string(pa_status status);
+
+/* Library version as major * 10000 + minor * 100 + patch. */
+int32_t pa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_H_ */

@@ -1,0 +1,161 @@
+"""ctypes binding of libpa.so: argument marshalling only.
+
+Every step of the path runs in the library's CUDA kernels.  These wrappers
+take torch tensors (which provide device memory and the current stream),
+check shapes and dtypes, pass raw pointers to the C ABI declared in
+include/pa.h, and raise on a non-zero status.  If the library is missing the
+import fails loudly; there is no fallback.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libpa.so")
+
+PA_OK = 0
+PA_ERR_INVALID_ARG = 1
+PA_ERR_UNSUPPORTED = 2
+PA_ERR_OUT_OF_RANGE = 4
+PA_ERR_CUDA = 8
+PA_ERR_TIMEOUT = 16
+
+PA_F32, PA_F16, PA_BF16 = 0, 1, 2
+BLOCK_SIZE = 16
+
+
+class PagedAttentionError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {error_string(code)} (status {code})")
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is not built; run `python -m paged_kv_cache_362_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    p, i32, i64, f32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+    lib.pa_reshape_and_cache.argtypes = [p, p, p, p, p, i64, i32, i32, i32, i32, ctypes.c_int, p, p]
+    lib.pa_reshape_and_cache.restype = ctypes.c_int
+    lib.pa_decode_workspace_size.argtypes = [i32, i32, i32, i32, i32, i32]
+    lib.pa_decode_workspace_size.restype = sz
+    lib.pa_decode.argtypes = [p, p, p, p, p, i32, p, i32, i32, i32, i32, i32, i32, f32, i32, i32, p, sz,
+                              ctypes.c_int, p, p]
+    lib.pa_decode.restype = ctypes.c_int
+    lib.pa_copy_blocks.argtypes = [p, p, p, i32, i32, i32, i32, i32, ctypes.c_int, p, p]
+    lib.pa_copy_blocks.restype = ctypes.c_int
+    lib.pa_get_error_string.argtypes = [ctypes.c_int]
+    lib.pa_get_error_string.restype = ctypes.c_char_p
+    lib.pa_version.argtypes = []
+    lib.pa_version.restype = i32
+    return lib
+
+
+LIB = _load()
+
+
+def error_string(code: int) -> str:
+    return LIB.pa_get_error_string(int(code)).decode()
+
+
+def version() -> int:
+    return int(LIB.pa_version())
+
+
+def _check(code: int, where: str):
+    if code != PA_OK:
+        raise PagedAttentionError(code, where)
+
+
+def _dtype_code(t) -> int:
+    import torch
+
+    return {torch.float32: PA_F32, torch.float16: PA_F16, torch.bfloat16: PA_BF16}[t.dtype]
+
+
+def _stream(stream):
+    import torch
+
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+def reshape_and_cache(key, value, key_cache, value_cache, slot_mapping, status=None, stream=None):
+    """Write each token's K/V into its slot (pa_reshape_and_cache).
+
+    key, value [T, Hkv, D]; key_cache, value_cache [NB, Hkv, 16, D];
+    slot_mapping int64 [T] (negative = skip); status: optional int32 device tensor.
+    """
+    assert key.is_contiguous() and value.is_contiguous() and key_cache.is_contiguous() and value_cache.is_contiguous()
+    assert slot_mapping.dtype.is_floating_point is False and slot_mapping.element_size() == 8
+    T, Hkv, D = key.shape
+    NB = key_cache.shape[0]
+    assert value.shape == key.shape and key_cache.shape == (NB, Hkv, BLOCK_SIZE, D) == value_cache.shape
+    assert key.dtype == value.dtype == key_cache.dtype == value_cache.dtype
+    _check(LIB.pa_reshape_and_cache(_ptr(key), _ptr(value), _ptr(key_cache), _ptr(value_cache), _ptr(slot_mapping),
+                                    T, NB, Hkv, D, BLOCK_SIZE, _dtype_code(key), _ptr(status), _stream(stream)),
+           "pa_reshape_and_cache")
+
+
+def decode_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, max_context_len, partition_size=0) -> int:
+    n = int(LIB.pa_decode_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, max_context_len,
+                                         partition_size))
+    if n == 0:
+        raise PagedAttentionError(PA_ERR_INVALID_ARG, "pa_decode_workspace_size")
+    return n
+
+
+def make_workspace(num_seqs, num_heads, num_kv_heads, head_dim, max_context_len, partition_size=0, device=None):
+    import torch
+
+    n = decode_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, max_context_len, partition_size)
+    return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def decode(out, q, key_cache, value_cache, block_tables, context_lens, scale, max_context_len, workspace,
+           partition_size=0, status=None, stream=None):
+    """One decode step of paged attention (pa_decode); writes ``out`` [B, Hq, D]."""
+    B, Hq, D = q.shape
+    NB, Hkv = key_cache.shape[0], key_cache.shape[1]
+    assert out.shape == q.shape and out.dtype == q.dtype == key_cache.dtype == value_cache.dtype
+    assert key_cache.shape == (NB, Hkv, BLOCK_SIZE, D) == value_cache.shape
+    assert block_tables.dtype.itemsize == 4 and context_lens.dtype.itemsize == 4
+    assert block_tables.shape[0] == B and context_lens.shape == (B,)
+    for t in (out, q, key_cache, value_cache, block_tables, context_lens, workspace):
+        assert t.is_contiguous()
+    _check(LIB.pa_decode(_ptr(out), _ptr(q), _ptr(key_cache), _ptr(value_cache), _ptr(block_tables),
+                         block_tables.shape[1], _ptr(context_lens), B, Hq, Hkv, D, BLOCK_SIZE, NB, float(scale),
+                         int(max_context_len), int(partition_size), _ptr(workspace),
+                         workspace.numel() * workspace.element_size(), _dtype_code(q), _ptr(status),
+                         _stream(stream)),
+           "pa_decode")
+
+
+def copy_blocks(key_cache, value_cache, block_pairs, status=None, stream=None):
+    """Copy-on-write clone of whole blocks (pa_copy_blocks); block_pairs int64 [N, 2] on the device."""
+    assert key_cache.is_contiguous() and value_cache.is_contiguous() and block_pairs.is_contiguous()
+    assert block_pairs.element_size() == 8 and block_pairs.dim() == 2 and block_pairs.shape[1] == 2
+    NB, Hkv, bs, D = key_cache.shape
+    _check(LIB.pa_copy_blocks(_ptr(key_cache), _ptr(value_cache), _ptr(block_pairs), block_pairs.shape[0], NB, Hkv,
+                              D, bs, _dtype_code(key_cache), _ptr(status), _stream(stream)),
+           "pa_copy_blocks")
+
+
+def check_copy_pairs(pairs_host, num_blocks: int) -> None:
+    """Host-side validation of copy pairs (ids in range, no repeated dst, no dst that is also a src)."""
+    import numpy as np
+
+    pr = np.asarray(pairs_host).reshape(-1, 2)
+    if pr.size and (pr.min() < 0 or pr.max() >= num_blocks):
+        raise ValueError("copy pair id outside the pool")
+    dst = pr[:, 1]
+    if len(np.unique(dst)) != len(dst):
+        raise ValueError("a destination block repeats")
+    if np.isin(dst, pr[:, 0]).any():
+        raise ValueError("a destination block is also a source")

@@ -1,0 +1,193 @@
+// C ABI of the library: host-side argument checks, workspace layout, launches.
+// See include/pa.h for the contract of every entry point.
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "pa_internal.h"
+
+namespace pa {
+
+cudaError_t device_info(DeviceInfo* out) {
+    static DeviceInfo cache[64];
+    static bool have[64] = {};
+    static std::mutex mu;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!have[dev]) {
+        DeviceInfo d{};
+        e = cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
+        e = cudaDeviceGetAttribute(&d.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+        if (e != cudaSuccess) return e;
+        cache[dev] = d;
+        have[dev] = true;
+    }
+    *out = cache[dev];
+    return cudaSuccess;
+}
+
+namespace {
+
+int elt_bytes(pa_dtype d) { return d == PA_F32 ? 4 : 2; }
+bool valid_dtype(int d) { return d == PA_F32 || d == PA_F16 || d == PA_BF16; }
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+int64_t ceil_div64(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// Partition size when the caller passes 0: the largest of 512/256/128/64
+// tokens that still yields enough (sequence, partition, KV head) items to keep
+// every SM of a B200 busy several times over.
+int auto_partition_size(int64_t num_seqs, int64_t num_kv_heads, int64_t max_context_len) {
+    int P = 512;
+    while (P > 64 && num_seqs * num_kv_heads * ceil_div64(max_context_len, P) < 8 * 148) P /= 2;
+    return P;
+}
+
+struct WsLayout {
+    int partition_size, max_parts;
+    int64_t max_items;
+    size_t off_items, off_m, off_l, off_o, total;
+};
+
+bool ws_layout(int64_t num_seqs, int64_t num_heads, int64_t num_kv_heads, int64_t head_dim,
+               int64_t max_context_len, int64_t partition_size, WsLayout* w) {
+    if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || max_context_len < 0) return false;
+    if (partition_size == 0) partition_size = auto_partition_size(num_seqs, num_kv_heads, max_context_len);
+    if (partition_size < kBlockSize || partition_size > kBlockSize * kMaxPartBlocks ||
+        partition_size % kBlockSize != 0)
+        return false;
+    const int64_t np = std::max<int64_t>(1, ceil_div64(max_context_len, partition_size));
+    w->partition_size = (int)partition_size;
+    w->max_parts = (int)np;
+    w->max_items = num_seqs * np * num_kv_heads;
+    const int64_t parts = np > 1 ? num_seqs * num_heads * np : 0;
+    w->off_items = 256;
+    w->off_m = round_up(w->off_items + (size_t)w->max_items * sizeof(int2), 256);
+    w->off_l = round_up(w->off_m + (size_t)parts * sizeof(float), 256);
+    w->off_o = round_up(w->off_l + (size_t)parts * sizeof(float), 256);
+    w->total = round_up(w->off_o + (size_t)parts * head_dim * sizeof(float), 256);
+    return true;
+}
+
+}  // namespace
+}  // namespace pa
+
+using namespace pa;
+
+extern "C" {
+
+pa_status pa_reshape_and_cache(const void* key, const void* value, void* key_cache, void* value_cache,
+                               const int64_t* slot_mapping, int64_t num_tokens, int32_t num_blocks,
+                               int32_t num_kv_heads, int32_t head_dim, int32_t block_size, pa_dtype dtype,
+                               int32_t* status, pa_stream_t stream) {
+    if (num_tokens < 0 || num_blocks <= 0 || num_kv_heads <= 0 || head_dim <= 0) return PA_ERR_INVALID_ARG;
+    if (!valid_dtype(dtype)) return PA_ERR_INVALID_ARG;
+    if (block_size != kBlockSize || (head_dim != 64 && head_dim != 128)) return PA_ERR_UNSUPPORTED;
+    if (num_tokens == 0) return PA_OK;
+    if (!key || !value || !key_cache || !value_cache || !slot_mapping) return PA_ERR_INVALID_ARG;
+    if (!aligned16(key) || !aligned16(value) || !aligned16(key_cache) || !aligned16(value_cache))
+        return PA_ERR_INVALID_ARG;
+    const cudaError_t e = launch_reshape_and_cache(key, value, key_cache, value_cache, slot_mapping, num_tokens,
+                                                   num_blocks, num_kv_heads, head_dim, elt_bytes(dtype), status,
+                                                   reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads, int32_t head_dim,
+                                int32_t max_context_len, int32_t partition_size) {
+    WsLayout w;
+    if (!ws_layout(num_seqs, num_heads, num_kv_heads, head_dim, max_context_len, partition_size, &w)) return 0;
+    return w.total;
+}
+
+pa_status pa_decode(void* out, const void* q, const void* key_cache, const void* value_cache,
+                    const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* context_lens,
+                    int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads, int32_t head_dim,
+                    int32_t block_size, int32_t num_blocks, float scale, int32_t max_context_len,
+                    int32_t partition_size, void* workspace, size_t workspace_bytes, pa_dtype dtype,
+                    int32_t* status, pa_stream_t stream) {
+    if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || num_blocks <= 0 ||
+        max_blocks_per_seq <= 0 || max_context_len < 0)
+        return PA_ERR_INVALID_ARG;
+    if (!valid_dtype(dtype) || !std::isfinite(scale)) return PA_ERR_INVALID_ARG;
+    if (num_heads % num_kv_heads != 0) return PA_ERR_INVALID_ARG;
+    if (block_size != kBlockSize || (head_dim != 64 && head_dim != 128) || num_kv_heads > 255)
+        return PA_ERR_UNSUPPORTED;
+    if (partition_size != 0 &&
+        (partition_size < kBlockSize || partition_size > kBlockSize * kMaxPartBlocks || partition_size % kBlockSize))
+        return PA_ERR_INVALID_ARG;
+    if ((int64_t)num_blocks * num_kv_heads * kBlockSize > INT32_MAX) return PA_ERR_UNSUPPORTED;
+    if (num_seqs == 0) return PA_OK;
+    if (!out || !q || !key_cache || !value_cache || !block_tables || !context_lens || !workspace)
+        return PA_ERR_INVALID_ARG;
+    if (!aligned16(out) || !aligned16(q) || !aligned16(key_cache) || !aligned16(value_cache) ||
+        (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return PA_ERR_INVALID_ARG;
+    WsLayout w;
+    if (!ws_layout(num_seqs, num_heads, num_kv_heads, head_dim, max_context_len, partition_size, &w))
+        return PA_ERR_INVALID_ARG;
+    if (workspace_bytes < w.total) return PA_ERR_INVALID_ARG;
+    if (w.max_items > INT32_MAX) return PA_ERR_UNSUPPORTED;
+
+    DecodeParams p{};
+    p.out = out;
+    p.q = q;
+    p.key_cache = key_cache;
+    p.value_cache = value_cache;
+    p.block_tables = block_tables;
+    p.context_lens = context_lens;
+    p.status = status;
+    p.num_seqs = num_seqs;
+    p.num_heads = num_heads;
+    p.num_kv_heads = num_kv_heads;
+    p.head_dim = head_dim;
+    p.group = num_heads / num_kv_heads;
+    p.max_blocks_per_seq = max_blocks_per_seq;
+    p.num_blocks = num_blocks;
+    p.ctx_cap = (int)std::min<int64_t>(max_context_len, (int64_t)max_blocks_per_seq * kBlockSize);
+    p.part_blocks = w.partition_size / kBlockSize;
+    p.max_parts = w.max_parts;
+    p.scale_log2 = scale * 1.4426950408889634f;  // log2(e)
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    p.n_items = reinterpret_cast<int32_t*>(ws);
+    p.items = reinterpret_cast<int2*>(ws + w.off_items);
+    p.part_m = reinterpret_cast<float*>(ws + w.off_m);
+    p.part_l = reinterpret_cast<float*>(ws + w.off_l);
+    p.part_o = reinterpret_cast<float*>(ws + w.off_o);
+    const cudaError_t e = launch_decode(p, dtype, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+pa_status pa_copy_blocks(void* key_cache, void* value_cache, const int64_t* block_pairs, int32_t num_pairs,
+                         int32_t num_blocks, int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                         pa_dtype dtype, int32_t* status, pa_stream_t stream) {
+    if (num_pairs < 0 || num_blocks <= 0 || num_kv_heads <= 0 || head_dim <= 0) return PA_ERR_INVALID_ARG;
+    if (!valid_dtype(dtype)) return PA_ERR_INVALID_ARG;
+    if (block_size != kBlockSize || (head_dim != 64 && head_dim != 128)) return PA_ERR_UNSUPPORTED;
+    if (num_pairs == 0) return PA_OK;
+    if (!key_cache || !value_cache || !block_pairs) return PA_ERR_INVALID_ARG;
+    if (!aligned16(key_cache) || !aligned16(value_cache)) return PA_ERR_INVALID_ARG;
+    const cudaError_t e = launch_copy_blocks(key_cache, value_cache, block_pairs, num_pairs, num_blocks,
+                                             num_kv_heads, head_dim, elt_bytes(dtype), status,
+                                             reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+const char* pa_get_error_string(pa_status s) {
+    const int v = (int)s;
+    if (v == PA_OK) return "PA_OK";
+    if (v & PA_ERR_INVALID_ARG) return "PA_ERR_INVALID_ARG: invalid argument";
+    if (v & PA_ERR_UNSUPPORTED) return "PA_ERR_UNSUPPORTED: configuration not supported";
+    if (v & PA_ERR_OUT_OF_RANGE) return "PA_ERR_OUT_OF_RANGE: block id, slot or context length out of range";
+    if (v & PA_ERR_CUDA) return "PA_ERR_CUDA: CUDA launch or query failed";
+    if (v & PA_ERR_TIMEOUT) return "PA_ERR_TIMEOUT: bounded wait inside a kernel expired";
+    return "unknown pa_status";
+}
+
+int32_t pa_version(void) { return 100; }
+
+}  // extern "C"

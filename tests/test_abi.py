@@ -1,0 +1,140 @@
+"""The C-ABI library loads, exports every declared symbol, and rejects bad host-side arguments.
+
+CPU only: every call here returns during host-side validation, before any CUDA call.
+"""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    src = open(os.path.join(ROOT, "include", "pa.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(pa_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = _declared_functions()
+    for n in ("pa_reshape_and_cache", "pa_decode", "pa_decode_workspace_size", "pa_copy_blocks",
+              "pa_get_error_string"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    import paged_kv_cache_362_b200 as pa
+
+    lib = ctypes.CDLL(pa.LIB_PATH)
+    missing = [n for n in _declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_error_strings_and_version():
+    import paged_kv_cache_362_b200 as pa
+
+    assert pa.error_string(0) == "PA_OK"
+    for code, word in ((1, "INVALID_ARG"), (2, "UNSUPPORTED"), (4, "OUT_OF_RANGE"), (8, "CUDA"), (16, "TIMEOUT")):
+        assert word in pa.error_string(code)
+    assert pa.version() >= 100
+
+
+def test_workspace_size_is_consistent():
+    import paged_kv_cache_362_b200 as pa
+
+    lib = pa._lib.LIB
+    # invalid arguments -> 0
+    assert lib.pa_decode_workspace_size(4, 28, 4, 128, 100, 24) == 0      # not a multiple of 16
+    assert lib.pa_decode_workspace_size(4, 28, 4, 128, 100, 1024) == 0    # above 512
+    assert lib.pa_decode_workspace_size(-1, 28, 4, 128, 100, 0) == 0
+    # one partition -> no partial buffers, only header + item list
+    small = lib.pa_decode_workspace_size(8, 28, 4, 128, 512, 512)
+    assert 256 < small < 4096
+    # 32k context, 512-token partitions: 64 partials of (D + 2) floats per (seq, head)
+    big = lib.pa_decode_workspace_size(8, 28, 4, 128, 32768, 512)
+    assert big >= 8 * 28 * 64 * (128 + 2) * 4
+    assert big % 256 == 0
+
+
+P = ctypes.c_void_p
+FAKE = P(0x1000)          # never dereferenced: every call below fails validation first
+
+
+def _rc(*args):
+    import paged_kv_cache_362_b200 as pa
+
+    return pa._lib.LIB.pa_reshape_and_cache(*args)
+
+
+def test_reshape_and_cache_validation():
+    import paged_kv_cache_362_b200 as pa
+
+    ok = dict(key=FAKE, value=FAKE, kc=FAKE, vc=FAKE, slots=FAKE)
+    args = lambda **o: [o.get("key", FAKE), o.get("value", FAKE), o.get("kc", FAKE), o.get("vc", FAKE),
+                        o.get("slots", FAKE), o.get("T", 4), o.get("NB", 8), o.get("Hkv", 2), o.get("D", 64),
+                        o.get("bs", 16), o.get("dt", 1), None, None]
+    assert _rc(*args(bs=8)) == pa.PA_ERR_UNSUPPORTED
+    assert _rc(*args(D=96)) == pa.PA_ERR_UNSUPPORTED
+    assert _rc(*args(T=-1)) == pa.PA_ERR_INVALID_ARG
+    assert _rc(*args(key=P(0))) == pa.PA_ERR_INVALID_ARG
+    assert _rc(*args(slots=P(0))) == pa.PA_ERR_INVALID_ARG
+    assert _rc(*args(dt=7)) == pa.PA_ERR_INVALID_ARG
+    assert _rc(*args(kc=P(0x1008))) == pa.PA_ERR_INVALID_ARG   # not 16-byte aligned
+    assert _rc(*args(T=0)) == pa.PA_OK                          # nothing to do
+    del ok
+
+
+def _dec(**o):
+    import paged_kv_cache_362_b200 as pa
+
+    a = [o.get("out", FAKE), o.get("q", FAKE), o.get("kc", FAKE), o.get("vc", FAKE), o.get("bt", FAKE),
+         o.get("MB", 4), o.get("cl", FAKE), o.get("B", 2), o.get("Hq", 4), o.get("Hkv", 2), o.get("D", 64),
+         o.get("bs", 16), o.get("NB", 8), ctypes.c_float(o.get("scale", 0.125)), o.get("maxctx", 64),
+         o.get("P", 0), o.get("ws", P(0x100000)), o.get("wsb", 1 << 20), o.get("dt", 1), None, None]
+    return pa._lib.LIB.pa_decode(*a)
+
+
+def test_decode_validation():
+    import paged_kv_cache_362_b200 as pa
+
+    assert _dec(Hq=5) == pa.PA_ERR_INVALID_ARG               # Hq not a multiple of Hkv
+    assert _dec(bs=32) == pa.PA_ERR_UNSUPPORTED
+    assert _dec(D=80) == pa.PA_ERR_UNSUPPORTED
+    assert _dec(Hkv=256, Hq=256) == pa.PA_ERR_UNSUPPORTED
+    assert _dec(P=24) == pa.PA_ERR_INVALID_ARG
+    assert _dec(P=1024) == pa.PA_ERR_INVALID_ARG
+    assert _dec(out=P(0)) == pa.PA_ERR_INVALID_ARG
+    assert _dec(ws=P(0)) == pa.PA_ERR_INVALID_ARG
+    assert _dec(ws=P(0x100010)) == pa.PA_ERR_INVALID_ARG     # workspace not 256-byte aligned
+    assert _dec(q=P(0x1004)) == pa.PA_ERR_INVALID_ARG
+    assert _dec(wsb=16) == pa.PA_ERR_INVALID_ARG             # workspace too small
+    assert _dec(scale=float("nan")) == pa.PA_ERR_INVALID_ARG
+    assert _dec(maxctx=-1) == pa.PA_ERR_INVALID_ARG
+    assert _dec(B=0) == pa.PA_OK
+
+
+def test_copy_blocks_validation():
+    import paged_kv_cache_362_b200 as pa
+
+    lib = pa._lib.LIB
+    assert lib.pa_copy_blocks(FAKE, FAKE, FAKE, -1, 8, 2, 64, 16, 1, None, None) == pa.PA_ERR_INVALID_ARG
+    assert lib.pa_copy_blocks(FAKE, FAKE, P(0), 3, 8, 2, 64, 16, 1, None, None) == pa.PA_ERR_INVALID_ARG
+    assert lib.pa_copy_blocks(FAKE, FAKE, FAKE, 3, 8, 2, 64, 12, 1, None, None) == pa.PA_ERR_UNSUPPORTED
+    assert lib.pa_copy_blocks(FAKE, FAKE, FAKE, 0, 8, 2, 64, 16, 1, None, None) == pa.PA_OK
+
+
+def test_host_copy_pair_checker():
+    import numpy as np
+
+    import paged_kv_cache_362_b200 as pa
+
+    pa.check_copy_pairs(np.array([[1, 3], [1, 4]]), 8)
+    with pytest.raises(ValueError):
+        pa.check_copy_pairs(np.array([[1, 3], [2, 3]]), 8)     # repeated dst
+    with pytest.raises(ValueError):
+        pa.check_copy_pairs(np.array([[1, 3], [3, 4]]), 8)     # dst that is also a src
+    with pytest.raises(ValueError):
+        pa.check_copy_pairs(np.array([[1, 9]]), 8)

@@ -159,7 +159,14 @@ def build_workload(cfg: WorkloadConfig, seed: int = 0, *, num_seqs: int | None =
         info.update(prefix_blocks=pre_blocks, parent_partial=parent_partial, shared_tokens_in_partial=r,
                     num_forks=nforks)
     else:
-        B = num_seqs or (len(context_lens) if context_lens is not None else cfg.num_seqs)
+        if num_seqs:
+            B = num_seqs
+        elif context_lens is not None:
+            B = len(context_lens)
+        elif cfg.ctx_kind == "fixed":
+            B = len(cfg.ctx_args)
+        else:
+            B = cfg.num_seqs
         if context_lens is not None:
             context = np.asarray(context_lens, dtype=np.int64)
         elif cfg.ctx_kind == "fixed" and num_seqs is not None and num_seqs != len(cfg.ctx_args):
