@@ -83,6 +83,32 @@ def dist_max(x: float) -> float:
     return float(t.item())
 
 
+def aggregate(kv_bytes_local: int, ms_local: float):
+    """Whole-job KV GB/s of a weak-scaling replica run and the max-over-ranks step time (ms).
+
+    Every rank processes its own replica; the job's throughput is the bytes all
+    ranks read divided by the slowest rank's step time.
+    """
+    import torch.distributed as dist
+
+    world = dist.get_world_size() if (dist.is_available() and dist.is_initialized()) else 1
+    ms = dist_max(ms_local)
+    total = dist_sum(float(kv_bytes_local))
+    return total / (ms * 1e-3) / 1e9, ms, world
+
+
+def dist_sum(x: float) -> float:
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()):
+        return x
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
 def dist_barrier():
     import torch.distributed as dist
 
@@ -416,10 +442,9 @@ def main():
     if status != 0:
         raise SystemExit(f"device status {status}: {w.pa.error_string(status)}")
 
-    ms = dist_max(float(np.mean(step_ms)))
+    value, ms, _ = aggregate(w.kv_bytes, float(np.mean(step_ms)))
+    total_bytes = dist_sum(float(w.kv_bytes))
     dec = dist_max(float(np.mean(dec_ms)))
-    total_bytes = w.kv_bytes * world
-    value = total_bytes / (ms * 1e-3) / 1e9
     achieved = w.kv_bytes / (dec * 1e-3) / 1e9
 
     e2e_ms, h2d, d2h = time_e2e(w, max(50, args.steps // 10), args.warmup, flush)

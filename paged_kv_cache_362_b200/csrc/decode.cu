@@ -36,6 +36,7 @@
 //  3. reduce  -- one warp per (b, h) of a multi-partition sequence:
 //                M = max m_p, L = sum l_p 2^(m_p - M),
 //                out = sum O_p 2^(m_p - M) / L.
+#include <cstdlib>
 #include <type_traits>
 #include <utility>
 
@@ -85,9 +86,10 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const DecodeParams p)
     // pass 2: place items (order inside a size class is irrelevant)
     for (int b0 = 0; b0 < p.num_seqs; b0 += blockDim.x) {
         const int b = b0 + threadIdx.x;
-        int nfull = 0, tail = -1;
+        int nfull = 0, tail = -1, ctx = 0;
         if (b < p.num_seqs) {
-            const int nblk = ceil_div_i(load_ctx(p, b, false), kBlockSize);
+            ctx = load_ctx(p, b, false);
+            const int nblk = ceil_div_i(ctx, kBlockSize);
             nfull = nblk / PB;
             const int t = nblk - nfull * PB;
             if (t > 0 || nblk == 0) tail = t;
@@ -104,10 +106,10 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const DecodeParams p)
         if (lane == 31 && incl) base = atomicAdd(&cursor[PB], incl);
         base = __shfl_sync(0xffffffffu, base, 31) + incl - mine;
         for (int j = 0; j < nfull; ++j)
-            for (int g = 0; g < Hkv; ++g) p.items[base + j * Hkv + g] = make_int2(b, (j << 8) | g);
+            for (int g = 0; g < Hkv; ++g) p.items[base + j * Hkv + g] = make_int4(b, (j << 8) | g, ctx, 0);
         if (tail >= 0) {
             const int tb = atomicAdd(&cursor[tail], Hkv);
-            for (int g = 0; g < Hkv; ++g) p.items[tb + g] = make_int2(b, (nfull << 8) | g);
+            for (int g = 0; g < Hkv; ++g) p.items[tb + g] = make_int4(b, (nfull << 8) | g, ctx, 0);
         }
     }
 }
@@ -116,12 +118,12 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const DecodeParams p)
 struct ItemGeom {
     int b, g, p, ctx, j0, nblk, nparts;
 };
-__device__ __forceinline__ ItemGeom item_geom(const DecodeParams& p, int2 it) {
+__device__ __forceinline__ ItemGeom item_geom(const DecodeParams& p, int4 it) {
     ItemGeom m;
     m.b = it.x;
     m.p = it.y >> 8;
     m.g = it.y & 255;
-    m.ctx = load_ctx(p, m.b, false);
+    m.ctx = it.z;
     const int nblk_total = ceil_div_i(m.ctx, kBlockSize);
     m.j0 = m.p * p.part_blocks;
     m.nblk = max(0, min(p.part_blocks, nblk_total - m.j0));
@@ -141,13 +143,20 @@ struct ItemMeta {
     int b, g, p, ctx, j0, nblk, nparts, pad;
 };
 
+// work-list entry and table row of one item, prefetched by the producer
+struct DescSlot {
+    int4 e;
+    int bt[kMaxPartBlocks];
+};
+
 template <int D, int NT, int NCW, int STAGES>
 struct TcCfg {
     static constexpr int kBoxes = D / 64;                    // 64-element (128 B) boxes per tile row
     static constexpr int kBoxBytes = kBlockSize * 128;       // 2 KB
     static constexpr int kTileBytes = kBlockSize * D * 2;    // one K or V tile
     static constexpr int kStageBytes = 2 * kTileBytes;
-    static constexpr int kISlots = 4;
+    static constexpr int kISlots = 4;                        // item metadata / Q ring
+    static constexpr int kDSlots = 4;                        // descriptor prefetch ring
     static constexpr int kHeadsPad = 8 * NT;
     static constexpr int kQBytes = kHeadsPad * D * 2;
     static constexpr int kMergeStride = D + 4;               // floats per head row (bank-conflict pad)
@@ -155,12 +164,14 @@ struct TcCfg {
     static constexpr int kOffQ = kOffStages + STAGES * kStageBytes;
     static constexpr int kOffMerge = kOffQ + kISlots * kQBytes;
     static constexpr int kOffMl = kOffMerge + NCW * kHeadsPad * kMergeStride * 4;
-    static constexpr int kOffMeta = kOffMl + NCW * kHeadsPad * 2 * 4;
+    static constexpr int kOffDesc = kOffMl + NCW * kHeadsPad * 2 * 4;
+    static constexpr int kOffMeta = kOffDesc + kDSlots * (int)sizeof(DescSlot);
     static constexpr int kOffBar = kOffMeta + kISlots * (int)sizeof(ItemMeta);
     static constexpr int kOffFlags = kOffBar + (2 * STAGES + 2 * kISlots) * 8;
     static constexpr int kBytes = kOffFlags + 16 + STAGES * 4;
     static constexpr int kSmemBytes = kBytes + 1024;         // slack for 1024-byte alignment
     static constexpr int kThreads = (NCW + 1) * 32;
+    static_assert(kOffDesc % 16 == 0 && sizeof(DescSlot) % 16 == 0, "cp.async 16-byte destinations");
 };
 
 template <typename T, int D, int NT, int NCW, int STAGES>
@@ -174,6 +185,7 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
     uint8_t* qbuf = smem + C::kOffQ;
     float* merge = reinterpret_cast<float*>(smem + C::kOffMerge);
     float* ml = reinterpret_cast<float*>(smem + C::kOffMl);
+    DescSlot* dsc = reinterpret_cast<DescSlot*>(smem + C::kOffDesc);
     ItemMeta* meta = reinterpret_cast<ItemMeta*>(smem + C::kOffMeta);
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
     uint64_t* empty = full + STAGES;
@@ -206,6 +218,7 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
     griddep_wait();
     const int n_items = *p.n_items;
     const int ctas = gridDim.x, cta = blockIdx.x;
+    const int PB = p.part_blocks;
 
     if (warp == NCW) {
         // ------------------------------------------------------------ producer
@@ -215,6 +228,40 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
         }
         const uint64_t pol = policy_evict_first();
         const size_t q_row_bytes = (size_t)D * 2;
+
+        // Descriptor pipeline, so that no global-memory latency sits between
+        // two items' tile loads: item k's work-list entry and table row land
+        // (cp.async) in slot k % kDSlots.  At the top of iteration i, entry(i),
+        // row(i) and entry(i+1) are visible and the group {row(i+1),
+        // entry(i+2)} is in flight; it completes while item i's tiles are
+        // being issued.
+        auto fetch_entry = [&](int it) {
+            const int r = item_rank(it, cta, ctas);
+            if (lane == 0 && r < n_items) cp_async_16(smem_u32(&dsc[it % C::kDSlots].e), &p.items[r]);
+        };
+        auto fetch_row = [&](int it) {
+            const int r = item_rank(it, cta, ctas);
+            if (r >= n_items) return;
+            const int4 e = dsc[it % C::kDSlots].e;
+            const int j0 = (e.y >> 8) * PB;
+            const int nblk = min(PB, ceil_div_i(e.z, kBlockSize) - j0);
+            if (lane < nblk)
+                cp_async_4(smem_u32(&dsc[it % C::kDSlots].bt[lane]),
+                           p.block_tables + (size_t)e.x * p.max_blocks_per_seq + j0 + lane);
+        };
+        fetch_entry(0);
+        cp_async_commit();
+        cp_async_wait_all();
+        __syncwarp();
+        fetch_row(0);
+        fetch_entry(1);
+        cp_async_commit();
+        cp_async_wait_all();
+        __syncwarp();
+        fetch_row(1);
+        fetch_entry(2);
+        cp_async_commit();
+
         uint32_t stage = 0;
         bool ok = true;
         for (int iter = 0; ok; ++iter) {
@@ -231,8 +278,8 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
                 }
                 break;
             }
-            const ItemGeom m = item_geom(p, p.items[rank]);
-            const int bt = lane < m.nblk ? p.block_tables[(size_t)m.b * p.max_blocks_per_seq + m.j0 + lane] : 0;
+            const DescSlot& d = dsc[iter % C::kDSlots];
+            const ItemGeom m = item_geom(p, d.e);
             if (lane == 0) {
                 meta[islot] = ItemMeta{m.b, m.g, m.p, m.ctx, m.j0, m.nblk, m.nparts, 0};
                 const uint32_t qbytes = (uint32_t)(G * q_row_bytes);
@@ -240,15 +287,10 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
                 bulk_load_1d(smem_u32(qbuf + islot * C::kQBytes),
                              static_cast<const uint8_t*>(p.q) + ((size_t)m.b * p.num_heads + (size_t)m.g * G) * q_row_bytes,
                              qbytes, &ifull[islot]);
-            }
-            for (int j = 0; j < m.nblk; ++j, ++stage) {
-                const int blk = __shfl_sync(0xffffffffu, bt, j);
-                const int s = stage % STAGES;
-                const uint32_t ph = (stage / STAGES) & 1;
-                int oks = 1;
-                if (lane == 0) oks = mbar_wait(&empty[s], ph ^ 1);
-                if (!__shfl_sync(0xffffffffu, oks, 0)) { ok = false; break; }
-                if (lane == 0) {
+                for (int j = 0; j < m.nblk; ++j, ++stage) {
+                    const int blk = d.bt[j];
+                    const int s = stage % STAGES;
+                    if (!mbar_wait(&empty[s], ((stage / STAGES) & 1) ^ 1)) { okw = 0; break; }
                     if (blk >= 0 && blk < p.num_blocks) {
                         stage_bad[s] = 0;
                         mbar_arrive_expect_tx(&full[s], C::kStageBytes);
@@ -267,20 +309,27 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
                     }
                 }
             }
-            if (*abort_flag) ok = false;
+            stage = __shfl_sync(0xffffffffu, stage, 0);
+            if (!__shfl_sync(0xffffffffu, okw, 0) || *abort_flag) { ok = false; break; }
+            // descriptors of items iter+2 and iter+3 start loading; item iter+1's are ready
+            cp_async_wait_all();
+            __syncwarp();
+            fetch_row(iter + 2);
+            fetch_entry(iter + 3);
+            cp_async_commit();
         }
+        cp_async_wait_all();
         if (!ok) {
             if (lane == 0) {
                 *abort_flag = 1;
                 set_status(p.status, PA_ERR_TIMEOUT);
-            }
-            // let copies already issued land before the CTA's memory is released
-            const uint32_t outstanding = stage < (uint32_t)STAGES ? stage : (uint32_t)STAGES;
-            if (lane == 0)
+                // let copies already issued land before the CTA's memory is released
+                const uint32_t outstanding = stage < (uint32_t)STAGES ? stage : (uint32_t)STAGES;
                 for (uint32_t k = 1; k <= outstanding; ++k) {
                     const uint32_t n = stage - k;
                     mbar_wait(&full[n % STAGES], (n / STAGES) & 1);
                 }
+            }
         }
         return;
     }
@@ -291,7 +340,17 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
     const int mi = lane >> 3, r8 = lane & 7;
     const float sl2 = p.scale_log2;
     constexpr int KS = D / 16;  // k-steps of QK^T == m-tiles of PV
+    constexpr bool kSplitP = std::is_same<T, __nv_bfloat16>::value;  // P as hi + lo bf16 pair
     uint32_t stage_base = 0;
+    // per-lane parts of the ldmatrix row addresses (tile-relative, bytes)
+    uint32_t koff[KS], voff[KS];
+#pragma unroll
+    for (int kk = 0; kk < KS; ++kk) {
+        const int kd0 = kk * 16 + 8 * (mi >> 1), ktok = r8 + 8 * (mi & 1);
+        koff[kk] = (kd0 >> 6) * C::kBoxBytes + ktok * 128 + ((((kd0 & 63) >> 3) ^ r8) << 4);
+        const int vd0 = kk * 16 + 8 * (mi & 1), vtok = r8 + 8 * (mi >> 1);
+        voff[kk] = C::kTileBytes + (vd0 >> 6) * C::kBoxBytes + vtok * 128 + ((((vd0 & 63) >> 3) ^ r8) << 4);
+    }
 
     for (int iter = 0;; ++iter) {
         const int islot = iter % C::kISlots;
@@ -339,31 +398,33 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
             }
             if (!stage_bad[s]) {
                 const int valid = min(kBlockSize, m.ctx - (m.j0 + j) * kBlockSize);
-                const uint32_t kbase = smem_u32(stages + s * C::kStageBytes);
-                const uint32_t vbase = kbase + C::kTileBytes;
+                const uint32_t tbase = smem_u32(stages + s * C::kStageBytes);
 
-                // ---- S^T[16 tokens x 8*NT heads] = K Q^T
-                float sacc[NT][4];
+                // ---- S^T[16 tokens x 8*NT heads] = K Q^T, two accumulator chains
+                float sa[NT][4], sb[NT][4];
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt) sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
-                const int ktok = r8 + 8 * (mi & 1);
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) sa[nt][c] = sb[nt][c] = 0.f;
 #pragma unroll
                 for (int kk = 0; kk < KS; ++kk) {
-                    const int d0 = kk * 16 + 8 * (mi >> 1);
-                    const uint32_t addr = kbase + (d0 >> 6) * C::kBoxBytes + ktok * 128 +
-                                          ((((d0 & 63) >> 3) ^ r8) << 4);
                     uint32_t a[4];
-                    ldsm_x4(addr, a[0], a[1], a[2], a[3]);
+                    ldsm_x4(tbase + koff[kk], a[0], a[1], a[2], a[3]);
 #pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) Mma<T>::run(sacc[nt], a, qf[nt][kk][0], qf[nt][kk][1]);
+                    for (int nt = 0; nt < NT; ++nt) {
+                        if (kk & 1) Mma<T>::run(sb[nt], a, qf[nt][kk][0], qf[nt][kk][1]);
+                        else Mma<T>::run(sa[nt], a, qf[nt][kk][0], qf[nt][kk][1]);
+                    }
                 }
 
                 // ---- online softmax per head column; P^T fragments for the PV product
-                uint32_t pb[NT][2];
+                uint32_t pb[NT][2], pl[NT][2];
+                bool rescale = false;
+                float al[NT][2];
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
-                    float s0 = sacc[nt][0] * sl2, s1 = sacc[nt][1] * sl2;
-                    float s2 = sacc[nt][2] * sl2, s3 = sacc[nt][3] * sl2;
+                    float s0 = (sa[nt][0] + sb[nt][0]) * sl2, s1 = (sa[nt][1] + sb[nt][1]) * sl2;
+                    float s2 = (sa[nt][2] + sb[nt][2]) * sl2, s3 = (sa[nt][3] + sb[nt][3]) * sl2;
                     if (gid >= valid) s0 = s1 = kNegInf;
                     if (gid + 8 >= valid) s2 = s3 = kNegInf;
                     float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
@@ -374,35 +435,49 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
                     }
                     const float mn0 = fmaxf(mrun[nt][0], mx0), mn1 = fmaxf(mrun[nt][1], mx1);
                     const float ms0 = mn0 == kNegInf ? 0.f : mn0, ms1 = mn1 == kNegInf ? 0.f : mn1;
-                    const float al0 = fast_exp2(mrun[nt][0] - ms0), al1 = fast_exp2(mrun[nt][1] - ms1);
+                    // alpha = 2^(m_old - m_new), exactly 1 when the running max did not move
+                    al[nt][0] = mn0 == mrun[nt][0] ? 1.f : fast_exp2(mrun[nt][0] - ms0);
+                    al[nt][1] = mn1 == mrun[nt][1] ? 1.f : fast_exp2(mrun[nt][1] - ms1);
+                    rescale |= (al[nt][0] != 1.f) | (al[nt][1] != 1.f);
                     mrun[nt][0] = mn0;
                     mrun[nt][1] = mn1;
                     const float p0 = fast_exp2(s0 - ms0), p1 = fast_exp2(s1 - ms1);
                     const float p2 = fast_exp2(s2 - ms0), p3 = fast_exp2(s3 - ms1);
-                    lrun[nt][0] = lrun[nt][0] * al0 + (p0 + p2);
-                    lrun[nt][1] = lrun[nt][1] * al1 + (p1 + p3);
-#pragma unroll
-                    for (int i = 0; i < KS; ++i) {
-                        o[nt][i][0] *= al0;
-                        o[nt][i][1] *= al1;
-                        o[nt][i][2] *= al0;
-                        o[nt][i][3] *= al1;
+                    lrun[nt][0] = lrun[nt][0] * al[nt][0] + (p0 + p2);
+                    lrun[nt][1] = lrun[nt][1] * al[nt][1] + (p1 + p3);
+                    const uint32_t h01 = Elt<T>::pack2(p0, p1), h23 = Elt<T>::pack2(p2, p3);
+                    pb[nt][0] = movmatrix_t(h01);
+                    pb[nt][1] = movmatrix_t(h23);
+                    if constexpr (kSplitP) {
+                        // remainder of p after bf16 rounding, itself in bf16: hi + lo carries ~16 bits
+                        const float2 f01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&h01));
+                        const float2 f23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&h23));
+                        pl[nt][0] = movmatrix_t(Elt<T>::pack2(p0 - f01.x, p1 - f01.y));
+                        pl[nt][1] = movmatrix_t(Elt<T>::pack2(p2 - f23.x, p3 - f23.y));
                     }
-                    pb[nt][0] = movmatrix_t(Elt<T>::pack2(p0, p1));
-                    pb[nt][1] = movmatrix_t(Elt<T>::pack2(p2, p3));
+                }
+                if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                        for (int i = 0; i < KS; ++i) {
+                            o[nt][i][0] *= al[nt][0];
+                            o[nt][i][1] *= al[nt][1];
+                            o[nt][i][2] *= al[nt][0];
+                            o[nt][i][3] *= al[nt][1];
+                        }
                 }
 
                 // ---- O^T[D x 8*NT] += V^T P^T
-                const int vtok = r8 + 8 * (mi >> 1);
 #pragma unroll
                 for (int i = 0; i < KS; ++i) {
-                    const int d0 = i * 16 + 8 * (mi & 1);
-                    const uint32_t addr = vbase + (d0 >> 6) * C::kBoxBytes + vtok * 128 +
-                                          ((((d0 & 63) >> 3) ^ r8) << 4);
                     uint32_t a[4];
-                    ldsm_x4_t(addr, a[0], a[1], a[2], a[3]);
+                    ldsm_x4_t(tbase + voff[i], a[0], a[1], a[2], a[3]);
 #pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) Mma<T>::run(o[nt][i], a, pb[nt][0], pb[nt][1]);
+                    for (int nt = 0; nt < NT; ++nt) {
+                        Mma<T>::run(o[nt][i], a, pb[nt][0], pb[nt][1]);
+                        if constexpr (kSplitP) Mma<T>::run(o[nt][i], a, pl[nt][0], pl[nt][1]);
+                    }
                 }
             }
             __syncwarp();
@@ -582,8 +657,16 @@ __global__ void __launch_bounds__(128) decode_reduce_kernel(const DecodeParams p
 // ===========================================================================
 namespace {
 
-constexpr int kNcw = 4;          // consumer warps per CTA
 constexpr int kStages = 16;      // shared-memory ring depth (one stage = one K and one V tile)
+
+// consumer warps per CTA: 4 by default; PA_TC_CONSUMER_WARPS=8 selects 8 (tuning)
+int tc_consumer_warps() {
+    static const int n = [] {
+        const char* e = getenv("PA_TC_CONSUMER_WARPS");
+        return (e && atoi(e) == 8) ? 8 : 4;
+    }();
+    return n;
+}
 
 PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
@@ -615,10 +698,10 @@ cudaError_t make_pool_map(CUtensorMap* map, const void* pool, pa_dtype dtype, in
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-template <typename T, int D, int NT>
+template <typename T, int D, int NT, int NCW>
 cudaError_t launch_tc(const DecodeParams& p, pa_dtype dtype, cudaStream_t stream, int max_items) {
-    using Cfg = TcCfg<D, NT, kNcw, kStages>;
-    auto kernel = decode_tc_kernel<T, D, NT, kNcw, kStages>;
+    using Cfg = TcCfg<D, NT, NCW, kStages>;
+    auto kernel = decode_tc_kernel<T, D, NT, NCW, kStages>;
     static bool attr_done = false;
     if (!attr_done) {
         cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
@@ -665,9 +748,15 @@ cudaError_t launch_all(const DecodeParams& p, pa_dtype dtype, cudaStream_t strea
     if constexpr (std::is_same<T, float>::value) {
         e = launch_simt<T, D>(p, stream, max_items);
     } else {
-        if (path == DecodePath::kTensorCore)
-            e = p.group <= 8 ? launch_tc<T, D, 1>(p, dtype, stream, max_items)
-                             : launch_tc<T, D, 2>(p, dtype, stream, max_items);
+        if (path == DecodePath::kTensorCore) {
+            const bool w8 = tc_consumer_warps() == 8;
+            if (p.group <= 8)
+                e = w8 ? launch_tc<T, D, 1, 8>(p, dtype, stream, max_items)
+                       : launch_tc<T, D, 1, 4>(p, dtype, stream, max_items);
+            else
+                e = w8 ? launch_tc<T, D, 2, 8>(p, dtype, stream, max_items)
+                       : launch_tc<T, D, 2, 4>(p, dtype, stream, max_items);
+        }
         else
             e = launch_simt<T, D>(p, stream, max_items);
     }

@@ -66,7 +66,7 @@ bool ws_layout(int64_t num_seqs, int64_t num_heads, int64_t num_kv_heads, int64_
     w->max_items = num_seqs * np * num_kv_heads;
     const int64_t parts = np > 1 ? num_seqs * num_heads * np : 0;
     w->off_items = 256;
-    w->off_m = round_up(w->off_items + (size_t)w->max_items * sizeof(int2), 256);
+    w->off_m = round_up(w->off_items + (size_t)w->max_items * sizeof(int4), 256);
     w->off_l = round_up(w->off_m + (size_t)parts * sizeof(float), 256);
     w->off_o = round_up(w->off_l + (size_t)parts * sizeof(float), 256);
     w->total = round_up(w->off_o + (size_t)parts * head_dim * sizeof(float), 256);
@@ -154,7 +154,7 @@ pa_status pa_decode(void* out, const void* q, const void* key_cache, const void*
     p.scale_log2 = scale * 1.4426950408889634f;  // log2(e)
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     p.n_items = reinterpret_cast<int32_t*>(ws);
-    p.items = reinterpret_cast<int2*>(ws + w.off_items);
+    p.items = reinterpret_cast<int4*>(ws + w.off_items);
     p.part_m = reinterpret_cast<float*>(ws + w.off_m);
     p.part_l = reinterpret_cast<float*>(ws + w.off_l);
     p.part_o = reinterpret_cast<float*>(ws + w.off_o);

@@ -134,6 +134,16 @@ __device__ __forceinline__ void bulk_load_1d(uint32_t dst, const void* src, uint
         "l"(src), "r"(bytes), "r"(smem_u32(bar))
         : "memory");
 }
+// per-thread async copies into shared memory (completion per thread via groups)
+__device__ __forceinline__ void cp_async_4(uint32_t dst, const void* src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -211,7 +221,7 @@ struct DecodeParams {
     float scale_log2;             // scale * log2(e)
     // workspace views
     int32_t* n_items;             // [1]
-    int2* items;                  // [max_items]: (b, (p << 8) | g), sorted by size, largest first
+    int4* items;                  // [max_items]: (b, (p << 8) | g, clamped ctx, 0), largest first
     float* part_m;                // [B, Hq, NP_max]   max logit (log2 units)
     float* part_l;                // [B, Hq, NP_max]   sum of 2^(s - m)
     float* part_o;                // [B, Hq, NP_max, D] unnormalised output
