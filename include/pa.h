@@ -157,6 +157,33 @@ pa_status pa_copy_blocks(void* key_cache, void* value_cache, const int64_t* bloc
                          int32_t head_dim, int32_t block_size, pa_dtype dtype, int32_t* status,
                          pa_stream_t stream);
 
+/*
+ * pa_decode_noalloc -- pa_decode without a caller-allocated workspace.
+ *
+ * The pages have no counterpart to this call; it exists for callers that
+ * cannot allocate device memory: code hosted by an engine that owns all
+ * device memory and gives its extensions no allocator, or a latency-critical
+ * loop that must not call cudaMalloc (which can synchronise the device).
+ * Arguments and results are those of pa_decode minus the workspace; the
+ * caller still passes every input and output buffer.
+ *
+ * The scratch is a fixed 32 MiB array in the library's device memory, held
+ * on every GPU that loads the library until the process exits.  A problem
+ * whose pa_decode_workspace_size() exceeds 32 MiB returns PA_ERR_UNSUPPORTED
+ * and enqueues nothing.  The first call made with a given device current
+ * looks up the array's device address (cudaGetSymbolAddress); make that first
+ * call before any stream capture begins.  No cudaMalloc or cudaFree is made.
+ * All calls share the one array: calls whose kernels overlap on the GPU (two
+ * streams, two host threads) race on it and give wrong results.  Nothing in
+ * it has to start at zero.
+ */
+pa_status pa_decode_noalloc(void* out, const void* q, const void* key_cache, const void* value_cache,
+                            const int32_t* block_tables, int32_t max_blocks_per_seq,
+                            const int32_t* context_lens, int32_t num_seqs, int32_t num_heads,
+                            int32_t num_kv_heads, int32_t head_dim, int32_t block_size, int32_t num_blocks,
+                            float scale, int32_t max_context_len, int32_t partition_size, pa_dtype dtype,
+                            int32_t* status, pa_stream_t stream);
+
 /* Static, human-readable name of a status code (or of the lowest bit set). */
 const char* pa_get_error_string(pa_status status);
 
