@@ -172,6 +172,13 @@ struct TcCfg {
     static constexpr int kSmemBytes = kBytes + 1024;         // slack for 1024-byte alignment
     static constexpr int kThreads = (NCW + 1) * 32;
     static_assert(kOffDesc % 16 == 0 && sizeof(DescSlot) % 16 == 0, "cp.async 16-byte destinations");
+    // Ring stage n and stage n + STAGES reuse one slot and one parity bit.  A
+    // consumer may only wait for stage n once stage n - STAGES (same slot, same
+    // parity) has been consumed, or it would take the old phase for the new
+    // one.  Within an item, block j goes to warp j % NCW, so with STAGES a
+    // multiple of NCW both stages belong to the same warp, which takes them in
+    // order; across items, the merge barrier at each item's end orders them.
+    static_assert(STAGES % NCW == 0, "ring depth must be a multiple of the consumer warps");
 };
 
 template <typename T, int D, int NT, int NCW, int STAGES>
