@@ -21,6 +21,7 @@ __global__ void __launch_bounds__(256) reshape_and_cache_kernel(
     const uint4* __restrict__ key, const uint4* __restrict__ value, uint4* __restrict__ key_cache,
     uint4* __restrict__ value_cache, const int64_t* __restrict__ slot_mapping, int64_t num_tokens,
     int num_kv_heads, int chunks_per_head, int64_t num_slots, int32_t* status) {
+    griddep_launch_dependents();
     griddep_wait();
     const int64_t chunks_per_token = (int64_t)num_kv_heads * chunks_per_head;
     const int64_t total = num_tokens * chunks_per_token;
@@ -48,6 +49,7 @@ __global__ void __launch_bounds__(256) copy_blocks_kernel(uint4* __restrict__ ke
                                                           const int64_t* __restrict__ pairs, int num_pairs,
                                                           int64_t num_blocks, int64_t block_chunks,
                                                           int32_t* status) {
+    griddep_launch_dependents();
     griddep_wait();
     const int k = blockIdx.x;
     if (k >= num_pairs) return;

@@ -37,6 +37,7 @@
 //                M = max m_p, L = sum l_p 2^(m_p - M),
 //                out = sum O_p 2^(m_p - M) / L.
 #include <cstdlib>
+#include <string>
 #include <type_traits>
 #include <utility>
 
@@ -51,67 +52,163 @@ constexpr float kNegInf = -__builtin_huge_valf();
 // ===========================================================================
 // 1. plan
 // ===========================================================================
+// Items are ordered by (class, size): first every item of the sequences that
+// span several partitions (their partial results must still be merged, so they
+// should finish early), then the single-partition sequences; within a class,
+// largest first.  Bucket key = class * (PB + 1) + (PB - blocks).
 __global__ void __launch_bounds__(1024) decode_plan_kernel(const DecodeParams p) {
-    __shared__ int cnt[kMaxPartBlocks + 1];
-    __shared__ int cursor[kMaxPartBlocks + 1];
+    constexpr int kThreads = 1024;
+    constexpr int kMaxKeys = 2 * (kMaxPartBlocks + 1);
+    __shared__ int cnt[kMaxKeys];
+    __shared__ int cursor[kMaxKeys];
+    __shared__ int preA[kThreads + 1];   // exclusive prefix of full-partition items, multi-partition class
+    __shared__ int preB[kThreads + 1];   // same, single-partition class
+    __shared__ int cctx[kThreads];
+    __shared__ int wsumA[kThreads / 32], wsumB[kThreads / 32];
+    __shared__ int nred;
+    // the partition kernel may launch now and set up; it waits for this grid to finish
+    griddep_launch_dependents();
     griddep_wait();
-    const int PB = p.part_blocks, Hkv = p.num_kv_heads;
-    const int lane = threadIdx.x & 31;
-    for (int i = threadIdx.x; i <= PB; i += blockDim.x) cnt[i] = 0;
+    const int PB = p.part_blocks, Hkv = p.num_kv_heads, KB = PB + 1;
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    for (int i = tid; i < 2 * KB; i += kThreads) cnt[i] = 0;
+    if (tid == 0) nred = 0;
+    for (int i = tid; i < p.num_seqs * Hkv; i += kThreads) p.merge_count[i] = 0;
     __syncthreads();
-    // pass 1: histogram of item sizes (in blocks)
-    for (int b0 = 0; b0 < p.num_seqs; b0 += blockDim.x) {
-        const int b = b0 + threadIdx.x;
-        int nfull = 0, tail = -1;
+    // pass 1: histogram of item keys (full-partition counts aggregated per warp)
+    for (int b0 = 0; b0 < p.num_seqs; b0 += kThreads) {
+        const int b = b0 + tid;
+        int fa = 0, fb = 0;
         if (b < p.num_seqs) {
             const int nblk = ceil_div_i(load_ctx(p, b, true), kBlockSize);
-            nfull = nblk / PB;
-            const int t = nblk - nfull * PB;
-            if (t > 0 || nblk == 0) tail = t;
+            const int nfull = nblk / PB, tail = nblk - nfull * PB;
+            const int cls = (nfull + (tail > 0)) > 1 ? 0 : 1;
+            (cls == 0 ? fa : fb) = nfull * Hkv;
+            if (tail > 0) atomicAdd(&cnt[cls * KB + PB - tail], Hkv);
+            if (nblk == 0) atomicAdd(&cnt[KB + PB], Hkv);
         }
-        const int wsum = __reduce_add_sync(0xffffffffu, nfull);
-        if (lane == 0 && wsum) atomicAdd(&cnt[PB], wsum);
-        if (tail >= 0) atomicAdd(&cnt[tail], 1);
+        fa = __reduce_add_sync(0xffffffffu, fa);
+        fb = __reduce_add_sync(0xffffffffu, fb);
+        if (lane == 0) {
+            if (fa) atomicAdd(&cnt[0], fa);
+            if (fb) atomicAdd(&cnt[KB], fb);
+        }
     }
     __syncthreads();
-    if (threadIdx.x == 0) {
-        int acc = 0;
-        for (int s = PB; s >= 0; --s) {
-            cursor[s] = acc;
-            acc += cnt[s] * Hkv;
+    // bucket offsets: warp 0 scans the (at most 66) keys, 3 per lane
+    if (wid == 0) {
+        int v[3], sum = 0;
+#pragma unroll
+        for (int k = 0; k < 3; ++k) {
+            const int key = lane * 3 + k;
+            v[k] = key < 2 * KB ? cnt[key] : 0;
+            sum += v[k];
         }
-        *p.n_items = acc;
-    }
-    __syncthreads();
-    // pass 2: place items (order inside a size class is irrelevant)
-    for (int b0 = 0; b0 < p.num_seqs; b0 += blockDim.x) {
-        const int b = b0 + threadIdx.x;
-        int nfull = 0, tail = -1, ctx = 0;
-        if (b < p.num_seqs) {
-            ctx = load_ctx(p, b, false);
-            const int nblk = ceil_div_i(ctx, kBlockSize);
-            nfull = nblk / PB;
-            const int t = nblk - nfull * PB;
-            if (t > 0 || nblk == 0) tail = t;
-        }
-        // warp-aggregated reservation in the full-partition class
-        const int mine = nfull * Hkv;
-        int incl = mine;
+        int incl = sum;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-            const int v = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += v;
+            const int u = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += u;
         }
-        int base = 0;
-        if (lane == 31 && incl) base = atomicAdd(&cursor[PB], incl);
-        base = __shfl_sync(0xffffffffu, base, 31) + incl - mine;
-        for (int j = 0; j < nfull; ++j)
-            for (int g = 0; g < Hkv; ++g) p.items[base + j * Hkv + g] = make_int4(b, (j << 8) | g, ctx, 0);
-        if (tail >= 0) {
-            const int tb = atomicAdd(&cursor[tail], Hkv);
-            for (int g = 0; g < Hkv; ++g) p.items[tb + g] = make_int4(b, (nfull << 8) | g, ctx, 0);
+        int acc = incl - sum;
+#pragma unroll
+        for (int k = 0; k < 3; ++k) {
+            const int key = lane * 3 + k;
+            if (key < 2 * KB) cursor[key] = acc;
+            acc += v[k];
+        }
+        if (lane == 31) {
+            *p.n_items = incl;
+            *p.item_counter = 0;
         }
     }
+    __syncthreads();
+    // pass 2: place items; order inside a bucket does not matter
+    for (int b0 = 0; b0 < p.num_seqs; b0 += kThreads) {
+        const int b = b0 + tid;
+        int nfull = 0, tail = 0, ctx = 0, nblk = 0;
+        if (b < p.num_seqs) {
+            ctx = load_ctx(p, b, false);
+            nblk = ceil_div_i(ctx, kBlockSize);
+            nfull = nblk / PB;
+            tail = nblk - nfull * PB;
+        }
+        const bool valid = b < p.num_seqs;
+        const bool multi = valid && (nfull + (tail > 0)) > 1;
+        if (valid && (tail > 0 || nblk == 0)) {
+            const int key = nblk == 0 ? KB + PB : (multi ? 0 : KB) + PB - tail;
+            const int tb = atomicAdd(&cursor[key], Hkv);
+            for (int g = 0; g < Hkv; ++g) p.items[tb + g] = make_int4(b, (nfull << 8) | g, ctx, 0);
+        }
+        // multi-partition sequences go to the reduce kernel's list
+        const unsigned mm = __ballot_sync(0xffffffffu, multi);
+        int rb = 0;
+        if (lane == 0 && mm) rb = atomicAdd(&nred, __popc(mm));
+        rb = __shfl_sync(0xffffffffu, rb, 0);
+        if (multi) p.red_seqs[rb + __popc(mm & ((1u << lane) - 1))] = b;
+        // block-wide exclusive scans of the full-partition item counts, per class
+        const int vA = multi ? nfull * Hkv : 0, vB = multi ? 0 : nfull * Hkv;
+        int ia = vA, ib = vB;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int ua = __shfl_up_sync(0xffffffffu, ia, o), ub = __shfl_up_sync(0xffffffffu, ib, o);
+            if (lane >= o) {
+                ia += ua;
+                ib += ub;
+            }
+        }
+        if (lane == 31) {
+            wsumA[wid] = ia;
+            wsumB[wid] = ib;
+        }
+        cctx[tid] = ctx;
+        __syncthreads();
+        if (wid == 0) {
+            int xa = wsumA[lane], xb = wsumB[lane];
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int ua = __shfl_up_sync(0xffffffffu, xa, o), ub = __shfl_up_sync(0xffffffffu, xb, o);
+                if (lane >= o) {
+                    xa += ua;
+                    xb += ub;
+                }
+            }
+            wsumA[lane] = xa;
+            wsumB[lane] = xb;
+        }
+        __syncthreads();
+        const int ea = ia - vA + (wid > 0 ? wsumA[wid - 1] : 0);
+        const int eb = ib - vB + (wid > 0 ? wsumB[wid - 1] : 0);
+        preA[tid] = ea;
+        preB[tid] = eb;
+        if (tid == kThreads - 1) {
+            preA[kThreads] = ea + vA;
+            preB[kThreads] = eb + vB;
+        }
+        __syncthreads();
+        // one thread per full-partition item: find its sequence by binary search over the prefix
+        for (int cls = 0; cls < 2; ++cls) {
+            const int* pre = cls == 0 ? preA : preB;
+            const int total = pre[kThreads], base = cursor[cls * KB];
+            for (int i = tid; i < total; i += kThreads) {
+                int lo = 0, hi = kThreads;
+                while (hi - lo > 1) {
+                    const int mid = (lo + hi) >> 1;
+                    if (pre[mid] <= i) lo = mid;
+                    else hi = mid;
+                }
+                const int r = i - pre[lo];
+                p.items[base + i] = make_int4(b0 + lo, ((r / Hkv) << 8) | (r % Hkv), cctx[lo], 0);
+            }
+        }
+        __syncthreads();
+        if (tid == 0) {
+            cursor[0] += preA[kThreads];
+            cursor[KB] += preB[kThreads];
+        }
+        __syncthreads();
+    }
+    if (tid == 0) *p.n_red = nred;
 }
 
 // geometry of one item, identical in every kernel
@@ -131,14 +228,56 @@ __device__ __forceinline__ ItemGeom item_geom(const DecodeParams& p, int4 it) {
     return m;
 }
 
-// snake assignment of sorted items to persistent CTAs
-__device__ __forceinline__ int item_rank(int iter, int cta, int ctas) {
-    return iter * ctas + ((iter & 1) ? (ctas - 1 - cta) : cta);
-}
-
 // ===========================================================================
 // 2a. partition kernel, tensor cores (fp16 / bf16)
 // ===========================================================================
+// Fused merge (single-warp CTAs, at most kFusedMaxParts partitions): one warp
+// combines every partition of (sequence b, KV head g) for the G query heads of
+// the group, out = sum_p O_p 2^(m_p - M) / sum_p l_p 2^(m_p - M).  The
+// partials were written by other CTAs: cache-global loads.
+constexpr int kFusedMaxParts = 16;
+
+template <typename T, int D>
+__device__ __forceinline__ void merge_group(const DecodeParams& p, int b, int g, int nparts, int lane) {
+    constexpr int E = D / 32;
+    using VecE = typename std::conditional<E == 4, float4, float2>::type;
+    const int G = p.group;
+    T* out = static_cast<T*>(p.out);
+    for (int h = 0; h < G; ++h) {
+        const size_t hq = (size_t)b * p.num_heads + (size_t)g * G + h;
+        const size_t base = hq * p.max_parts;
+        const float mq = lane < nparts ? __ldcg(p.part_m + base + lane) : kNegInf;
+        const float lq = lane < nparts ? __ldcg(p.part_l + base + lane) : 0.f;
+        VecE v[kFusedMaxParts];
+#pragma unroll
+        for (int q = 0; q < kFusedMaxParts; ++q)
+            if (q < nparts) v[q] = __ldcg(reinterpret_cast<const VecE*>(p.part_o + (base + q) * D + lane * E));
+        float M = mq;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+        const float Ms = M == kNegInf ? 0.f : M;
+        const float w = lane < nparts ? fast_exp2(mq - Ms) : 0.f;
+        float L = w * lq;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
+        float acc[E];
+#pragma unroll
+        for (int e = 0; e < E; ++e) acc[e] = 0.f;
+#pragma unroll
+        for (int q = 0; q < kFusedMaxParts; ++q) {
+            const float wq = __shfl_sync(0xffffffffu, w, q);
+            if (q < nparts) {
+                const float* f = reinterpret_cast<const float*>(&v[q]);
+#pragma unroll
+                for (int e = 0; e < E; ++e) acc[e] += wq * f[e];
+            }
+        }
+        const float inv = L > 0.f ? 1.f / L : 0.f;
+#pragma unroll
+        for (int e = 0; e < E; ++e) out[hq * D + lane * E + e] = Elt<T>::from_f(acc[e] * inv);
+    }
+}
+
 struct ItemMeta {
     int b, g, p, ctx, j0, nblk, nparts, pad;
 };
@@ -147,6 +286,8 @@ struct ItemMeta {
 struct DescSlot {
     int4 e;
     int bt[kMaxPartBlocks];
+    int rank;      // position in the work list (claimed from the shared counter)
+    int pad[3];
 };
 
 template <int D, int NT, int NCW, int STAGES>
@@ -155,34 +296,40 @@ struct TcCfg {
     static constexpr int kBoxBytes = kBlockSize * 128;       // 2 KB
     static constexpr int kTileBytes = kBlockSize * D * 2;    // one K or V tile
     static constexpr int kStageBytes = 2 * kTileBytes;
-    static constexpr int kISlots = 4;                        // item metadata / Q ring
+    static constexpr int kISlots = NCW == 1 ? 2 : 4;         // item metadata / Q ring
     static constexpr int kDSlots = 4;                        // descriptor prefetch ring
+    static constexpr int kMSlots = NCW == 1 ? 0 : 2;         // merge buffers (double-buffered; none for one warp)
     static constexpr int kHeadsPad = 8 * NT;
     static constexpr int kQBytes = kHeadsPad * D * 2;
     static constexpr int kMergeStride = D + 4;               // floats per head row (bank-conflict pad)
+    static constexpr int kMergeFloats = NCW * kHeadsPad * kMergeStride;   // one merge buffer
     static constexpr int kOffStages = 0;
     static constexpr int kOffQ = kOffStages + STAGES * kStageBytes;
     static constexpr int kOffMerge = kOffQ + kISlots * kQBytes;
-    static constexpr int kOffMl = kOffMerge + NCW * kHeadsPad * kMergeStride * 4;
-    static constexpr int kOffDesc = kOffMl + NCW * kHeadsPad * 2 * 4;
+    static constexpr int kOffMl = kOffMerge + kMSlots * kMergeFloats * 4;
+    static constexpr int kOffDesc = kOffMl + kMSlots * NCW * kHeadsPad * 2 * 4;
     static constexpr int kOffMeta = kOffDesc + kDSlots * (int)sizeof(DescSlot);
-    static constexpr int kOffBar = kOffMeta + kISlots * (int)sizeof(ItemMeta);
-    static constexpr int kOffFlags = kOffBar + (2 * STAGES + 2 * kISlots) * 8;
+    static constexpr int kQSlots = NCW == 1 ? 4 : 0;          // merge-task queue (single-warp CTAs)
+    static constexpr int kOffTasks = kOffMeta + kISlots * (int)sizeof(ItemMeta);
+    static constexpr int kOffBar = kOffTasks + kQSlots * 16;
+    static constexpr int kNumBars = 2 * STAGES + 2 * kISlots + 2 * kMSlots + 2 * kQSlots;
+    static constexpr int kOffFlags = kOffBar + kNumBars * 8;
     static constexpr int kBytes = kOffFlags + 16 + STAGES * 4;
     static constexpr int kSmemBytes = kBytes + 1024;         // slack for 1024-byte alignment
-    static constexpr int kThreads = (NCW + 1) * 32;
+    // warps: NCW consumers, one producer, and (single-warp CTAs) one merger
+    static constexpr int kWarps = NCW + 1 + (NCW == 1 ? 1 : 0);
+    static constexpr int kThreads = kWarps * 32;
     static_assert(kOffDesc % 16 == 0 && sizeof(DescSlot) % 16 == 0, "cp.async 16-byte destinations");
-    // Ring stage n and stage n + STAGES reuse one slot and one parity bit.  A
-    // consumer may only wait for stage n once stage n - STAGES (same slot, same
-    // parity) has been consumed, or it would take the old phase for the new
-    // one.  Within an item, block j goes to warp j % NCW, so with STAGES a
-    // multiple of NCW both stages belong to the same warp, which takes them in
-    // order; across items, the merge barrier at each item's end orders them.
+    // Ring stage n and stage n + STAGES reuse one slot and one parity bit, so a
+    // consumer may only wait for stage n once stage n - STAGES has landed, or it
+    // would take the old phase for the new one.  Stage n is consumed by warp
+    // n % NCW; with STAGES a multiple of NCW both stages belong to the same
+    // warp, which takes its stages in order.
     static_assert(STAGES % NCW == 0, "ring depth must be a multiple of the consumer warps");
 };
 
 template <typename T, int D, int NT, int NCW, int STAGES>
-__global__ void __launch_bounds__((NCW + 1) * 32, 1)
+__global__ void __launch_bounds__(TcCfg<D, NT, NCW, STAGES>::kThreads, 1)
     decode_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV) {
     using C = TcCfg<D, NT, NCW, STAGES>;
@@ -198,6 +345,11 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
     uint64_t* empty = full + STAGES;
     uint64_t* ifull = empty + STAGES;
     uint64_t* iempty = ifull + C::kISlots;
+    uint64_t* mfull = iempty + C::kISlots;       // all NCW warps deposited their item state
+    uint64_t* mempty = mfull + C::kMSlots;       // the item's merger has read the buffer
+    uint64_t* qfull = mempty + C::kMSlots;       // a merge task is queued
+    uint64_t* qempty = qfull + C::kQSlots;       // the merger took it
+    int4* tasks = reinterpret_cast<int4*>(smem + C::kOffTasks);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffFlags);
     volatile int* stage_bad = reinterpret_cast<volatile int*>(smem + C::kOffFlags + 16);
 
@@ -213,6 +365,14 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
             mbar_init(&ifull[i], 1);
             mbar_init(&iempty[i], NCW);
         }
+        for (int i = 0; i < C::kMSlots; ++i) {
+            mbar_init(&mfull[i], NCW);
+            mbar_init(&mempty[i], 1);
+        }
+        for (int i = 0; i < C::kQSlots; ++i) {
+            mbar_init(&qfull[i], 1);
+            mbar_init(&qempty[i], 1);
+        }
         *abort_flag = 0;
         mbar_fence_init();
     }
@@ -222,10 +382,32 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     __syncthreads();
 
+    griddep_launch_dependents();
     griddep_wait();
     const int n_items = *p.n_items;
-    const int ctas = gridDim.x, cta = blockIdx.x;
     const int PB = p.part_blocks;
+
+    if constexpr (NCW == 1) {
+        if (warp == NCW + 1) {
+            // -------------------------------------------------------- merger
+            // Takes (sequence, KV head) groups whose last partition this CTA
+            // finished and merges all their partitions, off the consumer's path.
+            for (int t = 0;; ++t) {
+                const int qs = t % C::kQSlots;
+                if (!__all_sync(0xffffffffu, mbar_wait(&qfull[qs], (t / C::kQSlots) & 1)) || *abort_flag) {
+                    *abort_flag = 1;
+                    break;
+                }
+                const int4 task = tasks[qs];
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&qempty[qs]);
+                if (task.x < 0) break;
+                __threadfence();
+                merge_group<T, D>(p, task.x, task.y, task.z, lane);
+            }
+            return;
+        }
+    }
 
     if (warp == NCW) {
         // ------------------------------------------------------------ producer
@@ -236,18 +418,21 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
         const uint64_t pol = policy_evict_first();
         const size_t q_row_bytes = (size_t)D * 2;
 
+        // Work is claimed dynamically from a counter the plan kernel reset, in the
+        // plan's largest-first order, so CTAs that finish early take more items.
         // Descriptor pipeline, so that no global-memory latency sits between
-        // two items' tile loads: item k's work-list entry and table row land
-        // (cp.async) in slot k % kDSlots.  At the top of iteration i, entry(i),
-        // row(i) and entry(i+1) are visible and the group {row(i+1),
-        // entry(i+2)} is in flight; it completes while item i's tiles are
-        // being issued.
-        auto fetch_entry = [&](int it) {
-            const int r = item_rank(it, cta, ctas);
-            if (lane == 0 && r < n_items) cp_async_16(smem_u32(&dsc[it % C::kDSlots].e), &p.items[r]);
+        // two items' tile loads: item k's claimed rank, work-list entry and
+        // table row land in slot k % kDSlots.  At the top of iteration i,
+        // entry(i), row(i) and entry(i+1) are visible, the group {row(i+1),
+        // entry(i+2)} is in flight, and the claim of item i+3 is in a register.
+        auto fetch_entry = [&](int it, int r) {
+            if (lane == 0) {
+                dsc[it % C::kDSlots].rank = r;
+                if (r < n_items) cp_async_16(smem_u32(&dsc[it % C::kDSlots].e), &p.items[r]);
+            }
         };
         auto fetch_row = [&](int it) {
-            const int r = item_rank(it, cta, ctas);
+            const int r = dsc[it % C::kDSlots].rank;
             if (r >= n_items) return;
             const int4 e = dsc[it % C::kDSlots].e;
             const int j0 = (e.y >> 8) * PB;
@@ -256,45 +441,105 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
                 cp_async_4(smem_u32(&dsc[it % C::kDSlots].bt[lane]),
                            p.block_tables + (size_t)e.x * p.max_blocks_per_seq + j0 + lane);
         };
-        fetch_entry(0);
+        // The first kStaticRounds items of every CTA are fixed (snake order over
+        // the largest-first list); after that CTAs claim the next item from the
+        // counter, so that CTAs which finish early take more of the small ones.
+        constexpr int kStaticRounds = 3;
+        const int ctas = gridDim.x, cta = blockIdx.x;
+        auto static_rank = [&](int it) { return it * ctas + ((it & 1) ? (ctas - 1 - cta) : cta); };
+        auto claim = [&](int it) {
+            if (it < kStaticRounds || p.static_schedule) return static_rank(it);
+            return kStaticRounds * ctas + atomicAdd(p.item_counter, 1);
+        };
+        int r0 = 0, r1 = 0, r2 = 0, claim_next = 0;
+        if (lane == 0) {
+            r0 = claim(0);
+            r1 = claim(1);
+            r2 = claim(2);
+            claim_next = claim(3);
+        }
+        fetch_entry(0, r0);
         cp_async_commit();
         cp_async_wait_all();
         __syncwarp();
         fetch_row(0);
-        fetch_entry(1);
+        fetch_entry(1, r1);
         cp_async_commit();
         cp_async_wait_all();
         __syncwarp();
         fetch_row(1);
-        fetch_entry(2);
+        fetch_entry(2, r2);
         cp_async_commit();
+        __syncwarp();
 
-        uint32_t stage = 0;
-        bool ok = true;
-        for (int iter = 0; ok; ++iter) {
-            const int rank = item_rank(iter, cta, ctas);
-            const int islot = iter % C::kISlots;
-            const uint32_t iph = (iter / C::kISlots) & 1;
+        // Item k's metadata and Q rows are published (and the Q copy issued) at
+        // the start of item k-1's tile stream, so they have landed by the time
+        // the consumers reach item k.  publish() returns 1 if item `it` was
+        // published, 0 at the end of the work list (sentinel published), -1 on
+        // a wait that timed out.
+        auto publish = [&](int it) -> int {
+            const int islot = it % C::kISlots;
             int okw = 1;
-            if (lane == 0) okw = mbar_wait(&iempty[islot], iph ^ 1);
-            if (!__shfl_sync(0xffffffffu, okw, 0)) { ok = false; break; }
-            if (rank >= n_items) {
+            if (lane == 0) okw = mbar_wait(&iempty[islot], ((it / C::kISlots) & 1) ^ 1);
+            if (!__shfl_sync(0xffffffffu, okw, 0)) return -1;
+            const DescSlot& dd = dsc[it % C::kDSlots];
+            if (dd.rank >= n_items) {
                 if (lane == 0) {
                     meta[islot].nblk = -1;
                     mbar_arrive(&ifull[islot]);
                 }
-                break;
+                return 0;
             }
-            const DescSlot& d = dsc[iter % C::kDSlots];
-            const ItemGeom m = item_geom(p, d.e);
             if (lane == 0) {
-                meta[islot] = ItemMeta{m.b, m.g, m.p, m.ctx, m.j0, m.nblk, m.nparts, 0};
+                const ItemGeom mm = item_geom(p, dd.e);
+                meta[islot] = ItemMeta{mm.b, mm.g, mm.p, mm.ctx, mm.j0, mm.nblk, mm.nparts, 0};
                 const uint32_t qbytes = (uint32_t)(G * q_row_bytes);
                 mbar_arrive_expect_tx(&ifull[islot], qbytes);
                 bulk_load_1d(smem_u32(qbuf + islot * C::kQBytes),
-                             static_cast<const uint8_t*>(p.q) + ((size_t)m.b * p.num_heads + (size_t)m.g * G) * q_row_bytes,
+                             static_cast<const uint8_t*>(p.q) +
+                                 ((size_t)mm.b * p.num_heads + (size_t)mm.g * G) * q_row_bytes,
                              qbytes, &ifull[islot]);
-                for (int j = 0; j < m.nblk; ++j, ++stage) {
+            }
+            return 1;
+        };
+
+        // With 4 item slots, item k+1 is published while item k streams; with 2
+        // (single-warp CTAs) that would hold the producer back to one item ahead
+        // of the consumer, so item k is published when its tiles start.
+        constexpr int kLook = C::kISlots >= 4 ? 1 : 0;
+        uint32_t stage = 0;
+        int npub = 0;  // items whose Q copy was issued
+        bool ok = true;
+        int pub = publish(0);
+        if (pub < 0) ok = false;
+        npub += pub > 0;
+        bool more = pub > 0;   // item iter exists
+        for (int iter = 0; ok && more; ++iter) {
+            if (kLook) {
+                pub = publish(iter + 1);
+                if (pub < 0) { ok = false; break; }
+                npub += pub > 0;
+                more = pub > 0;
+            } else if (iter > 0) {
+                pub = publish(iter);
+                if (pub < 0) { ok = false; break; }
+                npub += pub > 0;
+                if (pub == 0) break;
+            }
+            const DescSlot& d = dsc[iter % C::kDSlots];
+            const ItemGeom m = item_geom(p, d.e);
+            int okw = 1;
+            if (lane == 0) {
+                // each item starts on a stage that is a multiple of NCW, so block j
+                // always goes to consumer warp j % NCW wherever the item runs
+                // (bitwise-reproducible results); the padding stages carry no data
+                for (; stage % NCW != 0; ++stage) {
+                    const int s = stage % STAGES;
+                    if (!mbar_wait(&empty[s], ((stage / STAGES) & 1) ^ 1)) { okw = 0; break; }
+                    stage_bad[s] = 1;
+                    mbar_arrive(&full[s]);
+                }
+                for (int j = 0; j < m.nblk && okw; ++j, ++stage) {
                     const int blk = d.bt[j];
                     const int s = stage % STAGES;
                     if (!mbar_wait(&empty[s], ((stage / STAGES) & 1) ^ 1)) { okw = 0; break; }
@@ -318,12 +563,15 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
             }
             stage = __shfl_sync(0xffffffffu, stage, 0);
             if (!__shfl_sync(0xffffffffu, okw, 0) || *abort_flag) { ok = false; break; }
+            if (!kLook) more = true;
             // descriptors of items iter+2 and iter+3 start loading; item iter+1's are ready
             cp_async_wait_all();
             __syncwarp();
             fetch_row(iter + 2);
-            fetch_entry(iter + 3);
+            fetch_entry(iter + 3, claim_next);
+            if (lane == 0 && claim_next < n_items) claim_next = claim(iter + 4);
             cp_async_commit();
+            __syncwarp();
         }
         cp_async_wait_all();
         if (!ok) {
@@ -335,6 +583,11 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
                 for (uint32_t k = 1; k <= outstanding; ++k) {
                     const uint32_t n = stage - k;
                     mbar_wait(&full[n % STAGES], (n / STAGES) & 1);
+                }
+                const int qout = npub < C::kISlots ? npub : C::kISlots;
+                for (int k = 1; k <= qout; ++k) {
+                    const int it = npub - k;
+                    mbar_wait(&ifull[it % C::kISlots], (it / C::kISlots) & 1);
                 }
             }
         }
@@ -349,6 +602,7 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
     constexpr int KS = D / 16;  // k-steps of QK^T == m-tiles of PV
     constexpr bool kSplitP = std::is_same<T, __nv_bfloat16>::value;  // P as hi + lo bf16 pair
     uint32_t stage_base = 0;
+    int nq = 0;  // merge tasks queued (single-warp CTAs)
     // per-lane parts of the ldmatrix row addresses (tile-relative, bytes)
     uint32_t koff[KS], voff[KS];
 #pragma unroll
@@ -396,9 +650,24 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
             for (int i = 0; i < KS; ++i) o[nt][i][0] = o[nt][i][1] = o[nt][i][2] = o[nt][i][3] = 0.f;
         }
 
-        for (int j = cw; j < m.nblk; j += NCW) {
-            const uint32_t n = stage_base + j;
+        // padding stages in front of the item (see the producer), then the
+        // item's blocks: block j is stage item_base + j, owned by warp j % NCW
+        const uint32_t item_base = (stage_base + NCW - 1) / NCW * NCW;
+        for (uint32_t n = stage_base + (((uint32_t)cw + NCW - stage_base % NCW) % NCW); n < item_base; n += NCW) {
             const int s = n % STAGES;
+            if (!__all_sync(0xffffffffu, mbar_wait(&full[s], (n / STAGES) & 1)) || *abort_flag) {
+                *abort_flag = 1;
+                break;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[s]);
+        }
+        stage_base = item_base;
+        const uint32_t item_end = stage_base + (uint32_t)m.nblk;
+        uint32_t n = stage_base + (uint32_t)cw;
+        for (; n < item_end; n += NCW) {
+            const int s = n % STAGES;
+            const int j = (int)(n - stage_base);
             if (!__all_sync(0xffffffffu, mbar_wait(&full[s], (n / STAGES) & 1)) || *abort_flag) {
                 *abort_flag = 1;
                 break;
@@ -490,17 +759,85 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[s]);
         }
-        stage_base += (uint32_t)m.nblk;
+        stage_base = item_end;
+        if (*abort_flag) break;
 
-        // ---- merge the consumer warps' states, write output or partials
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
             for (int c = 0; c < 2; ++c)
 #pragma unroll
                 for (int off = 4; off < 32; off <<= 1) lrun[nt][c] += __shfl_xor_sync(0xffffffffu, lrun[nt][c], off);
+
+        if constexpr (NCW == 1) {
+            // ---- a single warp owns the whole item: write the result straight from
+            // the accumulator fragments (thread holds dims 16i+gid, 16i+gid+8 of heads
+            // 2*t4 and 2*t4+1 of each n-tile)
+            T* out = static_cast<T*>(p.out);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    const int h = nt * 8 + 2 * t4 + c;
+                    if (h >= G) continue;
+                    const size_t hq = (size_t)m.b * p.num_heads + (size_t)m.g * G + h;
+                    if (m.nparts == 1) {
+                        const float inv = lrun[nt][c] > 0.f ? 1.f / lrun[nt][c] : 0.f;
+#pragma unroll
+                        for (int i = 0; i < KS; ++i) {
+                            out[hq * D + i * 16 + gid] = Elt<T>::from_f(o[nt][i][c] * inv);
+                            out[hq * D + i * 16 + gid + 8] = Elt<T>::from_f(o[nt][i][2 + c] * inv);
+                        }
+                    } else {
+                        const size_t pi = hq * p.max_parts + m.p;
+#pragma unroll
+                        for (int i = 0; i < KS; ++i) {
+                            p.part_o[pi * D + i * 16 + gid] = o[nt][i][c];
+                            p.part_o[pi * D + i * 16 + gid + 8] = o[nt][i][2 + c];
+                        }
+                        if (gid == 0) {
+                            p.part_m[pi] = mrun[nt][c];
+                            p.part_l[pi] = lrun[nt][c];
+                        }
+                    }
+                }
+            if (p.fused_merge && m.nparts > 1) {
+                // the CTA that finishes the group's last partition queues it for its merger warp
+                __threadfence();
+                __syncwarp();
+                int prev = 0;
+                if (lane == 0) {
+                    prev = atomicAdd(&p.merge_count[(size_t)m.b * p.num_kv_heads + m.g], 1);
+                    __threadfence();
+                }
+                prev = __shfl_sync(0xffffffffu, prev, 0);
+                if (prev == m.nparts - 1) {
+                    const int qs = nq % C::kQSlots;
+                    if (!__all_sync(0xffffffffu, mbar_wait(&qempty[qs], ((nq / C::kQSlots) & 1) ^ 1))) {
+                        *abort_flag = 1;
+                        break;
+                    }
+                    if (lane == 0) {
+                        tasks[qs] = make_int4(m.b, m.g, m.nparts, 0);
+                        mbar_arrive(&qfull[qs]);
+                    }
+                    ++nq;
+                }
+            }
+            continue;
+        }
+
+        // ---- deposit this warp's state in merge buffer iter % 2 (no CTA-wide barrier)
+        const int mslot = iter & 1;
+        const uint32_t mph = (iter >> 1) & 1;
+        if (!__all_sync(0xffffffffu, mbar_wait(&mempty[mslot], mph ^ 1))) {
+            *abort_flag = 1;
+            break;
+        }
+        float* mbuf = merge + mslot * C::kMergeFloats;
+        float* mlb = ml + mslot * NCW * C::kHeadsPad * 2;
         {
-            float* mo = merge + cw * C::kHeadsPad * C::kMergeStride;
+            float* mo = mbuf + cw * C::kHeadsPad * C::kMergeStride;
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
                 const int h0 = nt * 8 + 2 * t4;
@@ -513,45 +850,70 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
                     mo[(h0 + 1) * C::kMergeStride + d + 8] = o[nt][i][3];
                 }
                 if (gid == 0) {
-                    ml[(cw * C::kHeadsPad + h0) * 2 + 0] = mrun[nt][0];
-                    ml[(cw * C::kHeadsPad + h0) * 2 + 1] = lrun[nt][0];
-                    ml[(cw * C::kHeadsPad + h0 + 1) * 2 + 0] = mrun[nt][1];
-                    ml[(cw * C::kHeadsPad + h0 + 1) * 2 + 1] = lrun[nt][1];
+                    mlb[(cw * C::kHeadsPad + h0) * 2 + 0] = mrun[nt][0];
+                    mlb[(cw * C::kHeadsPad + h0) * 2 + 1] = lrun[nt][0];
+                    mlb[(cw * C::kHeadsPad + h0 + 1) * 2 + 0] = mrun[nt][1];
+                    mlb[(cw * C::kHeadsPad + h0 + 1) * 2 + 1] = lrun[nt][1];
                 }
             }
         }
-        named_bar_sync(1, NCW * 32);
-        {
-            const int tid = cw * 32 + lane;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&mfull[mslot]);
+
+        // ---- the item's merger (warp iter % NCW) combines the NCW states and writes the result
+        if (cw == iter % NCW) {
+            if (!__all_sync(0xffffffffu, mbar_wait(&mfull[mslot], mph))) {
+                *abort_flag = 1;
+                break;
+            }
             T* out = static_cast<T*>(p.out);
-            for (int e = tid; e < G * D; e += NCW * 32) {
-                const int h = e / D, d = e - h * D;
+            for (int h = 0; h < G; ++h) {
+                float mw[NCW];
                 float M = kNegInf;
 #pragma unroll
-                for (int w = 0; w < NCW; ++w) M = fmaxf(M, ml[(w * C::kHeadsPad + h) * 2]);
+                for (int w = 0; w < NCW; ++w) {
+                    mw[w] = mlb[(w * C::kHeadsPad + h) * 2];
+                    M = fmaxf(M, mw[w]);
+                }
                 const float Ms = M == kNegInf ? 0.f : M;
-                float L = 0.f, acc = 0.f;
+                float L = 0.f;
 #pragma unroll
                 for (int w = 0; w < NCW; ++w) {
-                    const float sc = fast_exp2(ml[(w * C::kHeadsPad + h) * 2] - Ms);
-                    L += sc * ml[(w * C::kHeadsPad + h) * 2 + 1];
-                    acc += sc * merge[(w * C::kHeadsPad + h) * C::kMergeStride + d];
+                    mw[w] = fast_exp2(mw[w] - Ms);
+                    L += mw[w] * mlb[(w * C::kHeadsPad + h) * 2 + 1];
                 }
                 const size_t hq = (size_t)m.b * p.num_heads + (size_t)m.g * G + h;
-                if (m.nparts == 1) {
-                    out[hq * D + d] = Elt<T>::from_f(L > 0.f ? acc / L : 0.f);
-                } else {
-                    const size_t pi = hq * p.max_parts + m.p;
-                    p.part_o[pi * D + d] = acc;
-                    if (d == 0) {
-                        p.part_m[pi] = M;
-                        p.part_l[pi] = L;
+                const float inv = L > 0.f ? 1.f / L : 0.f;
+#pragma unroll
+                for (int k = 0; k < D / 32; ++k) {
+                    const int d = k * 32 + lane;
+                    float acc = 0.f;
+#pragma unroll
+                    for (int w = 0; w < NCW; ++w) acc += mw[w] * mbuf[(w * C::kHeadsPad + h) * C::kMergeStride + d];
+                    if (m.nparts == 1) {
+                        out[hq * D + d] = Elt<T>::from_f(acc * inv);
+                    } else {
+                        p.part_o[(hq * p.max_parts + m.p) * D + d] = acc;
                     }
                 }
+                if (m.nparts > 1 && lane == 0) {
+                    p.part_m[hq * p.max_parts + m.p] = M;
+                    p.part_l[hq * p.max_parts + m.p] = L;
+                }
             }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&mempty[mslot]);
         }
-        named_bar_sync(1, NCW * 32);
-        if (*abort_flag) break;
+    }
+    if constexpr (NCW == 1) {
+        // tell the merger warp there is nothing more
+        const int qs = nq % C::kQSlots;
+        const bool okq = __all_sync(0xffffffffu, mbar_wait(&qempty[qs], ((nq / C::kQSlots) & 1) ^ 1));
+        if (lane == 0) {
+            if (!okq) *abort_flag = 1;
+            tasks[qs] = make_int4(-1, 0, 0, 0);
+            mbar_arrive(&qfull[qs]);
+        }
     }
     if (*abort_flag && lane == 0) set_status(p.status, PA_ERR_TIMEOUT);
 }
@@ -627,36 +989,71 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(const DecodeParams
 // ===========================================================================
 // 3. reduce
 // ===========================================================================
+// Rows (sequence, query head) of the sequences the plan listed; a CTA takes
+// rows in turn.  Its 4 warps split a row's partitions (warp w takes partitions
+// w, w + 4, ...; lane l owns D/32 consecutive dims), then add up through
+// shared memory.  Loads are cache-global: the partials were written by other
+// SMs in the previous kernel.
 template <typename T, int D>
 __global__ void __launch_bounds__(128) decode_reduce_kernel(const DecodeParams p) {
-    constexpr int E = D / 32;
+    constexpr int kW = 4, E = D / 32, U = 8;
+    __shared__ float sacc[kW][D];
+    __shared__ float sl[kW];
     griddep_wait();
-    const long long wi = (long long)blockIdx.x * 4 + (threadIdx.x >> 5);
-    const int lane = threadIdx.x & 31;
-    if (wi >= (long long)p.num_seqs * p.num_heads) return;
-    const int b = (int)(wi / p.num_heads);
-    const int ctx = load_ctx(p, b, false);
-    const int nparts = max(1, ceil_div_i(ceil_div_i(ctx, kBlockSize), p.part_blocks));
-    if (nparts <= 1) return;
-    const size_t base = (size_t)wi * p.max_parts;
-    float M = kNegInf;
-    for (int q = lane; q < nparts; q += 32) M = fmaxf(M, p.part_m[base + q]);
+    const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int Hq = p.num_heads;
+    const long long n_rows = (long long)(*p.n_red) * Hq;
+    for (long long r = blockIdx.x; r < n_rows; r += gridDim.x) {
+        const int b = p.red_seqs[r / Hq], h = (int)(r % Hq);
+        const int ctx = load_ctx(p, b, false);
+        const int nparts = max(1, ceil_div_i(ceil_div_i(ctx, kBlockSize), p.part_blocks));
+        const size_t base = ((size_t)b * Hq + h) * p.max_parts;
+        float M = kNegInf;
+        for (int q = lane; q < nparts; q += 32) M = fmaxf(M, __ldcg(p.part_m + base + q));
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-    const float Ms = M == kNegInf ? 0.f : M;
-    float L = 0.f, acc[E];
+        for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+        const float Ms = M == kNegInf ? 0.f : M;
+        float L = 0.f, acc[E];
 #pragma unroll
-    for (int e = 0; e < E; ++e) acc[e] = 0.f;
-    for (int q = 0; q < nparts; ++q) {
-        const float sc = fast_exp2(p.part_m[base + q] - Ms);
-        L += sc * p.part_l[base + q];
-        const float* po = p.part_o + (base + q) * D + lane * E;
+        for (int e = 0; e < E; ++e) acc[e] = 0.f;
+        for (int q0 = wid; q0 < nparts; q0 += kW * U) {
+            float w[U], v[U][E];
 #pragma unroll
-        for (int e = 0; e < E; ++e) acc[e] += sc * po[e];
+            for (int u = 0; u < U; ++u) {
+                const int q = q0 + u * kW;
+                w[u] = 0.f;
+                if (q < nparts) {
+                    w[u] = fast_exp2(__ldcg(p.part_m + base + q) - Ms);
+                    L += w[u] * __ldcg(p.part_l + base + q);
+                    const float* po = p.part_o + (base + q) * D + lane * E;
+#pragma unroll
+                    for (int e = 0; e < E; ++e) v[u][e] = __ldcg(po + e);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < E; ++e) v[u][e] = 0.f;
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+#pragma unroll
+                for (int e = 0; e < E; ++e) acc[e] += w[u] * v[u][e];
+        }
+#pragma unroll
+        for (int e = 0; e < E; ++e) sacc[wid][lane * E + e] = acc[e];
+        if (lane == 0) sl[wid] = L;
+        __syncthreads();
+        if (threadIdx.x < D) {
+            float a = 0.f, lt = 0.f;
+#pragma unroll
+            for (int w2 = 0; w2 < kW; ++w2) {
+                a += sacc[w2][threadIdx.x];
+                lt += sl[w2];
+            }
+            static_cast<T*>(p.out)[((size_t)b * Hq + h) * D + threadIdx.x] =
+                Elt<T>::from_f(lt > 0.f ? a * (1.f / lt) : 0.f);
+        }
+        __syncthreads();
     }
-    T* out = static_cast<T*>(p.out) + (size_t)wi * D + lane * E;
-#pragma unroll
-    for (int e = 0; e < E; ++e) out[e] = Elt<T>::from_f(L > 0.f ? acc[e] / L : 0.f);
 }
 
 // ===========================================================================
@@ -664,15 +1061,26 @@ __global__ void __launch_bounds__(128) decode_reduce_kernel(const DecodeParams p
 // ===========================================================================
 namespace {
 
-constexpr int kStages = 16;      // shared-memory ring depth (one stage = one K and one V tile)
-
-// consumer warps per CTA: 4 by default; PA_TC_CONSUMER_WARPS=8 selects 8 (tuning)
-int tc_consumer_warps() {
-    static const int n = [] {
-        const char* e = getenv("PA_TC_CONSUMER_WARPS");
-        return (e && atoi(e) == 8) ? 8 : 4;
+// Shapes of the tensor-core partition kernel (consumer warps x ring stages; CTAs per SM
+// at D = 128 and a GQA group of at most 8, as shared memory allows):
+//   kPaired: 2 x 10 (80 KB ring), 2 CTAs per SM, warps merge through shared memory
+//   kQuad:   1 x 6  (48 KB ring), 4 CTAs per SM, one warp per item, no merge
+//   kTriple: 1 x 8  (64 KB ring), 3 CTAs per SM
+//   kPair1:  1 x 13 (104 KB ring), 2 CTAs per SM
+// The ring holds the bytes in flight that cover HBM latency; each consumer
+// warp holds one stage while it computes.  PA_TC_SHAPE selects one (tuning).
+enum class TcShape { kAuto, kPaired, kQuad, kTriple, kPair1 };
+TcShape tc_shape() {
+    static const TcShape s = [] {
+        const char* e = getenv("PA_TC_SHAPE");
+        const std::string v = e ? e : "";
+        if (v == "paired") return TcShape::kPaired;
+        if (v == "quad") return TcShape::kQuad;
+        if (v == "triple") return TcShape::kTriple;
+        if (v == "pair1") return TcShape::kPair1;
+        return TcShape::kAuto;
     }();
-    return n;
+    return s;
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
@@ -705,10 +1113,10 @@ cudaError_t make_pool_map(CUtensorMap* map, const void* pool, pa_dtype dtype, in
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-template <typename T, int D, int NT, int NCW>
+template <typename T, int D, int NT, int NCW, int STAGES>
 cudaError_t launch_tc(const DecodeParams& p, pa_dtype dtype, cudaStream_t stream, int max_items) {
-    using Cfg = TcCfg<D, NT, NCW, kStages>;
-    auto kernel = decode_tc_kernel<T, D, NT, NCW, kStages>;
+    using Cfg = TcCfg<D, NT, NCW, STAGES>;
+    auto kernel = decode_tc_kernel<T, D, NT, NCW, STAGES>;
     static bool attr_done = false;
     if (!attr_done) {
         cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
@@ -747,30 +1155,46 @@ cudaError_t launch_simt(const DecodeParams& p, cudaStream_t stream, int max_item
 }
 
 template <typename T, int D>
-cudaError_t launch_all(const DecodeParams& p, pa_dtype dtype, cudaStream_t stream) {
+cudaError_t launch_all(DecodeParams p, pa_dtype dtype, cudaStream_t stream) {
     const int max_items = p.num_seqs * p.max_parts * p.num_kv_heads;
     cudaError_t e = launch_pdl(decode_plan_kernel, dim3(1), dim3(1024), 0, stream, p);
     if (e != cudaSuccess) return e;
     const DecodePath path = decode_path(dtype, D, p.group);
+    bool fused = false;
     if constexpr (std::is_same<T, float>::value) {
         e = launch_simt<T, D>(p, stream, max_items);
     } else {
         if (path == DecodePath::kTensorCore) {
-            const bool w8 = tc_consumer_warps() == 8;
-            if (p.group <= 8)
-                e = w8 ? launch_tc<T, D, 1, 8>(p, dtype, stream, max_items)
-                       : launch_tc<T, D, 1, 4>(p, dtype, stream, max_items);
-            else
-                e = w8 ? launch_tc<T, D, 2, 8>(p, dtype, stream, max_items)
-                       : launch_tc<T, D, 2, 4>(p, dtype, stream, max_items);
+            TcShape sh = tc_shape();
+            // Automatic: sequences split into many partitions need the reduce kernel
+            // anyway and stream best with two 2-warp CTAs per SM; otherwise four
+            // single-warp CTAs per SM that merge partitions themselves.
+            if (sh == TcShape::kAuto) sh = p.max_parts > kFusedMaxParts ? TcShape::kPaired : TcShape::kQuad;
+            // single-warp shapes merge partitions in-kernel when there are few of them
+            fused = sh != TcShape::kPaired && p.max_parts > 1 && p.max_parts <= kFusedMaxParts;
+            p.fused_merge = fused ? 1 : 0;
+            if (p.group <= 8) {
+                switch (sh) {
+                    case TcShape::kPaired: e = launch_tc<T, D, 1, 2, 10>(p, dtype, stream, max_items); break;
+                    case TcShape::kTriple: e = launch_tc<T, D, 1, 1, 8>(p, dtype, stream, max_items); break;
+                    case TcShape::kPair1: e = launch_tc<T, D, 1, 1, 13>(p, dtype, stream, max_items); break;
+                    default: e = launch_tc<T, D, 1, 1, 6>(p, dtype, stream, max_items); break;
+                }
+            } else {
+                e = launch_tc<T, D, 2, 1, 6>(p, dtype, stream, max_items);
+            }
         }
         else
             e = launch_simt<T, D>(p, stream, max_items);
     }
     if (e != cudaSuccess) return e;
-    if (p.max_parts > 1) {
-        const long long warps = (long long)p.num_seqs * p.num_heads;
-        e = launch_pdl(decode_reduce_kernel<T, D>, dim3((unsigned)((warps + 3) / 4)), dim3(128), 0, stream, p);
+    if (p.max_parts > 1 && !fused) {
+        DeviceInfo dev;
+        e = device_info(&dev);
+        if (e != cudaSuccess) return e;
+        const long long rows = (long long)p.num_seqs * p.num_heads;
+        const long long cap = (long long)dev.sm_count * 8;
+        e = launch_pdl(decode_reduce_kernel<T, D>, dim3((unsigned)(rows < cap ? rows : cap)), dim3(128), 0, stream, p);
     }
     return e;
 }
@@ -783,7 +1207,14 @@ DecodePath decode_path(pa_dtype dtype, int head_dim, int group) {
     return DecodePath::kTensorCore;
 }
 
-cudaError_t launch_decode(const DecodeParams& p, pa_dtype dtype, cudaStream_t stream) {
+cudaError_t launch_decode(const DecodeParams& p_in, pa_dtype dtype, cudaStream_t stream) {
+    DecodeParams p = p_in;
+    // PA_SCHED=static disables dynamic claiming (tuning)
+    static const int static_sched = [] {
+        const char* e = getenv("PA_SCHED");
+        return (e && std::string(e) == "static") ? 1 : 0;
+    }();
+    p.static_schedule = static_sched;
     switch (dtype) {
         case PA_F32: return p.head_dim == 64 ? launch_all<float, 64>(p, dtype, stream)
                                              : launch_all<float, 128>(p, dtype, stream);

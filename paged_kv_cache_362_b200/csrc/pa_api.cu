@@ -50,7 +50,7 @@ int auto_partition_size(int64_t num_seqs, int64_t num_kv_heads, int64_t max_cont
 struct WsLayout {
     int partition_size, max_parts;
     int64_t max_items;
-    size_t off_items, off_m, off_l, off_o, total;
+    size_t off_items, off_red, off_cnt, off_m, off_l, off_o, total;
 };
 
 bool ws_layout(int64_t num_seqs, int64_t num_heads, int64_t num_kv_heads, int64_t head_dim,
@@ -66,7 +66,9 @@ bool ws_layout(int64_t num_seqs, int64_t num_heads, int64_t num_kv_heads, int64_
     w->max_items = num_seqs * np * num_kv_heads;
     const int64_t parts = np > 1 ? num_seqs * num_heads * np : 0;
     w->off_items = 256;
-    w->off_m = round_up(w->off_items + (size_t)w->max_items * sizeof(int4), 256);
+    w->off_red = round_up(w->off_items + (size_t)w->max_items * sizeof(int4), 256);
+    w->off_cnt = round_up(w->off_red + (size_t)num_seqs * sizeof(int32_t), 256);
+    w->off_m = round_up(w->off_cnt + (size_t)num_seqs * num_kv_heads * sizeof(int32_t), 256);
     w->off_l = round_up(w->off_m + (size_t)parts * sizeof(float), 256);
     w->off_o = round_up(w->off_l + (size_t)parts * sizeof(float), 256);
     w->total = round_up(w->off_o + (size_t)parts * head_dim * sizeof(float), 256);
@@ -154,6 +156,10 @@ pa_status pa_decode(void* out, const void* q, const void* key_cache, const void*
     p.scale_log2 = scale * 1.4426950408889634f;  // log2(e)
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     p.n_items = reinterpret_cast<int32_t*>(ws);
+    p.item_counter = reinterpret_cast<int32_t*>(ws) + 1;
+    p.n_red = reinterpret_cast<int32_t*>(ws) + 2;
+    p.red_seqs = reinterpret_cast<int32_t*>(ws + w.off_red);
+    p.merge_count = reinterpret_cast<int32_t*>(ws + w.off_cnt);
     p.items = reinterpret_cast<int4*>(ws + w.off_items);
     p.part_m = reinterpret_cast<float*>(ws + w.off_m);
     p.part_l = reinterpret_cast<float*>(ws + w.off_l);

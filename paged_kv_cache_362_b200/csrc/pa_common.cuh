@@ -91,14 +91,18 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
                  : "memory");
 }
+// The waiting thread is suspended until the phase completes or the hint (ns)
+// expires, so idle warps do not spin on issue slots.
+constexpr uint32_t kWaitHintNs = 100000;
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(kWaitHintNs)
         : "memory");
     return ok != 0;
 }
@@ -113,7 +117,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
     const uint64_t t0 = global_timer_ns();
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 255u) == 0 && global_timer_ns() - t0 > kWaitLimitNs) return false;
+        if ((i & 15u) == 0 && global_timer_ns() - t0 > kWaitLimitNs) return false;
     }
 }
 
@@ -220,7 +224,13 @@ struct DecodeParams {
     int max_parts;                // NP_max = ceil(max_context_len / partition_size)
     float scale_log2;             // scale * log2(e)
     // workspace views
-    int32_t* n_items;             // [1]
+    int32_t* n_items;             // [1] items in the work list
+    int32_t* item_counter;        // [1] next unclaimed item (reset to 0 by the plan kernel)
+    int static_schedule;          // 1: every item's CTA is fixed by the snake order (no claims)
+    int32_t* n_red;               // [1] sequences that span several partitions
+    int32_t* red_seqs;            // [num_seqs] their indices (order unspecified)
+    int32_t* merge_count;         // [num_seqs * num_kv_heads] partitions finished (reset by the plan kernel)
+    int fused_merge;              // 1: the partition kernel merges partitions itself (no reduce kernel)
     int4* items;                  // [max_items]: (b, (p << 8) | g, clamped ctx, 0), largest first
     float* part_m;                // [B, Hq, NP_max]   max logit (log2 units)
     float* part_l;                // [B, Hq, NP_max]   sum of 2^(s - m)
