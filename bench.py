@@ -203,7 +203,9 @@ class DeviceWorkload:
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
         self.kv_bytes = wl.kv_bytes()
         np_max = -(-self.max_ctx // self._resolved_partition())
-        self.launches_per_step = (1 if self.has_copy else 0) + 1 + 2 + (1 if np_max > 1 else 0)
+        # copy_blocks, reshape_and_cache, plan, partition kernel, and the reduce kernel
+        # when sequences span more partitions than the partition kernel merges itself (8)
+        self.launches_per_step = (1 if self.has_copy else 0) + 1 + 2 + (1 if np_max > 8 else 0)
 
     def _resolved_partition(self):
         if self.P:

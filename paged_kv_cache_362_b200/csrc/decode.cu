@@ -6,35 +6,42 @@
 // attention of q[b,h] over the sequence's K/V, which the kernel reaches by
 // walking the block table; the result is that of contiguous attention.
 //
-// How (three kernels, chained with programmatic dependent launch):
+// How (kernels chained with programmatic dependent launch):
 //
 //  1. plan    -- one CTA turns context_lens into a work list of items
-//                (sequence b, partition p, KV head g), largest first: all full
-//                partitions, then partial ones by decreasing block count,
-//                then empty sequences.  Partition p of b covers logical blocks
-//                [p*PB, min((p+1)*PB, ceil(ctx/16))).
-//  2. partition kernel -- persistent CTAs, one or two per SM.  CTA c takes
-//                items c, 2C-1-c, 2C+c, ... (snake order over the sorted list,
-//                which balances the load).  Per CTA:
-//                  * one producer warp streams, for each item, the Q rows of
-//                    the GQA group (1-D bulk copy) and every (block, KV head)
-//                    tile of K and of V (16 tokens x head_dim, contiguous
-//                    4 KB at D = 128) with 2-D TMA tensor copies into a ring of
+//                (sequence b, partition p, KV head g): first every item of the
+//                sequences that span several partitions, then the rest; within
+//                each class the largest first.  Partition p of b covers logical
+//                blocks [p*PB, min((p+1)*PB, ceil(ctx/16))).  It also lists the
+//                multi-partition sequences and zeroes their merge counters.
+//  2. partition kernel -- persistent CTAs (2 or 4 per SM).  CTA c takes items
+//                c, 2C-1-c, 2C+c, ... (snake order over the sorted list, which
+//                balances the load).  Per CTA:
+//                  * a producer warp streams, for each item, the Q rows of the
+//                    GQA group (1-D bulk copy) and every (block, KV head) tile
+//                    of K and of V (16 tokens x head_dim, contiguous 4 KB at
+//                    D = 128) with 2-D TMA tensor copies into a ring of
 //                    shared-memory stages, 128-byte swizzled, tracked by
-//                    mbarriers, evict-first in L2;
-//                  * consumer warps take the item's blocks round-robin and run
-//                    on tensor cores: S^T = K Q^T (m16n8k16, tokens x heads,
-//                    the GQA group padded to 8 or 16 columns), an online
-//                    softmax in fp32 (column max by warp shuffles, 2^x on
-//                    log2-scaled logits), then O^T += V^T P^T with P
-//                    transposed in registers (movmatrix);
-//                  * at the end of an item the consumer warps merge their
-//                    (max, sum, O) through shared memory and write either the
-//                    final output (single-partition sequence) or the
-//                    partition's (m, l, O) to the workspace.
+//                    mbarriers, evict-first in L2; work-list entries and table
+//                    rows are prefetched two items ahead with cp.async;
+//                  * consumer warps run each block on tensor cores:
+//                    S^T = K Q^T (m16n8k16, tokens x heads, the GQA group padded
+//                    to 8 or 16 columns), an online softmax in fp32 (column max
+//                    by warp shuffles, 2^x on log2-scaled logits), then
+//                    O^T += V^T P^T with P transposed in registers (movmatrix;
+//                    bf16 P carried as a hi + lo pair);
+//                  * with one consumer warp, the warp writes its item's result
+//                    straight from the accumulators (final row, or the
+//                    partition's (m, l, O)); the CTA that finishes the last
+//                    partition of a (sequence, KV head) hands it to a merger
+//                    warp that combines all partitions (when there are at most
+//                    16), so no reduce kernel runs;
+//                  * with two consumer warps, block j goes to warp j % 2 and
+//                    the warps' states are merged through a double-buffered
+//                    shared-memory slot by a rotating merger warp.
 //                A SIMT variant serves float32 and groups above 16.
-//  3. reduce  -- one warp per (b, h) of a multi-partition sequence:
-//                M = max m_p, L = sum l_p 2^(m_p - M),
+//  3. reduce  -- (sequences over 16 partitions, or two-warp CTAs) rows of the
+//                listed sequences: M = max m_p, L = sum l_p 2^(m_p - M),
 //                out = sum O_p 2^(m_p - M) / L.
 #include <cstdlib>
 #include <string>
@@ -52,17 +59,18 @@ constexpr float kNegInf = -__builtin_huge_valf();
 // ===========================================================================
 // 1. plan
 // ===========================================================================
-// Items are ordered by (class, size): first every item of the sequences that
-// span several partitions (their partial results must still be merged, so they
-// should finish early), then the single-partition sequences; within a class,
-// largest first.  Bucket key = class * (PB + 1) + (PB - blocks).
-__global__ void __launch_bounds__(1024) decode_plan_kernel(const DecodeParams p) {
-    constexpr int kThreads = 1024;
+// Item order.  Largest first (key = PB - blocks; empty sequences last), which
+// the snake assignment of the partition kernel turns into an even load; inside
+// a size class the items of sequences that span several partitions come
+// first.  With p.class_first, all items of those sequences come before the
+// others (each class largest first), so that their merges happen early.
+template <int kThreads>
+__global__ void __launch_bounds__(kThreads) decode_plan_kernel(const DecodeParams p) {
     constexpr int kMaxKeys = 2 * (kMaxPartBlocks + 1);
     __shared__ int cnt[kMaxKeys];
     __shared__ int cursor[kMaxKeys];
-    __shared__ int preA[kThreads + 1];   // exclusive prefix of full-partition items, multi-partition class
-    __shared__ int preB[kThreads + 1];   // same, single-partition class
+    __shared__ int preA[kThreads + 1];   // exclusive prefix of full-partition items, multi-partition sequences
+    __shared__ int preB[kThreads + 1];   // same, single-partition sequences
     __shared__ int cctx[kThreads];
     __shared__ int wsumA[kThreads / 32], wsumB[kThreads / 32];
     __shared__ int nred;
@@ -70,8 +78,11 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const DecodeParams p)
     griddep_launch_dependents();
     griddep_wait();
     const int PB = p.part_blocks, Hkv = p.num_kv_heads, KB = PB + 1;
+    const int nkeys = p.class_first ? 2 * KB : KB;
+    // key of an item of `blocks` blocks; single-partition class offset by KB when class_first
+    auto key_of = [&](int blocks, bool multi) { return ((p.class_first && !multi) ? KB : 0) + PB - blocks; };
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-    for (int i = tid; i < 2 * KB; i += kThreads) cnt[i] = 0;
+    for (int i = tid; i < nkeys; i += kThreads) cnt[i] = 0;
     if (tid == 0) nred = 0;
     for (int i = tid; i < p.num_seqs * Hkv; i += kThreads) p.merge_count[i] = 0;
     __syncthreads();
@@ -82,16 +93,16 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const DecodeParams p)
         if (b < p.num_seqs) {
             const int nblk = ceil_div_i(load_ctx(p, b, true), kBlockSize);
             const int nfull = nblk / PB, tail = nblk - nfull * PB;
-            const int cls = (nfull + (tail > 0)) > 1 ? 0 : 1;
-            (cls == 0 ? fa : fb) = nfull * Hkv;
-            if (tail > 0) atomicAdd(&cnt[cls * KB + PB - tail], Hkv);
-            if (nblk == 0) atomicAdd(&cnt[KB + PB], Hkv);
+            const bool multi = (nfull + (tail > 0)) > 1;
+            (multi ? fa : fb) = nfull * Hkv;
+            if (tail > 0) atomicAdd(&cnt[key_of(tail, multi)], Hkv);
+            if (nblk == 0) atomicAdd(&cnt[key_of(0, false)], Hkv);
         }
         fa = __reduce_add_sync(0xffffffffu, fa);
         fb = __reduce_add_sync(0xffffffffu, fb);
         if (lane == 0) {
-            if (fa) atomicAdd(&cnt[0], fa);
-            if (fb) atomicAdd(&cnt[KB], fb);
+            if (fa) atomicAdd(&cnt[key_of(PB, true)], fa);
+            if (fb) atomicAdd(&cnt[key_of(PB, false)], fb);
         }
     }
     __syncthreads();
@@ -101,7 +112,7 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const DecodeParams p)
 #pragma unroll
         for (int k = 0; k < 3; ++k) {
             const int key = lane * 3 + k;
-            v[k] = key < 2 * KB ? cnt[key] : 0;
+            v[k] = key < nkeys ? cnt[key] : 0;
             sum += v[k];
         }
         int incl = sum;
@@ -114,33 +125,33 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const DecodeParams p)
 #pragma unroll
         for (int k = 0; k < 3; ++k) {
             const int key = lane * 3 + k;
-            if (key < 2 * KB) cursor[key] = acc;
+            if (key < nkeys) cursor[key] = acc;
             acc += v[k];
         }
-        if (lane == 31) {
-            *p.n_items = incl;
-            *p.item_counter = 0;
-        }
+        if (lane == 31) *p.n_items = incl;
     }
     __syncthreads();
-    // pass 2: place items; order inside a bucket does not matter
+    // pass 2: place items
+    const int fkA = key_of(PB, true), fkB = key_of(PB, false);
     for (int b0 = 0; b0 < p.num_seqs; b0 += kThreads) {
         const int b = b0 + tid;
         int nfull = 0, tail = 0, ctx = 0, nblk = 0;
-        if (b < p.num_seqs) {
+        const bool valid = b < p.num_seqs;
+        if (valid) {
             ctx = load_ctx(p, b, false);
             nblk = ceil_div_i(ctx, kBlockSize);
             nfull = nblk / PB;
             tail = nblk - nfull * PB;
         }
-        const bool valid = b < p.num_seqs;
         const bool multi = valid && (nfull + (tail > 0)) > 1;
-        if (valid && (tail > 0 || nblk == 0)) {
-            const int key = nblk == 0 ? KB + PB : (multi ? 0 : KB) + PB - tail;
-            const int tb = atomicAdd(&cursor[key], Hkv);
+        const bool has_tail = valid && (tail > 0 || nblk == 0);
+        const int tkey = key_of(tail, multi);
+        // partial (and empty) partitions: multi-partition sequences first in their class
+        if (has_tail && multi) {
+            const int tb = atomicAdd(&cursor[tkey], Hkv);
             for (int g = 0; g < Hkv; ++g) p.items[tb + g] = make_int4(b, (nfull << 8) | g, ctx, 0);
         }
-        // multi-partition sequences go to the reduce kernel's list
+        // multi-partition sequences go to the reduce list
         const unsigned mm = __ballot_sync(0xffffffffu, multi);
         int rb = 0;
         if (lane == 0 && mm) rb = atomicAdd(&nred, __popc(mm));
@@ -162,9 +173,13 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const DecodeParams p)
             wsumB[wid] = ib;
         }
         cctx[tid] = ctx;
-        __syncthreads();
+        __syncthreads();   // (also orders the multi-partition tail reservations before the others)
+        if (has_tail && !multi) {
+            const int tb = atomicAdd(&cursor[tkey], Hkv);
+            for (int g = 0; g < Hkv; ++g) p.items[tb + g] = make_int4(b, (nfull << 8) | g, ctx, 0);
+        }
         if (wid == 0) {
-            int xa = wsumA[lane], xb = wsumB[lane];
+            int xa = lane < kThreads / 32 ? wsumA[lane] : 0, xb = lane < kThreads / 32 ? wsumB[lane] : 0;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
                 const int ua = __shfl_up_sync(0xffffffffu, xa, o), ub = __shfl_up_sync(0xffffffffu, xb, o);
@@ -173,8 +188,10 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const DecodeParams p)
                     xb += ub;
                 }
             }
-            wsumA[lane] = xa;
-            wsumB[lane] = xb;
+            if (lane < kThreads / 32) {
+                wsumA[lane] = xa;
+                wsumB[lane] = xb;
+            }
         }
         __syncthreads();
         const int ea = ia - vA + (wid > 0 ? wsumA[wid - 1] : 0);
@@ -186,10 +203,14 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const DecodeParams p)
             preB[kThreads] = eb + vB;
         }
         __syncthreads();
-        // one thread per full-partition item: find its sequence by binary search over the prefix
+        // full partitions, one thread per item, its sequence found by binary
+        // search over the prefix; class A before class B when they share a key
+        const int totalA = preA[kThreads], totalB = preB[kThreads];
+        const int baseA = cursor[fkA], baseB = cursor[fkB] + (fkA == fkB ? totalA : 0);
         for (int cls = 0; cls < 2; ++cls) {
             const int* pre = cls == 0 ? preA : preB;
-            const int total = pre[kThreads], base = cursor[cls * KB];
+            const int total = cls == 0 ? totalA : totalB;
+            const int base = cls == 0 ? baseA : baseB;
             for (int i = tid; i < total; i += kThreads) {
                 int lo = 0, hi = kThreads;
                 while (hi - lo > 1) {
@@ -203,8 +224,8 @@ __global__ void __launch_bounds__(1024) decode_plan_kernel(const DecodeParams p)
         }
         __syncthreads();
         if (tid == 0) {
-            cursor[0] += preA[kThreads];
-            cursor[KB] += preB[kThreads];
+            cursor[fkA] += totalA;
+            cursor[fkB] += totalB;
         }
         __syncthreads();
     }
@@ -234,48 +255,78 @@ __device__ __forceinline__ ItemGeom item_geom(const DecodeParams& p, int4 it) {
 // Fused merge (single-warp CTAs, at most kFusedMaxParts partitions): one warp
 // combines every partition of (sequence b, KV head g) for the G query heads of
 // the group, out = sum_p O_p 2^(m_p - M) / sum_p l_p 2^(m_p - M).  The
-// partials were written by other CTAs: cache-global loads.
-constexpr int kFusedMaxParts = 16;
+// partials were written by other CTAs: cache-global loads.  Round trips: one
+// for every (head, partition)'s m and l, then one per pair of heads for O.
+constexpr int kFusedMaxParts = 8;
 
 template <typename T, int D>
-__device__ __forceinline__ void merge_group(const DecodeParams& p, int b, int g, int nparts, int lane) {
+__device__ __forceinline__ void merge_group(const DecodeParams& p, int b, int g, int nparts, int lane,
+                                            float* s_w, float* s_inv) {
     constexpr int E = D / 32;
+    constexpr int MP = kFusedMaxParts;
     using VecE = typename std::conditional<E == 4, float4, float2>::type;
     const int G = p.group;
-    T* out = static_cast<T*>(p.out);
-    for (int h = 0; h < G; ++h) {
-        const size_t hq = (size_t)b * p.num_heads + (size_t)g * G + h;
-        const size_t base = hq * p.max_parts;
-        const float mq = lane < nparts ? __ldcg(p.part_m + base + lane) : kNegInf;
-        const float lq = lane < nparts ? __ldcg(p.part_l + base + lane) : 0.f;
-        VecE v[kFusedMaxParts];
+    const size_t hq0 = (size_t)b * p.num_heads + (size_t)g * G;
+    // (m, l) of entry e = h * MP + q, lane e % 32 slot e / 32; G <= 16 -> at most 4 slots
+    float mv[4], lv[4];
 #pragma unroll
-        for (int q = 0; q < kFusedMaxParts; ++q)
-            if (q < nparts) v[q] = __ldcg(reinterpret_cast<const VecE*>(p.part_o + (base + q) * D + lane * E));
-        float M = mq;
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-        const float Ms = M == kNegInf ? 0.f : M;
-        const float w = lane < nparts ? fast_exp2(mq - Ms) : 0.f;
-        float L = w * lq;
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
-        float acc[E];
-#pragma unroll
-        for (int e = 0; e < E; ++e) acc[e] = 0.f;
-#pragma unroll
-        for (int q = 0; q < kFusedMaxParts; ++q) {
-            const float wq = __shfl_sync(0xffffffffu, w, q);
-            if (q < nparts) {
-                const float* f = reinterpret_cast<const float*>(&v[q]);
-#pragma unroll
-                for (int e = 0; e < E; ++e) acc[e] += wq * f[e];
-            }
-        }
-        const float inv = L > 0.f ? 1.f / L : 0.f;
-#pragma unroll
-        for (int e = 0; e < E; ++e) out[hq * D + lane * E + e] = Elt<T>::from_f(acc[e] * inv);
+    for (int k = 0; k < 4; ++k) {
+        const int e = lane + 32 * k, h = e / MP, q = e % MP;
+        const bool ok = h < G && q < nparts;
+        const size_t pi = (hq0 + h) * p.max_parts + q;
+        mv[k] = ok ? __ldcg(p.part_m + pi) : kNegInf;
+        lv[k] = ok ? __ldcg(p.part_l + pi) : 0.f;
     }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        // the MP lanes of one head are consecutive: reduce over them
+        float M = mv[k];
+#pragma unroll
+        for (int off = 1; off < MP; off <<= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+        const float Ms = M == kNegInf ? 0.f : M;
+        const float w = mv[k] == kNegInf ? 0.f : fast_exp2(mv[k] - Ms);
+        float L = w * lv[k];
+#pragma unroll
+        for (int off = 1; off < MP; off <<= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
+        const int e = lane + 32 * k;
+        if (e / MP < G) {
+            s_w[e] = w;
+            if (e % MP == 0) s_inv[e / MP] = L > 0.f ? 1.f / L : 0.f;
+        }
+    }
+    __syncwarp();
+    T* out = static_cast<T*>(p.out);
+    for (int h0 = 0; h0 < G; h0 += 2) {
+        VecE v[2][MP];
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+            for (int q = 0; q < MP; ++q)
+                if (h0 + hh < G && q < nparts)
+                    v[hh][q] = __ldcg(reinterpret_cast<const VecE*>(p.part_o + ((hq0 + h0 + hh) * p.max_parts + q) * D +
+                                                                    lane * E));
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            const int h = h0 + hh;
+            if (h >= G) break;
+            float acc[E];
+#pragma unroll
+            for (int e = 0; e < E; ++e) acc[e] = 0.f;
+#pragma unroll
+            for (int q = 0; q < MP; ++q) {
+                if (q < nparts) {
+                    const float wq = s_w[h * MP + q];
+                    const float* f = reinterpret_cast<const float*>(&v[hh][q]);
+#pragma unroll
+                    for (int e = 0; e < E; ++e) acc[e] += wq * f[e];
+                }
+            }
+            const float inv = s_inv[h];
+#pragma unroll
+            for (int e = 0; e < E; ++e) out[(hq0 + h) * D + lane * E + e] = Elt<T>::from_f(acc[e] * inv);
+        }
+    }
+    __syncwarp();
 }
 
 struct ItemMeta {
@@ -286,7 +337,7 @@ struct ItemMeta {
 struct DescSlot {
     int4 e;
     int bt[kMaxPartBlocks];
-    int rank;      // position in the work list (claimed from the shared counter)
+    int rank;      // position in the work list
     int pad[3];
 };
 
@@ -311,7 +362,9 @@ struct TcCfg {
     static constexpr int kOffMeta = kOffDesc + kDSlots * (int)sizeof(DescSlot);
     static constexpr int kQSlots = NCW == 1 ? 4 : 0;          // merge-task queue (single-warp CTAs)
     static constexpr int kOffTasks = kOffMeta + kISlots * (int)sizeof(ItemMeta);
-    static constexpr int kOffBar = kOffTasks + kQSlots * 16;
+    static constexpr int kMergeW = NCW == 1 ? 128 + 16 : 0;   // merger's partition weights and 1/L
+    static constexpr int kOffMW = kOffTasks + kQSlots * 16;
+    static constexpr int kOffBar = kOffMW + kMergeW * 4;
     static constexpr int kNumBars = 2 * STAGES + 2 * kISlots + 2 * kMSlots + 2 * kQSlots;
     static constexpr int kOffFlags = kOffBar + kNumBars * 8;
     static constexpr int kBytes = kOffFlags + 16 + STAGES * 4;
@@ -384,7 +437,6 @@ __global__ void __launch_bounds__(TcCfg<D, NT, NCW, STAGES>::kThreads, 1)
 
     griddep_launch_dependents();
     griddep_wait();
-    const int n_items = *p.n_items;
     const int PB = p.part_blocks;
 
     if constexpr (NCW == 1) {
@@ -403,7 +455,8 @@ __global__ void __launch_bounds__(TcCfg<D, NT, NCW, STAGES>::kThreads, 1)
                 if (lane == 0) mbar_arrive(&qempty[qs]);
                 if (task.x < 0) break;
                 __threadfence();
-                merge_group<T, D>(p, task.x, task.y, task.z, lane);
+                float* s_w = reinterpret_cast<float*>(smem + C::kOffMW);
+                merge_group<T, D>(p, task.x, task.y, task.z, lane, s_w, s_w + 128);
             }
             return;
         }
@@ -418,13 +471,12 @@ __global__ void __launch_bounds__(TcCfg<D, NT, NCW, STAGES>::kThreads, 1)
         const uint64_t pol = policy_evict_first();
         const size_t q_row_bytes = (size_t)D * 2;
 
-        // Work is claimed dynamically from a counter the plan kernel reset, in the
-        // plan's largest-first order, so CTAs that finish early take more items.
         // Descriptor pipeline, so that no global-memory latency sits between
-        // two items' tile loads: item k's claimed rank, work-list entry and
-        // table row land in slot k % kDSlots.  At the top of iteration i,
-        // entry(i), row(i) and entry(i+1) are visible, the group {row(i+1),
-        // entry(i+2)} is in flight, and the claim of item i+3 is in a register.
+        // two items' tile loads: item k's rank, work-list entry and table row
+        // land in slot k % kDSlots.  At the top of iteration i, entry(i),
+        // row(i) and entry(i+1) are visible and the group {row(i+1),
+        // entry(i+2)} is in flight.
+        int n_items = 0;  // set once the plan's count has been read (below)
         auto fetch_entry = [&](int it, int r) {
             if (lane == 0) {
                 dsc[it % C::kDSlots].rank = r;
@@ -441,34 +493,32 @@ __global__ void __launch_bounds__(TcCfg<D, NT, NCW, STAGES>::kThreads, 1)
                 cp_async_4(smem_u32(&dsc[it % C::kDSlots].bt[lane]),
                            p.block_tables + (size_t)e.x * p.max_blocks_per_seq + j0 + lane);
         };
-        // The first kStaticRounds items of every CTA are fixed (snake order over
-        // the largest-first list); after that CTAs claim the next item from the
-        // counter, so that CTAs which finish early take more of the small ones.
-        constexpr int kStaticRounds = 3;
+        // Static schedule: CTA c takes ranks c, 2C-1-c, 2C+c, ... of the
+        // largest-first list (snake order), which balances the load without a
+        // shared counter (claiming items from one counter was measured slower:
+        // every CTA's claim goes to one address).
         const int ctas = gridDim.x, cta = blockIdx.x;
-        auto static_rank = [&](int it) { return it * ctas + ((it & 1) ? (ctas - 1 - cta) : cta); };
-        auto claim = [&](int it) {
-            if (it < kStaticRounds || p.static_schedule) return static_rank(it);
-            return kStaticRounds * ctas + atomicAdd(p.item_counter, 1);
-        };
-        int r0 = 0, r1 = 0, r2 = 0, claim_next = 0;
+        auto rank_of = [&](int it) { return it * ctas + ((it & 1) ? (ctas - 1 - cta) : cta); };
+        // the item count and this CTA's first work-list entry (rank = cta; the
+        // list holds at least gridDim.x entries) arrive in one round trip
+        int* s_nitems = const_cast<int*>(abort_flag) + 1;
         if (lane == 0) {
-            r0 = claim(0);
-            r1 = claim(1);
-            r2 = claim(2);
-            claim_next = claim(3);
+            cp_async_4(smem_u32(s_nitems), p.n_items);
+            cp_async_16(smem_u32(&dsc[0].e), &p.items[cta]);
         }
-        fetch_entry(0, r0);
         cp_async_commit();
         cp_async_wait_all();
         __syncwarp();
+        n_items = *s_nitems;
+        if (lane == 0) dsc[0].rank = cta < n_items ? cta : n_items;
+        __syncwarp();
         fetch_row(0);
-        fetch_entry(1, r1);
+        fetch_entry(1, rank_of(1));
         cp_async_commit();
         cp_async_wait_all();
         __syncwarp();
         fetch_row(1);
-        fetch_entry(2, r2);
+        fetch_entry(2, rank_of(2));
         cp_async_commit();
         __syncwarp();
 
@@ -568,8 +618,7 @@ __global__ void __launch_bounds__(TcCfg<D, NT, NCW, STAGES>::kThreads, 1)
             cp_async_wait_all();
             __syncwarp();
             fetch_row(iter + 2);
-            fetch_entry(iter + 3, claim_next);
-            if (lane == 0 && claim_next < n_items) claim_next = claim(iter + 4);
+            fetch_entry(iter + 3, rank_of(iter + 3));
             cp_async_commit();
             __syncwarp();
         }
@@ -1070,6 +1119,7 @@ namespace {
 // The ring holds the bytes in flight that cover HBM latency; each consumer
 // warp holds one stage while it computes.  PA_TC_SHAPE selects one (tuning).
 enum class TcShape { kAuto, kPaired, kQuad, kTriple, kPair1 };
+constexpr int kPairedMinParts = 32;
 TcShape tc_shape() {
     static const TcShape s = [] {
         const char* e = getenv("PA_TC_SHAPE");
@@ -1157,7 +1207,9 @@ cudaError_t launch_simt(const DecodeParams& p, cudaStream_t stream, int max_item
 template <typename T, int D>
 cudaError_t launch_all(DecodeParams p, pa_dtype dtype, cudaStream_t stream) {
     const int max_items = p.num_seqs * p.max_parts * p.num_kv_heads;
-    cudaError_t e = launch_pdl(decode_plan_kernel, dim3(1), dim3(1024), 0, stream, p);
+    // plan: one CTA; 256 threads cover typical batches in one pass, 1024 large ones
+    cudaError_t e = p.num_seqs <= 256 ? launch_pdl(decode_plan_kernel<256>, dim3(1), dim3(256), 0, stream, p)
+                                      : launch_pdl(decode_plan_kernel<1024>, dim3(1), dim3(1024), 0, stream, p);
     if (e != cudaSuccess) return e;
     const DecodePath path = decode_path(dtype, D, p.group);
     bool fused = false;
@@ -1166,10 +1218,11 @@ cudaError_t launch_all(DecodeParams p, pa_dtype dtype, cudaStream_t stream) {
     } else {
         if (path == DecodePath::kTensorCore) {
             TcShape sh = tc_shape();
-            // Automatic: sequences split into many partitions need the reduce kernel
-            // anyway and stream best with two 2-warp CTAs per SM; otherwise four
-            // single-warp CTAs per SM that merge partitions themselves.
-            if (sh == TcShape::kAuto) sh = p.max_parts > kFusedMaxParts ? TcShape::kPaired : TcShape::kQuad;
+            // Automatic: sequences split into many (> 32) partitions stream best with
+            // two 2-warp CTAs per SM (measured on 32k contexts); otherwise four
+            // single-warp CTAs per SM, which merge partitions themselves when there
+            // are at most kFusedMaxParts of them.
+            if (sh == TcShape::kAuto) sh = p.max_parts > kPairedMinParts ? TcShape::kPaired : TcShape::kQuad;
             // single-warp shapes merge partitions in-kernel when there are few of them
             fused = sh != TcShape::kPaired && p.max_parts > 1 && p.max_parts <= kFusedMaxParts;
             p.fused_merge = fused ? 1 : 0;
@@ -1209,12 +1262,13 @@ DecodePath decode_path(pa_dtype dtype, int head_dim, int group) {
 
 cudaError_t launch_decode(const DecodeParams& p_in, pa_dtype dtype, cudaStream_t stream) {
     DecodeParams p = p_in;
-    // PA_SCHED=static disables dynamic claiming (tuning)
-    static const int static_sched = [] {
-        const char* e = getenv("PA_SCHED");
-        return (e && std::string(e) == "static") ? 1 : 0;
+    // item order: multi-partition sequences' items first (measured best with
+    // the fused merge); PA_PLAN_ORDER=size orders all items by size (tuning)
+    static const int class_first = [] {
+        const char* e = getenv("PA_PLAN_ORDER");
+        return (e && std::string(e) == "size") ? 0 : 1;
     }();
-    p.static_schedule = static_sched;
+    p.class_first = class_first;
     switch (dtype) {
         case PA_F32: return p.head_dim == 64 ? launch_all<float, 64>(p, dtype, stream)
                                              : launch_all<float, 128>(p, dtype, stream);

@@ -156,8 +156,7 @@ pa_status pa_decode(void* out, const void* q, const void* key_cache, const void*
     p.scale_log2 = scale * 1.4426950408889634f;  // log2(e)
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     p.n_items = reinterpret_cast<int32_t*>(ws);
-    p.item_counter = reinterpret_cast<int32_t*>(ws) + 1;
-    p.n_red = reinterpret_cast<int32_t*>(ws) + 2;
+    p.n_red = reinterpret_cast<int32_t*>(ws) + 1;
     p.red_seqs = reinterpret_cast<int32_t*>(ws + w.off_red);
     p.merge_count = reinterpret_cast<int32_t*>(ws + w.off_cnt);
     p.items = reinterpret_cast<int4*>(ws + w.off_items);

@@ -225,12 +225,11 @@ struct DecodeParams {
     float scale_log2;             // scale * log2(e)
     // workspace views
     int32_t* n_items;             // [1] items in the work list
-    int32_t* item_counter;        // [1] next unclaimed item (reset to 0 by the plan kernel)
-    int static_schedule;          // 1: every item's CTA is fixed by the snake order (no claims)
     int32_t* n_red;               // [1] sequences that span several partitions
     int32_t* red_seqs;            // [num_seqs] their indices (order unspecified)
     int32_t* merge_count;         // [num_seqs * num_kv_heads] partitions finished (reset by the plan kernel)
     int fused_merge;              // 1: the partition kernel merges partitions itself (no reduce kernel)
+    int class_first;              // plan order: 1 = multi-partition sequences' items first
     int4* items;                  // [max_items]: (b, (p << 8) | g, clamped ctx, 0), largest first
     float* part_m;                // [B, Hq, NP_max]   max logit (log2 units)
     float* part_l;                // [B, Hq, NP_max]   sum of 2^(s - m)
