@@ -39,6 +39,25 @@ METRIC = "paged decode attention: achieved KV-read HBM GB/s (% of peak), seq/s"
 FALLBACK_HBM_GBS = 6650.0
 
 
+def profiled_traffic(workload: str):
+    """DRAM bytes per launch of the partition kernel from the committed ncu capture.
+
+    profiles/traffic.json records the capture together with a hash of the
+    decode source it was taken on; a changed kernel gets null, not a stale number.
+    """
+    import hashlib
+
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            t = json.load(f)
+        src = open(os.path.join(ROOT, t["source"]), "rb").read()
+        if hashlib.sha256(src).hexdigest()[:16] != t["source_sha256_16"]:
+            return None
+        return t[workload]["decode_tc_kernel_bytes"]
+    except Exception:
+        return None
+
+
 def measured_hbm_peak():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -202,20 +221,10 @@ class DeviceWorkload:
         self.out = torch.empty_like(self.q)
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
         self.kv_bytes = wl.kv_bytes()
-        np_max = -(-self.max_ctx // self._resolved_partition())
-        # copy_blocks, reshape_and_cache, plan, partition kernel, and the reduce kernel
-        # when sequences span more partitions than the partition kernel merges itself (8)
-        self.launches_per_step = (1 if self.has_copy else 0) + 1 + 2 + (1 if np_max > 8 else 0)
-
-    def _resolved_partition(self):
-        if self.P:
-            return self.P
-        # the library's automatic choice, restated only to count launches
-        c, B = self.cfg, self.wl.num_seqs
-        P = 512
-        while P > 64 and B * c.num_kv_heads * -(-self.max_ctx // P) < 8 * 148:
-            P //= 2
-        return P
+        # copy_blocks (when the step forks), reshape_and_cache, and the kernels pa_decode enqueues
+        self.decode_launches = pa.decode_launch_count(wl.num_seqs, c.num_heads, c.num_kv_heads, c.head_dim,
+                                                      self.max_ctx, self.P, c.dtype)
+        self.launches_per_step = (1 if self.has_copy else 0) + 1 + self.decode_launches
 
     def pre(self):
         if self.has_copy:
@@ -466,6 +475,7 @@ def main():
                 "decode_kv_gbs": round(sw.kv_bytes / (sd * 1e-3) / 1e9, 1),
                 "decode_frac_of_peak": round(sw.kv_bytes / (sd * 1e-3) / 1e9 / peak, 4),
                 "kv_bytes": sw.kv_bytes, "seq_per_s": round(sw.wl.num_seqs / (ss * 1e-3), 1),
+                "decode_launches": sw.decode_launches,
             }
             del sw
             torch.cuda.empty_cache()
@@ -493,8 +503,12 @@ def main():
             "pct_of_peak": round(100 * value / world / peak, 2),
             "seq_per_s": round(w.wl.num_seqs * world / (ms * 1e-3), 1),
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                         "frac": round(achieved / peak, 4), "traffic": None, "kernel": "pa_decode (plan + "
-                         "partition + reduce launches)", "peak_kind": peak_kind},
+                         "frac": round(achieved / peak, 4), "traffic": profiled_traffic(c.name),
+                         "algorithmic_bytes": w.kv_bytes,
+                         "kernel": f"pa_decode call ({w.decode_launches} launch(es): [plan +] attention "
+                                   "[+ reduce]), timed together; traffic = DRAM bytes of the attention kernel "
+                                   "from profiles/traffic.json",
+                         "peak_kind": peak_kind},
             "cpu_baseline": cpu,
             "e2e": {"value": round(total_bytes / (e2e * 1e-3) / 1e9, 2), "unit": "GB/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e, 5)},

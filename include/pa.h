@@ -129,9 +129,14 @@ size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_heads, int32_t num
  *   partition_size      tokens per partition: 0 = automatic, else a multiple
  *                       of 16 in [16, 512]
  *   workspace           device buffer of at least pa_decode_workspace_size()
- *                       bytes, 256-byte aligned; contents need no initialising
- *                       and are scratch between calls.  Calls that share a
- *                       workspace must not overlap in time.
+ *                       bytes, 256-byte aligned, ZERO-FILLED before its first
+ *                       use (cudaMemset).  It holds counters that each call
+ *                       leaves at zero for the next, whatever the sizes of the
+ *                       next problem; the rest is scratch.  After a call that
+ *                       reported PA_ERR_TIMEOUT, zero it again.  Calls that
+ *                       share a workspace must not overlap in time.
+ *
+ * The call enqueues pa_decode_launch_count() kernels on `stream`.
  */
 pa_status pa_decode(void* out, const void* q, const void* key_cache, const void* value_cache,
                     const int32_t* block_tables, int32_t max_blocks_per_seq,
@@ -139,6 +144,15 @@ pa_status pa_decode(void* out, const void* q, const void* key_cache, const void*
                     int32_t num_kv_heads, int32_t head_dim, int32_t block_size, int32_t num_blocks,
                     float scale, int32_t max_context_len, int32_t partition_size, void* workspace,
                     size_t workspace_bytes, pa_dtype dtype, int32_t* status, pa_stream_t stream);
+
+/*
+ * pa_decode_launch_count -- number of kernels pa_decode enqueues for these
+ * sizes on the current device (1 to 3: an optional planning kernel, the
+ * attention kernel, an optional reduce kernel).  Returns -1 for arguments
+ * pa_decode would reject, or when the device cannot be queried.
+ */
+int32_t pa_decode_launch_count(int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads, int32_t head_dim,
+                               int32_t max_context_len, int32_t partition_size, pa_dtype dtype);
 
 /*
  * pa_copy_blocks -- copy-on-write clone of whole blocks, in both pools.
@@ -171,11 +185,12 @@ pa_status pa_copy_blocks(void* key_cache, void* value_cache, const int64_t* bloc
  * on every GPU that loads the library until the process exits.  A problem
  * whose pa_decode_workspace_size() exceeds 32 MiB returns PA_ERR_UNSUPPORTED
  * and enqueues nothing.  The first call made with a given device current
- * looks up the array's device address (cudaGetSymbolAddress); make that first
+ * looks up the array's device address (cudaGetSymbolAddress), zero-fills it
+ * on `stream` and waits for that (cudaStreamSynchronize); make that first
  * call before any stream capture begins.  No cudaMalloc or cudaFree is made.
  * All calls share the one array: calls whose kernels overlap on the GPU (two
- * streams, two host threads) race on it and give wrong results.  Nothing in
- * it has to start at zero.
+ * streams, two host threads) race on it and give wrong results.  After a call
+ * that reported PA_ERR_TIMEOUT, stop using this entry point in the process.
  */
 pa_status pa_decode_noalloc(void* out, const void* q, const void* key_cache, const void* value_cache,
                             const int32_t* block_tables, int32_t max_blocks_per_seq,

@@ -18,6 +18,7 @@ from ._lib import (  # noqa: F401
     check_copy_pairs,
     copy_blocks,
     decode,
+    decode_launch_count,
     decode_workspace_size,
     error_string,
     make_workspace,

@@ -34,8 +34,12 @@ class PagedAttentionError(RuntimeError):
 
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"{LIB_PATH} is not built; run `python -m paged_kv_cache_362_b200.build`")
+        raise ImportError(f"{LIB_PATH} is not built; run `python paged_kv_cache_362_b200/build.py`")
     lib = ctypes.CDLL(LIB_PATH)
+    for sym in ("pa_reshape_and_cache", "pa_decode_workspace_size", "pa_decode", "pa_decode_launch_count",
+                "pa_copy_blocks", "pa_get_error_string", "pa_version"):
+        if not hasattr(lib, sym):
+            raise ImportError(f"{LIB_PATH} lacks {sym} (stale build); run `python paged_kv_cache_362_b200/build.py`")
     p, i32, i64, f32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
     lib.pa_reshape_and_cache.argtypes = [p, p, p, p, p, i64, i32, i32, i32, i32, ctypes.c_int, p, p]
     lib.pa_reshape_and_cache.restype = ctypes.c_int
@@ -44,6 +48,8 @@ def _load() -> ctypes.CDLL:
     lib.pa_decode.argtypes = [p, p, p, p, p, i32, p, i32, i32, i32, i32, i32, i32, f32, i32, i32, p, sz,
                               ctypes.c_int, p, p]
     lib.pa_decode.restype = ctypes.c_int
+    lib.pa_decode_launch_count.argtypes = [i32, i32, i32, i32, i32, i32, ctypes.c_int]
+    lib.pa_decode_launch_count.restype = i32
     lib.pa_copy_blocks.argtypes = [p, p, p, i32, i32, i32, i32, i32, ctypes.c_int, p, p]
     lib.pa_copy_blocks.restype = ctypes.c_int
     lib.pa_get_error_string.argtypes = [ctypes.c_int]
@@ -111,11 +117,23 @@ def decode_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, max_conte
     return n
 
 
+def decode_launch_count(num_seqs, num_heads, num_kv_heads, head_dim, max_context_len, partition_size=0,
+                        dtype="f16") -> int:
+    """Kernels one pa_decode call enqueues for these sizes on the current device."""
+    code = {"f32": 0, "f16": 1, "bf16": 2}[dtype]
+    n = int(LIB.pa_decode_launch_count(num_seqs, num_heads, num_kv_heads, head_dim, max_context_len,
+                                       partition_size, code))
+    if n < 0:
+        raise PagedAttentionError(PA_ERR_INVALID_ARG, "pa_decode_launch_count")
+    return n
+
+
 def make_workspace(num_seqs, num_heads, num_kv_heads, head_dim, max_context_len, partition_size=0, device=None):
     import torch
 
     n = decode_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, max_context_len, partition_size)
-    return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+    # zero-filled: pa_decode keeps merge counters in it that must start at zero
+    return torch.zeros(n, dtype=torch.uint8, device=device or "cuda")
 
 
 def decode(out, q, key_cache, value_cache, block_tables, context_lens, scale, max_context_len, workspace,

@@ -1,6 +1,8 @@
 """Build libpa.so (the C-ABI CUDA library) in-tree for sm_100a with nvcc.
 
-    python -m paged_kv_cache_362_b200.build [--force] [--verbose]
+    python paged_kv_cache_362_b200/build.py [--force] [--verbose]
+
+(run as a file: importing the package loads the library this builds)
 
 Each translation unit under csrc/ is compiled separately (in parallel), then
 linked into paged_kv_cache_362_b200/libpa.so with the CUDA runtime linked

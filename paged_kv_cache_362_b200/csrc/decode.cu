@@ -8,12 +8,15 @@
 //
 // How (kernels chained with programmatic dependent launch):
 //
-//  1. plan    -- one CTA turns context_lens into a work list of items
-//                (sequence b, partition p, KV head g): first every item of the
-//                sequences that span several partitions, then the rest; within
-//                each class the largest first.  Partition p of b covers logical
-//                blocks [p*PB, min((p+1)*PB, ceil(ctx/16))).  It also lists the
-//                multi-partition sequences and zeroes their merge counters.
+//  1. plan    -- the work list of items (sequence b, partition p, KV head g):
+//                every item of the sequences that span several partitions
+//                first, then the rest, each class largest first.  A sequence
+//                of nblk blocks has n = ceil(nblk / PB) partitions, the first
+//                n - 1 of PB blocks (see seq_parts).  For batches of up to
+//                256 sequences each CTA of the partition kernel derives its
+//                own items of the list from context_lens (no launch); a
+//                one-CTA plan kernel writes the whole list for larger
+//                batches, for many items per CTA and for the SIMT kernel.
 //  2. partition kernel -- persistent CTAs (2 or 4 per SM).  CTA c takes items
 //                c, 2C-1-c, 2C+c, ... (snake order over the sorted list, which
 //                balances the load).  Per CTA:
@@ -33,15 +36,16 @@
 //                  * with one consumer warp, the warp writes its item's result
 //                    straight from the accumulators (final row, or the
 //                    partition's (m, l, O)); the CTA that finishes the last
-//                    partition of a (sequence, KV head) hands it to a merger
-//                    warp that combines all partitions (when there are at most
-//                    16), so no reduce kernel runs;
+//                    partition of a (sequence, KV head) -- a per-group counter
+//                    in the workspace says which -- hands it to a merger warp
+//                    that combines all partitions (when there are at most 8)
+//                    and resets the counter, so no reduce kernel runs;
 //                  * with two consumer warps, block j goes to warp j % 2 and
 //                    the warps' states are merged through a double-buffered
 //                    shared-memory slot by a rotating merger warp.
 //                A SIMT variant serves float32 and groups above 16.
-//  3. reduce  -- (sequences over 16 partitions, or two-warp CTAs) rows of the
-//                listed sequences: M = max m_p, L = sum l_p 2^(m_p - M),
+//  3. reduce  -- (sequences over 8 partitions, or two-warp CTAs) rows of the
+//                multi-partition sequences: M = max m_p, L = sum l_p 2^(m_p - M),
 //                out = sum O_p 2^(m_p - M) / L.
 #include <cstdlib>
 #include <string>
@@ -59,177 +63,140 @@ constexpr float kNegInf = -__builtin_huge_valf();
 // ===========================================================================
 // 1. plan
 // ===========================================================================
+// Partitions.  A sequence of nblk blocks has n = max(1, ceil(nblk / PB))
+// partitions: partitions 0 .. nbig-1 hold `big` blocks, the others `small`.
+//  * full split (default): n - 1 partitions of PB blocks, then the remainder.
+//  * equal split (PA_SPLIT=equal, tuning): near-equal lengths, q + 1 blocks
+//    for the first r = nblk % n partitions and q = nblk / n for the rest.  It
+//    avoids small tail partitions, yet measured 1-6% slower on every workload.
+struct SeqParts {
+    int n, nbig, big, small;
+    __device__ __forceinline__ int start(int p) const { return p < nbig ? p * big : nbig * big + (p - nbig) * small; }
+    __device__ __forceinline__ int len(int p) const { return p < nbig ? big : small; }
+};
+__device__ __forceinline__ SeqParts seq_parts(int nblk, int PB, bool equal) {
+    SeqParts s;
+    s.n = max(1, ceil_div_i(nblk, PB));
+    if (equal) {
+        s.small = nblk / s.n;
+        s.big = s.small + 1;
+        s.nbig = nblk - s.small * s.n;
+    } else {
+        const int tail = nblk - (s.n - 1) * PB;   // 1 .. PB (0 for an empty sequence)
+        s.big = PB;
+        s.nbig = tail == PB ? s.n : s.n - 1;
+        s.small = tail == PB ? PB : tail;
+    }
+    return s;
+}
+
 // Item order.  Largest first (key = PB - blocks; empty sequences last), which
-// the snake assignment of the partition kernel turns into an even load; inside
-// a size class the items of sequences that span several partitions come
-// first.  With p.class_first, all items of those sequences come before the
-// others (each class largest first), so that their merges happen early.
+// the snake assignment of the partition kernel turns into an even load.  With
+// p.class_first (the default), all items of split sequences come before the
+// others, each class largest first, so that the merges of split sequences
+// happen early.  Inside a key the order is free; results do not depend on it.
+constexpr int kMaxKeys = 2 * (kMaxPartBlocks + 1);
+constexpr int kNoKey = 0xff;
+
+struct PlanKeys {
+    int PB, KB, Hkv, cf;
+    // key of an item of `blocks` blocks; single-partition class offset by KB when cf
+    __device__ __forceinline__ int key_of(int blocks, bool multi) const { return ((cf && !multi) ? KB : 0) + PB - blocks; }
+    __device__ __forceinline__ int nkeys() const { return cf ? 2 * KB : KB; }
+};
+
+// a sequence's items fall in at most two keys: nbig partitions of `big`
+// blocks and n - nbig of `small` blocks (kNoKey where there are none)
+__device__ __forceinline__ void seq_keys(const PlanKeys& K, const SeqParts& s, int& kbig, int& ksmall) {
+    const bool multi = s.n > 1;
+    kbig = s.nbig > 0 ? K.key_of(s.big, multi) : kNoKey;
+    ksmall = s.n > s.nbig ? K.key_of(s.small, multi) : kNoKey;
+}
+
+// Bucket offsets from the key counts: warp 0 scans the (at most 66) keys, 3
+// per lane, into off[0 .. nkeys] (off[nkeys] = total); returns the total on
+// lane 31.
+__device__ __forceinline__ int scan_keys(const int* cnt, int* off, int nkeys, int lane) {
+    static_assert(kMaxKeys <= 96, "the key scan covers 3 keys per lane");
+    int v[3], sum = 0;
+#pragma unroll
+    for (int k = 0; k < 3; ++k) {
+        const int key = lane * 3 + k;
+        v[k] = key < nkeys ? cnt[key] : 0;
+        sum += v[k];
+    }
+    int incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += u;
+    }
+    int acc = incl - sum;
+#pragma unroll
+    for (int k = 0; k < 3; ++k) {
+        const int key = lane * 3 + k;
+        if (key < nkeys) off[key] = acc;
+        acc += v[k];
+    }
+    if (lane == 31) off[nkeys] = incl;
+    return incl;
+}
+
+// One CTA writes the whole list (items of one key in arbitrary order) and
+// zeroes the merge counters of the problem.
 template <int kThreads>
 __global__ void __launch_bounds__(kThreads) decode_plan_kernel(const DecodeParams p) {
-    constexpr int kMaxKeys = 2 * (kMaxPartBlocks + 1);
     __shared__ int cnt[kMaxKeys];
-    __shared__ int cursor[kMaxKeys];
-    __shared__ int preA[kThreads + 1];   // exclusive prefix of full-partition items, multi-partition sequences
-    __shared__ int preB[kThreads + 1];   // same, single-partition sequences
-    __shared__ int cctx[kThreads];
-    __shared__ int wsumA[kThreads / 32], wsumB[kThreads / 32];
-    __shared__ int nred;
+    __shared__ int cursor[kMaxKeys + 1];
     // the partition kernel may launch now and set up; it waits for this grid to finish
     griddep_launch_dependents();
     griddep_wait();
-    const int PB = p.part_blocks, Hkv = p.num_kv_heads, KB = PB + 1;
-    const int nkeys = p.class_first ? 2 * KB : KB;
-    // key of an item of `blocks` blocks; single-partition class offset by KB when class_first
-    auto key_of = [&](int blocks, bool multi) { return ((p.class_first && !multi) ? KB : 0) + PB - blocks; };
+    const PlanKeys K{p.part_blocks, p.part_blocks + 1, p.num_kv_heads, p.class_first};
+    const int nkeys = K.nkeys(), Hkv = K.Hkv, B = p.num_seqs;
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     for (int i = tid; i < nkeys; i += kThreads) cnt[i] = 0;
-    if (tid == 0) nred = 0;
-    for (int i = tid; i < p.num_seqs * Hkv; i += kThreads) p.merge_count[i] = 0;
+    for (int i = tid; i < B * Hkv; i += kThreads) p.merge_count[i] = 0;
     __syncthreads();
-    // pass 1: histogram of item keys (full-partition counts aggregated per warp)
-    for (int b0 = 0; b0 < p.num_seqs; b0 += kThreads) {
-        const int b = b0 + tid;
-        int fa = 0, fb = 0;
-        if (b < p.num_seqs) {
-            const int nblk = ceil_div_i(load_ctx(p, b, true), kBlockSize);
-            const int nfull = nblk / PB, tail = nblk - nfull * PB;
-            const bool multi = (nfull + (tail > 0)) > 1;
-            (multi ? fa : fb) = nfull * Hkv;
-            if (tail > 0) atomicAdd(&cnt[key_of(tail, multi)], Hkv);
-            if (nblk == 0) atomicAdd(&cnt[key_of(0, false)], Hkv);
-        }
-        fa = __reduce_add_sync(0xffffffffu, fa);
-        fb = __reduce_add_sync(0xffffffffu, fb);
-        if (lane == 0) {
-            if (fa) atomicAdd(&cnt[key_of(PB, true)], fa);
-            if (fb) atomicAdd(&cnt[key_of(PB, false)], fb);
-        }
+    // pass 1: histogram of item keys
+    for (int b = tid; b < B; b += kThreads) {
+        const SeqParts sp = seq_parts(ceil_div_i(load_ctx(p, b, true), kBlockSize), K.PB, p.equal_split);
+        int kb, ks;
+        seq_keys(K, sp, kb, ks);
+        if (kb != kNoKey) atomicAdd(&cnt[kb], sp.nbig * Hkv);
+        if (ks != kNoKey) atomicAdd(&cnt[ks], (sp.n - sp.nbig) * Hkv);
     }
     __syncthreads();
-    // bucket offsets: warp 0 scans the (at most 66) keys, 3 per lane
     if (wid == 0) {
-        int v[3], sum = 0;
-#pragma unroll
-        for (int k = 0; k < 3; ++k) {
-            const int key = lane * 3 + k;
-            v[k] = key < nkeys ? cnt[key] : 0;
-            sum += v[k];
-        }
-        int incl = sum;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int u = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += u;
-        }
-        int acc = incl - sum;
-#pragma unroll
-        for (int k = 0; k < 3; ++k) {
-            const int key = lane * 3 + k;
-            if (key < nkeys) cursor[key] = acc;
-            acc += v[k];
-        }
-        if (lane == 31) *p.n_items = incl;
+        const int total = scan_keys(cnt, cursor, nkeys, lane);
+        if (lane == 31) p.hdr[kHdrItems] = total;
     }
     __syncthreads();
-    // pass 2: place items
-    const int fkA = key_of(PB, true), fkB = key_of(PB, false);
-    for (int b0 = 0; b0 < p.num_seqs; b0 += kThreads) {
-        const int b = b0 + tid;
-        int nfull = 0, tail = 0, ctx = 0, nblk = 0;
-        const bool valid = b < p.num_seqs;
-        if (valid) {
+    // pass 2: every lane reserves its sequence's slots; the warp then writes
+    // the items of its 32 sequences one sequence at a time
+    for (int b0 = wid * 32; b0 < B; b0 += kThreads) {
+        const int b = b0 + lane;
+        int ctx = 0, r = 0, n = 0, ob = 0, os = 0;
+        if (b < B) {
             ctx = load_ctx(p, b, false);
-            nblk = ceil_div_i(ctx, kBlockSize);
-            nfull = nblk / PB;
-            tail = nblk - nfull * PB;
+            const SeqParts sp = seq_parts(ceil_div_i(ctx, kBlockSize), K.PB, p.equal_split);
+            int kb, ks;
+            seq_keys(K, sp, kb, ks);
+            r = sp.nbig;
+            n = sp.n;
+            if (kb != kNoKey) ob = atomicAdd(&cursor[kb], r * Hkv);
+            if (ks != kNoKey) os = atomicAdd(&cursor[ks], (n - r) * Hkv);
         }
-        const bool multi = valid && (nfull + (tail > 0)) > 1;
-        const bool has_tail = valid && (tail > 0 || nblk == 0);
-        const int tkey = key_of(tail, multi);
-        // partial (and empty) partitions: multi-partition sequences first in their class
-        if (has_tail && multi) {
-            const int tb = atomicAdd(&cursor[tkey], Hkv);
-            for (int g = 0; g < Hkv; ++g) p.items[tb + g] = make_int4(b, (nfull << 8) | g, ctx, 0);
+        for (int l = 0; l < 32; ++l) {
+            const int bl = b0 + l;
+            if (bl >= B) break;
+            const int cl = __shfl_sync(0xffffffffu, ctx, l), rl = __shfl_sync(0xffffffffu, r, l);
+            const int nl = __shfl_sync(0xffffffffu, n, l);
+            const int obl = __shfl_sync(0xffffffffu, ob, l), osl = __shfl_sync(0xffffffffu, os, l);
+            for (int i = lane; i < rl * Hkv; i += 32) p.items[obl + i] = make_int4(bl, ((i / Hkv) << 8) | (i % Hkv), cl, 0);
+            for (int i = lane; i < (nl - rl) * Hkv; i += 32)
+                p.items[osl + i] = make_int4(bl, ((rl + i / Hkv) << 8) | (i % Hkv), cl, 0);
         }
-        // multi-partition sequences go to the reduce list
-        const unsigned mm = __ballot_sync(0xffffffffu, multi);
-        int rb = 0;
-        if (lane == 0 && mm) rb = atomicAdd(&nred, __popc(mm));
-        rb = __shfl_sync(0xffffffffu, rb, 0);
-        if (multi) p.red_seqs[rb + __popc(mm & ((1u << lane) - 1))] = b;
-        // block-wide exclusive scans of the full-partition item counts, per class
-        const int vA = multi ? nfull * Hkv : 0, vB = multi ? 0 : nfull * Hkv;
-        int ia = vA, ib = vB;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int ua = __shfl_up_sync(0xffffffffu, ia, o), ub = __shfl_up_sync(0xffffffffu, ib, o);
-            if (lane >= o) {
-                ia += ua;
-                ib += ub;
-            }
-        }
-        if (lane == 31) {
-            wsumA[wid] = ia;
-            wsumB[wid] = ib;
-        }
-        cctx[tid] = ctx;
-        __syncthreads();   // (also orders the multi-partition tail reservations before the others)
-        if (has_tail && !multi) {
-            const int tb = atomicAdd(&cursor[tkey], Hkv);
-            for (int g = 0; g < Hkv; ++g) p.items[tb + g] = make_int4(b, (nfull << 8) | g, ctx, 0);
-        }
-        if (wid == 0) {
-            int xa = lane < kThreads / 32 ? wsumA[lane] : 0, xb = lane < kThreads / 32 ? wsumB[lane] : 0;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int ua = __shfl_up_sync(0xffffffffu, xa, o), ub = __shfl_up_sync(0xffffffffu, xb, o);
-                if (lane >= o) {
-                    xa += ua;
-                    xb += ub;
-                }
-            }
-            if (lane < kThreads / 32) {
-                wsumA[lane] = xa;
-                wsumB[lane] = xb;
-            }
-        }
-        __syncthreads();
-        const int ea = ia - vA + (wid > 0 ? wsumA[wid - 1] : 0);
-        const int eb = ib - vB + (wid > 0 ? wsumB[wid - 1] : 0);
-        preA[tid] = ea;
-        preB[tid] = eb;
-        if (tid == kThreads - 1) {
-            preA[kThreads] = ea + vA;
-            preB[kThreads] = eb + vB;
-        }
-        __syncthreads();
-        // full partitions, one thread per item, its sequence found by binary
-        // search over the prefix; class A before class B when they share a key
-        const int totalA = preA[kThreads], totalB = preB[kThreads];
-        const int baseA = cursor[fkA], baseB = cursor[fkB] + (fkA == fkB ? totalA : 0);
-        for (int cls = 0; cls < 2; ++cls) {
-            const int* pre = cls == 0 ? preA : preB;
-            const int total = cls == 0 ? totalA : totalB;
-            const int base = cls == 0 ? baseA : baseB;
-            for (int i = tid; i < total; i += kThreads) {
-                int lo = 0, hi = kThreads;
-                while (hi - lo > 1) {
-                    const int mid = (lo + hi) >> 1;
-                    if (pre[mid] <= i) lo = mid;
-                    else hi = mid;
-                }
-                const int r = i - pre[lo];
-                p.items[base + i] = make_int4(b0 + lo, ((r / Hkv) << 8) | (r % Hkv), cctx[lo], 0);
-            }
-        }
-        __syncthreads();
-        if (tid == 0) {
-            cursor[fkA] += totalA;
-            cursor[fkB] += totalB;
-        }
-        __syncthreads();
     }
-    if (tid == 0) *p.n_red = nred;
 }
 
 // geometry of one item, identical in every kernel
@@ -242,10 +209,10 @@ __device__ __forceinline__ ItemGeom item_geom(const DecodeParams& p, int4 it) {
     m.p = it.y >> 8;
     m.g = it.y & 255;
     m.ctx = it.z;
-    const int nblk_total = ceil_div_i(m.ctx, kBlockSize);
-    m.j0 = m.p * p.part_blocks;
-    m.nblk = max(0, min(p.part_blocks, nblk_total - m.j0));
-    m.nparts = max(1, ceil_div_i(nblk_total, p.part_blocks));
+    const SeqParts sp = seq_parts(ceil_div_i(m.ctx, kBlockSize), p.part_blocks, p.equal_split);
+    m.j0 = sp.start(m.p);
+    m.nblk = sp.len(m.p);
+    m.nparts = sp.n;
     return m;
 }
 
@@ -341,6 +308,107 @@ struct DescSlot {
     int pad[3];
 };
 
+// ---------------------------------------------------------------------------
+// Self-planning: with p.self_plan set, no plan kernel runs; every CTA of the
+// partition kernel derives its own items of the largest-first list from
+// context_lens before its first tile copy.  The list has the plan kernel's
+// keys in the same order; inside a key the items go in sequence order.  Each
+// CTA reads all of context_lens (one round trip of cp.async), builds the key
+// histogram and its prefix, then each warp finds items rank by rank: the key
+// by binary search over the prefix, the sequence by a warp scan of the key's
+// per-sequence item counts.  Scratch lives in the tile ring, which is free
+// until the first copy.
+//
+// Fills own[0 .. n_own) with this CTA's items (ranks c, 2C-1-c, 2C+c, ...);
+// s_list[0] = list length, s_list[1] = n_own.  Called by every thread of the CTA.
+template <int kMaxOwn>
+__device__ void plan_own_items(const DecodeParams& p, int* scratch, int4* own, int* s_list) {
+    const int tid = threadIdx.x, nthr = blockDim.x, lane = tid & 31, wid = tid >> 5, nwarps = nthr >> 5;
+    const int B = p.num_seqs;
+    int* s_cnt = scratch;                        // [kMaxKeys]
+    int* s_off = s_cnt + kMaxKeys;               // [kMaxKeys + 1]
+    int* s_ctx = s_off + kMaxKeys + 2;           // [B] clamped context lengths
+    int* s_r = s_ctx + B;                        // [B] partitions of the longer length (nbig)
+    int* s_np = s_r + B;                         // [B] partitions
+    int* s_key = s_np + B;                       // [B] kbig | ksmall << 8
+    const PlanKeys K{p.part_blocks, p.part_blocks + 1, p.num_kv_heads, p.class_first};
+    const int nkeys = K.nkeys();
+    for (int b = tid; b < B; b += nthr) cp_async_4(smem_u32(&s_ctx[b]), p.context_lens + b);
+    cp_async_commit();
+    for (int i = tid; i < nkeys; i += nthr) s_cnt[i] = 0;
+    cp_async_wait_all();
+    __syncthreads();
+    // histogram of item keys; CTA 0 reports bad lengths
+    const bool report = blockIdx.x == 0;
+    for (int b = tid; b < B; b += nthr) {
+        const int c = clamp_ctx(p, s_ctx[b], report);
+        const SeqParts sp = seq_parts(ceil_div_i(c, kBlockSize), K.PB, p.equal_split);
+        int kb, ks;
+        seq_keys(K, sp, kb, ks);
+        s_ctx[b] = c;
+        s_r[b] = sp.nbig;
+        s_np[b] = sp.n;
+        s_key[b] = kb | (ks << 8);
+        if (kb != kNoKey) atomicAdd(&s_cnt[kb], sp.nbig * K.Hkv);
+        if (ks != kNoKey) atomicAdd(&s_cnt[ks], (sp.n - sp.nbig) * K.Hkv);
+    }
+    __syncthreads();
+    // bucket offsets and this CTA's share of the list
+    if (wid == 0) {
+        const int total = scan_keys(s_cnt, s_off, nkeys, lane);
+        if (lane == 31) {
+            const int C = gridDim.x, c = blockIdx.x;
+            const int full = total / C, rem = total - full * C;
+            int n_own = full + (((full & 1) ? C - 1 - c : c) < rem ? 1 : 0);
+            s_list[0] = total;
+            if (n_own > kMaxOwn) {   // excluded by the host: report it, and this CTA takes nothing
+                set_status(p.status, PA_ERR_UNSUPPORTED);
+                n_own = 0;
+                s_list[0] = 0;
+            }
+            s_list[1] = n_own;
+        }
+    }
+    __syncthreads();
+    const int n_own = s_list[1];
+    const int C = gridDim.x, c = blockIdx.x;
+    for (int it = wid; it < n_own; it += nwarps) {
+        const int r = it * C + ((it & 1) ? C - 1 - c : c);
+        int lo = 0, hi = nkeys;   // last key whose offset is <= r (never an empty one)
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (s_off[mid] <= r) lo = mid;
+            else hi = mid;
+        }
+        const int k = lo;
+        int j = r - s_off[k];     // index inside key k
+        for (int b0 = 0; b0 < B; b0 += 32) {
+            const int b = b0 + lane;
+            const int kk = b < B ? s_key[b] : (kNoKey | (kNoKey << 8));
+            const bool big = (kk & 0xff) == k, small = (kk >> 8) == k;
+            const int w = big ? s_r[b] * K.Hkv : (small ? (s_np[b] - s_r[b]) * K.Hkv : 0);
+            const int tot = __reduce_add_sync(0xffffffffu, w);
+            if (j >= tot) {
+                j -= tot;
+                continue;
+            }
+            int incl = w;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int u = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += u;
+            }
+            if (j >= incl - w && j < incl) {
+                const int local = j - (incl - w);
+                const int part = (big ? 0 : s_r[b]) + local / K.Hkv;
+                own[it] = make_int4(b, (part << 8) | (local % K.Hkv), s_ctx[b], 0);
+            }
+            break;
+        }
+    }
+    __syncthreads();
+}
+
 template <int D, int NT, int NCW, int STAGES>
 struct TcCfg {
     static constexpr int kBoxes = D / 64;                    // 64-element (128 B) boxes per tile row
@@ -364,15 +432,20 @@ struct TcCfg {
     static constexpr int kOffTasks = kOffMeta + kISlots * (int)sizeof(ItemMeta);
     static constexpr int kMergeW = NCW == 1 ? 128 + 16 : 0;   // merger's partition weights and 1/L
     static constexpr int kOffMW = kOffTasks + kQSlots * 16;
-    static constexpr int kOffBar = kOffMW + kMergeW * 4;
+    static constexpr int kMaxOwn = 64;                       // items a self-planning CTA can hold
+    static constexpr int kOffOwn = kOffMW + kMergeW * 4;
+    static constexpr int kOffBar = kOffOwn + kMaxOwn * 16;
     static constexpr int kNumBars = 2 * STAGES + 2 * kISlots + 2 * kMSlots + 2 * kQSlots;
     static constexpr int kOffFlags = kOffBar + kNumBars * 8;
     static constexpr int kBytes = kOffFlags + 16 + STAGES * 4;
     static constexpr int kSmemBytes = kBytes + 1024;         // slack for 1024-byte alignment
+    // largest batch a self-planning CTA can plan in its ring (4 ints per sequence)
+    static constexpr int kPlanSeqs = (STAGES * kStageBytes / 4 - 2 * kMaxKeys - 2) / 4;
     // warps: NCW consumers, one producer, and (single-warp CTAs) one merger
     static constexpr int kWarps = NCW + 1 + (NCW == 1 ? 1 : 0);
     static constexpr int kThreads = kWarps * 32;
     static_assert(kOffDesc % 16 == 0 && sizeof(DescSlot) % 16 == 0, "cp.async 16-byte destinations");
+    static_assert(kOffOwn % 16 == 0, "own-item list alignment");
     // Ring stage n and stage n + STAGES reuse one slot and one parity bit, so a
     // consumer may only wait for stage n once stage n - STAGES has landed, or it
     // would take the old phase for the new one.  Stage n is consumed by warp
@@ -438,6 +511,14 @@ __global__ void __launch_bounds__(TcCfg<D, NT, NCW, STAGES>::kThreads, 1)
     griddep_launch_dependents();
     griddep_wait();
     const int PB = p.part_blocks;
+    int4* own = reinterpret_cast<int4*>(smem + C::kOffOwn);
+    int* s_plan = const_cast<int*>(abort_flag) + 1;   // [0] list length, [1] own items (self-planning)
+    if (p.self_plan) {
+        plan_own_items<C::kMaxOwn>(p, reinterpret_cast<int*>(stages), own, s_plan);
+        // the scratch was written through the generic proxy; tile copies (async proxy) follow
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncthreads();
+    }
 
     if constexpr (NCW == 1) {
         if (warp == NCW + 1) {
@@ -457,6 +538,8 @@ __global__ void __launch_bounds__(TcCfg<D, NT, NCW, STAGES>::kThreads, 1)
                 __threadfence();
                 float* s_w = reinterpret_cast<float*>(smem + C::kOffMW);
                 merge_group<T, D>(p, task.x, task.y, task.z, lane, s_w, s_w + 128);
+                // every partition has arrived: the counter is free, leave it zeroed for the next call
+                if (lane == 0) p.merge_count[(size_t)task.x * p.num_kv_heads + task.y] = 0;
             }
             return;
         }
@@ -475,42 +558,52 @@ __global__ void __launch_bounds__(TcCfg<D, NT, NCW, STAGES>::kThreads, 1)
         // two items' tile loads: item k's rank, work-list entry and table row
         // land in slot k % kDSlots.  At the top of iteration i, entry(i),
         // row(i) and entry(i+1) are visible and the group {row(i+1),
-        // entry(i+2)} is in flight.
+        // entry(i+2)} is in flight.  A self-planning CTA has its entries in
+        // shared memory already (own[k] is item k).
+        const bool self_plan = p.self_plan != 0;
         int n_items = 0;  // set once the plan's count has been read (below)
         auto fetch_entry = [&](int it, int r) {
             if (lane == 0) {
                 dsc[it % C::kDSlots].rank = r;
-                if (r < n_items) cp_async_16(smem_u32(&dsc[it % C::kDSlots].e), &p.items[r]);
+                if (r < n_items) {
+                    if (self_plan) dsc[it % C::kDSlots].e = own[it];
+                    else cp_async_16(smem_u32(&dsc[it % C::kDSlots].e), &p.items[r]);
+                }
             }
         };
         auto fetch_row = [&](int it) {
             const int r = dsc[it % C::kDSlots].rank;
             if (r >= n_items) return;
-            const int4 e = dsc[it % C::kDSlots].e;
-            const int j0 = (e.y >> 8) * PB;
-            const int nblk = min(PB, ceil_div_i(e.z, kBlockSize) - j0);
-            if (lane < nblk)
+            const ItemGeom m = item_geom(p, dsc[it % C::kDSlots].e);
+            if (lane < m.nblk)
                 cp_async_4(smem_u32(&dsc[it % C::kDSlots].bt[lane]),
-                           p.block_tables + (size_t)e.x * p.max_blocks_per_seq + j0 + lane);
+                           p.block_tables + (size_t)m.b * p.max_blocks_per_seq + m.j0 + lane);
         };
         // Static schedule: CTA c takes ranks c, 2C-1-c, 2C+c, ... of the
         // largest-first list (snake order), which balances the load without a
-        // shared counter (claiming items from one counter was measured slower:
-        // every CTA's claim goes to one address).
+        // shared counter.  (Claiming the list's tail from a counter at run
+        // time was measured slower on every workload.)
         const int ctas = gridDim.x, cta = blockIdx.x;
         auto rank_of = [&](int it) { return it * ctas + ((it & 1) ? (ctas - 1 - cta) : cta); };
         // the item count and this CTA's first work-list entry (rank = cta; the
         // list holds at least gridDim.x entries) arrive in one round trip
-        int* s_nitems = const_cast<int*>(abort_flag) + 1;
-        if (lane == 0) {
-            cp_async_4(smem_u32(s_nitems), p.n_items);
-            cp_async_16(smem_u32(&dsc[0].e), &p.items[cta]);
+        if (self_plan) {
+            n_items = s_plan[0];
+            if (lane == 0) {
+                dsc[0].rank = cta < n_items ? cta : n_items;
+                if (cta < n_items) dsc[0].e = own[0];
+            }
+        } else {
+            if (lane == 0) {
+                cp_async_4(smem_u32(s_plan), &p.hdr[kHdrItems]);
+                cp_async_16(smem_u32(&dsc[0].e), &p.items[cta]);
+            }
+            cp_async_commit();
+            cp_async_wait_all();
+            __syncwarp();
+            n_items = s_plan[0];
+            if (lane == 0) dsc[0].rank = cta < n_items ? cta : n_items;
         }
-        cp_async_commit();
-        cp_async_wait_all();
-        __syncwarp();
-        n_items = *s_nitems;
-        if (lane == 0) dsc[0].rank = cta < n_items ? cta : n_items;
         __syncwarp();
         fetch_row(0);
         fetch_entry(1, rank_of(1));
@@ -976,7 +1069,7 @@ template <typename T, int D, int NW>
 __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(const DecodeParams p) {
     constexpr int E = D / 32;
     griddep_wait();
-    const int n_items = *p.n_items;
+    const int n_items = p.hdr[kHdrItems];
     const int G = p.group;
     const int lane = threadIdx.x & 31;
     const T* qp = static_cast<const T*>(p.q);
@@ -1038,11 +1131,12 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(const DecodeParams
 // ===========================================================================
 // 3. reduce
 // ===========================================================================
-// Rows (sequence, query head) of the sequences the plan listed; a CTA takes
-// rows in turn.  Its 4 warps split a row's partitions (warp w takes partitions
-// w, w + 4, ...; lane l owns D/32 consecutive dims), then add up through
-// shared memory.  Loads are cache-global: the partials were written by other
-// SMs in the previous kernel.
+// Rows (sequence, query head); a CTA takes rows in turn and skips those of
+// sequences with one partition, which the partition kernel finished.  Its 4
+// warps split a row's partitions (warp w takes partitions w, w + 4, ...; lane
+// l owns D/32 consecutive dims), then add up through shared memory.  Loads
+// are cache-global: the partials were written by other SMs in the previous
+// kernel.
 template <typename T, int D>
 __global__ void __launch_bounds__(128) decode_reduce_kernel(const DecodeParams p) {
     constexpr int kW = 4, E = D / 32, U = 8;
@@ -1051,11 +1145,12 @@ __global__ void __launch_bounds__(128) decode_reduce_kernel(const DecodeParams p
     griddep_wait();
     const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int Hq = p.num_heads;
-    const long long n_rows = (long long)(*p.n_red) * Hq;
+    const long long n_rows = (long long)p.num_seqs * Hq;
     for (long long r = blockIdx.x; r < n_rows; r += gridDim.x) {
-        const int b = p.red_seqs[r / Hq], h = (int)(r % Hq);
+        const int b = (int)(r / Hq), h = (int)(r % Hq);
         const int ctx = load_ctx(p, b, false);
         const int nparts = max(1, ceil_div_i(ceil_div_i(ctx, kBlockSize), p.part_blocks));
+        if (nparts == 1) continue;   // (uniform over the CTA)
         const size_t base = ((size_t)b * Hq + h) * p.max_parts;
         float M = kNegInf;
         for (int q = lane; q < nparts; q += 32) M = fmaxf(M, __ldcg(p.part_m + base + q));
@@ -1163,8 +1258,48 @@ cudaError_t make_pool_map(CUtensorMap* map, const void* pool, pa_dtype dtype, in
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+template <int NT_, int NCW_, int ST_>
+struct TcTag {
+    static constexpr int NT = NT_, NCW = NCW_, ST = ST_;
+};
+
+// calls f(TcTag<NT, NCW, STAGES>{}) for the kernel instance of a shape
+template <typename F>
+cudaError_t dispatch_shape(int group, TcShape sh, F&& f) {
+    if (group > 8) return f(TcTag<2, 1, 6>{});
+    switch (sh) {
+        case TcShape::kPaired: return f(TcTag<1, 2, 10>{});
+        case TcShape::kTriple: return f(TcTag<1, 1, 8>{});
+        case TcShape::kPair1: return f(TcTag<1, 1, 13>{});
+        default: return f(TcTag<1, 1, 6>{});
+    }
+}
+
+constexpr int kSelfPlanMaxSeqs = 256;
+
+// PA_SELF_PLAN=0 keeps the plan kernel for every shape (tuning and tests)
+bool self_plan_allowed() {
+    static const bool on = [] {
+        const char* e = getenv("PA_SELF_PLAN");
+        return !(e && std::string(e) == "0");
+    }();
+    return on;
+}
+
+// What launch_decode enqueues for a problem.
+struct DecodeChoice {
+    bool tc = false;         // tensor-core partition kernel (else SIMT)
+    TcShape shape = TcShape::kAuto;
+    bool fused = false;      // the partition kernel merges partitions (no reduce kernel)
+    bool self_plan = false;  // CTAs plan their own items (no plan kernel)
+    bool reduce = false;
+    int grid = 1;            // partition-kernel CTAs
+    int launches = 0;
+};
+
+// grid of a tensor-core instance (one wave of resident CTAs) and whether it can self-plan
 template <typename T, int D, int NT, int NCW, int STAGES>
-cudaError_t launch_tc(const DecodeParams& p, pa_dtype dtype, cudaStream_t stream, int max_items) {
+cudaError_t tc_choice(const DecodeParams& p, long long max_items, DecodeChoice* c) {
     using Cfg = TcCfg<D, NT, NCW, STAGES>;
     auto kernel = decode_tc_kernel<T, D, NT, NCW, STAGES>;
     static bool attr_done = false;
@@ -1173,10 +1308,7 @@ cudaError_t launch_tc(const DecodeParams& p, pa_dtype dtype, cudaStream_t stream
         if (e != cudaSuccess) return e;
         attr_done = true;
     }
-    CUtensorMap mk, mv;
-    cudaError_t e = make_pool_map(&mk, p.key_cache, dtype, p.num_blocks, p.num_kv_heads, D);
-    if (e != cudaSuccess) return e;
-    e = make_pool_map(&mv, p.value_cache, dtype, p.num_blocks, p.num_kv_heads, D);
+    cudaError_t e = prefer_max_shared(reinterpret_cast<const void*>(kernel));
     if (e != cudaSuccess) return e;
     DeviceInfo dev;
     e = device_info(&dev);
@@ -1185,19 +1317,66 @@ cudaError_t launch_tc(const DecodeParams& p, pa_dtype dtype, cudaStream_t stream
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&ctas_per_sm, kernel, Cfg::kThreads, Cfg::kSmemBytes);
     if (e != cudaSuccess) return e;
     if (ctas_per_sm < 1) return cudaErrorInvalidConfiguration;
-    int grid = dev.sm_count * ctas_per_sm;
+    long long grid = (long long)dev.sm_count * ctas_per_sm;
     if (grid > max_items) grid = max_items;
     if (grid < 1) grid = 1;
-    return launch_pdl(kernel, dim3(grid), dim3(Cfg::kThreads), Cfg::kSmemBytes, stream, p, mk, mv);
+    c->grid = (int)grid;
+    // Each self-planning CTA scans all of context_lens; past a few hundred
+    // sequences one plan kernel is cheaper (measured: equal at 256, the plan
+    // kernel 3.6% faster at 1024, self-planning 2-11% faster at 8 and 32).
+    c->self_plan = self_plan_allowed() && p.num_seqs <= kSelfPlanMaxSeqs && p.num_seqs <= Cfg::kPlanSeqs &&
+                   (long long)p.num_seqs * p.num_kv_heads <= kCounterSlots &&
+                   (max_items + grid - 1) / grid <= Cfg::kMaxOwn;
+    return cudaSuccess;
 }
 
 template <typename T, int D>
-cudaError_t launch_simt(const DecodeParams& p, cudaStream_t stream, int max_items) {
+cudaError_t choose(const DecodeParams& p, pa_dtype dtype, DecodeChoice* c) {
+    const long long max_items = (long long)p.num_seqs * p.max_parts * p.num_kv_heads;
+    *c = DecodeChoice{};
+    if constexpr (!std::is_same<T, float>::value) {
+        if (decode_path(dtype, D, p.group) == DecodePath::kTensorCore) {
+            c->tc = true;
+            TcShape sh = tc_shape();
+            // Automatic: sequences split into many (> 32) partitions stream best with
+            // two 2-warp CTAs per SM (measured on 32k contexts); otherwise four
+            // single-warp CTAs per SM, which merge partitions themselves when there
+            // are at most kFusedMaxParts of them.
+            if (sh == TcShape::kAuto) sh = p.max_parts > kPairedMinParts ? TcShape::kPaired : TcShape::kQuad;
+            c->shape = sh;
+            const bool one_warp = p.group > 8 || sh != TcShape::kPaired;
+            c->fused = one_warp && p.max_parts > 1 && p.max_parts <= kFusedMaxParts;
+            const cudaError_t e = dispatch_shape(p.group, sh, [&](auto tag) {
+                using Tg = decltype(tag);
+                return tc_choice<T, D, Tg::NT, Tg::NCW, Tg::ST>(p, max_items, c);
+            });
+            if (e != cudaSuccess) return e;
+        }
+    }
+    c->reduce = p.max_parts > 1 && !c->fused;
+    c->launches = (c->self_plan ? 0 : 1) + 1 + (c->reduce ? 1 : 0);
+    return cudaSuccess;
+}
+
+template <typename T, int D, int NT, int NCW, int STAGES>
+cudaError_t launch_tc(const DecodeParams& p, pa_dtype dtype, cudaStream_t stream, int grid) {
+    using Cfg = TcCfg<D, NT, NCW, STAGES>;
+    CUtensorMap mk, mv;
+    cudaError_t e = make_pool_map(&mk, p.key_cache, dtype, p.num_blocks, p.num_kv_heads, D);
+    if (e != cudaSuccess) return e;
+    e = make_pool_map(&mv, p.value_cache, dtype, p.num_blocks, p.num_kv_heads, D);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(decode_tc_kernel<T, D, NT, NCW, STAGES>, dim3(grid), dim3(Cfg::kThreads), Cfg::kSmemBytes,
+                      stream, p, mk, mv);
+}
+
+template <typename T, int D>
+cudaError_t launch_simt(const DecodeParams& p, cudaStream_t stream, long long max_items) {
     DeviceInfo dev;
     cudaError_t e = device_info(&dev);
     if (e != cudaSuccess) return e;
     constexpr int NW = 4;
-    long long want = ((long long)max_items * p.group + NW - 1) / NW;
+    long long want = (max_items * p.group + NW - 1) / NW;
     long long cap = (long long)dev.sm_count * 8;
     int grid = (int)(want < cap ? want : cap);
     if (grid < 1) grid = 1;
@@ -1206,42 +1385,31 @@ cudaError_t launch_simt(const DecodeParams& p, cudaStream_t stream, int max_item
 
 template <typename T, int D>
 cudaError_t launch_all(DecodeParams p, pa_dtype dtype, cudaStream_t stream) {
-    const int max_items = p.num_seqs * p.max_parts * p.num_kv_heads;
-    // plan: one CTA; 256 threads cover typical batches in one pass, 1024 large ones
-    cudaError_t e = p.num_seqs <= 256 ? launch_pdl(decode_plan_kernel<256>, dim3(1), dim3(256), 0, stream, p)
-                                      : launch_pdl(decode_plan_kernel<1024>, dim3(1), dim3(1024), 0, stream, p);
+    DecodeChoice c;
+    cudaError_t e = choose<T, D>(p, dtype, &c);
     if (e != cudaSuccess) return e;
-    const DecodePath path = decode_path(dtype, D, p.group);
-    bool fused = false;
+    p.fused_merge = c.fused ? 1 : 0;
+    p.self_plan = c.self_plan ? 1 : 0;
+    if (!c.self_plan) {
+        // plan: one CTA; 256 threads cover typical batches in one pass, 1024 large ones
+        e = p.num_seqs <= 256 ? launch_pdl(decode_plan_kernel<256>, dim3(1), dim3(256), 0, stream, p)
+                              : launch_pdl(decode_plan_kernel<1024>, dim3(1), dim3(1024), 0, stream, p);
+        if (e != cudaSuccess) return e;
+    }
     if constexpr (std::is_same<T, float>::value) {
-        e = launch_simt<T, D>(p, stream, max_items);
+        e = launch_simt<T, D>(p, stream, (long long)p.num_seqs * p.max_parts * p.num_kv_heads);
     } else {
-        if (path == DecodePath::kTensorCore) {
-            TcShape sh = tc_shape();
-            // Automatic: sequences split into many (> 32) partitions stream best with
-            // two 2-warp CTAs per SM (measured on 32k contexts); otherwise four
-            // single-warp CTAs per SM, which merge partitions themselves when there
-            // are at most kFusedMaxParts of them.
-            if (sh == TcShape::kAuto) sh = p.max_parts > kPairedMinParts ? TcShape::kPaired : TcShape::kQuad;
-            // single-warp shapes merge partitions in-kernel when there are few of them
-            fused = sh != TcShape::kPaired && p.max_parts > 1 && p.max_parts <= kFusedMaxParts;
-            p.fused_merge = fused ? 1 : 0;
-            if (p.group <= 8) {
-                switch (sh) {
-                    case TcShape::kPaired: e = launch_tc<T, D, 1, 2, 10>(p, dtype, stream, max_items); break;
-                    case TcShape::kTriple: e = launch_tc<T, D, 1, 1, 8>(p, dtype, stream, max_items); break;
-                    case TcShape::kPair1: e = launch_tc<T, D, 1, 1, 13>(p, dtype, stream, max_items); break;
-                    default: e = launch_tc<T, D, 1, 1, 6>(p, dtype, stream, max_items); break;
-                }
-            } else {
-                e = launch_tc<T, D, 2, 1, 6>(p, dtype, stream, max_items);
-            }
+        if (c.tc) {
+            e = dispatch_shape(p.group, c.shape, [&](auto tag) {
+                using Tg = decltype(tag);
+                return launch_tc<T, D, Tg::NT, Tg::NCW, Tg::ST>(p, dtype, stream, c.grid);
+            });
+        } else {
+            e = launch_simt<T, D>(p, stream, (long long)p.num_seqs * p.max_parts * p.num_kv_heads);
         }
-        else
-            e = launch_simt<T, D>(p, stream, max_items);
     }
     if (e != cudaSuccess) return e;
-    if (p.max_parts > 1 && !fused) {
+    if (c.reduce) {
         DeviceInfo dev;
         e = device_info(&dev);
         if (e != cudaSuccess) return e;
@@ -1250,6 +1418,27 @@ cudaError_t launch_all(DecodeParams p, pa_dtype dtype, cudaStream_t stream) {
         e = launch_pdl(decode_reduce_kernel<T, D>, dim3((unsigned)(rows < cap ? rows : cap)), dim3(128), 0, stream, p);
     }
     return e;
+}
+
+// partition lengths: full partitions and the remainder last (measured best);
+// PA_SPLIT=equal gives near-equal lengths (tuning)
+int equal_split() {
+    static const int v = [] {
+        const char* e = getenv("PA_SPLIT");
+        return (e && std::string(e) == "equal") ? 1 : 0;
+    }();
+    return v;
+}
+
+int class_first_order() {
+    // item order: every item of the split sequences first, so that their
+    // merges happen early (measured best with the fused merge);
+    // PA_PLAN_ORDER=size orders all items by size alone (tuning)
+    static const int cf = [] {
+        const char* e = getenv("PA_PLAN_ORDER");
+        return (e && std::string(e) == "size") ? 0 : 1;
+    }();
+    return cf;
 }
 
 }  // namespace
@@ -1262,13 +1451,8 @@ DecodePath decode_path(pa_dtype dtype, int head_dim, int group) {
 
 cudaError_t launch_decode(const DecodeParams& p_in, pa_dtype dtype, cudaStream_t stream) {
     DecodeParams p = p_in;
-    // item order: multi-partition sequences' items first (measured best with
-    // the fused merge); PA_PLAN_ORDER=size orders all items by size (tuning)
-    static const int class_first = [] {
-        const char* e = getenv("PA_PLAN_ORDER");
-        return (e && std::string(e) == "size") ? 0 : 1;
-    }();
-    p.class_first = class_first;
+    p.class_first = class_first_order();
+    p.equal_split = equal_split();
     switch (dtype) {
         case PA_F32: return p.head_dim == 64 ? launch_all<float, 64>(p, dtype, stream)
                                              : launch_all<float, 128>(p, dtype, stream);
@@ -1278,6 +1462,20 @@ cudaError_t launch_decode(const DecodeParams& p_in, pa_dtype dtype, cudaStream_t
                                               : launch_all<__nv_bfloat16, 128>(p, dtype, stream);
     }
     return cudaErrorInvalidValue;
+}
+
+cudaError_t decode_launch_count(const DecodeParams& p, pa_dtype dtype, int* launches) {
+    DecodeChoice c;
+    cudaError_t e = cudaErrorInvalidValue;
+    switch (dtype) {
+        case PA_F32: e = p.head_dim == 64 ? choose<float, 64>(p, dtype, &c) : choose<float, 128>(p, dtype, &c); break;
+        case PA_F16: e = p.head_dim == 64 ? choose<__half, 64>(p, dtype, &c) : choose<__half, 128>(p, dtype, &c); break;
+        case PA_BF16:
+            e = p.head_dim == 64 ? choose<__nv_bfloat16, 64>(p, dtype, &c) : choose<__nv_bfloat16, 128>(p, dtype, &c);
+            break;
+    }
+    if (e == cudaSuccess) *launches = c.launches;
+    return e;
 }
 
 }  // namespace pa

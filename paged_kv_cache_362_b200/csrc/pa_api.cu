@@ -30,6 +30,20 @@ cudaError_t device_info(DeviceInfo* out) {
     return cudaSuccess;
 }
 
+cudaError_t prefer_max_shared(const void* kernel) {
+    static std::mutex mu;
+    static const void* done[256];
+    static int n = 0;
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < n; ++i)
+        if (done[i] == kernel) return cudaSuccess;
+    const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                               cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
+    if (n < 256) done[n++] = kernel;
+    return cudaSuccess;
+}
+
 namespace {
 
 int elt_bytes(pa_dtype d) { return d == PA_F32 ? 4 : 2; }
@@ -47,10 +61,16 @@ int auto_partition_size(int64_t num_seqs, int64_t num_kv_heads, int64_t max_cont
     return P;
 }
 
+// Workspace: a 256-byte header (the plan kernel's list length), the merge
+// counters, the work list, then the partitions' (m, l, O).  The merge counters
+// sit at the same place for every problem, in a region of at least
+// kCounterSlots entries, so a workspace reused for problems of another shape
+// still finds them zeroed: every call leaves its counters at zero, and no
+// other region ever overlaps the first kCounterSlots.
 struct WsLayout {
     int partition_size, max_parts;
     int64_t max_items;
-    size_t off_items, off_red, off_cnt, off_m, off_l, off_o, total;
+    size_t off_items, off_cnt, off_m, off_l, off_o, total;
 };
 
 bool ws_layout(int64_t num_seqs, int64_t num_heads, int64_t num_kv_heads, int64_t head_dim,
@@ -65,10 +85,10 @@ bool ws_layout(int64_t num_seqs, int64_t num_heads, int64_t num_kv_heads, int64_
     w->max_parts = (int)np;
     w->max_items = num_seqs * np * num_kv_heads;
     const int64_t parts = np > 1 ? num_seqs * num_heads * np : 0;
-    w->off_items = 256;
-    w->off_red = round_up(w->off_items + (size_t)w->max_items * sizeof(int4), 256);
-    w->off_cnt = round_up(w->off_red + (size_t)num_seqs * sizeof(int32_t), 256);
-    w->off_m = round_up(w->off_cnt + (size_t)num_seqs * num_kv_heads * sizeof(int32_t), 256);
+    w->off_cnt = 256;
+    const int64_t counters = std::max<int64_t>(kCounterSlots, num_seqs * num_kv_heads);
+    w->off_items = round_up(w->off_cnt + (size_t)counters * sizeof(int32_t), 256);
+    w->off_m = round_up(w->off_items + (size_t)w->max_items * sizeof(int4), 256);
     w->off_l = round_up(w->off_m + (size_t)parts * sizeof(float), 256);
     w->off_o = round_up(w->off_l + (size_t)parts * sizeof(float), 256);
     w->total = round_up(w->off_o + (size_t)parts * head_dim * sizeof(float), 256);
@@ -155,9 +175,7 @@ pa_status pa_decode(void* out, const void* q, const void* key_cache, const void*
     p.max_parts = w.max_parts;
     p.scale_log2 = scale * 1.4426950408889634f;  // log2(e)
     uint8_t* ws = static_cast<uint8_t*>(workspace);
-    p.n_items = reinterpret_cast<int32_t*>(ws);
-    p.n_red = reinterpret_cast<int32_t*>(ws) + 1;
-    p.red_seqs = reinterpret_cast<int32_t*>(ws + w.off_red);
+    p.hdr = reinterpret_cast<int32_t*>(ws);
     p.merge_count = reinterpret_cast<int32_t*>(ws + w.off_cnt);
     p.items = reinterpret_cast<int4*>(ws + w.off_items);
     p.part_m = reinterpret_cast<float*>(ws + w.off_m);
@@ -165,6 +183,25 @@ pa_status pa_decode(void* out, const void* q, const void* key_cache, const void*
     p.part_o = reinterpret_cast<float*>(ws + w.off_o);
     const cudaError_t e = launch_decode(p, dtype, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+int32_t pa_decode_launch_count(int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads, int32_t head_dim,
+                               int32_t max_context_len, int32_t partition_size, pa_dtype dtype) {
+    if (num_seqs <= 0 || num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads != 0) return -1;
+    if (!valid_dtype(dtype) || (head_dim != 64 && head_dim != 128) || num_kv_heads > 255) return -1;
+    WsLayout w;
+    if (!ws_layout(num_seqs, num_heads, num_kv_heads, head_dim, max_context_len, partition_size, &w)) return -1;
+    if (w.max_items > INT32_MAX) return -1;
+    DecodeParams p{};
+    p.num_seqs = num_seqs;
+    p.num_heads = num_heads;
+    p.num_kv_heads = num_kv_heads;
+    p.head_dim = head_dim;
+    p.group = num_heads / num_kv_heads;
+    p.part_blocks = w.partition_size / kBlockSize;
+    p.max_parts = w.max_parts;
+    int n = 0;
+    return decode_launch_count(p, dtype, &n) == cudaSuccess ? n : -1;
 }
 
 pa_status pa_copy_blocks(void* key_cache, void* value_cache, const int64_t* block_pairs, int32_t num_pairs,

@@ -209,6 +209,10 @@ __device__ __forceinline__ int ceil_div_i(int a, int b) { return (a + b - 1) / b
 // ---------------------------------------------------------------------------
 // decode: shared parameter block and work-item encoding
 // ---------------------------------------------------------------------------
+// Workspace header words (int32): kHdrItems = length of the work list
+// written by the plan kernel.
+constexpr int kHdrItems = 0;
+
 struct DecodeParams {
     void* out;                    // [B, Hq, D]
     const void* q;                // [B, Hq, D]
@@ -224,26 +228,29 @@ struct DecodeParams {
     int max_parts;                // NP_max = ceil(max_context_len / partition_size)
     float scale_log2;             // scale * log2(e)
     // workspace views
-    int32_t* n_items;             // [1] items in the work list
-    int32_t* n_red;               // [1] sequences that span several partitions
-    int32_t* red_seqs;            // [num_seqs] their indices (order unspecified)
-    int32_t* merge_count;         // [num_seqs * num_kv_heads] partitions finished (reset by the plan kernel)
+    int32_t* hdr;                 // [64] header words, indices kHdr* below
+    int32_t* merge_count;         // [num_seqs * num_kv_heads] partitions finished; zero between calls
+                                  // (each merger resets the counter it completes)
     int fused_merge;              // 1: the partition kernel merges partitions itself (no reduce kernel)
-    int class_first;              // plan order: 1 = multi-partition sequences' items first
-    int4* items;                  // [max_items]: (b, (p << 8) | g, clamped ctx, 0), largest first
+    int class_first;              // item order: 1 = multi-partition sequences' items first
+    int self_plan;                // 1: each partition-kernel CTA derives its own items (no plan kernel)
+    int equal_split;              // 1: a sequence's partitions have near-equal lengths (else full + remainder)
+    int4* items;                  // [max_items]: (b, (p << 8) | g, clamped ctx, 0), largest first (plan kernel)
     float* part_m;                // [B, Hq, NP_max]   max logit (log2 units)
     float* part_l;                // [B, Hq, NP_max]   sum of 2^(s - m)
     float* part_o;                // [B, Hq, NP_max, D] unnormalised output
 };
 
 // context length as every decode kernel sees it: clamped into [0, ctx_cap]
-__device__ __forceinline__ int load_ctx(const DecodeParams& p, int b, bool flag) {
-    int c = p.context_lens[b];
+__device__ __forceinline__ int clamp_ctx(const DecodeParams& p, int c, bool flag) {
     if (c < 0 || c > p.ctx_cap) {
         if (flag) set_status(p.status, PA_ERR_OUT_OF_RANGE);
         c = c < 0 ? 0 : p.ctx_cap;
     }
     return c;
+}
+__device__ __forceinline__ int load_ctx(const DecodeParams& p, int b, bool flag) {
+    return clamp_ctx(p, p.context_lens[b], flag);
 }
 
 }  // namespace pa

@@ -27,8 +27,21 @@ cudaError_t launch_copy_blocks(void* key_cache, void* value_cache, const int64_t
 enum class DecodePath { kTensorCore, kSimt };
 DecodePath decode_path(pa_dtype dtype, int head_dim, int group);
 
-// Plan + partition kernel + (if any sequence spans several partitions) reduce.
+// Merge counters the workspace always reserves (at a fixed offset); problems
+// with more (sequence, KV head) pairs than this use the plan kernel, which
+// zeroes the counters it uses.
+constexpr int kCounterSlots = 16384;
+
+// [plan] + partition kernel + (if sequences span several partitions and the
+// partition kernel does not merge them) reduce.
 cudaError_t launch_decode(const DecodeParams& p, pa_dtype dtype, cudaStream_t stream);
+
+// Number of kernels launch_decode enqueues for these sizes (p's pointers unused).
+cudaError_t decode_launch_count(const DecodeParams& p, pa_dtype dtype, int* launches);
+
+// Every library kernel asks for the same (maximum) shared-memory carveout, so
+// that SMs need not reconfigure L1/shared memory between chained kernels.
+cudaError_t prefer_max_shared(const void* kernel);
 
 // Launch with programmatic stream serialisation so a kernel's launch overlaps
 // the tail of its predecessor; every kernel calls griddep_wait() before it
@@ -36,6 +49,8 @@ cudaError_t launch_decode(const DecodeParams& p, pa_dtype dtype, cudaStream_t st
 template <typename... KArgs, typename... Args>
 cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
                        Args&&... args) {
+    const cudaError_t ce = prefer_max_shared(reinterpret_cast<const void*>(kernel));
+    if (ce != cudaSuccess) return ce;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
     cfg.blockDim = block;

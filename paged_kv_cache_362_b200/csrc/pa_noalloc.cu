@@ -11,10 +11,11 @@
 // module is loaded holds it until the process exits.  Problems whose
 // workspace (pa_decode_workspace_size) exceeds it are rejected.
 //
-// All calls share the one array.  Nothing in it has to start at zero -- each
-// call's plan kernel rewrites the item count and the work list before the
-// other kernels read them -- but calls whose kernels overlap on the GPU (two
-// streams, or two host threads) race on it and give wrong results.
+// All calls share the one array; calls whose kernels overlap on the GPU (two
+// streams, or two host threads) race on it and give wrong results.  The first
+// call on a device zero-fills it (the state pa_decode asks of a fresh
+// workspace: its merge counters at zero); every call that completes leaves
+// them zeroed again.
 #include <mutex>
 
 #include "pa_internal.h"
@@ -32,8 +33,10 @@ std::mutex g_mu;
 void* g_scratch_addr[kMaxDevices] = {};
 
 // Device address of g_decode_scratch on the current device, resolved on the
-// first call made with that device current.
-cudaError_t scratch_address(void** out) {
+// first call made with that device current.  That first call also zero-fills
+// the array on `stream` and waits for it, so the state pa_decode expects of a
+// fresh workspace does not rest on how the module was loaded.
+cudaError_t scratch_address(void** out, cudaStream_t stream) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
@@ -42,6 +45,10 @@ cudaError_t scratch_address(void** out) {
     if (g_scratch_addr[dev] == nullptr) {
         void* p = nullptr;
         e = cudaGetSymbolAddress(&p, g_decode_scratch);
+        if (e != cudaSuccess) return e;
+        e = cudaMemsetAsync(p, 0, kStaticScratchBytes, stream);
+        if (e != cudaSuccess) return e;
+        e = cudaStreamSynchronize(stream);
         if (e != cudaSuccess) return e;
         g_scratch_addr[dev] = p;
     }
@@ -63,7 +70,7 @@ extern "C" pa_status pa_decode_noalloc(void* out, const void* q, const void* key
     if (need == 0) return PA_ERR_INVALID_ARG;
     if (need > kStaticScratchBytes) return PA_ERR_UNSUPPORTED;  // problem too large for the fixed scratch
     void* scratch = nullptr;
-    if (scratch_address(&scratch) != cudaSuccess) return PA_ERR_CUDA;
+    if (scratch_address(&scratch, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return PA_ERR_CUDA;
     return pa_decode(out, q, key_cache, value_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs,
                      num_heads, num_kv_heads, head_dim, block_size, num_blocks, scale, max_context_len,
                      partition_size, scratch, kStaticScratchBytes, dtype, status, stream);

@@ -50,9 +50,14 @@ def test_workspace_size_is_consistent():
     assert lib.pa_decode_workspace_size(4, 28, 4, 128, 100, 24) == 0      # not a multiple of 16
     assert lib.pa_decode_workspace_size(4, 28, 4, 128, 100, 1024) == 0    # above 512
     assert lib.pa_decode_workspace_size(-1, 28, 4, 128, 100, 0) == 0
-    # one partition -> no partial buffers, only header + item list
+    # one partition -> no partial buffers: header, the fixed 16384-entry merge
+    # counter region (int32) and the item list
+    counters = 16384 * 4
     small = lib.pa_decode_workspace_size(8, 28, 4, 128, 512, 512)
-    assert 256 < small < 4096
+    assert 256 + counters < small < 256 + counters + 4096
+    # the counter region grows with the (sequence, KV head) pairs beyond that
+    huge = lib.pa_decode_workspace_size(8192, 32, 8, 128, 16, 16)
+    assert huge >= 256 + 8192 * 8 * 4 + 8192 * 8 * 16
     # 32k context, 512-token partitions: 64 partials of (D + 2) floats per (seq, head)
     big = lib.pa_decode_workspace_size(8, 28, 4, 128, 32768, 512)
     assert big >= 8 * 28 * 64 * (128 + 2) * 4
