@@ -89,6 +89,18 @@ __device__ __forceinline__ SeqParts seq_parts(int nblk, int PB, bool equal) {
     }
     return s;
 }
+// the same, without a division for the common single-partition case
+__device__ __forceinline__ SeqParts seq_parts_fast(int nblk, int PB, bool equal) {
+    if (nblk <= PB) {
+        SeqParts s;
+        s.n = 1;
+        s.big = equal ? nblk + 1 : PB;
+        s.nbig = (!equal && nblk == PB) ? 1 : 0;
+        s.small = nblk;
+        return s;
+    }
+    return seq_parts(nblk, PB, equal);
+}
 
 // Item order.  Largest first (key = PB - blocks; empty sequences last), which
 // the snake assignment of the partition kernel turns into an even load.  With
@@ -159,7 +171,7 @@ __global__ void __launch_bounds__(kThreads) decode_plan_kernel(const DecodeParam
     __syncthreads();
     // pass 1: histogram of item keys
     for (int b = tid; b < B; b += kThreads) {
-        const SeqParts sp = seq_parts(ceil_div_i(load_ctx(p, b, true), kBlockSize), K.PB, p.equal_split);
+        const SeqParts sp = seq_parts_fast(ceil_div_i(load_ctx(p, b, true), kBlockSize), K.PB, p.equal_split);
         int kb, ks;
         seq_keys(K, sp, kb, ks);
         if (kb != kNoKey) atomicAdd(&cnt[kb], sp.nbig * Hkv);
@@ -178,7 +190,7 @@ __global__ void __launch_bounds__(kThreads) decode_plan_kernel(const DecodeParam
         int ctx = 0, r = 0, n = 0, ob = 0, os = 0;
         if (b < B) {
             ctx = load_ctx(p, b, false);
-            const SeqParts sp = seq_parts(ceil_div_i(ctx, kBlockSize), K.PB, p.equal_split);
+            const SeqParts sp = seq_parts_fast(ceil_div_i(ctx, kBlockSize), K.PB, p.equal_split);
             int kb, ks;
             seq_keys(K, sp, kb, ks);
             r = sp.nbig;
@@ -209,7 +221,7 @@ __device__ __forceinline__ ItemGeom item_geom(const DecodeParams& p, int4 it) {
     m.p = it.y >> 8;
     m.g = it.y & 255;
     m.ctx = it.z;
-    const SeqParts sp = seq_parts(ceil_div_i(m.ctx, kBlockSize), p.part_blocks, p.equal_split);
+    const SeqParts sp = seq_parts_fast(ceil_div_i(m.ctx, kBlockSize), p.part_blocks, p.equal_split);
     m.j0 = sp.start(m.p);
     m.nblk = sp.len(m.p);
     m.nparts = sp.n;
@@ -342,7 +354,7 @@ __device__ void plan_own_items(const DecodeParams& p, int* scratch, int4* own, i
     const bool report = blockIdx.x == 0;
     for (int b = tid; b < B; b += nthr) {
         const int c = clamp_ctx(p, s_ctx[b], report);
-        const SeqParts sp = seq_parts(ceil_div_i(c, kBlockSize), K.PB, p.equal_split);
+        const SeqParts sp = seq_parts_fast(ceil_div_i(c, kBlockSize), K.PB, p.equal_split);
         int kb, ks;
         seq_keys(K, sp, kb, ks);
         s_ctx[b] = c;
@@ -444,6 +456,9 @@ struct TcCfg {
     // warps: NCW consumers, one producer, and (single-warp CTAs) one merger
     static constexpr int kWarps = NCW + 1 + (NCW == 1 ? 1 : 0);
     static constexpr int kThreads = kWarps * 32;
+    // CTAs per SM the shape is sized for (shared memory at D = 128); the
+    // register budget is capped to match
+    static constexpr int kMinBlocks = (NCW == 2 || NT == 2 || STAGES >= 13) ? 2 : (STAGES >= 8 ? 3 : 4);
     static_assert(kOffDesc % 16 == 0 && sizeof(DescSlot) % 16 == 0, "cp.async 16-byte destinations");
     static_assert(kOffOwn % 16 == 0, "own-item list alignment");
     // Ring stage n and stage n + STAGES reuse one slot and one parity bit, so a
@@ -455,7 +470,7 @@ struct TcCfg {
 };
 
 template <typename T, int D, int NT, int NCW, int STAGES>
-__global__ void __launch_bounds__(TcCfg<D, NT, NCW, STAGES>::kThreads, 1)
+__global__ void __launch_bounds__(TcCfg<D, NT, NCW, STAGES>::kThreads, TcCfg<D, NT, NCW, STAGES>::kMinBlocks)
     decode_tc_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV) {
     using C = TcCfg<D, NT, NCW, STAGES>;
@@ -514,6 +529,14 @@ __global__ void __launch_bounds__(TcCfg<D, NT, NCW, STAGES>::kThreads, 1)
     int4* own = reinterpret_cast<int4*>(smem + C::kOffOwn);
     int* s_plan = const_cast<int*>(abort_flag) + 1;   // [0] list length, [1] own items (self-planning)
     if (p.self_plan) {
+        {   // warm L2 with this CTA's share of the block tables: the rows are read right after planning
+            const char* bt = reinterpret_cast<const char*>(p.block_tables);
+            const size_t bytes = (size_t)p.num_seqs * p.max_blocks_per_seq * sizeof(int32_t);
+            const size_t share = (bytes + gridDim.x - 1) / gridDim.x;
+            const size_t lo = share * blockIdx.x, hi = min(bytes, lo + share);
+            for (size_t off = lo + (size_t)threadIdx.x * 128; off < hi; off += (size_t)blockDim.x * 128)
+                prefetch_l2(bt + off);
+        }
         plan_own_items<C::kMaxOwn>(p, reinterpret_cast<int*>(stages), own, s_plan);
         // the scratch was written through the generic proxy; tile copies (async proxy) follow
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -806,100 +829,157 @@ __global__ void __launch_bounds__(TcCfg<D, NT, NCW, STAGES>::kThreads, 1)
         }
         stage_base = item_base;
         const uint32_t item_end = stage_base + (uint32_t)m.nblk;
-        uint32_t n = stage_base + (uint32_t)cw;
-        for (; n < item_end; n += NCW) {
-            const int s = n % STAGES;
-            const int j = (int)(n - stage_base);
-            if (!__all_sync(0xffffffffu, mbar_wait(&full[s], (n / STAGES) & 1)) || *abort_flag) {
-                *abort_flag = 1;
-                break;
-            }
-            if (!stage_bad[s]) {
-                const int valid = min(kBlockSize, m.ctx - (m.j0 + j) * kBlockSize);
-                const uint32_t tbase = smem_u32(stages + s * C::kStageBytes);
 
-                // ---- S^T[16 tokens x 8*NT heads] = K Q^T, two accumulator chains
-                float sa[NT][4], sb[NT][4];
+        // One step of NB blocks (tiles at tb[], valid token counts vl[]):
+        // S^T = K Q^T for each block (two accumulator chains per block, the
+        // blocks' chains interleaved), one online-softmax update over all NB*16
+        // tokens, then O^T += V^T P^T for each block.
+        auto step = [&](auto nb_tag, const uint32_t* tb, const int* vl) {
+            constexpr int NB = decltype(nb_tag)::value;
+            float sa[NB][NT][4], sb[NB][NT][4];
+#pragma unroll
+            for (int bb = 0; bb < NB; ++bb)
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) sa[nt][c] = sb[nt][c] = 0.f;
+                    for (int c = 0; c < 4; ++c) sa[bb][nt][c] = sb[bb][nt][c] = 0.f;
 #pragma unroll
-                for (int kk = 0; kk < KS; ++kk) {
+            for (int kk = 0; kk < KS; ++kk) {
+#pragma unroll
+                for (int bb = 0; bb < NB; ++bb) {
                     uint32_t a[4];
-                    ldsm_x4(tbase + koff[kk], a[0], a[1], a[2], a[3]);
+                    ldsm_x4(tb[bb] + koff[kk], a[0], a[1], a[2], a[3]);
 #pragma unroll
                     for (int nt = 0; nt < NT; ++nt) {
-                        if (kk & 1) Mma<T>::run(sb[nt], a, qf[nt][kk][0], qf[nt][kk][1]);
-                        else Mma<T>::run(sa[nt], a, qf[nt][kk][0], qf[nt][kk][1]);
+                        if (kk & 1) Mma<T>::run(sb[bb][nt], a, qf[nt][kk][0], qf[nt][kk][1]);
+                        else Mma<T>::run(sa[bb][nt], a, qf[nt][kk][0], qf[nt][kk][1]);
                     }
                 }
+            }
 
-                // ---- online softmax per head column; P^T fragments for the PV product
-                uint32_t pb[NT][2], pl[NT][2];
-                bool rescale = false;
-                float al[NT][2];
+            // ---- online softmax per head column; P^T fragments for the PV product
+            uint32_t pb[NB][NT][2], pl[NB][NT][2];
+            bool rescale = false;
+            float al[NT][2];
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    float s0 = (sa[nt][0] + sb[nt][0]) * sl2, s1 = (sa[nt][1] + sb[nt][1]) * sl2;
-                    float s2 = (sa[nt][2] + sb[nt][2]) * sl2, s3 = (sa[nt][3] + sb[nt][3]) * sl2;
-                    if (gid >= valid) s0 = s1 = kNegInf;
-                    if (gid + 8 >= valid) s2 = s3 = kNegInf;
-                    float mx0 = fmaxf(s0, s2), mx1 = fmaxf(s1, s3);
+            for (int nt = 0; nt < NT; ++nt) {
+                float sv[NB][4];
+                float mx0 = kNegInf, mx1 = kNegInf;
 #pragma unroll
-                    for (int off = 4; off < 32; off <<= 1) {
-                        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
-                        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
-                    }
-                    const float mn0 = fmaxf(mrun[nt][0], mx0), mn1 = fmaxf(mrun[nt][1], mx1);
-                    const float ms0 = mn0 == kNegInf ? 0.f : mn0, ms1 = mn1 == kNegInf ? 0.f : mn1;
-                    // alpha = 2^(m_old - m_new), exactly 1 when the running max did not move
-                    al[nt][0] = mn0 == mrun[nt][0] ? 1.f : fast_exp2(mrun[nt][0] - ms0);
-                    al[nt][1] = mn1 == mrun[nt][1] ? 1.f : fast_exp2(mrun[nt][1] - ms1);
-                    rescale |= (al[nt][0] != 1.f) | (al[nt][1] != 1.f);
-                    mrun[nt][0] = mn0;
-                    mrun[nt][1] = mn1;
-                    const float p0 = fast_exp2(s0 - ms0), p1 = fast_exp2(s1 - ms1);
-                    const float p2 = fast_exp2(s2 - ms0), p3 = fast_exp2(s3 - ms1);
-                    lrun[nt][0] = lrun[nt][0] * al[nt][0] + (p0 + p2);
-                    lrun[nt][1] = lrun[nt][1] * al[nt][1] + (p1 + p3);
+                for (int bb = 0; bb < NB; ++bb) {
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) sv[bb][c] = (sa[bb][nt][c] + sb[bb][nt][c]) * sl2;
+                    if (gid >= vl[bb]) sv[bb][0] = sv[bb][1] = kNegInf;
+                    if (gid + 8 >= vl[bb]) sv[bb][2] = sv[bb][3] = kNegInf;
+                    mx0 = fmaxf(mx0, fmaxf(sv[bb][0], sv[bb][2]));
+                    mx1 = fmaxf(mx1, fmaxf(sv[bb][1], sv[bb][3]));
+                }
+#pragma unroll
+                for (int off = 4; off < 32; off <<= 1) {
+                    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+                    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+                }
+                const float mn0 = fmaxf(mrun[nt][0], mx0), mn1 = fmaxf(mrun[nt][1], mx1);
+                const float ms0 = mn0 == kNegInf ? 0.f : mn0, ms1 = mn1 == kNegInf ? 0.f : mn1;
+                // alpha = 2^(m_old - m_new), exactly 1 when the running max did not move
+                al[nt][0] = mn0 == mrun[nt][0] ? 1.f : fast_exp2(mrun[nt][0] - ms0);
+                al[nt][1] = mn1 == mrun[nt][1] ? 1.f : fast_exp2(mrun[nt][1] - ms1);
+                rescale |= (al[nt][0] != 1.f) | (al[nt][1] != 1.f);
+                mrun[nt][0] = mn0;
+                mrun[nt][1] = mn1;
+                float l0 = 0.f, l1 = 0.f;
+#pragma unroll
+                for (int bb = 0; bb < NB; ++bb) {
+                    const float p0 = fast_exp2(sv[bb][0] - ms0), p1 = fast_exp2(sv[bb][1] - ms1);
+                    const float p2 = fast_exp2(sv[bb][2] - ms0), p3 = fast_exp2(sv[bb][3] - ms1);
+                    l0 += p0 + p2;
+                    l1 += p1 + p3;
                     const uint32_t h01 = Elt<T>::pack2(p0, p1), h23 = Elt<T>::pack2(p2, p3);
-                    pb[nt][0] = movmatrix_t(h01);
-                    pb[nt][1] = movmatrix_t(h23);
+                    pb[bb][nt][0] = movmatrix_t(h01);
+                    pb[bb][nt][1] = movmatrix_t(h23);
                     if constexpr (kSplitP) {
                         // remainder of p after bf16 rounding, itself in bf16: hi + lo carries ~16 bits
                         const float2 f01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&h01));
                         const float2 f23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&h23));
-                        pl[nt][0] = movmatrix_t(Elt<T>::pack2(p0 - f01.x, p1 - f01.y));
-                        pl[nt][1] = movmatrix_t(Elt<T>::pack2(p2 - f23.x, p3 - f23.y));
+                        pl[bb][nt][0] = movmatrix_t(Elt<T>::pack2(p0 - f01.x, p1 - f01.y));
+                        pl[bb][nt][1] = movmatrix_t(Elt<T>::pack2(p2 - f23.x, p3 - f23.y));
                     }
                 }
-                if (__any_sync(0xffffffffu, rescale)) {
+                lrun[nt][0] = lrun[nt][0] * al[nt][0] + l0;
+                lrun[nt][1] = lrun[nt][1] * al[nt][1] + l1;
+            }
+            if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll
-                    for (int nt = 0; nt < NT; ++nt)
+                for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-                        for (int i = 0; i < KS; ++i) {
-                            o[nt][i][0] *= al[nt][0];
-                            o[nt][i][1] *= al[nt][1];
-                            o[nt][i][2] *= al[nt][0];
-                            o[nt][i][3] *= al[nt][1];
-                        }
-                }
+                    for (int i = 0; i < KS; ++i) {
+                        o[nt][i][0] *= al[nt][0];
+                        o[nt][i][1] *= al[nt][1];
+                        o[nt][i][2] *= al[nt][0];
+                        o[nt][i][3] *= al[nt][1];
+                    }
+            }
 
-                // ---- O^T[D x 8*NT] += V^T P^T
+            // ---- O^T[D x 8*NT] += V^T P^T
 #pragma unroll
-                for (int i = 0; i < KS; ++i) {
+            for (int i = 0; i < KS; ++i) {
+#pragma unroll
+                for (int bb = 0; bb < NB; ++bb) {
                     uint32_t a[4];
-                    ldsm_x4_t(tbase + voff[i], a[0], a[1], a[2], a[3]);
+                    ldsm_x4_t(tb[bb] + voff[i], a[0], a[1], a[2], a[3]);
 #pragma unroll
                     for (int nt = 0; nt < NT; ++nt) {
-                        Mma<T>::run(o[nt][i], a, pb[nt][0], pb[nt][1]);
-                        if constexpr (kSplitP) Mma<T>::run(o[nt][i], a, pl[nt][0], pl[nt][1]);
+                        Mma<T>::run(o[nt][i], a, pb[bb][nt][0], pb[bb][nt][1]);
+                        if constexpr (kSplitP) Mma<T>::run(o[nt][i], a, pl[bb][nt][0], pl[bb][nt][1]);
                     }
                 }
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[s]);
+        };
+        auto tile_of = [&](uint32_t n) { return smem_u32(stages + (n % STAGES) * C::kStageBytes); };
+        auto valid_of = [&](uint32_t n) { return min(kBlockSize, m.ctx - (m.j0 + (int)(n - stage_base)) * kBlockSize); };
+        auto wait_full = [&](uint32_t n) {
+            if (!__all_sync(0xffffffffu, mbar_wait(&full[n % STAGES], (n / STAGES) & 1)) || *abort_flag) {
+                *abort_flag = 1;
+                return false;
+            }
+            return true;
+        };
+        // A single consumer warp takes the item's blocks two at a time, which
+        // halves the dependent latency per block (the warp has no other warp
+        // to hide it behind); with several consumer warps, block j goes to
+        // warp j % NCW one at a time.  (Two n-tiles of heads leave no
+        // registers for pairs.)
+        constexpr bool kPairs = NCW == 1 && NT == 1;
+        uint32_t n = stage_base + (uint32_t)cw;
+        while (n < item_end) {
+            if (kPairs && n + 1 < item_end) {
+                if (!wait_full(n) || !wait_full(n + 1)) break;
+                const bool bad0 = stage_bad[n % STAGES] != 0, bad1 = stage_bad[(n + 1) % STAGES] != 0;
+                const uint32_t tb[2] = {tile_of(n), tile_of(n + 1)};
+                const int vl[2] = {valid_of(n), valid_of(n + 1)};
+                if (!bad0 && !bad1) {
+                    step(std::integral_constant<int, 2>{}, tb, vl);
+                } else {   // a block the producer skipped (bad id) holds no data
+                    if (!bad0) step(std::integral_constant<int, 1>{}, tb, vl);
+                    if (!bad1) step(std::integral_constant<int, 1>{}, tb + 1, vl + 1);
+                }
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(&empty[n % STAGES]);
+                    mbar_arrive(&empty[(n + 1) % STAGES]);
+                }
+                n += 2;
+            } else {
+                if (!wait_full(n)) break;
+                if (!stage_bad[n % STAGES]) {
+                    const uint32_t tb[1] = {tile_of(n)};
+                    const int vl[1] = {valid_of(n)};
+                    step(std::integral_constant<int, 1>{}, tb, vl);
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[n % STAGES]);
+                n += NCW;
+            }
         }
         stage_base = item_end;
         if (*abort_flag) break;
