@@ -39,19 +39,31 @@ METRIC = "paged decode attention: achieved KV-read HBM GB/s (% of peak), seq/s"
 FALLBACK_HBM_GBS = 6650.0
 
 
-def profiled_traffic(workload: str):
-    """DRAM bytes per launch of the partition kernel from the committed ncu capture.
+def kernel_source_hash() -> str:
+    """Hash of the device code the profiles were taken on.
 
-    profiles/traffic.json records the capture together with a hash of the
-    decode source it was taken on; a changed kernel gets null, not a stale number.
+    The device part of csrc/decode.cu (up to its host-side section) and
+    csrc/pa_common.cuh: host-side launch choices do not change the kernels.
     """
     import hashlib
 
+    csrc = os.path.join(ROOT, "paged_kv_cache_362_b200", "csrc")
+    dec = open(os.path.join(csrc, "decode.cu"), "rb").read()
+    dec = dec.split(b"\n// host side\n")[0]
+    common = open(os.path.join(csrc, "pa_common.cuh"), "rb").read()
+    return hashlib.sha256(dec + common).hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per launch of the attention kernel from the committed ncu capture.
+
+    profiles/traffic.json records the capture together with a hash of the
+    device code it was taken on; a changed kernel gets null, not a stale number.
+    """
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
             t = json.load(f)
-        src = open(os.path.join(ROOT, t["source"]), "rb").read()
-        if hashlib.sha256(src).hexdigest()[:16] != t["source_sha256_16"]:
+        if kernel_source_hash() != t["source_sha256_16"]:
             return None
         return t[workload]["decode_tc_kernel_bytes"]
     except Exception:

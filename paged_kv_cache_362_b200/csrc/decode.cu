@@ -17,7 +17,7 @@
 //                own items of the list from context_lens (no launch); a
 //                one-CTA plan kernel writes the whole list for larger
 //                batches, for many items per CTA and for the SIMT kernel.
-//  2. partition kernel -- persistent CTAs (2 or 4 per SM).  CTA c takes items
+//  2. partition kernel -- persistent CTAs (4 per SM).  CTA c takes items
 //                c, 2C-1-c, 2C+c, ... (snake order over the sorted list, which
 //                balances the load).  Per CTA:
 //                  * a producer warp streams, for each item, the Q rows of the
@@ -27,7 +27,7 @@
 //                    shared-memory stages, 128-byte swizzled, tracked by
 //                    mbarriers, evict-first in L2; work-list entries and table
 //                    rows are prefetched two items ahead with cp.async;
-//                  * consumer warps run each block on tensor cores:
+//                  * consumer warps run two blocks per step on tensor cores:
 //                    S^T = K Q^T (m16n8k16, tokens x heads, the GQA group padded
 //                    to 8 or 16 columns), an online softmax in fp32 (column max
 //                    by warp shuffles, 2^x on log2-scaled logits), then
@@ -40,9 +40,9 @@
 //                    in the workspace says which -- hands it to a merger warp
 //                    that combines all partitions (when there are at most 8)
 //                    and resets the counter, so no reduce kernel runs;
-//                  * with two consumer warps, block j goes to warp j % 2 and
-//                    the warps' states are merged through a double-buffered
-//                    shared-memory slot by a rotating merger warp.
+//                  * (tuning shape) with two consumer warps, block j goes to
+//                    warp j % 2 and the warps' states are merged through a
+//                    double-buffered shared-memory slot by a rotating merger.
 //                A SIMT variant serves float32 and groups above 16.
 //  3. reduce  -- (sequences over 8 partitions, or two-warp CTAs) rows of the
 //                multi-partition sequences: M = max m_p, L = sum l_p 2^(m_p - M),
@@ -231,25 +231,30 @@ __device__ __forceinline__ ItemGeom item_geom(const DecodeParams& p, int4 it) {
 // ===========================================================================
 // 2a. partition kernel, tensor cores (fp16 / bf16)
 // ===========================================================================
-// Fused merge (single-warp CTAs, at most kFusedMaxParts partitions): one warp
-// combines every partition of (sequence b, KV head g) for the G query heads of
-// the group, out = sum_p O_p 2^(m_p - M) / sum_p l_p 2^(m_p - M).  The
+// Fused merge (single-warp CTAs, at most kFusedMaxParts = 8 partitions): one
+// warp combines every partition of (sequence b, KV head g) for the G query
+// heads of the group, out = sum_p O_p 2^(m_p - M) / sum_p l_p 2^(m_p - M).  The
 // partials were written by other CTAs: cache-global loads.  Round trips: one
-// for every (head, partition)'s m and l, then one per pair of heads for O.
+// for every (head, partition)'s m and l, then one per two or four heads for O.
+// (Sixteen partitions per warp were measured slower than the reduce kernel.)
 constexpr int kFusedMaxParts = 8;
 
-template <typename T, int D>
+template <typename T, int D, int GMAX>
 __device__ __forceinline__ void merge_group(const DecodeParams& p, int b, int g, int nparts, int lane,
                                             float* s_w, float* s_inv) {
     constexpr int E = D / 32;
     constexpr int MP = kFusedMaxParts;
+    constexpr int kSlots = GMAX * MP / 32;
+    // heads whose partial rows are in flight together (4 fits the register
+    // budget of the D = 128, 8-head shape without raising it; 2 elsewhere)
+    constexpr int HP = (D == 128 && GMAX == 8) ? 4 : 2;
     using VecE = typename std::conditional<E == 4, float4, float2>::type;
     const int G = p.group;
     const size_t hq0 = (size_t)b * p.num_heads + (size_t)g * G;
-    // (m, l) of entry e = h * MP + q, lane e % 32 slot e / 32; G <= 16 -> at most 4 slots
-    float mv[4], lv[4];
+    // (m, l) of entry e = h * MP + q: lane e % 32, slot e / 32
+    float mv[kSlots], lv[kSlots];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
+    for (int k = 0; k < kSlots; ++k) {
         const int e = lane + 32 * k, h = e / MP, q = e % MP;
         const bool ok = h < G && q < nparts;
         const size_t pi = (hq0 + h) * p.max_parts + q;
@@ -257,7 +262,7 @@ __device__ __forceinline__ void merge_group(const DecodeParams& p, int b, int g,
         lv[k] = ok ? __ldcg(p.part_l + pi) : 0.f;
     }
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
+    for (int k = 0; k < kSlots; ++k) {
         // the MP lanes of one head are consecutive: reduce over them
         float M = mv[k];
 #pragma unroll
@@ -274,18 +279,19 @@ __device__ __forceinline__ void merge_group(const DecodeParams& p, int b, int g,
         }
     }
     __syncwarp();
+    // out = sum_q w_q O_q / L, lane l owning dims [l*E, l*E + E)
     T* out = static_cast<T*>(p.out);
-    for (int h0 = 0; h0 < G; h0 += 2) {
-        VecE v[2][MP];
+    for (int h0 = 0; h0 < G; h0 += HP) {
+        VecE v[HP][MP];
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh)
+        for (int hh = 0; hh < HP; ++hh)
 #pragma unroll
             for (int q = 0; q < MP; ++q)
                 if (h0 + hh < G && q < nparts)
                     v[hh][q] = __ldcg(reinterpret_cast<const VecE*>(p.part_o + ((hq0 + h0 + hh) * p.max_parts + q) * D +
                                                                     lane * E));
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
+        for (int hh = 0; hh < HP; ++hh) {
             const int h = h0 + hh;
             if (h >= G) break;
             float acc[E];
@@ -442,7 +448,8 @@ struct TcCfg {
     static constexpr int kOffMeta = kOffDesc + kDSlots * (int)sizeof(DescSlot);
     static constexpr int kQSlots = NCW == 1 ? 4 : 0;          // merge-task queue (single-warp CTAs)
     static constexpr int kOffTasks = kOffMeta + kISlots * (int)sizeof(ItemMeta);
-    static constexpr int kMergeW = NCW == 1 ? 128 + 16 : 0;   // merger's partition weights and 1/L
+    // merger's partition weights (heads x kFusedMaxParts) and 1/L (heads)
+    static constexpr int kMergeW = NCW == 1 ? kHeadsPad * kFusedMaxParts + kHeadsPad : 0;
     static constexpr int kOffMW = kOffTasks + kQSlots * 16;
     static constexpr int kMaxOwn = 64;                       // items a self-planning CTA can hold
     static constexpr int kOffOwn = kOffMW + kMergeW * 4;
@@ -560,7 +567,8 @@ __global__ void __launch_bounds__(TcCfg<D, NT, NCW, STAGES>::kThreads, TcCfg<D, 
                 if (task.x < 0) break;
                 __threadfence();
                 float* s_w = reinterpret_cast<float*>(smem + C::kOffMW);
-                merge_group<T, D>(p, task.x, task.y, task.z, lane, s_w, s_w + 128);
+                merge_group<T, D, C::kHeadsPad>(p, task.x, task.y, task.z, lane, s_w,
+                                                s_w + C::kHeadsPad * kFusedMaxParts);
                 // every partition has arrived: the counter is free, leave it zeroed for the next call
                 if (lane == 0) p.merge_count[(size_t)task.x * p.num_kv_heads + task.y] = 0;
             }
@@ -944,19 +952,19 @@ __global__ void __launch_bounds__(TcCfg<D, NT, NCW, STAGES>::kThreads, TcCfg<D, 
             }
             return true;
         };
-        // A single consumer warp takes the item's blocks two at a time, which
-        // halves the dependent latency per block (the warp has no other warp
-        // to hide it behind); with several consumer warps, block j goes to
-        // warp j % NCW one at a time.  (Two n-tiles of heads leave no
-        // registers for pairs.)
-        constexpr bool kPairs = NCW == 1 && NT == 1;
+        // Block j belongs to warp j % NCW, which takes its blocks two at a
+        // time (j and j + NCW): that interleaves two blocks' dependent chains,
+        // which the warp has no other warp to hide behind.  (Two n-tiles of
+        // heads leave no registers for pairs.)
+        constexpr bool kPairs = NT == 1;
         uint32_t n = stage_base + (uint32_t)cw;
         while (n < item_end) {
-            if (kPairs && n + 1 < item_end) {
-                if (!wait_full(n) || !wait_full(n + 1)) break;
-                const bool bad0 = stage_bad[n % STAGES] != 0, bad1 = stage_bad[(n + 1) % STAGES] != 0;
-                const uint32_t tb[2] = {tile_of(n), tile_of(n + 1)};
-                const int vl[2] = {valid_of(n), valid_of(n + 1)};
+            if (kPairs && n + NCW < item_end) {
+                const uint32_t n1 = n + NCW;
+                if (!wait_full(n) || !wait_full(n1)) break;
+                const bool bad0 = stage_bad[n % STAGES] != 0, bad1 = stage_bad[n1 % STAGES] != 0;
+                const uint32_t tb[2] = {tile_of(n), tile_of(n1)};
+                const int vl[2] = {valid_of(n), valid_of(n1)};
                 if (!bad0 && !bad1) {
                     step(std::integral_constant<int, 2>{}, tb, vl);
                 } else {   // a block the producer skipped (bad id) holds no data
@@ -966,9 +974,9 @@ __global__ void __launch_bounds__(TcCfg<D, NT, NCW, STAGES>::kThreads, TcCfg<D, 
                 __syncwarp();
                 if (lane == 0) {
                     mbar_arrive(&empty[n % STAGES]);
-                    mbar_arrive(&empty[(n + 1) % STAGES]);
+                    mbar_arrive(&empty[n1 % STAGES]);
                 }
-                n += 2;
+                n += 2 * NCW;
             } else {
                 if (!wait_full(n)) break;
                 if (!stage_bad[n % STAGES]) {
@@ -1292,9 +1300,10 @@ namespace {
 //   kTriple: 1 x 8  (64 KB ring), 3 CTAs per SM
 //   kPair1:  1 x 13 (104 KB ring), 2 CTAs per SM
 // The ring holds the bytes in flight that cover HBM latency; each consumer
-// warp holds one stage while it computes.  PA_TC_SHAPE selects one (tuning).
+// warp holds two stages while it computes.  kQuad is the automatic choice
+// (measured best on every workload once consumers took two blocks per step);
+// PA_TC_SHAPE selects another (tuning).
 enum class TcShape { kAuto, kPaired, kQuad, kTriple, kPair1 };
-constexpr int kPairedMinParts = 32;
 TcShape tc_shape() {
     static const TcShape s = [] {
         const char* e = getenv("PA_TC_SHAPE");
@@ -1418,11 +1427,9 @@ cudaError_t choose(const DecodeParams& p, pa_dtype dtype, DecodeChoice* c) {
         if (decode_path(dtype, D, p.group) == DecodePath::kTensorCore) {
             c->tc = true;
             TcShape sh = tc_shape();
-            // Automatic: sequences split into many (> 32) partitions stream best with
-            // two 2-warp CTAs per SM (measured on 32k contexts); otherwise four
-            // single-warp CTAs per SM, which merge partitions themselves when there
-            // are at most kFusedMaxParts of them.
-            if (sh == TcShape::kAuto) sh = p.max_parts > kPairedMinParts ? TcShape::kPaired : TcShape::kQuad;
+            // Automatic: four single-warp CTAs per SM, which merge partitions
+            // themselves when there are at most kFusedMaxParts of them.
+            if (sh == TcShape::kAuto) sh = TcShape::kQuad;
             c->shape = sh;
             const bool one_warp = p.group > 8 || sh != TcShape::kPaired;
             c->fused = one_warp && p.max_parts > 1 && p.max_parts <= kFusedMaxParts;
