@@ -207,7 +207,7 @@ class ClockSampler:
 # workload on the device
 # ---------------------------------------------------------------------------
 class DeviceWorkload:
-    def __init__(self, name: str, seed: int, partition_size: int | None = None):
+    def __init__(self, name: str, seed: int, partition_size: int | None = None, placement: str | None = None):
         import torch
 
         import paged_kv_cache_362_b200 as pa
@@ -215,7 +215,7 @@ class DeviceWorkload:
 
         self.pa = pa
         self.cfg = get_config(name)
-        self.wl = build_workload(self.cfg, seed=seed)
+        self.wl = build_workload(self.cfg, seed=seed, placement=placement)
         self.P = self.cfg.partition_size if partition_size is None else partition_size
         dev = torch.device("cuda")
         v = device_values(self.wl, dev)
@@ -247,6 +247,23 @@ class DeviceWorkload:
         c = self.cfg
         self.pa.decode(self.out, self.q, self.kc, self.vc, self.bt, self.cl, c.scale, self.max_ctx, self.ws,
                        partition_size=self.P, status=self.status)
+
+
+def unique_kv_bytes(wl) -> int:
+    """K/V bytes of the distinct physical blocks a decode step reads (shared blocks once)."""
+    c = wl.cfg
+    seen = {}
+    for b in range(wl.num_seqs):
+        n = int(wl.context_lens[b])
+        for j in range(-(-n // 16)):
+            blk = int(wl.block_tables[b, j])
+            seen[blk] = max(seen.get(blk, 0), min(16, n - 16 * j))
+    elt = {"f32": 4, "f16": 2, "bf16": 2}[c.dtype]
+    return sum(seen.values()) * c.num_kv_heads * c.head_dim * 2 * elt
+
+
+def pct3(xs):
+    return [round(float(v), 5) for v in np.percentile(np.asarray(xs), [10, 50, 90])]
 
 
 def time_steps(w: DeviceWorkload, steps: int, warmup: int, flush, use_graph: bool):
@@ -367,10 +384,20 @@ def _oracle_run(cfg, sub, v, threads):
                     cfg.dtype, cfg.num_kv_heads, num_threads=threads)
 
 
-def oracle_sample_throughput(name: str, seed: int, budget_s: float, max_seqs: int):
+def cpu_model() -> str:
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def oracle_sample_throughput(name: str, seed: int, budget_s: float, max_seqs: int, threads: int | None = None):
     """fp64 C oracle on a bounded sample of the workload: (KV GB/s, seq/s, threads, sample text)."""
     cfg, sub, v, total = _oracle_subproblem(name, seed, max_seqs, seed + 7)
-    threads = os.cpu_count() or 1
+    threads = threads or os.cpu_count() or 1
     reps, t0 = 0, time.perf_counter()
     while True:
         _oracle_run(cfg, sub, v, threads)
@@ -380,7 +407,7 @@ def oracle_sample_throughput(name: str, seed: int, budget_s: float, max_seqs: in
             break
     per = el / reps
     sample = (f"{sub.num_seqs} of {total} sequences of {name} (seed {seed}), {reps} run(s), "
-              f"fp64 C oracle with OpenMP")
+              f"fp64 C oracle with OpenMP on {threads} thread(s)")
     return sub.kv_bytes() / per / 1e9, sub.num_seqs / per, threads, sample, per
 
 
@@ -474,6 +501,7 @@ def main():
     e2e = dist_max(float(np.mean(e2e_ms)))
 
     secondary = {}
+    placement = {}
     if not args.no_secondary:
         for name in ("long32k", "qwen_layer", "shared_prefix"):
             if name == args.workload:
@@ -482,7 +510,12 @@ def main():
             s_step, s_dec = time_steps(sw, max(50, args.steps // 10), args.warmup, flush, use_graph)
             sd = dist_max(float(np.mean(s_dec)))
             ss = dist_max(float(np.mean(s_step)))
-            secondary[name] = {
+            if name == "shared_prefix":
+                ub = unique_kv_bytes(sw.wl)
+                unique_note = {"unique_kv_bytes": ub, "decode_unique_gbs": round(ub / (sd * 1e-3) / 1e9, 1)}
+            else:
+                unique_note = {}
+            secondary[name] = {"decode_ms_p10_p50_p90": pct3(s_dec), **unique_note,
                 "decode_ms": round(sd, 5), "step_ms": round(ss, 5),
                 "decode_kv_gbs": round(sw.kv_bytes / (sd * 1e-3) / 1e9, 1),
                 "decode_frac_of_peak": round(sw.kv_bytes / (sd * 1e-3) / 1e9 / peak, 4),
@@ -491,12 +524,27 @@ def main():
             }
             del sw
             torch.cuda.empty_cache()
+        # cost of scattered blocks: the same sequences with contiguous (identity) placement
+        for name in ("churned256", "long32k"):
+            res = {}
+            for pl in (None, "identity"):
+                pw = DeviceWorkload(name, args.seed + rank, placement=pl)
+                _, p_dec = time_steps(pw, max(50, args.steps // 10), args.warmup, flush, use_graph)
+                res[pl or pw.cfg.placement] = dist_max(float(np.mean(p_dec)))
+                del pw
+                torch.cuda.empty_cache()
+            (shuf, ms_s), (_, ms_i) = list(res.items())
+            placement[name] = {f"decode_ms_{shuf}": round(ms_s, 5), "decode_ms_identity": round(ms_i, 5),
+                               "overhead_pct": round(100 * (ms_s / ms_i - 1), 2)}
 
     cpu = None
     if rank == 0 and world == 1:
         gbs, sps, threads, sample, _ = oracle_sample_throughput(args.workload, args.seed, args.cpu_budget,
                                                                 args.cpu_seqs)
-        cpu = {"value": round(gbs, 4), "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": sample}
+        gbs1, _, _, sample1, _ = oracle_sample_throughput(args.workload, args.seed, args.cpu_budget / 4,
+                                                          max(1, args.cpu_seqs // 8), threads=1)
+        cpu = {"value": round(gbs, 4), "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": sample,
+               "value_1_thread": round(gbs1, 4), "sample_1_thread": sample1, "cpu_model": cpu_model()}
 
     if rank == 0:
         c = w.cfg
@@ -524,6 +572,8 @@ def main():
             "cpu_baseline": cpu,
             "e2e": {"value": round(total_bytes / (e2e * 1e-3) / 1e9, 2), "unit": "GB/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e, 5)},
+            "step_ms_p10_p50_p90": pct3(step_ms), "decode_ms_p10_p50_p90": pct3(dec_ms),
+            "placement_overhead": placement,
             "gpu_launches": w.launches_per_step * args.steps,
             "clocks": clk,
             "secondary": secondary,

@@ -468,6 +468,9 @@ struct TcCfg {
     static constexpr int kMinBlocks = (NCW == 2 || NT == 2 || STAGES >= 13) ? 2 : (STAGES >= 8 ? 3 : 4);
     static_assert(kOffDesc % 16 == 0 && sizeof(DescSlot) % 16 == 0, "cp.async 16-byte destinations");
     static_assert(kOffOwn % 16 == 0, "own-item list alignment");
+    // the shared memory a shape is sized for: kMinBlocks CTAs per SM (228 KB,
+    // 1 KB reserved per CTA)
+    static_assert(kMinBlocks * (kSmemBytes + 1024) <= 228 * 1024 || D != 128, "shape no longer fits its CTAs per SM");
     // Ring stage n and stage n + STAGES reuse one slot and one parity bit, so a
     // consumer may only wait for stage n once stage n - STAGES has landed, or it
     // would take the old phase for the new one.  Stage n is consumed by warp
