@@ -384,6 +384,42 @@ def _oracle_run(cfg, sub, v, threads):
                     cfg.dtype, cfg.num_kv_heads, num_threads=threads)
 
 
+def block_manager_step(name: str, seed: int, steps: int = 200):
+    """Host time of the block manager's part of a decode step for the workload's batch.
+
+    The workload's sequences are added to a C++ block manager (pa_block_manager.h)
+    with their context lengths; a quarter of them are then forked (shared
+    prefixes), and each step appends one token to every sequence and reads the
+    block tables for pa_decode.  Returns a dict for the JSON line.
+    """
+    import paged_kv_cache_362_b200 as pa
+    from workloads import build_workload, get_config
+
+    cfg = get_config(name)
+    wl = build_workload(cfg, seed=seed)
+    nseq = wl.num_seqs
+    ctx = wl.context_lens.astype(int)
+    need = int(sum(-(-c // 16) + (steps + 15) // 16 + 1 for c in ctx)) * 2
+    bm = pa.BlockManager(need, 16)
+    for i, c in enumerate(ctx):
+        bm.add_sequence(i, int(c))
+    forks = list(range(nseq, nseq + nseq // 4))
+    for j, child in enumerate(forks):
+        bm.fork(j, child)
+    ids = np.arange(nseq + len(forks), dtype=np.int64)
+    mb = -(-(int(ctx.max()) + steps + 16) // 16)
+    copies = 0
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        _, pairs = bm.append_tokens(ids)
+        copies += len(pairs)
+        bm.block_tables(ids, mb)
+    per = (time.perf_counter() - t0) / steps
+    return {"workload": name, "sequences": int(ids.size), "forked": len(forks), "steps": steps,
+            "us_per_step": round(per * 1e6, 1), "copy_pairs_total": copies,
+            "what": "append one token per sequence (slot mapping, copy-on-write pairs) + block tables, host C++"}
+
+
 def cpu_model() -> str:
     try:
         for line in open("/proc/cpuinfo"):
@@ -546,6 +582,8 @@ def main():
         cpu = {"value": round(gbs, 4), "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": sample,
                "value_1_thread": round(gbs1, 4), "sample_1_thread": sample1, "cpu_model": cpu_model()}
 
+    bm_step = block_manager_step(args.workload, args.seed) if rank == 0 else None
+
     if rank == 0:
         c = w.cfg
         line = {
@@ -574,6 +612,7 @@ def main():
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e, 5)},
             "step_ms_p10_p50_p90": pct3(step_ms), "decode_ms_p10_p50_p90": pct3(dec_ms),
             "placement_overhead": placement,
+            "block_manager": bm_step,
             "gpu_launches": w.launches_per_step * args.steps,
             "clocks": clk,
             "secondary": secondary,

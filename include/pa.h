@@ -60,7 +60,8 @@ typedef enum {
     PA_ERR_UNSUPPORTED = 2,   /* valid but not implemented: block_size != 16, head_dim, dtype */
     PA_ERR_OUT_OF_RANGE = 4,  /* device: block id, slot or context length outside its range */
     PA_ERR_CUDA = 8,          /* a CUDA launch or query failed */
-    PA_ERR_TIMEOUT = 16       /* device: a bounded wait inside a kernel gave up */
+    PA_ERR_TIMEOUT = 16,      /* device: a bounded wait inside a kernel gave up */
+    PA_ERR_NO_BLOCKS = 32     /* block manager (pa_block_manager.h): not enough free blocks */
 } pa_status;
 
 typedef enum { PA_F32 = 0, PA_F16 = 1, PA_BF16 = 2 } pa_dtype;

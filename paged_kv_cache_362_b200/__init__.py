@@ -10,10 +10,12 @@ from ._lib import (  # noqa: F401
     LIB_PATH,
     PA_ERR_CUDA,
     PA_ERR_INVALID_ARG,
+    PA_ERR_NO_BLOCKS,
     PA_ERR_OUT_OF_RANGE,
     PA_ERR_TIMEOUT,
     PA_ERR_UNSUPPORTED,
     PA_OK,
+    BlockManager,
     PagedAttentionError,
     check_copy_pairs,
     copy_blocks,

@@ -21,6 +21,7 @@ PA_ERR_UNSUPPORTED = 2
 PA_ERR_OUT_OF_RANGE = 4
 PA_ERR_CUDA = 8
 PA_ERR_TIMEOUT = 16
+PA_ERR_NO_BLOCKS = 32
 
 PA_F32, PA_F16, PA_BF16 = 0, 1, 2
 BLOCK_SIZE = 16
@@ -37,7 +38,7 @@ def _load() -> ctypes.CDLL:
         raise ImportError(f"{LIB_PATH} is not built; run `python paged_kv_cache_362_b200/build.py`")
     lib = ctypes.CDLL(LIB_PATH)
     for sym in ("pa_reshape_and_cache", "pa_decode_workspace_size", "pa_decode", "pa_decode_launch_count",
-                "pa_copy_blocks", "pa_get_error_string", "pa_version"):
+                "pa_copy_blocks", "pa_get_error_string", "pa_version", "pa_bm_create", "pa_bm_append_tokens"):
         if not hasattr(lib, sym):
             raise ImportError(f"{LIB_PATH} lacks {sym} (stale build); run `python paged_kv_cache_362_b200/build.py`")
     p, i32, i64, f32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
@@ -52,6 +53,30 @@ def _load() -> ctypes.CDLL:
     lib.pa_decode_launch_count.restype = i32
     lib.pa_copy_blocks.argtypes = [p, p, p, i32, i32, i32, i32, i32, ctypes.c_int, p, p]
     lib.pa_copy_blocks.restype = ctypes.c_int
+    # host block manager (pa_block_manager.h)
+    lib.pa_bm_create.argtypes = [i32, i32]
+    lib.pa_bm_create.restype = p
+    lib.pa_bm_destroy.argtypes = [p]
+    lib.pa_bm_destroy.restype = None
+    for fn in ("pa_bm_num_blocks", "pa_bm_num_free_blocks", "pa_bm_num_sequences"):
+        getattr(lib, fn).argtypes = [p]
+        getattr(lib, fn).restype = i32
+    lib.pa_bm_ref_count.argtypes = [p, i32]
+    lib.pa_bm_ref_count.restype = i32
+    lib.pa_bm_add_sequence.argtypes = [p, i64, i32, p]
+    lib.pa_bm_add_sequence.restype = ctypes.c_int
+    lib.pa_bm_fork.argtypes = [p, i64, i64]
+    lib.pa_bm_fork.restype = ctypes.c_int
+    lib.pa_bm_append_tokens.argtypes = [p, p, i32, p, p, p]
+    lib.pa_bm_append_tokens.restype = ctypes.c_int
+    lib.pa_bm_free_sequence.argtypes = [p, i64]
+    lib.pa_bm_free_sequence.restype = ctypes.c_int
+    lib.pa_bm_block_tables.argtypes = [p, p, i32, i32, p, p]
+    lib.pa_bm_block_tables.restype = ctypes.c_int
+    lib.pa_bm_sequence_blocks.argtypes = [p, i64]
+    lib.pa_bm_sequence_blocks.restype = i32
+    lib.pa_bm_sequence_length.argtypes = [p, i64]
+    lib.pa_bm_sequence_length.restype = i64
     lib.pa_get_error_string.argtypes = [ctypes.c_int]
     lib.pa_get_error_string.restype = ctypes.c_char_p
     lib.pa_version.argtypes = []
@@ -177,3 +202,86 @@ def check_copy_pairs(pairs_host, num_blocks: int) -> None:
         raise ValueError("a destination block repeats")
     if np.isin(dst, pr[:, 0]).any():
         raise ValueError("a destination block is also a source")
+
+
+class BlockManager:
+    """Host block manager (pa_block_manager.h): allocation, sharing, copy-on-write, slot mappings.
+
+    Arrays in and out are NumPy (host); ``append_tokens`` returns the slot
+    mapping for pa_reshape_and_cache and the copy pairs for pa_copy_blocks.
+    """
+
+    def __init__(self, num_blocks: int, block_size: int = BLOCK_SIZE):
+        self._h = LIB.pa_bm_create(num_blocks, block_size)
+        if not self._h:
+            raise PagedAttentionError(PA_ERR_INVALID_ARG, "pa_bm_create")
+        self.block_size = block_size
+
+    def close(self):
+        if self._h:
+            LIB.pa_bm_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        self.close()
+
+    @property
+    def num_blocks(self) -> int:
+        return int(LIB.pa_bm_num_blocks(self._h))
+
+    @property
+    def num_free_blocks(self) -> int:
+        return int(LIB.pa_bm_num_free_blocks(self._h))
+
+    @property
+    def num_sequences(self) -> int:
+        return int(LIB.pa_bm_num_sequences(self._h))
+
+    def ref_count(self, block: int) -> int:
+        return int(LIB.pa_bm_ref_count(self._h, block))
+
+    def sequence_blocks(self, seq_id: int) -> int:
+        return int(LIB.pa_bm_sequence_blocks(self._h, seq_id))
+
+    def sequence_length(self, seq_id: int) -> int:
+        return int(LIB.pa_bm_sequence_length(self._h, seq_id))
+
+    def add_sequence(self, seq_id: int, num_tokens: int):
+        import numpy as np
+
+        slots = np.empty(num_tokens, dtype=np.int64)
+        _check(LIB.pa_bm_add_sequence(self._h, seq_id, num_tokens, slots.ctypes.data if num_tokens else None),
+               "pa_bm_add_sequence")
+        return slots
+
+    def fork(self, parent_id: int, child_id: int) -> None:
+        _check(LIB.pa_bm_fork(self._h, parent_id, child_id), "pa_bm_fork")
+
+    def append_tokens(self, seq_ids):
+        """(slot_mapping int64 [n], copy_pairs int64 [k, 2]) for one new token per listed sequence."""
+        import numpy as np
+
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        n = ids.shape[0]
+        slots = np.empty(n, dtype=np.int64)
+        pairs = np.empty((max(n, 1), 2), dtype=np.int64)
+        k = ctypes.c_int32(0)
+        _check(LIB.pa_bm_append_tokens(self._h, ids.ctypes.data, n, slots.ctypes.data, pairs.ctypes.data,
+                                       ctypes.byref(k)), "pa_bm_append_tokens")
+        return slots, pairs[:k.value].copy()
+
+    def free_sequence(self, seq_id: int) -> None:
+        _check(LIB.pa_bm_free_sequence(self._h, seq_id), "pa_bm_free_sequence")
+
+    def block_tables(self, seq_ids, max_blocks_per_seq: int):
+        """(block_tables int32 [n, max_blocks_per_seq] padded with -1, context_lens int32 [n])."""
+        import numpy as np
+
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        n = ids.shape[0]
+        bt = np.empty((n, max_blocks_per_seq), dtype=np.int32)
+        cl = np.empty(n, dtype=np.int32)
+        _check(LIB.pa_bm_block_tables(self._h, ids.ctypes.data, n, max_blocks_per_seq, bt.ctypes.data,
+                                      cl.ctypes.data), "pa_bm_block_tables")
+        return bt, cl
+

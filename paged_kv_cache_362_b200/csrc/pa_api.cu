@@ -227,6 +227,7 @@ const char* pa_get_error_string(pa_status s) {
     if (v & PA_ERR_OUT_OF_RANGE) return "PA_ERR_OUT_OF_RANGE: block id, slot or context length out of range";
     if (v & PA_ERR_CUDA) return "PA_ERR_CUDA: CUDA launch or query failed";
     if (v & PA_ERR_TIMEOUT) return "PA_ERR_TIMEOUT: bounded wait inside a kernel expired";
+    if (v & PA_ERR_NO_BLOCKS) return "PA_ERR_NO_BLOCKS: not enough free blocks in the pool";
     return "unknown pa_status";
 }
 
