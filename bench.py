@@ -420,6 +420,34 @@ def block_manager_step(name: str, seed: int, steps: int = 200):
             "what": "append one token per sequence (slot mapping, copy-on-write pairs) + block tables, host C++"}
 
 
+def swap_bandwidth(w, nblocks: int = 4096, reps: int = 5):
+    """pa_swap_blocks between the workload's device pools and pinned host pools, both ways (GB/s)."""
+    import torch
+
+    pa = w.pa
+    shape = (nblocks,) + tuple(w.kc.shape[1:])
+    hk = torch.empty(shape, dtype=w.kc.dtype).pin_memory()
+    hv = torch.empty(shape, dtype=w.kc.dtype).pin_memory()
+    rng = np.random.default_rng(3)
+    dev_ids = rng.choice(w.kc.shape[0], size=nblocks, replace=False)
+    out_pairs = torch.from_numpy(np.stack([dev_ids, np.arange(nblocks)], 1).astype(np.int64)).cuda()
+    in_pairs = torch.from_numpy(np.stack([np.arange(nblocks), dev_ids], 1).astype(np.int64)).cuda()
+    nbytes = 2 * hk.numel() * hk.element_size()
+    res = {"blocks": nblocks, "bytes": nbytes}
+    for name, args in (("device_to_host_gbs", (w.kc, w.vc, hk, hv, out_pairs)),
+                       ("host_to_device_gbs", (hk, hv, w.kc, w.vc, in_pairs))):
+        pa.swap_blocks(*args)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            pa.swap_blocks(*args)
+        e1.record()
+        torch.cuda.synchronize()
+        res[name] = round(nbytes * reps / (e0.elapsed_time(e1) * 1e-3) / 1e9, 1)
+    return res
+
+
 def cpu_model() -> str:
     try:
         for line in open("/proc/cpuinfo"):
@@ -583,6 +611,7 @@ def main():
                "value_1_thread": round(gbs1, 4), "sample_1_thread": sample1, "cpu_model": cpu_model()}
 
     bm_step = block_manager_step(args.workload, args.seed) if rank == 0 else None
+    swap = swap_bandwidth(w) if rank == 0 and not args.no_secondary else None
 
     if rank == 0:
         c = w.cfg
@@ -613,6 +642,7 @@ def main():
             "step_ms_p10_p50_p90": pct3(step_ms), "decode_ms_p10_p50_p90": pct3(dec_ms),
             "placement_overhead": placement,
             "block_manager": bm_step,
+            "swap": swap,
             "gpu_launches": w.launches_per_step * args.steps,
             "clocks": clk,
             "secondary": secondary,

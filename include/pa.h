@@ -173,6 +173,31 @@ pa_status pa_copy_blocks(void* key_cache, void* value_cache, const int64_t* bloc
                          pa_stream_t stream);
 
 /*
+ * pa_swap_blocks -- copy whole blocks from one pool to another of the same
+ * shape, for evicting blocks to CPU memory and bringing them back
+ * ("PagedAttention, Visualized", Part 3: the operating-system table, where
+ * swapping to disk corresponds to evicting blocks to CPU memory; an evicted
+ * sequence's shared blocks stay, because others still use them).  The block
+ * manager (pa_block_manager.h) produces the pairs.
+ *
+ * For each pair k < num_pairs with (s, d) = (block_pairs[2k], block_pairs[2k+1]):
+ *     dst_key_cache[d] = src_key_cache[s];  dst_value_cache[d] = src_value_cache[s]
+ * (all num_kv_heads * 16 * head_dim elements; bit-exact).  Either pool may be
+ * pinned host memory that the device addresses directly (cudaHostAlloc or
+ * cudaMallocHost memory, which unified addressing maps at the same pointer):
+ * swapping out is device -> host, swapping in host -> device.  A pair with an
+ * id outside [0, src_num_blocks) or [0, dst_num_blocks) is skipped and sets
+ * PA_ERR_OUT_OF_RANGE.  No dst may repeat.  The source pool must not be
+ * written by other work until the call has completed on `stream`.
+ *
+ *   block_pairs   int64 [num_pairs][2], device-addressable (device or pinned host)
+ */
+pa_status pa_swap_blocks(const void* src_key_cache, const void* src_value_cache, void* dst_key_cache,
+                         void* dst_value_cache, const int64_t* block_pairs, int32_t num_pairs, int32_t src_num_blocks,
+                         int32_t dst_num_blocks, int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                         pa_dtype dtype, int32_t* status, pa_stream_t stream);
+
+/*
  * pa_decode_noalloc -- pa_decode without a caller-allocated workspace.
  *
  * The pages have no counterpart to this call; it exists for callers that

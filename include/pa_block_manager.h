@@ -50,14 +50,17 @@ extern "C" {
 
 typedef struct pa_block_manager pa_block_manager;
 
-/* A pool of num_blocks blocks of block_size tokens (1 .. 1024; the kernels
- * take 16).  Returns NULL for invalid arguments or when memory runs out. */
-pa_block_manager* pa_bm_create(int32_t num_blocks, int32_t block_size);
+/* A pool of num_blocks device blocks of block_size tokens (1 .. 1024; the
+ * kernels take 16) and a pool of num_host_blocks blocks in CPU memory that
+ * swapped-out sequences move to (0: no swapping).  Returns NULL for invalid
+ * arguments or when memory runs out. */
+pa_block_manager* pa_bm_create(int32_t num_blocks, int32_t block_size, int32_t num_host_blocks);
 void pa_bm_destroy(pa_block_manager* bm);
 
 int32_t pa_bm_num_blocks(const pa_block_manager* bm);
 int32_t pa_bm_num_free_blocks(const pa_block_manager* bm);
 int32_t pa_bm_num_sequences(const pa_block_manager* bm);
+int32_t pa_bm_num_free_host_blocks(const pa_block_manager* bm);
 
 /* References to a block (0 = free), or -1 for an id outside the pool. */
 int32_t pa_bm_ref_count(const pa_block_manager* bm, int32_t block);
@@ -94,8 +97,32 @@ pa_status pa_bm_fork(pa_block_manager* bm, int64_t parent_id, int64_t child_id);
 pa_status pa_bm_append_tokens(pa_block_manager* bm, const int64_t* seq_ids, int32_t n, int64_t* slot_mapping,
                               int64_t* copy_pairs, int32_t* num_copy_pairs);
 
-/* pa_bm_free_sequence -- drop the sequence; its blocks lose one reference each. */
+/* pa_bm_free_sequence -- drop the sequence (resident or swapped out); its
+ * device blocks lose one reference each, its host blocks are free again. */
 pa_status pa_bm_free_sequence(pa_block_manager* bm, int64_t seq_id);
+
+/*
+ * pa_bm_swap_out -- evict a resident sequence to the host pool under memory
+ * pressure ("PagedAttention, Visualized", Part 3: swapping to disk is
+ * evicting blocks to CPU memory; shared blocks stay, since others still use
+ * them).  Every block only this sequence references gets a host block and is
+ * freed on the device; shared blocks keep the sequence's reference.  pairs
+ * (int64 [n][2], capacity = the sequence's block count) receives (device
+ * block, host block) for pa_swap_blocks from the device pools to the host
+ * pools; run that copy before the freed device blocks are written again.  A
+ * swapped-out sequence cannot be appended to, forked or decoded.
+ */
+pa_status pa_bm_swap_out(pa_block_manager* bm, int64_t seq_id, int64_t* pairs, int32_t* num_pairs);
+
+/*
+ * pa_bm_swap_in -- bring a swapped-out sequence back: a fresh device block for
+ * each of its host blocks; pairs receives (host block, device block) for
+ * pa_swap_blocks from the host pools to the device pools.
+ */
+pa_status pa_bm_swap_in(pa_block_manager* bm, int64_t seq_id, int64_t* pairs, int32_t* num_pairs);
+
+/* 1 if the sequence is swapped out, 0 if resident, -1 for an unknown id. */
+int32_t pa_bm_is_swapped(const pa_block_manager* bm, int64_t seq_id);
 
 /*
  * pa_bm_block_tables -- the pa_decode inputs for n sequences:

@@ -15,7 +15,10 @@ It follows the pages' description step by step:
     writes into a block others still reference first gets its own copy of it
     (digest, section "Copy-on-write: when two requests share a prefix");
   * a finished request gives its blocks back; a block is free again when no
-    request references it.
+    request references it;
+  * under memory pressure a request is evicted to CPU memory, the OS's
+    swapping; its shared blocks stay, because others still use them
+    ("PagedAttention, Visualized", Part 3).
 
 The pages say nothing about which free block is handed out next.  The reading
 taken (and stated in the library's header): a stack, the most recently freed
@@ -31,13 +34,15 @@ class NoBlocks(Exception):
 
 
 class BlockModel:
-    def __init__(self, num_blocks: int, block_size: int):
+    def __init__(self, num_blocks: int, block_size: int, num_host_blocks: int = 0):
         self.num_blocks = num_blocks
         self.block_size = block_size
         self.refs = [0] * num_blocks
         self.free = list(range(num_blocks - 1, -1, -1))   # the end of the list is handed out next
+        self.host_free = list(range(num_host_blocks - 1, -1, -1))
         self.tables: dict[int, list[int]] = {}
         self.lengths: dict[int, int] = {}
+        self.on_host: dict[int, list[bool]] = {}            # swapped-out requests: which entries are host blocks
 
     # --- pool ---------------------------------------------------------------
     def _take(self) -> int:
@@ -107,8 +112,46 @@ class BlockModel:
     def free_sequence(self, sid: int) -> None:
         table = self.tables.pop(sid)
         del self.lengths[sid]
-        for b in reversed(table):
-            self._release(b)
+        host = self.on_host.pop(sid, [False] * len(table))
+        for b, h in zip(reversed(table), reversed(host)):
+            if h:
+                self.host_free.append(b)
+            else:
+                self._release(b)
+
+    def swap_out(self, sid: int) -> list[tuple[int, int]]:
+        """Evict a request: its private blocks move to host blocks, (device, host) pairs."""
+        assert sid in self.tables and sid not in self.on_host
+        table = self.tables[sid]
+        private = [j for j, b in enumerate(table) if self.refs[b] == 1]
+        if len(private) > len(self.host_free):
+            raise NoBlocks()
+        host = [False] * len(table)
+        pairs = []
+        for j in private:
+            h = self.host_free.pop()
+            pairs.append((table[j], h))
+            self._release(table[j])
+            table[j] = h
+            host[j] = True
+        self.on_host[sid] = host
+        return pairs
+
+    def swap_in(self, sid: int) -> list[tuple[int, int]]:
+        """Bring an evicted request back: a fresh device block per host block, (host, device) pairs."""
+        host = self.on_host[sid]
+        table = self.tables[sid]
+        if sum(host) > len(self.free):
+            raise NoBlocks()
+        pairs = []
+        for j, h in enumerate(host):
+            if h:
+                d = self._take()
+                pairs.append((table[j], d))
+                self.host_free.append(table[j])
+                table[j] = d
+        del self.on_host[sid]
+        return pairs
 
     def block_tables(self, sids: list[int], max_blocks: int) -> tuple[list[list[int]], list[int]]:
         rows = []

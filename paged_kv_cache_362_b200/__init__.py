@@ -25,5 +25,6 @@ from ._lib import (  # noqa: F401
     error_string,
     make_workspace,
     reshape_and_cache,
+    swap_blocks,
     version,
 )

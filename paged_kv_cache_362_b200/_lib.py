@@ -54,11 +54,11 @@ def _load() -> ctypes.CDLL:
     lib.pa_copy_blocks.argtypes = [p, p, p, i32, i32, i32, i32, i32, ctypes.c_int, p, p]
     lib.pa_copy_blocks.restype = ctypes.c_int
     # host block manager (pa_block_manager.h)
-    lib.pa_bm_create.argtypes = [i32, i32]
+    lib.pa_bm_create.argtypes = [i32, i32, i32]
     lib.pa_bm_create.restype = p
     lib.pa_bm_destroy.argtypes = [p]
     lib.pa_bm_destroy.restype = None
-    for fn in ("pa_bm_num_blocks", "pa_bm_num_free_blocks", "pa_bm_num_sequences"):
+    for fn in ("pa_bm_num_blocks", "pa_bm_num_free_blocks", "pa_bm_num_sequences", "pa_bm_num_free_host_blocks"):
         getattr(lib, fn).argtypes = [p]
         getattr(lib, fn).restype = i32
     lib.pa_bm_ref_count.argtypes = [p, i32]
@@ -71,6 +71,13 @@ def _load() -> ctypes.CDLL:
     lib.pa_bm_append_tokens.restype = ctypes.c_int
     lib.pa_bm_free_sequence.argtypes = [p, i64]
     lib.pa_bm_free_sequence.restype = ctypes.c_int
+    for fn in ("pa_bm_swap_out", "pa_bm_swap_in"):
+        getattr(lib, fn).argtypes = [p, i64, p, p]
+        getattr(lib, fn).restype = ctypes.c_int
+    lib.pa_bm_is_swapped.argtypes = [p, i64]
+    lib.pa_bm_is_swapped.restype = i32
+    lib.pa_swap_blocks.argtypes = [p, p, p, p, p, i32, i32, i32, i32, i32, i32, ctypes.c_int, p, p]
+    lib.pa_swap_blocks.restype = ctypes.c_int
     lib.pa_bm_block_tables.argtypes = [p, p, i32, i32, p, p]
     lib.pa_bm_block_tables.restype = ctypes.c_int
     lib.pa_bm_sequence_blocks.argtypes = [p, i64]
@@ -190,6 +197,26 @@ def copy_blocks(key_cache, value_cache, block_pairs, status=None, stream=None):
            "pa_copy_blocks")
 
 
+def swap_blocks(src_key_cache, src_value_cache, dst_key_cache, dst_value_cache, block_pairs, status=None,
+                stream=None):
+    """Whole blocks between two pools (pa_swap_blocks); either side may be pinned host memory.
+
+    block_pairs int64 [N, 2] (src block, dst block), on the device or in pinned host memory.
+    """
+    for t in (src_key_cache, src_value_cache, dst_key_cache, dst_value_cache, block_pairs):
+        assert t.is_contiguous()
+        assert t.is_cuda or t.is_pinned(), "pools and pairs must be device memory or pinned host memory"
+    assert block_pairs.element_size() == 8 and block_pairs.dim() == 2 and block_pairs.shape[1] == 2
+    assert src_key_cache.dtype == dst_key_cache.dtype == src_value_cache.dtype == dst_value_cache.dtype
+    NBs, Hkv, bs, D = src_key_cache.shape
+    NBd = dst_key_cache.shape[0]
+    assert dst_key_cache.shape[1:] == src_key_cache.shape[1:]
+    _check(LIB.pa_swap_blocks(_ptr(src_key_cache), _ptr(src_value_cache), _ptr(dst_key_cache), _ptr(dst_value_cache),
+                              _ptr(block_pairs), block_pairs.shape[0], NBs, NBd, Hkv, D, bs,
+                              _dtype_code(src_key_cache), _ptr(status), _stream(stream)),
+           "pa_swap_blocks")
+
+
 def check_copy_pairs(pairs_host, num_blocks: int) -> None:
     """Host-side validation of copy pairs (ids in range, no repeated dst, no dst that is also a src)."""
     import numpy as np
@@ -211,8 +238,8 @@ class BlockManager:
     mapping for pa_reshape_and_cache and the copy pairs for pa_copy_blocks.
     """
 
-    def __init__(self, num_blocks: int, block_size: int = BLOCK_SIZE):
-        self._h = LIB.pa_bm_create(num_blocks, block_size)
+    def __init__(self, num_blocks: int, block_size: int = BLOCK_SIZE, num_host_blocks: int = 0):
+        self._h = LIB.pa_bm_create(num_blocks, block_size, num_host_blocks)
         if not self._h:
             raise PagedAttentionError(PA_ERR_INVALID_ARG, "pa_bm_create")
         self.block_size = block_size
@@ -236,6 +263,29 @@ class BlockManager:
     @property
     def num_sequences(self) -> int:
         return int(LIB.pa_bm_num_sequences(self._h))
+
+    @property
+    def num_free_host_blocks(self) -> int:
+        return int(LIB.pa_bm_num_free_host_blocks(self._h))
+
+    def is_swapped(self, seq_id: int) -> bool:
+        return int(LIB.pa_bm_is_swapped(self._h, seq_id)) == 1
+
+    def _swap(self, fn, seq_id: int, where: str):
+        import numpy as np
+
+        pairs = np.empty((max(self.sequence_blocks(seq_id), 1), 2), dtype=np.int64)
+        k = ctypes.c_int32(0)
+        _check(fn(self._h, seq_id, pairs.ctypes.data, ctypes.byref(k)), where)
+        return pairs[:k.value].copy()
+
+    def swap_out(self, seq_id: int):
+        """(device block, host block) pairs for swap_blocks(device pools -> host pools)."""
+        return self._swap(LIB.pa_bm_swap_out, seq_id, "pa_bm_swap_out")
+
+    def swap_in(self, seq_id: int):
+        """(host block, device block) pairs for swap_blocks(host pools -> device pools)."""
+        return self._swap(LIB.pa_bm_swap_in, seq_id, "pa_bm_swap_in")
 
     def ref_count(self, block: int) -> int:
         return int(LIB.pa_bm_ref_count(self._h, block))

@@ -19,7 +19,9 @@
 namespace {
 
 struct Sequence {
-    std::vector<int32_t> blocks;  // physical block of each logical block
+    std::vector<int32_t> blocks;  // physical block of each logical block (a host block where on_host)
+    std::vector<uint8_t> on_host; // while swapped out: 1 where the block lives in the host pool
+    bool swapped = false;
     int64_t len = 0;              // tokens
     int64_t pending = 0;          // scratch of pa_bm_append_tokens: tokens of this call counted so far
     int64_t pending_blocks = 0;   // scratch: fresh blocks this call appends to the table
@@ -32,6 +34,8 @@ struct pa_block_manager {
     int32_t block_size = 16;
     std::vector<int32_t> ref;          // references per block (0 = free)
     std::vector<int32_t> free_stack;   // top = back: the next block handed out
+    int32_t num_host_blocks = 0;
+    std::vector<int32_t> host_free;    // the host pool's free blocks, handed out the same way
     std::unordered_map<int64_t, Sequence> seqs;
     // scratch of pa_bm_append_tokens, kept between calls to avoid allocations
     std::vector<Sequence*> batch;      // sequence of each token
@@ -52,8 +56,8 @@ struct pa_block_manager {
 
 extern "C" {
 
-pa_block_manager* pa_bm_create(int32_t num_blocks, int32_t block_size) {
-    if (num_blocks <= 0 || block_size <= 0 || block_size > 1024) return nullptr;
+pa_block_manager* pa_bm_create(int32_t num_blocks, int32_t block_size, int32_t num_host_blocks) {
+    if (num_blocks <= 0 || block_size <= 0 || block_size > 1024 || num_host_blocks < 0) return nullptr;
     if ((int64_t)num_blocks * block_size > INT64_MAX / 2) return nullptr;
     pa_block_manager* bm = new (std::nothrow) pa_block_manager;
     if (!bm) return nullptr;
@@ -64,6 +68,9 @@ pa_block_manager* pa_bm_create(int32_t num_blocks, int32_t block_size) {
         bm->copied.assign(num_blocks, 0);
         bm->free_stack.resize(num_blocks);
         for (int32_t i = 0; i < num_blocks; ++i) bm->free_stack[i] = num_blocks - 1 - i;   // pops 0, 1, 2, ...
+        bm->num_host_blocks = num_host_blocks;
+        bm->host_free.resize(num_host_blocks);
+        for (int32_t i = 0; i < num_host_blocks; ++i) bm->host_free[i] = num_host_blocks - 1 - i;
     } catch (...) {
         delete bm;
         return nullptr;
@@ -76,6 +83,7 @@ void pa_bm_destroy(pa_block_manager* bm) { delete bm; }
 int32_t pa_bm_num_blocks(const pa_block_manager* bm) { return bm ? bm->num_blocks : 0; }
 int32_t pa_bm_num_free_blocks(const pa_block_manager* bm) { return bm ? (int32_t)bm->free_stack.size() : 0; }
 int32_t pa_bm_num_sequences(const pa_block_manager* bm) { return bm ? (int32_t)bm->seqs.size() : 0; }
+int32_t pa_bm_num_free_host_blocks(const pa_block_manager* bm) { return bm ? (int32_t)bm->host_free.size() : 0; }
 
 int32_t pa_bm_ref_count(const pa_block_manager* bm, int32_t block) {
     if (!bm || block < 0 || block >= bm->num_blocks) return -1;
@@ -105,7 +113,7 @@ pa_status pa_bm_add_sequence(pa_block_manager* bm, int64_t seq_id, int32_t num_t
 pa_status pa_bm_fork(pa_block_manager* bm, int64_t parent_id, int64_t child_id) {
     if (!bm) return PA_ERR_INVALID_ARG;
     auto it = bm->seqs.find(parent_id);
-    if (it == bm->seqs.end() || bm->seqs.count(child_id)) return PA_ERR_INVALID_ARG;
+    if (it == bm->seqs.end() || it->second.swapped || bm->seqs.count(child_id)) return PA_ERR_INVALID_ARG;
     try {
         Sequence child = it->second;   // same table: shared blocks
         for (int32_t b : child.blocks) ++bm->ref[b];
@@ -138,7 +146,7 @@ pa_status pa_bm_append_tokens(pa_block_manager* bm, const int64_t* seq_ids, int3
     int32_t k = 0;
     for (; k < n; ++k) {
         auto it = bm->seqs.find(seq_ids[k]);
-        if (it == bm->seqs.end()) {
+        if (it == bm->seqs.end() || it->second.swapped) {
             ok = false;
             break;
         }
@@ -207,9 +215,77 @@ pa_status pa_bm_free_sequence(pa_block_manager* bm, int64_t seq_id) {
     auto it = bm->seqs.find(seq_id);
     if (it == bm->seqs.end()) return PA_ERR_INVALID_ARG;
     // release from the last block back, so the prompt's first block is handed out first again
-    for (auto b = it->second.blocks.rbegin(); b != it->second.blocks.rend(); ++b) bm->drop(*b);
+    const Sequence& sq = it->second;
+    for (size_t j = sq.blocks.size(); j-- > 0;) {
+        if (sq.swapped && sq.on_host[j]) bm->host_free.push_back(sq.blocks[j]);
+        else bm->drop(sq.blocks[j]);
+    }
     bm->seqs.erase(it);
     return PA_OK;
+}
+
+pa_status pa_bm_swap_out(pa_block_manager* bm, int64_t seq_id, int64_t* pairs, int32_t* num_pairs) {
+    if (!bm || !pairs || !num_pairs) return PA_ERR_INVALID_ARG;
+    *num_pairs = 0;
+    auto it = bm->seqs.find(seq_id);
+    if (it == bm->seqs.end() || it->second.swapped) return PA_ERR_INVALID_ARG;
+    Sequence& s = it->second;
+    int64_t need = 0;   // blocks only this sequence holds move; shared ones stay for the others
+    for (int32_t b : s.blocks) need += bm->ref[b] == 1;
+    if (need > (int64_t)bm->host_free.size()) return PA_ERR_NO_BLOCKS;
+    try {
+        s.on_host.assign(s.blocks.size(), 0);
+    } catch (...) {
+        return PA_ERR_INVALID_ARG;
+    }
+    int32_t k = 0;
+    for (size_t j = 0; j < s.blocks.size(); ++j) {
+        const int32_t b = s.blocks[j];
+        if (bm->ref[b] != 1) continue;
+        const int32_t h = bm->host_free.back();
+        bm->host_free.pop_back();
+        pairs[2 * k] = b;
+        pairs[2 * k + 1] = h;
+        ++k;
+        bm->drop(b);
+        s.blocks[j] = h;
+        s.on_host[j] = 1;
+    }
+    s.swapped = true;
+    *num_pairs = k;
+    return PA_OK;
+}
+
+pa_status pa_bm_swap_in(pa_block_manager* bm, int64_t seq_id, int64_t* pairs, int32_t* num_pairs) {
+    if (!bm || !pairs || !num_pairs) return PA_ERR_INVALID_ARG;
+    *num_pairs = 0;
+    auto it = bm->seqs.find(seq_id);
+    if (it == bm->seqs.end() || !it->second.swapped) return PA_ERR_INVALID_ARG;
+    Sequence& s = it->second;
+    int64_t need = 0;
+    for (uint8_t h : s.on_host) need += h;
+    if (need > (int64_t)bm->free_stack.size()) return PA_ERR_NO_BLOCKS;
+    int32_t k = 0;
+    for (size_t j = 0; j < s.blocks.size(); ++j) {
+        if (!s.on_host[j]) continue;
+        const int32_t h = s.blocks[j];
+        const int32_t d = bm->take();
+        pairs[2 * k] = h;
+        pairs[2 * k + 1] = d;
+        ++k;
+        bm->host_free.push_back(h);
+        s.blocks[j] = d;
+    }
+    s.on_host.clear();
+    s.swapped = false;
+    *num_pairs = k;
+    return PA_OK;
+}
+
+int32_t pa_bm_is_swapped(const pa_block_manager* bm, int64_t seq_id) {
+    if (!bm) return -1;
+    auto it = bm->seqs.find(seq_id);
+    return it == bm->seqs.end() ? -1 : (it->second.swapped ? 1 : 0);
 }
 
 pa_status pa_bm_block_tables(const pa_block_manager* bm, const int64_t* seq_ids, int32_t n,
@@ -218,7 +294,7 @@ pa_status pa_bm_block_tables(const pa_block_manager* bm, const int64_t* seq_ids,
     if (n > 0 && (!seq_ids || !block_tables || !context_lens)) return PA_ERR_INVALID_ARG;
     for (int32_t k = 0; k < n; ++k) {   // validate everything before writing anything
         auto it = bm->seqs.find(seq_ids[k]);
-        if (it == bm->seqs.end() || (int64_t)it->second.blocks.size() > max_blocks_per_seq ||
+        if (it == bm->seqs.end() || it->second.swapped || (int64_t)it->second.blocks.size() > max_blocks_per_seq ||
             it->second.len > INT32_MAX)
             return PA_ERR_INVALID_ARG;
     }

@@ -64,6 +64,30 @@ __global__ void __launch_bounds__(256) copy_blocks_kernel(uint4* __restrict__ ke
     for (int64_t i = threadIdx.x; i < block_chunks; i += blockDim.x) d[i] = s[i];
 }
 
+// Whole blocks between two pools of the same shape, either of which may be
+// pinned host memory the device addresses (swap out / swap in).  Grid: (pair,
+// K or V); 16-byte chunks, consecutive threads on consecutive chunks, so the
+// transfers over PCIe are full 128-byte lines.
+__global__ void __launch_bounds__(256) swap_blocks_kernel(const uint4* __restrict__ src_key,
+                                                          const uint4* __restrict__ src_value,
+                                                          uint4* __restrict__ dst_key, uint4* __restrict__ dst_value,
+                                                          const int64_t* __restrict__ pairs, int num_pairs,
+                                                          int64_t src_blocks, int64_t dst_blocks,
+                                                          int64_t block_chunks, int32_t* status) {
+    griddep_launch_dependents();
+    griddep_wait();
+    const int k = blockIdx.x;
+    if (k >= num_pairs) return;
+    const int64_t src = pairs[2 * k], dst = pairs[2 * k + 1];
+    if (src < 0 || src >= src_blocks || dst < 0 || dst >= dst_blocks) {
+        if (blockIdx.y == 0 && threadIdx.x == 0) set_status(status, PA_ERR_OUT_OF_RANGE);
+        return;
+    }
+    const uint4* s = (blockIdx.y == 0 ? src_key : src_value) + src * block_chunks;
+    uint4* d = (blockIdx.y == 0 ? dst_key : dst_value) + dst * block_chunks;
+    for (int64_t i = threadIdx.x; i < block_chunks; i += blockDim.x) d[i] = s[i];
+}
+
 cudaError_t launch_reshape_and_cache(const void* key, const void* value, void* key_cache, void* value_cache,
                                      const int64_t* slot_mapping, int64_t num_tokens, int32_t num_blocks,
                                      int32_t num_kv_heads, int32_t head_dim, int elt_bytes, int32_t* status,
@@ -91,6 +115,18 @@ cudaError_t launch_copy_blocks(void* key_cache, void* value_cache, const int64_t
     return launch_pdl(copy_blocks_kernel, dim3(num_pairs, 2), dim3(256), 0, stream,
                       static_cast<uint4*>(key_cache), static_cast<uint4*>(value_cache), block_pairs, (int)num_pairs,
                       (int64_t)num_blocks, block_chunks, status);
+}
+
+cudaError_t launch_swap_blocks(const void* src_key, const void* src_value, void* dst_key, void* dst_value,
+                               const int64_t* block_pairs, int32_t num_pairs, int32_t src_num_blocks,
+                               int32_t dst_num_blocks, int32_t num_kv_heads, int32_t head_dim, int elt_bytes,
+                               int32_t* status, cudaStream_t stream) {
+    if (num_pairs == 0) return cudaSuccess;
+    const int64_t block_chunks = (int64_t)num_kv_heads * kBlockSize * head_dim * elt_bytes / 16;
+    return launch_pdl(swap_blocks_kernel, dim3(num_pairs, 2), dim3(256), 0, stream,
+                      static_cast<const uint4*>(src_key), static_cast<const uint4*>(src_value),
+                      static_cast<uint4*>(dst_key), static_cast<uint4*>(dst_value), block_pairs, (int)num_pairs,
+                      (int64_t)src_num_blocks, (int64_t)dst_num_blocks, block_chunks, status);
 }
 
 }  // namespace pa

@@ -219,6 +219,26 @@ pa_status pa_copy_blocks(void* key_cache, void* value_cache, const int64_t* bloc
     return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
+pa_status pa_swap_blocks(const void* src_key_cache, const void* src_value_cache, void* dst_key_cache,
+                         void* dst_value_cache, const int64_t* block_pairs, int32_t num_pairs, int32_t src_num_blocks,
+                         int32_t dst_num_blocks, int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                         pa_dtype dtype, int32_t* status, pa_stream_t stream) {
+    if (num_pairs < 0 || src_num_blocks <= 0 || dst_num_blocks <= 0 || num_kv_heads <= 0 || head_dim <= 0)
+        return PA_ERR_INVALID_ARG;
+    if (!valid_dtype(dtype)) return PA_ERR_INVALID_ARG;
+    if (block_size != kBlockSize || (head_dim != 64 && head_dim != 128)) return PA_ERR_UNSUPPORTED;
+    if (num_pairs == 0) return PA_OK;
+    if (!src_key_cache || !src_value_cache || !dst_key_cache || !dst_value_cache || !block_pairs)
+        return PA_ERR_INVALID_ARG;
+    if (!aligned16(src_key_cache) || !aligned16(src_value_cache) || !aligned16(dst_key_cache) ||
+        !aligned16(dst_value_cache))
+        return PA_ERR_INVALID_ARG;
+    const cudaError_t e = launch_swap_blocks(src_key_cache, src_value_cache, dst_key_cache, dst_value_cache,
+                                             block_pairs, num_pairs, src_num_blocks, dst_num_blocks, num_kv_heads,
+                                             head_dim, elt_bytes(dtype), status, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
 const char* pa_get_error_string(pa_status s) {
     const int v = (int)s;
     if (v == PA_OK) return "PA_OK";

@@ -23,6 +23,11 @@ cudaError_t launch_copy_blocks(void* key_cache, void* value_cache, const int64_t
                                int32_t num_blocks, int32_t num_kv_heads, int32_t head_dim, int elt_bytes,
                                int32_t* status, cudaStream_t stream);
 
+cudaError_t launch_swap_blocks(const void* src_key, const void* src_value, void* dst_key, void* dst_value,
+                               const int64_t* block_pairs, int32_t num_pairs, int32_t src_num_blocks,
+                               int32_t dst_num_blocks, int32_t num_kv_heads, int32_t head_dim, int elt_bytes,
+                               int32_t* status, cudaStream_t stream);
+
 // Which main decode kernel serves a shape.
 enum class DecodePath { kTensorCore, kSimt };
 DecodePath decode_path(pa_dtype dtype, int head_dim, int group);

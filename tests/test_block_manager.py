@@ -7,11 +7,13 @@ CPU only.  Three kinds of checks:
     history; a fork shares blocks and a write into a shared block clones it first
     (digest, "Copy-on-write: when two requests share a prefix");
   * operation by operation, the C++ manager equals oracle/block_model.py on seeded
-    random workloads (slots, copy pairs, free counts, references, tables);
+    random workloads (slots, copy pairs, swap pairs, free counts, references,
+    tables), with requests evicted to a host pool and brought back;
   * a data-level invariant that holds for any correct manager: with every token
     written to its slot and every copy applied, each request reads back exactly its
     own token history through its block table -- its prefix as it was at the fork,
-    then its own tokens -- whatever the other requests wrote.
+    then its own tokens -- whatever the other requests wrote, and after a round
+    trip through the host pool.
 """
 
 import json
@@ -132,6 +134,32 @@ def test_exact_accounting_when_sharers_append_together():
     assert slots.tolist() == [1 * 16 + 8, 0 * 16 + 8]
 
 
+def test_swap_moves_private_blocks_and_keeps_shared_ones():
+    """Eviction moves only what the request alone holds; its shared prefix stays on the device."""
+    pa = _pa()
+    bm = pa.BlockManager(16, 16, 8)
+    bm.add_sequence(1, 40)                        # blocks 0, 1, 2
+    bm.fork(1, 2)
+    bm.append_tokens([2])                         # 2 copies block 2 -> 3; shares 0 and 1
+    out = bm.swap_out(2)
+    assert out.tolist() == [[3, 0]]               # only the private block, to host block 0
+    assert bm.is_swapped(2) and bm.ref_count(0) == 2 and bm.ref_count(3) == 0
+    with pytest.raises(pa.PagedAttentionError):
+        bm.append_tokens([2])                     # no appends while evicted
+    with pytest.raises(pa.PagedAttentionError):
+        bm.block_tables([2], 4)
+    back = bm.swap_in(2)
+    assert back.tolist() == [[0, 3]]              # the freed block 3 is handed out again
+    bt, cl = bm.block_tables([2], 4)
+    assert bt.tolist() == [[0, 1, 3, -1]] and cl.tolist() == [41]
+    assert bm.num_free_host_blocks == 8
+    bm2 = pa.BlockManager(4, 16, 0)               # no host pool: nothing can be evicted
+    bm2.add_sequence(1, 5)
+    with pytest.raises(pa.PagedAttentionError) as e:
+        bm2.swap_out(1)
+    assert e.value.code == pa.PA_ERR_NO_BLOCKS
+
+
 def test_argument_errors():
     pa = _pa()
     bm = pa.BlockManager(8, 16)
@@ -160,9 +188,11 @@ def _random_ops(rng, steps):
             yield ("fork", parent, next_id)
             live.append(next_id)
             next_id += 1
-        elif r < 0.85:
+        elif r < 0.78:
             k = int(rng.integers(1, min(len(live), 12) + 1))
             yield ("append", [int(x) for x in rng.choice(live, size=k, replace=True)])
+        elif r < 0.85:
+            yield ("swap", int(rng.choice(live)))
         else:
             sid = int(rng.choice(live))
             live.remove(sid)
@@ -173,11 +203,18 @@ def _random_ops(rng, steps):
 @pytest.mark.parametrize("block_size", [16, 4])
 def test_matches_model_and_keeps_every_history(seed, block_size):
     pa = _pa()
-    nb = 48
-    bm, model = pa.BlockManager(nb, block_size), BlockModel(nb, block_size)
+    nb, nh = 48, 24
+    bm, model = pa.BlockManager(nb, block_size, nh), BlockModel(nb, block_size, nh)
     rng = np.random.default_rng(seed)
     pool = np.full(nb * block_size, -1, dtype=np.int64)     # token written in each slot
+    host = np.full(nh * block_size, -1, dtype=np.int64)     # the host pool, for swapped-out blocks
     history: dict[int, list[int]] = {}
+    swapped: set[int] = set()
+
+    def move(src, dst, pairs):
+        for a, b in pairs:
+            dst[b * block_size:(b + 1) * block_size] = src[a * block_size:(a + 1) * block_size]
+
     token = 0
     for op in _random_ops(rng, 400):
         if op[0] == "add":
@@ -195,15 +232,47 @@ def test_matches_model_and_keeps_every_history(seed, block_size):
             token += n
             pool[got] = toks
             history[sid] = toks
+        elif op[0] == "swap":
+            _, sid = op
+            if sid not in history:
+                continue
+            if sid in swapped:
+                try:
+                    exp = model.swap_in(sid)
+                except NoBlocks:
+                    with pytest.raises(pa.PagedAttentionError) as e:
+                        bm.swap_in(sid)
+                    assert e.value.code == pa.PA_ERR_NO_BLOCKS
+                    continue
+                got = bm.swap_in(sid)
+                assert [tuple(p) for p in got.tolist()] == exp
+                move(host, pool, got)
+                swapped.discard(sid)
+            else:
+                try:
+                    exp = model.swap_out(sid)
+                except NoBlocks:
+                    with pytest.raises(pa.PagedAttentionError) as e:
+                        bm.swap_out(sid)
+                    assert e.value.code == pa.PA_ERR_NO_BLOCKS
+                    continue
+                got = bm.swap_out(sid)
+                assert [tuple(p) for p in got.tolist()] == exp
+                move(pool, host, got)
+                # the freed device blocks are written by others from now on
+                for d, _ in got.tolist():
+                    pool[d * block_size:(d + 1) * block_size] = -7
+                swapped.add(sid)
+            assert bm.is_swapped(sid) == (sid in swapped)
         elif op[0] == "fork":
             _, parent, child = op
-            if parent not in history:
+            if parent not in history or parent in swapped:
                 continue
             model.fork(parent, child)
             bm.fork(parent, child)
             history[child] = list(history[parent])
         elif op[0] == "append":
-            sids = [s for s in op[1] if s in history]
+            sids = [s for s in op[1] if s in history and s not in swapped]
             if not sids:
                 continue
             try:
@@ -230,11 +299,14 @@ def test_matches_model_and_keeps_every_history(seed, block_size):
             model.free_sequence(sid)
             bm.free_sequence(sid)
             del history[sid]
+            swapped.discard(sid)
         # state equal after every operation
         assert bm.num_free_blocks == len(model.free)
+        assert bm.num_free_host_blocks == len(model.host_free)
         assert [bm.ref_count(b) for b in range(nb)] == model.refs
-        if history:
-            sids = sorted(history)
+        resident = [s_ for s_ in history if s_ not in swapped]
+        if resident:
+            sids = sorted(resident)
             mb = max(len(model.tables[s]) for s in sids) or 1
             bt, cl = bm.block_tables(sids, mb)
             exp_bt, exp_cl = model.block_tables(sids, mb)

@@ -73,3 +73,63 @@ def test_decode_loop_with_forks_and_copy_on_write():
     for sid in live:
         bm.free_sequence(sid)
     assert bm.num_free_blocks == NB
+
+
+def test_swap_out_and_in_through_pinned_host_memory():
+    """A request is evicted to pinned host pools, its device blocks are reused, it comes back intact."""
+    import torch
+
+    import paged_kv_cache_362_b200 as pa
+
+    rng = np.random.default_rng(5)
+    NB, NH, Hkv, Hq, D, dt = 64, 32, 4, 28, 128, "bf16"
+    scale = 1.0 / np.sqrt(D)
+    bm = pa.BlockManager(NB, 16, NH)
+    shape = (NB, Hkv, 16, D)
+    # N(0, 1) values as bf16 bit patterns (the top half of the fp32 bits)
+    bits = lambda s: (rng.standard_normal(s).astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    kc_h, vc_h = bits(shape), bits(shape)
+    kc, vc = to_device(kc_h, dt), to_device(vc_h, dt)
+    hk = torch.empty((NH, Hkv, 16, D), dtype=torch.bfloat16).pin_memory()
+    hv = torch.empty((NH, Hkv, 16, D), dtype=torch.bfloat16).pin_memory()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for sid, n in ((1, 300), (2, 70)):
+        bm.add_sequence(sid, n)
+    bm.fork(1, 3)
+    bm.append_tokens([3])                       # 3 clones 1's partial block: it owns that one, shares the rest
+    bt0, cl0 = bm.block_tables([1, 2, 3], 32)
+    q = bits((3, Hq, D))
+    before = torch.empty((3, Hq, D), dtype=torch.bfloat16, device="cuda")
+    ws = pa.make_workspace(3, Hq, Hkv, D, 512)
+    q_d = to_device(q, dt)
+    pa.decode(before, q_d, kc, vc, torch.from_numpy(bt0).cuda(), torch.from_numpy(cl0).cuda(), scale, 512, ws)
+    # evict 1 and 2; their private blocks go to the host pools
+    moved = {}
+    for sid in (1, 2):
+        pairs = bm.swap_out(sid)
+        moved[sid] = pairs
+        pa.swap_blocks(kc, vc, hk, hv, torch.from_numpy(pairs).cuda(), status=status)
+    torch.cuda.synchronize()
+    for sid, pairs in moved.items():
+        for d, h in pairs.tolist():
+            assert np.array_equal(hk[h].view(torch.int16).numpy().view(np.uint16), kc_h[d])
+            assert np.array_equal(hv[h].view(torch.int16).numpy().view(np.uint16), vc_h[d])
+    # 1's shared blocks stayed for 3; the freed blocks are overwritten by a new request
+    assert len(moved[1]) < bm.sequence_blocks(1)
+    slots = bm.add_sequence(9, 16 * bm.num_free_blocks)
+    junk = torch.zeros((len(slots), Hkv, D), dtype=torch.bfloat16, device="cuda")
+    pa.reshape_and_cache(junk, junk, kc, vc, torch.from_numpy(slots).cuda(), status=status)
+    bm.free_sequence(9)
+    # bring them back (pinned pairs this time) and decode again: the same bits as before the eviction
+    for sid in (1, 2):
+        pairs = torch.from_numpy(bm.swap_in(sid)).pin_memory()
+        pa.swap_blocks(hk, hv, kc, vc, pairs, status=status)
+    bt1, cl1 = bm.block_tables([1, 2, 3], 32)
+    after = torch.empty_like(before)
+    pa.decode(after, q_d, kc, vc, torch.from_numpy(bt1).cuda(), torch.from_numpy(cl1).cuda(), scale, 512, ws)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    assert torch.equal(before.view(torch.int16), after.view(torch.int16))
+    # and the result is the oracle's on the original pools through the original tables
+    ref = c_oracle.decode(q, kc_h, vc_h, bt0, cl0, scale, dt, Hkv)
+    compare(out_f64(after), ref, dt, "after swap round trip")
