@@ -448,6 +448,54 @@ def swap_bandwidth(w, nblocks: int = 4096, reps: int = 5):
     return res
 
 
+def prefill_throughput(seed: int, reps: int = 20):
+    """pa_prefill on chunked prompts (4 sequences: 512 new tokens on 3,584 cached ones, Qwen-shaped
+    heads, bf16): causal attention TFLOP/s against the measured bf16 tensor peak."""
+    import torch
+
+    import paged_kv_cache_362_b200 as pa
+
+    B, past, chunk, Hq, Hkv, D = 4, 3584, 512, 28, 4, 128
+    ctx = past + chunk
+    nbps = ctx // 16
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    kc = torch.randn((B * nbps, Hkv, 16, D), generator=g, device="cuda").to(torch.bfloat16)
+    vc = torch.randn((B * nbps, Hkv, 16, D), generator=g, device="cuda").to(torch.bfloat16)
+    perm = np.random.default_rng(seed).permutation(B * nbps).astype(np.int32)
+    bt = torch.from_numpy(perm.reshape(B, nbps)).cuda()
+    q = torch.randn((B * chunk, Hq, D), generator=g, device="cuda").to(torch.bfloat16)
+    out = torch.empty_like(q)
+    qs = torch.arange(0, B * chunk + 1, chunk, dtype=torch.int32, device="cuda")
+    cl = torch.full((B,), ctx, dtype=torch.int32, device="cuda")
+    args = (out, q, kc, vc, bt, qs, cl, 1 / D ** 0.5, chunk)
+    for _ in range(3):
+        pa.prefill(*args)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        pa.prefill(*args)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    flops = 4 * Hq * D * B * sum(past + i + 1 for i in range(chunk))
+    tf = flops / (ms * 1e-3) / 1e12
+    peak, _ = measured_bf16_peak()
+    return {"workload": f"{B} sequences x ({chunk} new on {past} cached tokens), 28/4 heads, D 128, bf16",
+            "ms": round(ms, 4), "tflops": round(tf, 1), "peak_tflops": peak, "frac": round(tf / peak, 4)}
+
+
+def measured_bf16_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            v = json.load(f).get("bf16_tflops")
+        if v:
+            return float(v), "measured"
+    except Exception:
+        pass
+    return 1590.0, "fallback"
+
+
 def cpu_model() -> str:
     try:
         for line in open("/proc/cpuinfo"):
@@ -612,6 +660,7 @@ def main():
 
     bm_step = block_manager_step(args.workload, args.seed) if rank == 0 else None
     swap = swap_bandwidth(w) if rank == 0 and not args.no_secondary else None
+    prefill_res = prefill_throughput(args.seed) if rank == 0 and not args.no_secondary else None
 
     if rank == 0:
         c = w.cfg
@@ -643,6 +692,7 @@ def main():
             "placement_overhead": placement,
             "block_manager": bm_step,
             "swap": swap,
+            "prefill": prefill_res,
             "gpu_launches": w.launches_per_step * args.steps,
             "clocks": clk,
             "secondary": secondary,

@@ -173,6 +173,37 @@ pa_status pa_copy_blocks(void* key_cache, void* value_cache, const int64_t* bloc
                          pa_stream_t stream);
 
 /*
+ * pa_prefill -- causal attention of a chunk of new query tokens per sequence
+ * over everything the sequence has in the paged cache (prompt processing, and
+ * chunked prefill on top of an existing context).
+ *
+ * Sequence b's new tokens are q rows [query_start[b], query_start[b+1]); with
+ * n = context_lens[b] tokens in the cache, the new ones included (written
+ * first with pa_reshape_and_cache), and L = query_start[b+1] - query_start[b],
+ * query row i < L sits at position p = n - L + i and attends to positions
+ * 0 .. p through the block table ("PagedAttention" digest, sections
+ * "PagedAttention in one picture" and "Why the attention kernel works at
+ * all"): with g = h / (num_heads / num_kv_heads),
+ *     out[query_start[b] + i][h][:] = sum_{j <= p} softmax_j(scale * q . K_j) V_j
+ * computed in fp32 from the stored values and rounded to the element type.
+ *
+ *   out, q          [query_start[num_seqs]][num_heads][head_dim], 16-byte aligned
+ *   block_tables    int32 [num_seqs][max_blocks_per_seq]; entries outside
+ *                   [0, num_blocks) set PA_ERR_OUT_OF_RANGE and contribute nothing
+ *   query_start     int32 [num_seqs + 1], nondecreasing, device
+ *   context_lens    int32 [num_seqs], device; n < L or n > max_blocks_per_seq * 16
+ *                   sets PA_ERR_OUT_OF_RANGE and leaves that sequence's rows unwritten
+ *   max_query_len   host-side upper bound of the L (sizes the grid)
+ * Supported: float16 and bfloat16, head_dim 64 or 128, at most 16 query heads
+ * per KV head (PA_ERR_UNSUPPORTED otherwise).  No workspace.
+ */
+pa_status pa_prefill(void* out, const void* q, const void* key_cache, const void* value_cache,
+                     const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* query_start,
+                     const int32_t* context_lens, int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads,
+                     int32_t head_dim, int32_t block_size, int32_t num_blocks, float scale, int32_t max_query_len,
+                     pa_dtype dtype, int32_t* status, pa_stream_t stream);
+
+/*
  * pa_swap_blocks -- copy whole blocks from one pool to another of the same
  * shape, for evicting blocks to CPU memory and bringing them back
  * ("PagedAttention, Visualized", Part 3: the operating-system table, where

@@ -66,3 +66,14 @@ def decode_pairs(pairs, q, key_cache, value_cache, block_tables, context_lens, s
     if rc != 0:
         raise IndexError(f"C oracle status {rc}")
     return out
+
+
+def prefill(q, key_cache, value_cache, block_tables, query_start, context_lens, scale, dtype, num_kv_heads,
+            num_threads: int = 0) -> np.ndarray:
+    """fp64 [T, Hq, D] causal prefill: row at position p attends to positions 0 .. p (a decode of p + 1 tokens)."""
+    from .reference import prefill_rows
+
+    seqs, pos = prefill_rows(np.asarray(query_start), np.asarray(context_lens))
+    bt = np.ascontiguousarray(np.asarray(block_tables)[seqs], dtype=np.int32)
+    return decode(q, key_cache, value_cache, bt, (pos + 1).astype(np.int32), scale, dtype, num_kv_heads,
+                  num_threads=num_threads)

@@ -165,6 +165,32 @@ def decode(q: np.ndarray, key_cache: np.ndarray, value_cache: np.ndarray,
     return out
 
 
+def prefill_rows(query_start: np.ndarray, context_lens: np.ndarray):
+    """For every new query row: (sequence, position).  Row i of sequence b (of L
+    new tokens, n tokens in the cache in all) sits at position n - L + i."""
+    seqs, pos = [], []
+    for b in range(len(context_lens)):
+        L = int(query_start[b + 1] - query_start[b])
+        n = int(context_lens[b])
+        for i in range(L):
+            seqs.append(b)
+            pos.append(n - L + i)
+    return np.array(seqs, dtype=np.int64), np.array(pos, dtype=np.int64)
+
+
+def prefill(q: np.ndarray, key_cache: np.ndarray, value_cache: np.ndarray, block_tables: np.ndarray,
+            query_start: np.ndarray, context_lens: np.ndarray, scale: float, dtype: str,
+            num_kv_heads: int) -> np.ndarray:
+    """Causal attention of each new query row over the cache up to its own position (fp64 [T, Hq, D]).
+
+    By definition the row at position p sees exactly the keys 0 .. p: it is the
+    decode of a sequence whose context is the first p + 1 tokens.
+    """
+    seqs, pos = prefill_rows(query_start, context_lens)
+    return decode(q, key_cache, value_cache, block_tables[seqs], (pos + 1).astype(np.int32), scale, dtype,
+                  num_kv_heads)
+
+
 # ---------------------------------------------------------------------------
 # Split-context partitions and their merge.  Softmax over a union of disjoint
 # token sets can be rebuilt from each set's (max, sum of exp, unnormalised

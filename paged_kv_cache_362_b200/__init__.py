@@ -24,6 +24,7 @@ from ._lib import (  # noqa: F401
     decode_workspace_size,
     error_string,
     make_workspace,
+    prefill,
     reshape_and_cache,
     swap_blocks,
     version,

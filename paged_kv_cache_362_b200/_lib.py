@@ -38,7 +38,7 @@ def _load() -> ctypes.CDLL:
         raise ImportError(f"{LIB_PATH} is not built; run `python paged_kv_cache_362_b200/build.py`")
     lib = ctypes.CDLL(LIB_PATH)
     for sym in ("pa_reshape_and_cache", "pa_decode_workspace_size", "pa_decode", "pa_decode_launch_count",
-                "pa_copy_blocks", "pa_get_error_string", "pa_version", "pa_bm_create", "pa_bm_append_tokens"):
+                "pa_copy_blocks", "pa_get_error_string", "pa_version", "pa_bm_create", "pa_bm_append_tokens", "pa_prefill", "pa_swap_blocks"):
         if not hasattr(lib, sym):
             raise ImportError(f"{LIB_PATH} lacks {sym} (stale build); run `python paged_kv_cache_362_b200/build.py`")
     p, i32, i64, f32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
@@ -76,6 +76,8 @@ def _load() -> ctypes.CDLL:
         getattr(lib, fn).restype = ctypes.c_int
     lib.pa_bm_is_swapped.argtypes = [p, i64]
     lib.pa_bm_is_swapped.restype = i32
+    lib.pa_prefill.argtypes = [p, p, p, p, p, i32, p, p, i32, i32, i32, i32, i32, i32, f32, i32, ctypes.c_int, p, p]
+    lib.pa_prefill.restype = ctypes.c_int
     lib.pa_swap_blocks.argtypes = [p, p, p, p, p, i32, i32, i32, i32, i32, i32, ctypes.c_int, p, p]
     lib.pa_swap_blocks.restype = ctypes.c_int
     lib.pa_bm_block_tables.argtypes = [p, p, i32, i32, p, p]
@@ -185,6 +187,27 @@ def decode(out, q, key_cache, value_cache, block_tables, context_lens, scale, ma
                          workspace.numel() * workspace.element_size(), _dtype_code(q), _ptr(status),
                          _stream(stream)),
            "pa_decode")
+
+
+def prefill(out, q, key_cache, value_cache, block_tables, query_start, context_lens, scale, max_query_len,
+            status=None, stream=None):
+    """Causal attention of each sequence's new query rows over its paged cache (pa_prefill).
+
+    q, out [T, Hq, D]; query_start int32 [B + 1]; context_lens int32 [B] (the new tokens included,
+    already written with reshape_and_cache).
+    """
+    T, Hq, D = q.shape
+    NB, Hkv = key_cache.shape[0], key_cache.shape[1]
+    assert out.shape == q.shape and out.dtype == q.dtype == key_cache.dtype == value_cache.dtype
+    assert block_tables.dtype.itemsize == 4 and context_lens.dtype.itemsize == 4 and query_start.dtype.itemsize == 4
+    B = context_lens.shape[0]
+    assert query_start.shape == (B + 1,) and block_tables.shape[0] == B
+    for t in (out, q, key_cache, value_cache, block_tables, query_start, context_lens):
+        assert t.is_contiguous()
+    _check(LIB.pa_prefill(_ptr(out), _ptr(q), _ptr(key_cache), _ptr(value_cache), _ptr(block_tables),
+                          block_tables.shape[1], _ptr(query_start), _ptr(context_lens), B, Hq, Hkv, D, BLOCK_SIZE, NB,
+                          float(scale), int(max_query_len), _dtype_code(q), _ptr(status), _stream(stream)),
+           "pa_prefill")
 
 
 def copy_blocks(key_cache, value_cache, block_pairs, status=None, stream=None):

@@ -219,6 +219,46 @@ pa_status pa_copy_blocks(void* key_cache, void* value_cache, const int64_t* bloc
     return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
+pa_status pa_prefill(void* out, const void* q, const void* key_cache, const void* value_cache,
+                     const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* query_start,
+                     const int32_t* context_lens, int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads,
+                     int32_t head_dim, int32_t block_size, int32_t num_blocks, float scale, int32_t max_query_len,
+                     pa_dtype dtype, int32_t* status, pa_stream_t stream) {
+    if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || num_blocks <= 0 ||
+        max_blocks_per_seq <= 0 || max_query_len < 0)
+        return PA_ERR_INVALID_ARG;
+    if (!valid_dtype(dtype) || !std::isfinite(scale) || num_heads % num_kv_heads != 0) return PA_ERR_INVALID_ARG;
+    if (block_size != kBlockSize || (head_dim != 64 && head_dim != 128) || dtype == PA_F32 ||
+        num_heads / num_kv_heads > 16)
+        return PA_ERR_UNSUPPORTED;
+    if ((int64_t)num_blocks * num_kv_heads * kBlockSize * head_dim > INT64_MAX / 4) return PA_ERR_UNSUPPORTED;
+    if (num_seqs == 0 || max_query_len == 0) return PA_OK;
+    if (!out || !q || !key_cache || !value_cache || !block_tables || !query_start || !context_lens)
+        return PA_ERR_INVALID_ARG;
+    if (!aligned16(out) || !aligned16(q) || !aligned16(key_cache) || !aligned16(value_cache))
+        return PA_ERR_INVALID_ARG;
+    PrefillParams p{};
+    p.out = out;
+    p.q = q;
+    p.key_cache = key_cache;
+    p.value_cache = value_cache;
+    p.block_tables = block_tables;
+    p.query_start = query_start;
+    p.context_lens = context_lens;
+    p.status = status;
+    p.num_seqs = num_seqs;
+    p.num_heads = num_heads;
+    p.num_kv_heads = num_kv_heads;
+    p.head_dim = head_dim;
+    p.group = num_heads / num_kv_heads;
+    p.max_blocks_per_seq = max_blocks_per_seq;
+    p.num_blocks = num_blocks;
+    p.max_query_len = max_query_len;
+    p.scale_log2 = scale * 1.4426950408889634f;  // log2(e)
+    const cudaError_t e = launch_prefill(p, dtype, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
 pa_status pa_swap_blocks(const void* src_key_cache, const void* src_value_cache, void* dst_key_cache,
                          void* dst_value_cache, const int64_t* block_pairs, int32_t num_pairs, int32_t src_num_blocks,
                          int32_t dst_num_blocks, int32_t num_kv_heads, int32_t head_dim, int32_t block_size,

@@ -147,6 +147,7 @@ __device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src) {
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_group1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 
 __device__ __forceinline__ void prefetch_l2(const void* p) {
     asm volatile("prefetch.global.L2 [%0];" ::"l"(p) : "memory");
@@ -242,6 +243,21 @@ struct DecodeParams {
     float* part_m;                // [B, Hq, NP_max]   max logit (log2 units)
     float* part_l;                // [B, Hq, NP_max]   sum of 2^(s - m)
     float* part_o;                // [B, Hq, NP_max, D] unnormalised output
+};
+
+// paged prefill (pa_prefill)
+struct PrefillParams {
+    void* out;                    // [T, Hq, D]
+    const void* q;                // [T, Hq, D]
+    const void* key_cache;        // [NB, Hkv, 16, D]
+    const void* value_cache;
+    const int32_t* block_tables;  // [B, MB]
+    const int32_t* query_start;   // [B + 1]: sequence b's queries are rows [query_start[b], query_start[b+1])
+    const int32_t* context_lens;  // [B]: tokens in the cache, the new ones included
+    int32_t* status;
+    int num_seqs, num_heads, num_kv_heads, head_dim, group;
+    int max_blocks_per_seq, num_blocks, max_query_len;
+    float scale_log2;
 };
 
 // context length as every decode kernel sees it: clamped into [0, ctx_cap]

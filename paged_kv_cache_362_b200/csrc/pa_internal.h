@@ -28,6 +28,9 @@ cudaError_t launch_swap_blocks(const void* src_key, const void* src_value, void*
                                int32_t dst_num_blocks, int32_t num_kv_heads, int32_t head_dim, int elt_bytes,
                                int32_t* status, cudaStream_t stream);
 
+// Causal attention of each sequence's new query tokens over its paged cache.
+cudaError_t launch_prefill(const PrefillParams& p, pa_dtype dtype, cudaStream_t stream);
+
 // Which main decode kernel serves a shape.
 enum class DecodePath { kTensorCore, kSimt };
 DecodePath decode_path(pa_dtype dtype, int head_dim, int group);

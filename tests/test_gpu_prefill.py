@@ -1,0 +1,116 @@
+"""GPU parity of paged prefill (pa_prefill) against the fp64 oracle.
+
+Whole prompts and chunks on top of an existing context, ragged chunk lengths
+(1, 15, 16, 17, ...), GQA groups 1 to 16, head_dim 64 and 128, fp16 and bf16;
+every output element is compared.  Also: a bad block id is flagged and
+contributes nothing, and the result does not depend on where blocks live.
+"""
+
+import numpy as np
+import pytest
+
+from oracle import c_oracle
+from parity import compare, out_f64, to_device
+
+pytestmark = pytest.mark.gpu
+
+
+def _case(rng, ctxs, chunks, Hq, Hkv, D, dtype, extra_blocks=3):
+    B = len(ctxs)
+    mb = max(-(-c // 16) for c in ctxs)
+    nb = sum(-(-c // 16) for c in ctxs) + extra_blocks
+    perm = rng.permutation(nb)
+    bt = np.full((B, mb), -1, dtype=np.int32)
+    k = 0
+    for b, c in enumerate(ctxs):
+        for j in range(-(-c // 16)):
+            bt[b, j] = perm[k]
+            k += 1
+    npdt = np.float16 if dtype == "f16" else np.float32
+
+    def draw(shape):
+        x = rng.standard_normal(shape).astype(np.float32)
+        return x.astype(np.float16) if dtype == "f16" else (x.view(np.uint32) >> 16).astype(np.uint16)
+
+    kc, vc = draw((nb, Hkv, 16, D)), draw((nb, Hkv, 16, D))
+    qs = np.concatenate([[0], np.cumsum(chunks)]).astype(np.int32)
+    q = draw((int(qs[-1]), Hq, D))
+    del npdt
+    return q, kc, vc, bt, qs, np.array(ctxs, dtype=np.int32)
+
+
+def _run(q, kc, vc, bt, qs, cl, scale, dtype, status=None):
+    import torch
+
+    import paged_kv_cache_362_b200 as pa
+
+    out = torch.full(q.shape, float("nan"), dtype=torch.float16 if dtype == "f16" else torch.bfloat16,
+                     device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda") if status is None else status
+    pa.prefill(out, to_device(q, dtype), to_device(kc, dtype), to_device(vc, dtype), torch.from_numpy(bt).cuda(),
+               torch.from_numpy(qs).cuda(), torch.from_numpy(cl).cuda(), scale, int(np.diff(qs).max()), status=st)
+    torch.cuda.synchronize()
+    return out, int(st.item())
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+@pytest.mark.parametrize("heads", [(28, 4), (8, 8), (16, 2), (32, 2)], ids=lambda h: f"{h[0]}x{h[1]}")
+@pytest.mark.parametrize("D", [64, 128])
+def test_prompts_and_chunks_every_element(dtype, heads, D):
+    Hq, Hkv = heads
+    rng = np.random.default_rng(Hq + D)
+    # (context, new tokens): whole prompts, chunks on a context, ragged lengths around 16
+    ctxs = [1, 15, 17, 64, 300, 96, 129, 40]
+    chunks = [1, 15, 16, 33, 300, 17, 1, 40]
+    q, kc, vc, bt, qs, cl = _case(rng, ctxs, chunks, Hq, Hkv, D, dtype)
+    scale = 1.0 / np.sqrt(D)
+    out, st = _run(q, kc, vc, bt, qs, cl, scale, dtype)
+    assert st == 0
+    ref = c_oracle.prefill(q, kc, vc, bt, qs, cl, scale, dtype, Hkv)
+    compare(out_f64(out), ref, dtype, f"{dtype} {heads} D={D}")
+
+
+def test_long_chunk_on_long_context():
+    rng = np.random.default_rng(7)
+    ctxs, chunks = [4096, 2500], [512, 700]
+    q, kc, vc, bt, qs, cl = _case(rng, ctxs, chunks, 28, 4, 128, "bf16")
+    out, st = _run(q, kc, vc, bt, qs, cl, 1 / np.sqrt(128), "bf16")
+    assert st == 0
+    ref = c_oracle.prefill(q, kc, vc, bt, qs, cl, 1 / np.sqrt(128), "bf16", 4)
+    compare(out_f64(out), ref, "bf16", "long")
+
+
+def test_placement_does_not_change_the_bits():
+    import torch
+
+    rng = np.random.default_rng(9)
+    q, kc, vc, bt, qs, cl = _case(rng, [200, 90], [200, 30], 28, 4, 128, "f16")
+    a, _ = _run(q, kc, vc, bt, qs, cl, 0.09, "f16")
+    perm = rng.permutation(kc.shape[0])
+    kc2, vc2 = np.empty_like(kc), np.empty_like(vc)
+    kc2[perm], vc2[perm] = kc, vc
+    bt2 = np.where(bt >= 0, perm[np.maximum(bt, 0)], -1).astype(np.int32)
+    b, _ = _run(q, kc2, vc2, bt2, qs, cl, 0.09, "f16")
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+def test_bad_block_flagged_and_skipped():
+    import paged_kv_cache_362_b200 as pa
+
+    rng = np.random.default_rng(4)
+    q, kc, vc, bt, qs, cl = _case(rng, [64], [20], 8, 2, 64, "f16")
+    bt_bad = bt.copy()
+    bt_bad[0, 1] = 10_000            # keys 16..31 are unreachable
+    out, st = _run(q, kc, vc, bt_bad, qs, cl, 0.125, "f16")
+    assert st & pa.PA_ERR_OUT_OF_RANGE
+    # the oracle without those 16 keys: rows see their visible keys except positions 16..31
+    from oracle import reference as R
+
+    seqs, pos = R.prefill_rows(qs, cl)
+    got = out_f64(out)
+    for t, p_ in enumerate(pos):
+        keys = [i for i in range(int(p_) + 1) if not 16 <= i < 32]
+        K = np.stack([kc[bt[0, i // 16], :, i % 16] for i in keys], axis=1).astype(np.float64)
+        V = np.stack([vc[bt[0, i // 16], :, i % 16] for i in keys], axis=1).astype(np.float64)
+        ref = np.stack([R.attention_f64(q[t, h].astype(np.float64), K[h // 4], V[h // 4], 0.125) for h in range(8)])
+        compare(got[t], ref, "f16", f"row {t}")
