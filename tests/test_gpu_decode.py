@@ -191,3 +191,31 @@ def test_full_size_step_sampled(name):
     mabs, mrel = compare(got, ref, wl.cfg.dtype, name)
     print(f"{name}: max abs {mabs:.2e} max rel {mrel:.2e} over {len(seqs)} sequences")
     torch.cuda.synchronize()
+
+
+def test_extreme_sizes():
+    """The largest shapes the workspace and grids see: one 262,144-token context (512 partitions,
+    reduce kernel) and 8,192 short sequences (planning kernel, counters beyond the fixed region)."""
+    import torch
+
+    pa = _pa()
+    # one very long sequence, MQA group of 8
+    cfg = get_config("qwen_layer", dtype="bf16", num_heads=8, num_kv_heads=1, head_dim=128, num_blocks=16400,
+                     ctx_kind="fixed", ctx_args=(262144,))
+    wl = build_workload(cfg, seed=21)
+    case = DeviceCase(wl, device_draw=True)
+    sub = case.host_subproblem([0])
+    out = _decode(case, partition_size=512)
+    assert int(case.status.item()) == 0
+    compare(out_f64(out), oracle_step(sub, cfg, do_copy=False, do_write=False), "bf16", "262144 tokens")
+    del case
+    torch.cuda.empty_cache()
+    # many short sequences
+    cfg = get_config("qwen_layer", dtype="f16", num_blocks=8192 * 3 + 8, ctx_kind="uniform", ctx_args=(1, 40))
+    wl = build_workload(cfg, seed=22, num_seqs=8192)
+    case = DeviceCase(wl, device_draw=True)
+    seqs = _seq_sample(wl, n=24, seed=3)
+    sub = case.host_subproblem(seqs)
+    out = _decode(case, partition_size=16)
+    assert int(case.status.item()) == 0
+    compare(out_f64(out)[seqs], oracle_step(sub, cfg, do_copy=False, do_write=False), "f16", "8192 sequences")
