@@ -5,8 +5,10 @@
 One step is one layer's decode step of the named workload, through the
 library's C ABI: copy-on-write block copies (workloads that have them), the
 cache write of each sequence's new token, then paged decode attention.
-Inputs are seeded synthetic tensors resident in HBM; L2 is flushed (a
-256 MiB write) before every timed step, outside the step's events.
+Inputs are seeded synthetic tensors resident in HBM; L2 is flushed before
+every timed step, outside the step's events: a 256 MiB write, then a 256 MiB
+read of another buffer, so that the write's dirty lines are written back
+during the flush (the decode after a write-only flush is reported too).
 
 Printed (rank 0, one JSON line): KV-read GB/s of the whole step (``value``),
 % of the measured HBM peak, sequences/s, the decode launch's roofline
@@ -207,7 +209,8 @@ class ClockSampler:
 # workload on the device
 # ---------------------------------------------------------------------------
 class DeviceWorkload:
-    def __init__(self, name: str, seed: int, partition_size: int | None = None, placement: str | None = None):
+    def __init__(self, name: str, seed: int, partition_size: int | None = None, placement: str | None = None,
+                 block_size: int | None = None):
         import torch
 
         import paged_kv_cache_362_b200 as pa
@@ -215,6 +218,10 @@ class DeviceWorkload:
 
         self.pa = pa
         self.cfg = get_config(name)
+        if block_size is not None and block_size != self.cfg.block_size:
+            # the same sequences in blocks of another size; the pool keeps its token capacity
+            self.cfg = get_config(name, block_size=block_size,
+                                  num_blocks=self.cfg.num_blocks * self.cfg.block_size // block_size)
         self.wl = build_workload(self.cfg, seed=seed, placement=placement)
         self.P = self.cfg.partition_size if partition_size is None else partition_size
         dev = torch.device("cuda")
@@ -252,12 +259,13 @@ class DeviceWorkload:
 def unique_kv_bytes(wl) -> int:
     """K/V bytes of the distinct physical blocks a decode step reads (shared blocks once)."""
     c = wl.cfg
+    bs = c.block_size
     seen = {}
     for b in range(wl.num_seqs):
         n = int(wl.context_lens[b])
-        for j in range(-(-n // 16)):
+        for j in range(-(-n // bs)):
             blk = int(wl.block_tables[b, j])
-            seen[blk] = max(seen.get(blk, 0), min(16, n - 16 * j))
+            seen[blk] = max(seen.get(blk, 0), min(bs, n - bs * j))
     elt = {"f32": 4, "f16": 2, "bf16": 2}[c.dtype]
     return sum(seen.values()) * c.num_kv_heads * c.head_dim * 2 * elt
 
@@ -591,8 +599,18 @@ def main():
     if not torch.cuda.is_available():
         raise SystemExit("bench.py needs a CUDA device")
     peak, peak_kind = measured_hbm_peak()
+    # L2 flush before every timed step: write 256 MiB (twice the L2), then read
+    # another 256 MiB so that the write's dirty lines are written back during
+    # the flush rather than during the step that follows
     flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
-    flush = lambda: flush_buf.zero_()
+    flush_rd = torch.ones(64 << 20, dtype=torch.float32, device="cuda")
+    flush_acc = torch.zeros((), dtype=torch.float32, device="cuda")
+
+    def flush():
+        flush_buf.zero_()
+        torch.sum(flush_rd, dim=0, out=flush_acc)
+
+    flush_write_only = lambda: flush_buf.zero_()
     use_graph = not args.no_graph
 
     w = DeviceWorkload(args.workload, args.seed + rank, args.partition_size)
@@ -611,6 +629,10 @@ def main():
 
     e2e_ms, h2d, d2h = time_e2e(w, max(50, args.steps // 10), args.warmup, flush)
     e2e = dist_max(float(np.mean(e2e_ms)))
+    # the same decode after a write-only flush: the step then also pays for
+    # writing back up to an L2 of the flush's dirty lines
+    _, wo_dec = time_steps(w, max(50, args.steps // 10), args.warmup, flush_write_only, use_graph)
+    wo = dist_max(float(np.mean(wo_dec)))
 
     secondary = {}
     placement = {}
@@ -649,6 +671,32 @@ def main():
             placement[name] = {f"decode_ms_{shuf}": round(ms_s, 5), "decode_ms_identity": round(ms_i, 5),
                                "overhead_pct": round(100 * (ms_s / ms_i - 1), 2)}
 
+    # the block-size trade-off: the same sequences in 8-, 16- and 32-token blocks
+    sweep = {}
+    if not args.no_secondary:
+        for name in ("churned256", "long32k"):
+            rows = {}
+            for bs in (8, 16, 32):
+                bw = DeviceWorkload(name, args.seed + rank, block_size=bs)
+                _, b_dec = time_steps(bw, max(50, args.steps // 10), args.warmup, flush, use_graph)
+                bd = dist_max(float(np.mean(b_dec)))
+                cl = bw.wl.context_lens.astype(np.int64)
+                nblk = -(-cl // bs)
+                rows[str(bs)] = {
+                    "decode_ms": round(bd, 5), "decode_ms_p10_p50_p90": pct3(b_dec),
+                    "decode_kv_gbs": round(bw.kv_bytes / (bd * 1e-3) / 1e9, 1),
+                    "decode_frac_of_peak": round(bw.kv_bytes / (bd * 1e-3) / 1e9 / peak, 4),
+                    "blocks": int(nblk.sum()), "block_table_bytes": int(nblk.sum()) * 4,
+                    "wasted_slots": int((nblk * bs - cl).sum()),
+                    "wasted_pct": round(100 * float((nblk * bs - cl).sum()) / float((nblk * bs).sum()), 2),
+                    "decode_launches": bw.decode_launches,
+                }
+                if int(bw.status.item()) != 0:
+                    raise SystemExit(f"device status {int(bw.status.item())} at block size {bs}")
+                del bw
+                torch.cuda.empty_cache()
+            sweep[name] = rows
+
     cpu = None
     if rank == 0 and world == 1:
         gbs, sps, threads, sample, _ = oracle_sample_throughput(args.workload, args.seed, args.cpu_budget,
@@ -669,11 +717,13 @@ def main():
             "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": c.dtype, "data": "synthetic",
             "config": {"workload": c.name, "num_seqs": w.wl.num_seqs, "num_heads": c.num_heads,
-                       "num_kv_heads": c.num_kv_heads, "head_dim": c.head_dim, "block_size": 16,
+                       "num_kv_heads": c.num_kv_heads, "head_dim": c.head_dim, "block_size": c.block_size,
                        "num_blocks": c.num_blocks, "mean_context": float(np.mean(w.wl.context_lens)),
                        "max_context": w.max_ctx, "partition_size": w.P or "auto",
                        "parallelism": f"replicas x{world}",
-                       "l2": "flushed before every timed step (256 MiB write, outside the step's events)",
+                       "l2": "flushed before every timed step, outside its events: a 256 MiB write, then a "
+                             "256 MiB read of another buffer (so the flush's dirty lines are written back before "
+                             "the step)",
                        "cuda_graph": use_graph,
                        "step": ("copy_blocks + " if w.has_copy else "") + "reshape_and_cache + decode"},
             "pct_of_peak": round(100 * value / world / peak, 2),
@@ -684,12 +734,16 @@ def main():
                          "kernel": f"pa_decode call ({w.decode_launches} launch(es): [plan +] attention "
                                    "[+ reduce]), timed together; traffic = DRAM bytes of the attention kernel "
                                    "from profiles/traffic.json",
-                         "peak_kind": peak_kind},
+                         "peak_kind": peak_kind,
+                         "after_write_only_flush": {"decode_ms": round(wo, 5),
+                                                    "achieved": round(w.kv_bytes / (wo * 1e-3) / 1e9, 1),
+                                                    "frac": round(w.kv_bytes / (wo * 1e-3) / 1e9 / peak, 4)}},
             "cpu_baseline": cpu,
             "e2e": {"value": round(total_bytes / (e2e * 1e-3) / 1e9, 2), "unit": "GB/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e, 5)},
             "step_ms_p10_p50_p90": pct3(step_ms), "decode_ms_p10_p50_p90": pct3(dec_ms),
             "placement_overhead": placement,
+            "block_size_sweep": sweep,
             "block_manager": bm_step,
             "swap": swap,
             "prefill": prefill_res,

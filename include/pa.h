@@ -2,8 +2,8 @@
  * pa.h -- C ABI of the B200 (sm_100a) paged KV-cache decode-attention library.
  *
  * What the library implements is the hot path the pages describe:
- *   - the KV cache lives in a shared pool of fixed-size physical blocks of 16
- *     tokens, and each request reaches its blocks through a block table that
+ *   - the KV cache lives in a shared pool of fixed-size physical blocks (16
+ *     tokens by default), and each request reaches its blocks through a block table that
  *     maps logical block index -> physical block index ("PagedAttention"
  *     digest, section "PagedAttention in one picture");
  *   - each decoded token appends one K/V entry inside the current logical
@@ -33,12 +33,18 @@
  *    `*status` when `status` is not NULL.  `status` is a device int32 the
  *    caller zeroes and reads back after synchronising.  Kernels never trap.
  *  * Dtypes: q, K, V, out and the appended key/value share one element type.
- *  * Pool layout (both key_cache and value_cache):
- *        [num_blocks][num_kv_heads][block_size = 16][head_dim]   row-major,
- *    so one (block, KV head) tile of 16 tokens is a contiguous run of
- *    16 * head_dim elements.  Slot s of the pool is block s / 16, offset s % 16.
+ *  * Pool layout (both key_cache and value_cache), with BS = block_size:
+ *        [num_blocks][num_kv_heads][BS][head_dim]   row-major,
+ *    so one (block, KV head) tile of BS tokens is a contiguous run of
+ *    BS * head_dim elements.  Slot s of the pool is block s / BS, offset s % BS.
  *  * GQA: query head h uses KV head h / (num_heads / num_kv_heads).
- *  * Supported: block_size 16; head_dim 64 or 128; float32, float16, bfloat16.
+ *  * Supported: block_size 8, 16 or 32 (pa_prefill: 16); head_dim 64 or 128;
+ *    float32, float16, bfloat16.  16 is the pages' default: smaller blocks
+ *    waste fewer slots in a sequence's last block but need longer block
+ *    tables and more, smaller reads ("PagedAttention" digest,
+ *    "Misconceptions").
+ *  * Slots of a block past a sequence's context may hold anything (NaN bit
+ *    patterns included): the attention calls never let them reach a result.
  */
 #ifndef PA_H_
 #define PA_H_
@@ -57,7 +63,7 @@ typedef struct CUstream_st* pa_stream_t;
 typedef enum {
     PA_OK = 0,
     PA_ERR_INVALID_ARG = 1,   /* null pointer, negative size, misaligned buffer, small workspace */
-    PA_ERR_UNSUPPORTED = 2,   /* valid but not implemented: block_size != 16, head_dim, dtype */
+    PA_ERR_UNSUPPORTED = 2,   /* valid but not implemented: block_size, head_dim, dtype */
     PA_ERR_OUT_OF_RANGE = 4,  /* device: block id, slot or context length outside its range */
     PA_ERR_CUDA = 8,          /* a CUDA launch or query failed */
     PA_ERR_TIMEOUT = 16,      /* device: a bounded wait inside a kernel gave up */
@@ -70,9 +76,9 @@ typedef enum { PA_F32 = 0, PA_F16 = 1, PA_BF16 = 2 } pa_dtype;
  * pa_reshape_and_cache -- write the K/V of newly decoded tokens into the pool.
  *
  * For every token t < num_tokens with s = slot_mapping[t] >= 0:
- *     key_cache  [s / 16][h][s % 16][:] = key  [t][h][:]   for all h < num_kv_heads
- *     value_cache[s / 16][h][s % 16][:] = value[t][h][:]
- * A negative slot is padding and writes nothing.  A slot >= num_blocks * 16
+ *     key_cache  [s / BS][h][s % BS][:] = key  [t][h][:]   for all h < num_kv_heads
+ *     value_cache[s / BS][h][s % BS][:] = value[t][h][:]
+ * A negative slot is padding and writes nothing.  A slot >= num_blocks * BS
  * writes nothing and sets PA_ERR_OUT_OF_RANGE in *status.  The copy is
  * bit-exact.  Distinct tokens must name distinct slots (otherwise which one
  * lands is unspecified).
@@ -106,8 +112,8 @@ size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_heads, int32_t num
  *
  * For every sequence b < num_seqs and query head h < num_heads, with
  * n = context_lens[b] and g = h / (num_heads / num_kv_heads):
- *     K_i = key_cache  [block_tables[b][i / 16]][g][i % 16][:]   (i < n)
- *     V_i = value_cache[block_tables[b][i / 16]][g][i % 16][:]
+ *     K_i = key_cache  [block_tables[b][i / BS]][g][i % BS][:]   (i < n)
+ *     V_i = value_cache[block_tables[b][i / BS]][g][i % BS][:]
  *     out[b][h][:] = sum_i softmax_i(scale * q[b][h][:] . K_i) V_i
  * computed in fp32 from the stored values and rounded to the element type.
  * n = 0 gives a zero row.  The context is split into partitions of
@@ -120,11 +126,14 @@ size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_heads, int32_t num
  *   key_cache,
  *   value_cache         pools, layout above
  *   block_tables        int32 [num_seqs][max_blocks_per_seq]; only the first
- *                       ceil(n / 16) entries of row b are read, each must be
- *                       in [0, num_blocks) (else PA_ERR_OUT_OF_RANGE and the
- *                       block is skipped)
+ *                       ceil(n / BS) entries of row b are read, each must be
+ *                       in [0, num_blocks): else PA_ERR_OUT_OF_RANGE, and the
+ *                       16-token tile holding the bad block contributes
+ *                       nothing (with 8-token blocks that includes the other
+ *                       block of the tile; with 32-token blocks, both tiles
+ *                       of the block)
  *   context_lens        int32 [num_seqs]; a value outside
- *                       [0, min(max_context_len, max_blocks_per_seq * 16)] is
+ *                       [0, min(max_context_len, max_blocks_per_seq * BS)] is
  *                       clamped into that range and sets PA_ERR_OUT_OF_RANGE
  *   max_context_len     host-side upper bound of context_lens (sizes the split)
  *   partition_size      tokens per partition: 0 = automatic, else a multiple
@@ -160,7 +169,7 @@ int32_t pa_decode_launch_count(int32_t num_seqs, int32_t num_heads, int32_t num_
  *
  * For each pair k < num_pairs with (src, dst) = (block_pairs[2k], block_pairs[2k+1]):
  *     key_cache[dst] = key_cache[src];  value_cache[dst] = value_cache[src]
- * (all num_kv_heads * 16 * head_dim elements; bit-exact).  A pair with an id
+ * (all num_kv_heads * BS * head_dim elements; bit-exact).  A pair with an id
  * outside [0, num_blocks) is skipped and sets PA_ERR_OUT_OF_RANGE.  No dst
  * may repeat and no dst may also be a src in the same call (that would be a
  * write/write or read/write race); the result is then unspecified.
@@ -194,8 +203,8 @@ pa_status pa_copy_blocks(void* key_cache, void* value_cache, const int64_t* bloc
  *   context_lens    int32 [num_seqs], device; n < L or n > max_blocks_per_seq * 16
  *                   sets PA_ERR_OUT_OF_RANGE and leaves that sequence's rows unwritten
  *   max_query_len   host-side upper bound of the L (sizes the grid)
- * Supported: float16 and bfloat16, head_dim 64 or 128, at most 16 query heads
- * per KV head (PA_ERR_UNSUPPORTED otherwise).  No workspace.
+ * Supported: block_size 16, float16 and bfloat16, head_dim 64 or 128, at most
+ * 16 query heads per KV head (PA_ERR_UNSUPPORTED otherwise).  No workspace.
  */
 pa_status pa_prefill(void* out, const void* q, const void* key_cache, const void* value_cache,
                      const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* query_start,
@@ -213,7 +222,7 @@ pa_status pa_prefill(void* out, const void* q, const void* key_cache, const void
  *
  * For each pair k < num_pairs with (s, d) = (block_pairs[2k], block_pairs[2k+1]):
  *     dst_key_cache[d] = src_key_cache[s];  dst_value_cache[d] = src_value_cache[s]
- * (all num_kv_heads * 16 * head_dim elements; bit-exact).  Either pool may be
+ * (all num_kv_heads * BS * head_dim elements; bit-exact).  Either pool may be
  * pinned host memory that the device addresses directly (cudaHostAlloc or
  * cudaMallocHost memory, which unified addressing maps at the same pointer):
  * swapping out is device -> host, swapping in host -> device.  A pair with an

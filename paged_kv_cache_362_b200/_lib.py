@@ -129,17 +129,17 @@ def _ptr(t):
 def reshape_and_cache(key, value, key_cache, value_cache, slot_mapping, status=None, stream=None):
     """Write each token's K/V into its slot (pa_reshape_and_cache).
 
-    key, value [T, Hkv, D]; key_cache, value_cache [NB, Hkv, 16, D];
+    key, value [T, Hkv, D]; key_cache, value_cache [NB, Hkv, block_size, D] (block_size 8, 16 or 32);
     slot_mapping int64 [T] (negative = skip); status: optional int32 device tensor.
     """
     assert key.is_contiguous() and value.is_contiguous() and key_cache.is_contiguous() and value_cache.is_contiguous()
     assert slot_mapping.dtype.is_floating_point is False and slot_mapping.element_size() == 8
     T, Hkv, D = key.shape
-    NB = key_cache.shape[0]
-    assert value.shape == key.shape and key_cache.shape == (NB, Hkv, BLOCK_SIZE, D) == value_cache.shape
+    NB, bs = key_cache.shape[0], key_cache.shape[2]
+    assert value.shape == key.shape and key_cache.shape == (NB, Hkv, bs, D) == value_cache.shape
     assert key.dtype == value.dtype == key_cache.dtype == value_cache.dtype
     _check(LIB.pa_reshape_and_cache(_ptr(key), _ptr(value), _ptr(key_cache), _ptr(value_cache), _ptr(slot_mapping),
-                                    T, NB, Hkv, D, BLOCK_SIZE, _dtype_code(key), _ptr(status), _stream(stream)),
+                                    T, NB, Hkv, D, bs, _dtype_code(key), _ptr(status), _stream(stream)),
            "pa_reshape_and_cache")
 
 
@@ -172,17 +172,20 @@ def make_workspace(num_seqs, num_heads, num_kv_heads, head_dim, max_context_len,
 
 def decode(out, q, key_cache, value_cache, block_tables, context_lens, scale, max_context_len, workspace,
            partition_size=0, status=None, stream=None):
-    """One decode step of paged attention (pa_decode); writes ``out`` [B, Hq, D]."""
+    """One decode step of paged attention (pa_decode); writes ``out`` [B, Hq, D].
+
+    The block size (8, 16 or 32 tokens) is the pools' dimension 2.
+    """
     B, Hq, D = q.shape
-    NB, Hkv = key_cache.shape[0], key_cache.shape[1]
+    NB, Hkv, bs = key_cache.shape[0], key_cache.shape[1], key_cache.shape[2]
     assert out.shape == q.shape and out.dtype == q.dtype == key_cache.dtype == value_cache.dtype
-    assert key_cache.shape == (NB, Hkv, BLOCK_SIZE, D) == value_cache.shape
+    assert key_cache.shape == (NB, Hkv, bs, D) == value_cache.shape
     assert block_tables.dtype.itemsize == 4 and context_lens.dtype.itemsize == 4
     assert block_tables.shape[0] == B and context_lens.shape == (B,)
     for t in (out, q, key_cache, value_cache, block_tables, context_lens, workspace):
         assert t.is_contiguous()
     _check(LIB.pa_decode(_ptr(out), _ptr(q), _ptr(key_cache), _ptr(value_cache), _ptr(block_tables),
-                         block_tables.shape[1], _ptr(context_lens), B, Hq, Hkv, D, BLOCK_SIZE, NB, float(scale),
+                         block_tables.shape[1], _ptr(context_lens), B, Hq, Hkv, D, bs, NB, float(scale),
                          int(max_context_len), int(partition_size), _ptr(workspace),
                          workspace.numel() * workspace.element_size(), _dtype_code(q), _ptr(status),
                          _stream(stream)),
@@ -197,15 +200,16 @@ def prefill(out, q, key_cache, value_cache, block_tables, query_start, context_l
     already written with reshape_and_cache).
     """
     T, Hq, D = q.shape
-    NB, Hkv = key_cache.shape[0], key_cache.shape[1]
+    NB, Hkv, bs = key_cache.shape[0], key_cache.shape[1], key_cache.shape[2]
     assert out.shape == q.shape and out.dtype == q.dtype == key_cache.dtype == value_cache.dtype
+    assert key_cache.shape == value_cache.shape
     assert block_tables.dtype.itemsize == 4 and context_lens.dtype.itemsize == 4 and query_start.dtype.itemsize == 4
     B = context_lens.shape[0]
     assert query_start.shape == (B + 1,) and block_tables.shape[0] == B
     for t in (out, q, key_cache, value_cache, block_tables, query_start, context_lens):
         assert t.is_contiguous()
     _check(LIB.pa_prefill(_ptr(out), _ptr(q), _ptr(key_cache), _ptr(value_cache), _ptr(block_tables),
-                          block_tables.shape[1], _ptr(query_start), _ptr(context_lens), B, Hq, Hkv, D, BLOCK_SIZE, NB,
+                          block_tables.shape[1], _ptr(query_start), _ptr(context_lens), B, Hq, Hkv, D, bs, NB,
                           float(scale), int(max_query_len), _dtype_code(q), _ptr(status), _stream(stream)),
            "pa_prefill")
 

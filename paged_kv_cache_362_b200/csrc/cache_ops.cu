@@ -16,11 +16,11 @@
 
 namespace pa {
 
-// key/value [T, Hkv, D] -> pools [NB, Hkv, 16, D];  chunk = 16 bytes
+// key/value [T, Hkv, D] -> pools [NB, Hkv, block_size, D];  chunk = 16 bytes
 __global__ void __launch_bounds__(256) reshape_and_cache_kernel(
     const uint4* __restrict__ key, const uint4* __restrict__ value, uint4* __restrict__ key_cache,
     uint4* __restrict__ value_cache, const int64_t* __restrict__ slot_mapping, int64_t num_tokens,
-    int num_kv_heads, int chunks_per_head, int64_t num_slots, int32_t* status) {
+    int num_kv_heads, int chunks_per_head, int block_size, int64_t num_slots, int32_t* status) {
     griddep_launch_dependents();
     griddep_wait();
     const int64_t chunks_per_token = (int64_t)num_kv_heads * chunks_per_head;
@@ -35,9 +35,9 @@ __global__ void __launch_bounds__(256) reshape_and_cache_kernel(
             if (r == 0) set_status(status, PA_ERR_OUT_OF_RANGE);
             continue;
         }
-        const int64_t blk = s / kBlockSize, off = s % kBlockSize;
+        const int64_t blk = s / block_size, off = s % block_size;
         const int64_t h = r / chunks_per_head, c = r - h * chunks_per_head;
-        const int64_t dst = ((blk * num_kv_heads + h) * kBlockSize + off) * chunks_per_head + c;
+        const int64_t dst = ((blk * num_kv_heads + h) * block_size + off) * chunks_per_head + c;
         key_cache[dst] = key[i];
         value_cache[dst] = value[i];
     }
@@ -90,7 +90,8 @@ __global__ void __launch_bounds__(256) swap_blocks_kernel(const uint4* __restric
 
 cudaError_t launch_reshape_and_cache(const void* key, const void* value, void* key_cache, void* value_cache,
                                      const int64_t* slot_mapping, int64_t num_tokens, int32_t num_blocks,
-                                     int32_t num_kv_heads, int32_t head_dim, int elt_bytes, int32_t* status,
+                                     int32_t num_kv_heads, int32_t head_dim, int32_t block_size, int elt_bytes,
+                                     int32_t* status,
                                      cudaStream_t stream) {
     if (num_tokens == 0) return cudaSuccess;
     DeviceInfo dev;
@@ -104,14 +105,14 @@ cudaError_t launch_reshape_and_cache(const void* key, const void* value, void* k
     return launch_pdl(reshape_and_cache_kernel, dim3(grid), dim3(256), 0, stream,
                       static_cast<const uint4*>(key), static_cast<const uint4*>(value),
                       static_cast<uint4*>(key_cache), static_cast<uint4*>(value_cache), slot_mapping, num_tokens,
-                      (int)num_kv_heads, chunks_per_head, (int64_t)num_blocks * kBlockSize, status);
+                      (int)num_kv_heads, chunks_per_head, (int)block_size, (int64_t)num_blocks * block_size, status);
 }
 
 cudaError_t launch_copy_blocks(void* key_cache, void* value_cache, const int64_t* block_pairs, int32_t num_pairs,
-                               int32_t num_blocks, int32_t num_kv_heads, int32_t head_dim, int elt_bytes,
-                               int32_t* status, cudaStream_t stream) {
+                               int32_t num_blocks, int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                               int elt_bytes, int32_t* status, cudaStream_t stream) {
     if (num_pairs == 0) return cudaSuccess;
-    const int64_t block_chunks = (int64_t)num_kv_heads * kBlockSize * head_dim * elt_bytes / 16;
+    const int64_t block_chunks = (int64_t)num_kv_heads * block_size * head_dim * elt_bytes / 16;
     return launch_pdl(copy_blocks_kernel, dim3(num_pairs, 2), dim3(256), 0, stream,
                       static_cast<uint4*>(key_cache), static_cast<uint4*>(value_cache), block_pairs, (int)num_pairs,
                       (int64_t)num_blocks, block_chunks, status);
@@ -119,10 +120,10 @@ cudaError_t launch_copy_blocks(void* key_cache, void* value_cache, const int64_t
 
 cudaError_t launch_swap_blocks(const void* src_key, const void* src_value, void* dst_key, void* dst_value,
                                const int64_t* block_pairs, int32_t num_pairs, int32_t src_num_blocks,
-                               int32_t dst_num_blocks, int32_t num_kv_heads, int32_t head_dim, int elt_bytes,
-                               int32_t* status, cudaStream_t stream) {
+                               int32_t dst_num_blocks, int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                               int elt_bytes, int32_t* status, cudaStream_t stream) {
     if (num_pairs == 0) return cudaSuccess;
-    const int64_t block_chunks = (int64_t)num_kv_heads * kBlockSize * head_dim * elt_bytes / 16;
+    const int64_t block_chunks = (int64_t)num_kv_heads * block_size * head_dim * elt_bytes / 16;
     return launch_pdl(swap_blocks_kernel, dim3(num_pairs, 2), dim3(256), 0, stream,
                       static_cast<const uint4*>(src_key), static_cast<const uint4*>(src_value),
                       static_cast<uint4*>(dst_key), static_cast<uint4*>(dst_value), block_pairs, (int)num_pairs,

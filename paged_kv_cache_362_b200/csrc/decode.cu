@@ -21,9 +21,10 @@
 //                c, 2C-1-c, 2C+c, ... (snake order over the sorted list, which
 //                balances the load).  Per CTA:
 //                  * a producer warp streams, for each item, the Q rows of the
-//                    GQA group (1-D bulk copy) and every (block, KV head) tile
-//                    of K and of V (16 tokens x head_dim, contiguous 4 KB at
-//                    D = 128) with 2-D TMA tensor copies into a ring of
+//                    GQA group (1-D bulk copy) and every 16-token tile of K and
+//                    of V of the KV head (one 16-token block, contiguous 4 KB at
+//                    D = 128; half of a 32-token block; or two 8-token blocks)
+//                    with 2-D TMA tensor copies into a ring of
 //                    shared-memory stages, 128-byte swizzled, tracked by
 //                    mbarriers, evict-first in L2; work-list entries and table
 //                    rows are prefetched two items ahead with cp.async;
@@ -171,7 +172,7 @@ __global__ void __launch_bounds__(kThreads) decode_plan_kernel(const DecodeParam
     __syncthreads();
     // pass 1: histogram of item keys
     for (int b = tid; b < B; b += kThreads) {
-        const SeqParts sp = seq_parts_fast(ceil_div_i(load_ctx(p, b, true), kBlockSize), K.PB, p.equal_split);
+        const SeqParts sp = seq_parts_fast(ceil_div_i(load_ctx(p, b, true), kChunk), K.PB, p.equal_split);
         int kb, ks;
         seq_keys(K, sp, kb, ks);
         if (kb != kNoKey) atomicAdd(&cnt[kb], sp.nbig * Hkv);
@@ -190,7 +191,7 @@ __global__ void __launch_bounds__(kThreads) decode_plan_kernel(const DecodeParam
         int ctx = 0, r = 0, n = 0, ob = 0, os = 0;
         if (b < B) {
             ctx = load_ctx(p, b, false);
-            const SeqParts sp = seq_parts_fast(ceil_div_i(ctx, kBlockSize), K.PB, p.equal_split);
+            const SeqParts sp = seq_parts_fast(ceil_div_i(ctx, kChunk), K.PB, p.equal_split);
             int kb, ks;
             seq_keys(K, sp, kb, ks);
             r = sp.nbig;
@@ -221,7 +222,7 @@ __device__ __forceinline__ ItemGeom item_geom(const DecodeParams& p, int4 it) {
     m.p = it.y >> 8;
     m.g = it.y & 255;
     m.ctx = it.z;
-    const SeqParts sp = seq_parts_fast(ceil_div_i(m.ctx, kBlockSize), p.part_blocks, p.equal_split);
+    const SeqParts sp = seq_parts_fast(ceil_div_i(m.ctx, kChunk), p.part_blocks, p.equal_split);
     m.j0 = sp.start(m.p);
     m.nblk = sp.len(m.p);
     m.nparts = sp.n;
@@ -321,7 +322,8 @@ struct ItemMeta {
 // work-list entry and table row of one item, prefetched by the producer
 struct DescSlot {
     int4 e;
-    int bt[kMaxPartBlocks];
+    int bt[kMaxPartBlocks];    // per chunk: its block (8-token blocks: the first of its two)
+    int bt2[kMaxPartBlocks];   // 8-token blocks: the chunk's second block, if the context reaches it
     int rank;      // position in the work list
     int pad[3];
 };
@@ -360,7 +362,7 @@ __device__ void plan_own_items(const DecodeParams& p, int* scratch, int4* own, i
     const bool report = blockIdx.x == 0;
     for (int b = tid; b < B; b += nthr) {
         const int c = clamp_ctx(p, s_ctx[b], report);
-        const SeqParts sp = seq_parts_fast(ceil_div_i(c, kBlockSize), K.PB, p.equal_split);
+        const SeqParts sp = seq_parts_fast(ceil_div_i(c, kChunk), K.PB, p.equal_split);
         int kb, ks;
         seq_keys(K, sp, kb, ks);
         s_ctx[b] = c;
@@ -430,8 +432,8 @@ __device__ void plan_own_items(const DecodeParams& p, int* scratch, int4* own, i
 template <int D, int NT, int NCW, int STAGES>
 struct TcCfg {
     static constexpr int kBoxes = D / 64;                    // 64-element (128 B) boxes per tile row
-    static constexpr int kBoxBytes = kBlockSize * 128;       // 2 KB
-    static constexpr int kTileBytes = kBlockSize * D * 2;    // one K or V tile
+    static constexpr int kBoxBytes = kChunk * 128;           // 2 KB: 16 rows x 128 B
+    static constexpr int kTileBytes = kChunk * D * 2;        // one K or V tile (16 tokens)
     static constexpr int kStageBytes = 2 * kTileBytes;
     static constexpr int kISlots = NCW == 1 ? 2 : 4;         // item metadata / Q ring
     static constexpr int kDSlots = 4;                        // descriptor prefetch ring
@@ -609,9 +611,23 @@ __global__ void __launch_bounds__(TcCfg<D, NT, NCW, STAGES>::kThreads, TcCfg<D, 
             const int r = dsc[it % C::kDSlots].rank;
             if (r >= n_items) return;
             const ItemGeom m = item_geom(p, dsc[it % C::kDSlots].e);
-            if (lane < m.nblk)
-                cp_async_4(smem_u32(&dsc[it % C::kDSlots].bt[lane]),
-                           p.block_tables + (size_t)m.b * p.max_blocks_per_seq + m.j0 + lane);
+            if (lane < m.nblk) {
+                // chunk c is block c (16-token blocks), the half (c & 1) of block
+                // c / 2 (32-token blocks) or blocks 2c and 2c + 1 (8-token blocks,
+                // the second only where the context reaches it)
+                DescSlot& ds = dsc[it % C::kDSlots];
+                const int32_t* row = p.block_tables + (size_t)m.b * p.max_blocks_per_seq;
+                const int c = m.j0 + lane;
+                if (p.block_size == kChunk) {
+                    cp_async_4(smem_u32(&ds.bt[lane]), row + c);
+                } else if (p.block_size > kChunk) {
+                    cp_async_4(smem_u32(&ds.bt[lane]), row + (c >> 1));
+                } else {
+                    cp_async_4(smem_u32(&ds.bt[lane]), row + 2 * c);
+                    if (2 * c + 1 < ceil_div_i(m.ctx, p.block_size))
+                        cp_async_4(smem_u32(&ds.bt2[lane]), row + 2 * c + 1);
+                }
+            }
         };
         // Static schedule: CTA c takes ranks c, 2C-1-c, 2C+c, ... of the
         // largest-first list (snake order), which balances the load without a
@@ -716,21 +732,51 @@ __global__ void __launch_bounds__(TcCfg<D, NT, NCW, STAGES>::kThreads, TcCfg<D, 
                     stage_bad[s] = 1;
                     mbar_arrive(&full[s]);
                 }
+                const int bs = p.block_size;
+                const int nphys = ceil_div_i(m.ctx, bs);   // blocks the context occupies
                 for (int j = 0; j < m.nblk && okw; ++j, ++stage) {
+                    const int c = m.j0 + j;
                     const int blk = d.bt[j];
+                    // 8-token blocks: the chunk's second block, absent past the context
+                    const bool has1 = bs < kChunk && 2 * c + 1 < nphys;
+                    const int blk1 = has1 ? d.bt2[j] : 0;
                     const int s = stage % STAGES;
                     if (!mbar_wait(&empty[s], ((stage / STAGES) & 1) ^ 1)) { okw = 0; break; }
-                    if (blk >= 0 && blk < p.num_blocks) {
+                    if (blk >= 0 && blk < p.num_blocks && blk1 >= 0 && blk1 < p.num_blocks) {
                         stage_bad[s] = 0;
-                        mbar_arrive_expect_tx(&full[s], C::kStageBytes);
-                        const int y = (blk * p.num_kv_heads + m.g) * kBlockSize;
                         const uint32_t kdst = smem_u32(stages + s * C::kStageBytes);
+                        if (bs >= kChunk) {
+                            // one 16-row box per 64 columns: the block, or its half c & 1
+                            mbar_arrive_expect_tx(&full[s], C::kStageBytes);
+                            const int y = (blk * p.num_kv_heads + m.g) * bs + (bs > kChunk ? (c & 1) * kChunk : 0);
 #pragma unroll
-                        for (int h = 0; h < C::kBoxes; ++h)
-                            tma_load_2d(kdst + h * C::kBoxBytes, &tmK, h * 64, y, &full[s], pol);
+                            for (int h = 0; h < C::kBoxes; ++h)
+                                tma_load_2d(kdst + h * C::kBoxBytes, &tmK, h * 64, y, &full[s], pol);
 #pragma unroll
-                        for (int h = 0; h < C::kBoxes; ++h)
-                            tma_load_2d(kdst + C::kTileBytes + h * C::kBoxBytes, &tmV, h * 64, y, &full[s], pol);
+                            for (int h = 0; h < C::kBoxes; ++h)
+                                tma_load_2d(kdst + C::kTileBytes + h * C::kBoxBytes, &tmV, h * 64, y, &full[s],
+                                            pol);
+                        } else {
+                            // 8-row boxes: rows 0-7 of the tile from the first block,
+                            // rows 8-15 (1 KB further, the next 128-byte swizzle atom,
+                            // so the tile's layout is that of one 16-row box) from the
+                            // second; past the context, rows 8-15 keep stale data that
+                            // the consumer masks (K) and clears (V)
+                            mbar_arrive_expect_tx(&full[s], has1 ? C::kStageBytes : C::kStageBytes / 2);
+                            const int y0 = blk * p.num_kv_heads + m.g, y1 = blk1 * p.num_kv_heads + m.g;
+#pragma unroll
+                            for (int h = 0; h < C::kBoxes; ++h) {
+                                tma_load_2d(kdst + h * C::kBoxBytes, &tmK, h * 64, y0 * bs, &full[s], pol);
+                                tma_load_2d(kdst + C::kTileBytes + h * C::kBoxBytes, &tmV, h * 64, y0 * bs,
+                                            &full[s], pol);
+                                if (has1) {
+                                    tma_load_2d(kdst + h * C::kBoxBytes + C::kBoxBytes / 2, &tmK, h * 64, y1 * bs,
+                                                &full[s], pol);
+                                    tma_load_2d(kdst + C::kTileBytes + h * C::kBoxBytes + C::kBoxBytes / 2, &tmV,
+                                                h * 64, y1 * bs, &full[s], pol);
+                                }
+                            }
+                        }
                     } else {
                         stage_bad[s] = 1;
                         set_status(p.status, PA_ERR_OUT_OF_RANGE);
@@ -947,7 +993,25 @@ __global__ void __launch_bounds__(TcCfg<D, NT, NCW, STAGES>::kThreads, TcCfg<D, 
             }
         };
         auto tile_of = [&](uint32_t n) { return smem_u32(stages + (n % STAGES) * C::kStageBytes); };
-        auto valid_of = [&](uint32_t n) { return min(kBlockSize, m.ctx - (m.j0 + (int)(n - stage_base)) * kBlockSize); };
+        auto valid_of = [&](uint32_t n) { return min(kChunk, m.ctx - (m.j0 + (int)(n - stage_base)) * kChunk); };
+        // The last chunk of a sequence is partly past the context.  Its rows
+        // there hold whatever the pool (or an earlier stage) held: the logits
+        // of those rows are masked, but a probability of 0 times a NaN in V
+        // is still NaN, so the V rows past the context are zeroed first.
+        // Returns whether it wrote (the stage then needs a proxy fence before
+        // the tensor copies refill it).
+        auto clear_v_tail = [&](uint32_t n) {
+            const int vl = valid_of(n);
+            if (vl >= kChunk) return false;
+            const uint32_t vt = tile_of(n) + C::kTileBytes;
+            const int per_box = (kChunk - vl) * 8;   // 16-byte pieces past row vl in one 128-byte-wide box
+            for (int i = lane; i < C::kBoxes * per_box; i += 32) {
+                const int bx = i / per_box, r = i - bx * per_box;
+                st_shared_zero16(vt + bx * C::kBoxBytes + vl * 128 + r * 16);
+            }
+            __syncwarp();
+            return true;
+        };
         auto wait_full = [&](uint32_t n) {
             if (!__all_sync(0xffffffffu, mbar_wait(&full[n % STAGES], (n / STAGES) & 1)) || *abort_flag) {
                 *abort_flag = 1;
@@ -968,12 +1032,15 @@ __global__ void __launch_bounds__(TcCfg<D, NT, NCW, STAGES>::kThreads, TcCfg<D, 
                 const bool bad0 = stage_bad[n % STAGES] != 0, bad1 = stage_bad[n1 % STAGES] != 0;
                 const uint32_t tb[2] = {tile_of(n), tile_of(n1)};
                 const int vl[2] = {valid_of(n), valid_of(n1)};
+                // only the later chunk of the pair can end a sequence
+                const bool cleared = !bad1 && clear_v_tail(n1);
                 if (!bad0 && !bad1) {
                     step(std::integral_constant<int, 2>{}, tb, vl);
                 } else {   // a block the producer skipped (bad id) holds no data
                     if (!bad0) step(std::integral_constant<int, 1>{}, tb, vl);
                     if (!bad1) step(std::integral_constant<int, 1>{}, tb + 1, vl + 1);
                 }
+                if (cleared) fence_proxy_async_shared();
                 __syncwarp();
                 if (lane == 0) {
                     mbar_arrive(&empty[n % STAGES]);
@@ -982,11 +1049,14 @@ __global__ void __launch_bounds__(TcCfg<D, NT, NCW, STAGES>::kThreads, TcCfg<D, 
                 n += 2 * NCW;
             } else {
                 if (!wait_full(n)) break;
+                bool cleared = false;
                 if (!stage_bad[n % STAGES]) {
+                    cleared = clear_v_tail(n);
                     const uint32_t tb[1] = {tile_of(n)};
                     const int vl[1] = {valid_of(n)};
                     step(std::integral_constant<int, 1>{}, tb, vl);
                 }
+                if (cleared) fence_proxy_async_shared();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&empty[n % STAGES]);
                 n += NCW;
@@ -1179,17 +1249,24 @@ __global__ void __launch_bounds__(NW * 32) decode_simt_kernel(const DecodeParams
             acc[e] = 0.f;
         }
         float mrun = kNegInf, lrun = 0.f;
+        const int bs = p.block_size;
+        const int32_t* row = p.block_tables + (size_t)m.b * p.max_blocks_per_seq;
         for (int j = 0; j < m.nblk; ++j) {
-            const int blk = p.block_tables[(size_t)m.b * p.max_blocks_per_seq + m.j0 + j];
-            if (blk < 0 || blk >= p.num_blocks) {
+            // the 16-token chunk's block (8-token blocks: its two blocks); a bad
+            // id drops the whole chunk, as in the tensor-core kernel
+            const int pos0 = (m.j0 + j) * kChunk;
+            const int ntok = min(kChunk, m.ctx - pos0);
+            const int blk0 = row[pos0 / bs];
+            const int blk1 = ntok > bs ? row[pos0 / bs + 1] : blk0;
+            if (blk0 < 0 || blk0 >= p.num_blocks || blk1 < 0 || blk1 >= p.num_blocks) {
                 if (lane == 0) set_status(p.status, PA_ERR_OUT_OF_RANGE);
                 continue;
             }
-            const int ntok = min(kBlockSize, m.ctx - (m.j0 + j) * kBlockSize);
-            const size_t tile = ((size_t)blk * p.num_kv_heads + m.g) * kBlockSize * D;
             for (int t = 0; t < ntok; ++t) {
-                const T* kr = kc + tile + (size_t)t * D + lane * E;
-                const T* vr = vc + tile + (size_t)t * D + lane * E;
+                const int pos = pos0 + t;
+                const size_t tok = (((size_t)(t < bs ? blk0 : blk1) * p.num_kv_heads + m.g) * bs + pos % bs) * D;
+                const T* kr = kc + tok + lane * E;
+                const T* vr = vc + tok + lane * E;
                 float dot = 0.f;
 #pragma unroll
                 for (int e = 0; e < E; ++e) dot += qv[e] * Elt<T>::to_f(kr[e]);
@@ -1240,7 +1317,7 @@ __global__ void __launch_bounds__(128) decode_reduce_kernel(const DecodeParams p
     for (long long r = blockIdx.x; r < n_rows; r += gridDim.x) {
         const int b = (int)(r / Hq), h = (int)(r % Hq);
         const int ctx = load_ctx(p, b, false);
-        const int nparts = max(1, ceil_div_i(ceil_div_i(ctx, kBlockSize), p.part_blocks));
+        const int nparts = max(1, ceil_div_i(ceil_div_i(ctx, kChunk), p.part_blocks));
         if (nparts == 1) continue;   // (uniform over the CTA)
         const size_t base = ((size_t)b * Hq + h) * p.max_parts;
         float M = kNegInf;
@@ -1333,14 +1410,15 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
 }
 
 // 2-D view of a pool: rows of head_dim elements, one row per (block, KV head, slot);
-// a box is 16 rows x 64 elements (128 B), 128-byte swizzled in shared memory.
+// a box is 16 rows (8 for 8-token blocks) x 64 elements (128 B), 128-byte
+// swizzled in shared memory.
 cudaError_t make_pool_map(CUtensorMap* map, const void* pool, pa_dtype dtype, int num_blocks, int num_kv_heads,
-                          int head_dim) {
+                          int head_dim, int block_size) {
     auto encode = get_encode_fn();
     if (!encode) return cudaErrorNotSupported;
-    const cuuint64_t dims[2] = {(cuuint64_t)head_dim, (cuuint64_t)num_blocks * num_kv_heads * kBlockSize};
+    const cuuint64_t dims[2] = {(cuuint64_t)head_dim, (cuuint64_t)num_blocks * num_kv_heads * block_size};
     const cuuint64_t strides[1] = {(cuuint64_t)head_dim * 2};
-    const cuuint32_t box[2] = {64, (cuuint32_t)kBlockSize};
+    const cuuint32_t box[2] = {64, (cuuint32_t)(block_size < kChunk ? block_size : kChunk)};
     const cuuint32_t estr[2] = {1, 1};
     const CUtensorMapDataType dt =
         dtype == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
@@ -1452,9 +1530,9 @@ template <typename T, int D, int NT, int NCW, int STAGES>
 cudaError_t launch_tc(const DecodeParams& p, pa_dtype dtype, cudaStream_t stream, int grid) {
     using Cfg = TcCfg<D, NT, NCW, STAGES>;
     CUtensorMap mk, mv;
-    cudaError_t e = make_pool_map(&mk, p.key_cache, dtype, p.num_blocks, p.num_kv_heads, D);
+    cudaError_t e = make_pool_map(&mk, p.key_cache, dtype, p.num_blocks, p.num_kv_heads, D, p.block_size);
     if (e != cudaSuccess) return e;
-    e = make_pool_map(&mv, p.value_cache, dtype, p.num_blocks, p.num_kv_heads, D);
+    e = make_pool_map(&mv, p.value_cache, dtype, p.num_blocks, p.num_kv_heads, D, p.block_size);
     if (e != cudaSuccess) return e;
     return launch_pdl(decode_tc_kernel<T, D, NT, NCW, STAGES>, dim3(grid), dim3(Cfg::kThreads), Cfg::kSmemBytes,
                       stream, p, mk, mv);

@@ -77,8 +77,7 @@ bool ws_layout(int64_t num_seqs, int64_t num_heads, int64_t num_kv_heads, int64_
                int64_t max_context_len, int64_t partition_size, WsLayout* w) {
     if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || max_context_len < 0) return false;
     if (partition_size == 0) partition_size = auto_partition_size(num_seqs, num_kv_heads, max_context_len);
-    if (partition_size < kBlockSize || partition_size > kBlockSize * kMaxPartBlocks ||
-        partition_size % kBlockSize != 0)
+    if (partition_size < kChunk || partition_size > kChunk * kMaxPartBlocks || partition_size % kChunk != 0)
         return false;
     const int64_t np = std::max<int64_t>(1, ceil_div64(max_context_len, partition_size));
     w->partition_size = (int)partition_size;
@@ -108,13 +107,13 @@ pa_status pa_reshape_and_cache(const void* key, const void* value, void* key_cac
                                int32_t* status, pa_stream_t stream) {
     if (num_tokens < 0 || num_blocks <= 0 || num_kv_heads <= 0 || head_dim <= 0) return PA_ERR_INVALID_ARG;
     if (!valid_dtype(dtype)) return PA_ERR_INVALID_ARG;
-    if (block_size != kBlockSize || (head_dim != 64 && head_dim != 128)) return PA_ERR_UNSUPPORTED;
+    if (!block_size_supported(block_size) || (head_dim != 64 && head_dim != 128)) return PA_ERR_UNSUPPORTED;
     if (num_tokens == 0) return PA_OK;
     if (!key || !value || !key_cache || !value_cache || !slot_mapping) return PA_ERR_INVALID_ARG;
     if (!aligned16(key) || !aligned16(value) || !aligned16(key_cache) || !aligned16(value_cache))
         return PA_ERR_INVALID_ARG;
     const cudaError_t e = launch_reshape_and_cache(key, value, key_cache, value_cache, slot_mapping, num_tokens,
-                                                   num_blocks, num_kv_heads, head_dim, elt_bytes(dtype), status,
+                                                   num_blocks, num_kv_heads, head_dim, block_size, elt_bytes(dtype), status,
                                                    reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
@@ -137,12 +136,12 @@ pa_status pa_decode(void* out, const void* q, const void* key_cache, const void*
         return PA_ERR_INVALID_ARG;
     if (!valid_dtype(dtype) || !std::isfinite(scale)) return PA_ERR_INVALID_ARG;
     if (num_heads % num_kv_heads != 0) return PA_ERR_INVALID_ARG;
-    if (block_size != kBlockSize || (head_dim != 64 && head_dim != 128) || num_kv_heads > 255)
+    if (!block_size_supported(block_size) || (head_dim != 64 && head_dim != 128) || num_kv_heads > 255)
         return PA_ERR_UNSUPPORTED;
     if (partition_size != 0 &&
-        (partition_size < kBlockSize || partition_size > kBlockSize * kMaxPartBlocks || partition_size % kBlockSize))
+        (partition_size < kChunk || partition_size > kChunk * kMaxPartBlocks || partition_size % kChunk))
         return PA_ERR_INVALID_ARG;
-    if ((int64_t)num_blocks * num_kv_heads * kBlockSize > INT32_MAX) return PA_ERR_UNSUPPORTED;
+    if ((int64_t)num_blocks * num_kv_heads * block_size > INT32_MAX) return PA_ERR_UNSUPPORTED;
     if (num_seqs == 0) return PA_OK;
     if (!out || !q || !key_cache || !value_cache || !block_tables || !context_lens || !workspace)
         return PA_ERR_INVALID_ARG;
@@ -170,8 +169,9 @@ pa_status pa_decode(void* out, const void* q, const void* key_cache, const void*
     p.group = num_heads / num_kv_heads;
     p.max_blocks_per_seq = max_blocks_per_seq;
     p.num_blocks = num_blocks;
-    p.ctx_cap = (int)std::min<int64_t>(max_context_len, (int64_t)max_blocks_per_seq * kBlockSize);
-    p.part_blocks = w.partition_size / kBlockSize;
+    p.block_size = block_size;
+    p.ctx_cap = (int)std::min<int64_t>(max_context_len, (int64_t)max_blocks_per_seq * block_size);
+    p.part_blocks = w.partition_size / kChunk;
     p.max_parts = w.max_parts;
     p.scale_log2 = scale * 1.4426950408889634f;  // log2(e)
     uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -198,7 +198,7 @@ int32_t pa_decode_launch_count(int32_t num_seqs, int32_t num_heads, int32_t num_
     p.num_kv_heads = num_kv_heads;
     p.head_dim = head_dim;
     p.group = num_heads / num_kv_heads;
-    p.part_blocks = w.partition_size / kBlockSize;
+    p.part_blocks = w.partition_size / kChunk;
     p.max_parts = w.max_parts;
     int n = 0;
     return decode_launch_count(p, dtype, &n) == cudaSuccess ? n : -1;
@@ -209,12 +209,12 @@ pa_status pa_copy_blocks(void* key_cache, void* value_cache, const int64_t* bloc
                          pa_dtype dtype, int32_t* status, pa_stream_t stream) {
     if (num_pairs < 0 || num_blocks <= 0 || num_kv_heads <= 0 || head_dim <= 0) return PA_ERR_INVALID_ARG;
     if (!valid_dtype(dtype)) return PA_ERR_INVALID_ARG;
-    if (block_size != kBlockSize || (head_dim != 64 && head_dim != 128)) return PA_ERR_UNSUPPORTED;
+    if (!block_size_supported(block_size) || (head_dim != 64 && head_dim != 128)) return PA_ERR_UNSUPPORTED;
     if (num_pairs == 0) return PA_OK;
     if (!key_cache || !value_cache || !block_pairs) return PA_ERR_INVALID_ARG;
     if (!aligned16(key_cache) || !aligned16(value_cache)) return PA_ERR_INVALID_ARG;
     const cudaError_t e = launch_copy_blocks(key_cache, value_cache, block_pairs, num_pairs, num_blocks,
-                                             num_kv_heads, head_dim, elt_bytes(dtype), status,
+                                             num_kv_heads, head_dim, block_size, elt_bytes(dtype), status,
                                              reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
@@ -228,10 +228,10 @@ pa_status pa_prefill(void* out, const void* q, const void* key_cache, const void
         max_blocks_per_seq <= 0 || max_query_len < 0)
         return PA_ERR_INVALID_ARG;
     if (!valid_dtype(dtype) || !std::isfinite(scale) || num_heads % num_kv_heads != 0) return PA_ERR_INVALID_ARG;
-    if (block_size != kBlockSize || (head_dim != 64 && head_dim != 128) || dtype == PA_F32 ||
+    if (block_size != kChunk || (head_dim != 64 && head_dim != 128) || dtype == PA_F32 ||
         num_heads / num_kv_heads > 16)
         return PA_ERR_UNSUPPORTED;
-    if ((int64_t)num_blocks * num_kv_heads * kBlockSize * head_dim > INT64_MAX / 4) return PA_ERR_UNSUPPORTED;
+    if ((int64_t)num_blocks * num_kv_heads * kChunk * head_dim > INT64_MAX / 4) return PA_ERR_UNSUPPORTED;
     if (num_seqs == 0 || max_query_len == 0) return PA_OK;
     if (!out || !q || !key_cache || !value_cache || !block_tables || !query_start || !context_lens)
         return PA_ERR_INVALID_ARG;
@@ -266,7 +266,7 @@ pa_status pa_swap_blocks(const void* src_key_cache, const void* src_value_cache,
     if (num_pairs < 0 || src_num_blocks <= 0 || dst_num_blocks <= 0 || num_kv_heads <= 0 || head_dim <= 0)
         return PA_ERR_INVALID_ARG;
     if (!valid_dtype(dtype)) return PA_ERR_INVALID_ARG;
-    if (block_size != kBlockSize || (head_dim != 64 && head_dim != 128)) return PA_ERR_UNSUPPORTED;
+    if (!block_size_supported(block_size) || (head_dim != 64 && head_dim != 128)) return PA_ERR_UNSUPPORTED;
     if (num_pairs == 0) return PA_OK;
     if (!src_key_cache || !src_value_cache || !dst_key_cache || !dst_value_cache || !block_pairs)
         return PA_ERR_INVALID_ARG;
@@ -275,7 +275,8 @@ pa_status pa_swap_blocks(const void* src_key_cache, const void* src_value_cache,
         return PA_ERR_INVALID_ARG;
     const cudaError_t e = launch_swap_blocks(src_key_cache, src_value_cache, dst_key_cache, dst_value_cache,
                                              block_pairs, num_pairs, src_num_blocks, dst_num_blocks, num_kv_heads,
-                                             head_dim, elt_bytes(dtype), status, reinterpret_cast<cudaStream_t>(stream));
+                                             head_dim, block_size, elt_bytes(dtype), status,
+                                             reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 

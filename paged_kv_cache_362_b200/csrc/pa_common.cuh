@@ -16,8 +16,13 @@
 
 namespace pa {
 
-constexpr int kBlockSize = 16;          // tokens per physical block
-constexpr int kMaxPartBlocks = 32;      // partition_size <= 512 tokens
+// The attention kernels step through a sequence 16 tokens at a time (one
+// 16-row MMA tile, a "chunk"); a physical block holds 8, 16 or 32 tokens, so
+// a chunk is two blocks, one block or half a block.  Partitions are counted
+// in chunks.
+constexpr int kChunk = 16;              // tokens per tile step
+constexpr int kMaxPartBlocks = 32;      // chunks per partition: partition_size <= 512 tokens
+__host__ __device__ constexpr bool block_size_supported(int bs) { return bs == 8 || bs == 16 || bs == 32; }
 
 // ---------------------------------------------------------------------------
 // element types
@@ -149,6 +154,15 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_group1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 
+// 16 zero bytes at a shared-memory address
+__device__ __forceinline__ void st_shared_zero16(uint32_t addr) {
+    asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(addr), "r"(0) : "memory");
+}
+// orders this thread's generic-proxy shared-memory accesses before later
+// async-proxy ones (tensor copies that refill the same bytes)
+__device__ __forceinline__ void fence_proxy_async_shared() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
 __device__ __forceinline__ void prefetch_l2(const void* p) {
     asm volatile("prefetch.global.L2 [%0];" ::"l"(p) : "memory");
 }
@@ -220,15 +234,16 @@ constexpr int kHdrItems = 0;
 struct DecodeParams {
     void* out;                    // [B, Hq, D]
     const void* q;                // [B, Hq, D]
-    const void* key_cache;        // [NB, Hkv, 16, D]
+    const void* key_cache;        // [NB, Hkv, block_size, D]
     const void* value_cache;
     const int32_t* block_tables;  // [B, MB]
     const int32_t* context_lens;  // [B]
     int32_t* status;
     int num_seqs, num_heads, num_kv_heads, head_dim, group;
     int max_blocks_per_seq, num_blocks;
-    int ctx_cap;                  // min(max_context_len, MB * 16)
-    int part_blocks;              // PB: blocks per partition
+    int block_size;               // tokens per physical block: 8, 16 or 32
+    int ctx_cap;                  // min(max_context_len, MB * block_size)
+    int part_blocks;              // PB: chunks (16 tokens) per partition
     int max_parts;                // NP_max = ceil(max_context_len / partition_size)
     float scale_log2;             // scale * log2(e)
     // workspace views

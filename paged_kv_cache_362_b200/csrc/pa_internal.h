@@ -16,17 +16,18 @@ cudaError_t device_info(DeviceInfo* out);
 
 cudaError_t launch_reshape_and_cache(const void* key, const void* value, void* key_cache, void* value_cache,
                                      const int64_t* slot_mapping, int64_t num_tokens, int32_t num_blocks,
-                                     int32_t num_kv_heads, int32_t head_dim, int elt_bytes, int32_t* status,
+                                     int32_t num_kv_heads, int32_t head_dim, int32_t block_size, int elt_bytes,
+                                     int32_t* status,
                                      cudaStream_t stream);
 
 cudaError_t launch_copy_blocks(void* key_cache, void* value_cache, const int64_t* block_pairs, int32_t num_pairs,
-                               int32_t num_blocks, int32_t num_kv_heads, int32_t head_dim, int elt_bytes,
-                               int32_t* status, cudaStream_t stream);
+                               int32_t num_blocks, int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                               int elt_bytes, int32_t* status, cudaStream_t stream);
 
 cudaError_t launch_swap_blocks(const void* src_key, const void* src_value, void* dst_key, void* dst_value,
                                const int64_t* block_pairs, int32_t num_pairs, int32_t src_num_blocks,
-                               int32_t dst_num_blocks, int32_t num_kv_heads, int32_t head_dim, int elt_bytes,
-                               int32_t* status, cudaStream_t stream);
+                               int32_t dst_num_blocks, int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                               int elt_bytes, int32_t* status, cudaStream_t stream);
 
 // Causal attention of each sequence's new query tokens over its paged cache.
 cudaError_t launch_prefill(const PrefillParams& p, pa_dtype dtype, cudaStream_t stream);

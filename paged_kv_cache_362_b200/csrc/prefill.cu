@@ -12,6 +12,8 @@
 // with K_j, V_j of KV head h / G.  The new tokens' K/V must already be in the
 // cache (pa_reshape_and_cache).
 //
+// Blocks of 16 tokens (the block size of the pages' default).
+//
 // How: one CTA per (16-query tile, KV head, sequence), one warp per query
 // head of the GQA group, so each K/V block is loaded once into shared memory
 // (cp.async, double-buffered) for all G heads and 16 queries.  Per block a
@@ -33,7 +35,7 @@ constexpr int kQTile = 16;
 template <int D>
 struct PrefillCfg {
     static constexpr int kRow = D + 8;                 // padded smem row (halves): conflict-free ldmatrix
-    static constexpr int kTileBytes = kBlockSize * kRow * 2;
+    static constexpr int kTileBytes = kChunk * kRow * 2;
     static constexpr int kQBytes = kQTile * kRow * 2;  // one head's query tile
 };
 
@@ -48,14 +50,14 @@ __global__ void __launch_bounds__(16 * 32) prefill_kernel(PrefillParams p) {
     const int qs = p.query_start[b], qlen = p.query_start[b + 1] - qs;
     if (i0 >= qlen || qlen <= 0) return;
     int n = p.context_lens[b];
-    if (n < qlen || n > p.max_blocks_per_seq * kBlockSize) {   // a query position outside the cache
+    if (n < qlen || n > p.max_blocks_per_seq * kChunk) {   // a query position outside the cache
         if (threadIdx.x == 0) set_status(p.status, PA_ERR_OUT_OF_RANGE);
         return;
     }
     const int rows = min(kQTile, qlen - i0);
     const int pos0 = n - qlen + i0;                  // position of query row 0 of the tile
     const int kend = pos0 + rows;                    // keys [0, kend) are visible to some row
-    const int nkb = ceil_div_i(kend, kBlockSize);
+    const int nkb = ceil_div_i(kend, kChunk);
     uint8_t* qsm = smem;                                              // [G][16][kRow]
     uint8_t* kv = smem + G * C::kQBytes;                              // [2 stages][K, V][16][kRow]
     __shared__ int bad[2];                                            // the stage's block id was out of range
@@ -72,7 +74,11 @@ __global__ void __launch_bounds__(16 * 32) prefill_kernel(PrefillParams p) {
             v = *reinterpret_cast<const uint4*>(q + ((size_t)(qs + i0 + r) * p.num_heads + g * G + hh) * D + k * 8);
         *reinterpret_cast<uint4*>(qsm + hh * C::kQBytes + r * C::kRow * 2 + k * 16) = v;
     }
-    // K and V tiles of key block kb into stage st (zeros and a status bit for a bad block id)
+    // K and V tiles of key block kb into stage st (zeros and a status bit for a
+    // bad block id).  Rows at or past kend are zero-filled, not loaded: no
+    // query of the tile sees them, and the slots past the context hold
+    // whatever the pool held (NaN bit patterns in a fresh allocation), which
+    // a masked probability of 0 would still carry into O (0 * NaN = NaN).
     auto load_block = [&](int kb, int st) {
         const int blk = p.block_tables[(size_t)b * p.max_blocks_per_seq + kb];
         const bool good = blk >= 0 && blk < p.num_blocks;
@@ -80,11 +86,11 @@ __global__ void __launch_bounds__(16 * 32) prefill_kernel(PrefillParams p) {
             bad[st] = !good;   // its keys are masked: the block contributes nothing
             if (!good) set_status(p.status, PA_ERR_OUT_OF_RANGE);
         }
-        const size_t base = ((size_t)blk * p.num_kv_heads + g) * kBlockSize * D;
-        for (int c = threadIdx.x; c < 2 * kBlockSize * kChunks; c += nthr) {
-            const int which = c / (kBlockSize * kChunks), r = (c / kChunks) % kBlockSize, k = c % kChunks;
+        const size_t base = ((size_t)blk * p.num_kv_heads + g) * kChunk * D;
+        for (int c = threadIdx.x; c < 2 * kChunk * kChunks; c += nthr) {
+            const int which = c / (kChunk * kChunks), r = (c / kChunks) % kChunk, k = c % kChunks;
             uint8_t* dst = kv + (st * 2 + which) * C::kTileBytes + r * C::kRow * 2 + k * 16;
-            if (good) cp_async_16(smem_u32(dst), (which ? vc : kc) + base + r * D + k * 8);
+            if (good && kb * kChunk + r < kend) cp_async_16(smem_u32(dst), (which ? vc : kc) + base + r * D + k * 8);
             else *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
         }
     };
@@ -125,7 +131,7 @@ __global__ void __launch_bounds__(16 * 32) prefill_kernel(PrefillParams p) {
                 Mma<T>::run(s[1], a, bq[2], bq[3]);
             }
             // ---- causal mask and online softmax per query row (rows gid and gid + 8)
-            const int key0 = kb * kBlockSize;
+            const int key0 = kb * kChunk;
             const bool skip = bad[st] != 0;
             float mx[2] = {kNegInfP, kNegInfP};
 #pragma unroll

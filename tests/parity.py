@@ -96,6 +96,20 @@ class DeviceCase:
         self.copy_pairs = torch.from_numpy(np.ascontiguousarray(wl.copy_pairs)).to(device)
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
 
+    def poison_unread(self):
+        """NaN into every pool slot no sequence reads (the tails of last blocks, unused blocks)."""
+        import torch
+
+        from workloads import unread_slots
+
+        blk, off = unread_slots(self.wl)
+        dev = self.dev["key_cache"].device
+        bi = torch.from_numpy(blk).to(dev)
+        oi = torch.from_numpy(off).to(dev)
+        for k in ("key_cache", "value_cache"):
+            self.dev[k][bi, :, oi, :] = float("nan")
+        return int(blk.size)
+
     def host_subproblem(self, seqs):
         """Compact host copy (pre-step) of everything the oracle needs for sequences ``seqs``.
 
@@ -105,8 +119,9 @@ class DeviceCase:
         import torch
 
         wl = self.wl
+        bs = wl.cfg.block_size
         seqs = list(seqs)
-        nblk = [-(-int(wl.context_lens[b]) // 16) for b in seqs]
+        nblk = [-(-int(wl.context_lens[b]) // bs) for b in seqs]
         used = set()
         for b, n in zip(seqs, nblk):
             used.update(int(x) for x in wl.block_tables[b, :n])
@@ -130,7 +145,7 @@ class DeviceCase:
             s = int(wl.slot_mapping[t])
             keys.append(key_h[t])
             vals.append(val_h[t])
-            slots.append(remap[s // 16] * 16 + s % 16)
+            slots.append(remap[s // bs] * bs + s % bs)
         q = to_host(self.dev["q"], self.dtype)[seqs]
         return dict(q=q, key_cache=kc, value_cache=vc, block_tables=bt,
                     context_lens=wl.context_lens[seqs].copy(),

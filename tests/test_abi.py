@@ -81,7 +81,10 @@ def test_reshape_and_cache_validation():
     args = lambda **o: [o.get("key", FAKE), o.get("value", FAKE), o.get("kc", FAKE), o.get("vc", FAKE),
                         o.get("slots", FAKE), o.get("T", 4), o.get("NB", 8), o.get("Hkv", 2), o.get("D", 64),
                         o.get("bs", 16), o.get("dt", 1), None, None]
-    assert _rc(*args(bs=8)) == pa.PA_ERR_UNSUPPORTED
+    for bs in (4, 12, 64):                                      # block sizes: 8, 16 and 32 only
+        assert _rc(*args(bs=bs)) == pa.PA_ERR_UNSUPPORTED
+    for bs in (8, 32):                                          # supported: fails on the null key instead
+        assert _rc(*args(bs=bs, key=P(0))) == pa.PA_ERR_INVALID_ARG
     assert _rc(*args(D=96)) == pa.PA_ERR_UNSUPPORTED
     assert _rc(*args(T=-1)) == pa.PA_ERR_INVALID_ARG
     assert _rc(*args(key=P(0))) == pa.PA_ERR_INVALID_ARG
@@ -106,7 +109,12 @@ def test_decode_validation():
     import paged_kv_cache_362_b200 as pa
 
     assert _dec(Hq=5) == pa.PA_ERR_INVALID_ARG               # Hq not a multiple of Hkv
-    assert _dec(bs=32) == pa.PA_ERR_UNSUPPORTED
+    for bs in (4, 24, 64):
+        assert _dec(bs=bs) == pa.PA_ERR_UNSUPPORTED
+    for bs in (8, 32):
+        assert _dec(bs=bs, out=P(0)) == pa.PA_ERR_INVALID_ARG
+    # pool rows (blocks x KV heads x block size) index the tensor copies in int32
+    assert _dec(bs=32, NB=1 << 25) == pa.PA_ERR_UNSUPPORTED
     assert _dec(D=80) == pa.PA_ERR_UNSUPPORTED
     assert _dec(Hkv=256, Hq=256) == pa.PA_ERR_UNSUPPORTED
     assert _dec(P=24) == pa.PA_ERR_INVALID_ARG
@@ -129,6 +137,23 @@ def test_copy_blocks_validation():
     assert lib.pa_copy_blocks(FAKE, FAKE, P(0), 3, 8, 2, 64, 16, 1, None, None) == pa.PA_ERR_INVALID_ARG
     assert lib.pa_copy_blocks(FAKE, FAKE, FAKE, 3, 8, 2, 64, 12, 1, None, None) == pa.PA_ERR_UNSUPPORTED
     assert lib.pa_copy_blocks(FAKE, FAKE, FAKE, 0, 8, 2, 64, 16, 1, None, None) == pa.PA_OK
+
+
+def test_prefill_and_swap_validation():
+    import paged_kv_cache_362_b200 as pa
+
+    lib = pa._lib.LIB
+    pf = lambda bs, dt=1, out=FAKE: lib.pa_prefill(out, FAKE, FAKE, FAKE, FAKE, 4, FAKE, FAKE, 2, 4, 2, 64, bs, 8,
+                                                   ctypes.c_float(0.125), 16, dt, None, None)
+    assert pf(8) == pa.PA_ERR_UNSUPPORTED                   # prefill reads 16-token blocks only
+    assert pf(32) == pa.PA_ERR_UNSUPPORTED
+    assert pf(16, dt=0) == pa.PA_ERR_UNSUPPORTED            # float32
+    assert pf(16, out=P(0)) == pa.PA_ERR_INVALID_ARG
+    sw = lambda bs, n=3: lib.pa_swap_blocks(FAKE, FAKE, FAKE, FAKE, P(0), n, 8, 8, 2, 64, bs, 1, None, None)
+    assert sw(12) == pa.PA_ERR_UNSUPPORTED
+    for bs in (8, 16, 32):
+        assert sw(bs) == pa.PA_ERR_INVALID_ARG              # null pairs
+        assert sw(bs, n=0) == pa.PA_OK
 
 
 def test_host_copy_pair_checker():

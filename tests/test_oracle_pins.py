@@ -82,3 +82,78 @@ def test_c_oracle_rejects_out_of_pool_block():
         c_oracle.decode(q, kc, vc, bt, cl, 1.0, "f32", 1)
     with pytest.raises(IndexError):
         R.decode(q, kc, vc, bt, cl, 1.0, "f32", 1)
+
+
+def _relayout(kc, vc, tables, ctx, bs, rng):
+    """The same per-sequence K/V rows in a pool of block size ``bs``, blocks placed at random."""
+    B = len(ctx)
+    nblk = [-(-int(n) // bs) for n in ctx]
+    nb = sum(nblk) + 3
+    Hkv, D = kc.shape[1], kc.shape[3]
+    bs0 = kc.shape[2]
+    k2 = rng.standard_normal((nb, Hkv, bs, D)).astype(kc.dtype)
+    v2 = rng.standard_normal((nb, Hkv, bs, D)).astype(vc.dtype)
+    perm = rng.permutation(nb)
+    t2 = np.full((B, max(1, max(nblk))), -1, dtype=np.int32)
+    k = 0
+    for b in range(B):
+        for j in range(nblk[b]):
+            t2[b, j] = perm[k]
+            k += 1
+        for i in range(int(ctx[b])):
+            src = tables[b, i // bs0]
+            k2[t2[b, i // bs], :, i % bs] = kc[src, :, i % bs0]
+            v2[t2[b, i // bs], :, i % bs] = vc[src, :, i % bs0]
+    return k2, v2, t2
+
+
+@pytest.mark.parametrize("bs", [1, 4, 8, 32])
+def test_oracle_output_does_not_depend_on_block_size(bs):
+    """Paging changes where K/V rows live, not the attention ("PagedAttention" digest, "Why the attention
+    kernel works at all"): the same rows in pools of another block size give the same bits."""
+    rng = np.random.default_rng(bs)
+    ctx = np.array([1, 7, 8, 9, 16, 33, 70], dtype=np.int32)
+    Hq, Hkv, D = 6, 2, 16
+    # a pool of block size 16 with random rows, then the same rows re-laid at bs
+    nb = sum(-(-int(n) // 16) for n in ctx)
+    k16 = rng.standard_normal((nb, Hkv, 16, D)).astype(np.float32)
+    v16 = rng.standard_normal((nb, Hkv, 16, D)).astype(np.float32)
+    t16 = np.full((len(ctx), 5), -1, dtype=np.int32)
+    k = 0
+    for b, n in enumerate(ctx):
+        for j in range(-(-int(n) // 16)):
+            t16[b, j] = k
+            k += 1
+    q = rng.standard_normal((len(ctx), Hq, D)).astype(np.float32)
+    kb, vb, tb = _relayout(k16, v16, t16, ctx, bs, rng)
+    a = R.decode(q, k16, v16, t16, ctx, 0.25, "f32", Hkv)
+    b = R.decode(q, kb, vb, tb, ctx, 0.25, "f32", Hkv)
+    assert np.array_equal(a, b)
+    c = c_oracle.decode(q, kb, vb, tb, ctx, 0.25, "f32", Hkv)
+    assert np.allclose(a, c, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("bs", [8, 16, 32])
+def test_oracle_never_reads_past_the_context(bs):
+    """Slots past a sequence's context (the tail of its last block, unused blocks) may hold NaN: the oracle's
+    result is unchanged, bit for bit, and finite."""
+    from workloads import build_workload, get_config, host_values, poison_unread_slots, unread_slots
+
+    ctx = (0, 1, 7, 8, 9, 15, 17, 31, 33, 100)
+    need = sum(-(-c // bs) for c in ctx)
+    cfg = get_config("qwen_layer", dtype="f16", num_heads=8, num_kv_heads=2, head_dim=64, block_size=bs,
+                     num_blocks=need + 5, ctx_kind="fixed", ctx_args=ctx)
+    wl = build_workload(cfg, seed=bs)
+    vh = host_values(wl)
+    before = c_oracle.decode(vh["q"], vh["key_cache"], vh["value_cache"], wl.block_tables, wl.context_lens,
+                             cfg.scale, "f16", 2)
+    n = poison_unread_slots(wl, vh)
+    # exactly the slots past each context: block tails plus the 5 unused blocks
+    assert n == need * bs - sum(ctx) + 5 * bs
+    blk, off = unread_slots(wl)
+    for b, c in enumerate(ctx):
+        for i in range(c):
+            assert not ((blk == wl.block_tables[b, i // bs]) & (off == i % bs)).any()
+    after = c_oracle.decode(vh["q"], vh["key_cache"], vh["value_cache"], wl.block_tables, wl.context_lens,
+                            cfg.scale, "f16", 2)
+    assert np.isfinite(after).all() and np.array_equal(before, after)

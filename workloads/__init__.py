@@ -8,4 +8,5 @@ that computes a result.
 """
 
 from .configs import CONFIGS, WorkloadConfig, get_config  # noqa: F401
-from .gen import Workload, build_workload, host_values, device_values  # noqa: F401
+from .gen import (Workload, build_workload, device_values, host_values, poison_unread_slots,  # noqa: F401
+                  unread_slots)

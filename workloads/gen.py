@@ -284,3 +284,43 @@ def device_values(wl: Workload, device, seed: int | None = None) -> dict:
         "key_cache": normal((wl.num_blocks, c.num_kv_heads, c.block_size, c.head_dim)),
         "value_cache": normal((wl.num_blocks, c.num_kv_heads, c.block_size, c.head_dim)),
     }
+
+
+# bit patterns of a quiet NaN in each storage dtype (bf16 held as uint16)
+_NAN_BITS = {"f16": np.float16(np.nan), "bf16": np.uint16(0x7FC0), "f32": np.float32(np.nan)}
+
+
+def unread_slots(wl: Workload):
+    """Slots of the pool that no sequence of the workload reads: (blocks, offsets).
+
+    A block in the middle of a table is read whole; a sequence's last block
+    up to its context; a copy-pair source whole (its copy is read).  Every
+    other slot -- the tail of last blocks, unreferenced blocks -- may hold
+    anything in a real pool; tests fill them with NaN.
+    """
+    bs = wl.cfg.block_size
+    extent = np.zeros(wl.num_blocks, dtype=np.int64)
+    for b in range(wl.num_seqs):
+        n = int(wl.context_lens[b])
+        nb = _ceil_div(n, bs)
+        if nb == 0:
+            continue
+        row = wl.block_tables[b, :nb].astype(np.int64)
+        ok = (row >= 0) & (row < wl.num_blocks)
+        mid = row[:-1][ok[:-1]]
+        extent[mid] = bs
+        if ok[-1]:
+            extent[row[-1]] = max(extent[row[-1]], n - (nb - 1) * bs)
+    for src, _ in np.asarray(wl.copy_pairs).reshape(-1, 2):
+        extent[int(src)] = bs
+    blk, off = np.nonzero(np.arange(bs)[None, :] >= extent[:, None])
+    return blk, off
+
+
+def poison_unread_slots(wl: Workload, vals: dict) -> int:
+    """Write NaN into every unread slot of the host pools in ``vals`` (in place); returns the slot count."""
+    blk, off = unread_slots(wl)
+    nan = _NAN_BITS[wl.cfg.dtype]
+    for k in ("key_cache", "value_cache"):
+        vals[k][blk, :, off, :] = nan
+    return int(blk.size)
