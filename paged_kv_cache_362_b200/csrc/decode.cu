@@ -1646,4 +1646,6 @@ cudaError_t decode_launch_count(const DecodeParams& p, pa_dtype dtype, int* laun
     return e;
 }
 
+int decode_fused_max_parts() { return kFusedMaxParts; }
+
 }  // namespace pa

@@ -48,6 +48,10 @@ cudaError_t launch_decode(const DecodeParams& p, pa_dtype dtype, cudaStream_t st
 // Number of kernels launch_decode enqueues for these sizes (p's pointers unused).
 cudaError_t decode_launch_count(const DecodeParams& p, pa_dtype dtype, int* launches);
 
+// Most partitions per sequence that the attention kernel merges itself (more
+// take the reduce kernel).
+int decode_fused_max_parts();
+
 // Every library kernel asks for the same (maximum) shared-memory carveout, so
 // that SMs need not reconfigure L1/shared memory between chained kernels.
 cudaError_t prefer_max_shared(const void* kernel);

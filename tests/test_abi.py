@@ -168,3 +168,18 @@ def test_host_copy_pair_checker():
         pa.check_copy_pairs(np.array([[1, 3], [3, 4]]), 8)     # dst that is also a src
     with pytest.raises(ValueError):
         pa.check_copy_pairs(np.array([[1, 9]]), 8)
+
+
+def test_auto_partition_size():
+    """partition_size 0: enough items for every SM, and no reduce kernel where one wave of CTAs still fills."""
+    import paged_kv_cache_362_b200 as pa
+
+    ws = lambda B, mc, P: pa._lib.LIB.pa_decode_workspace_size(B, 28, 4, 128, mc, P)
+    # 32 sequences of up to 2048 tokens: 256-token partitions (8 per sequence, merged by the attention kernel),
+    # not the 128 that the item count alone would pick
+    assert ws(32, 2048, 0) == ws(32, 2048, 256) != ws(32, 2048, 128)
+    # 256 sequences of up to 4096 tokens, 8 of up to 32768: 512
+    assert ws(256, 4096, 0) == ws(256, 4096, 512) != ws(256, 4096, 256)
+    assert ws(8, 32768, 0) == ws(8, 32768, 512)
+    # one sequence of 2048: 64-token partitions, the smallest, since even they give too few items
+    assert ws(1, 2048, 0) == ws(1, 2048, 64) != ws(1, 2048, 128)
