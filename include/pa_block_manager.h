@@ -51,9 +51,10 @@ extern "C" {
 typedef struct pa_block_manager pa_block_manager;
 
 /* A pool of num_blocks device blocks of block_size tokens (1 .. 1024; the
- * kernels take 16) and a pool of num_host_blocks blocks in CPU memory that
- * swapped-out sequences move to (0: no swapping).  Returns NULL for invalid
- * arguments or when memory runs out. */
+ * attention and cache kernels take 8, 16 or 32, prefill 16) and a pool of
+ * num_host_blocks blocks in CPU memory that swapped-out sequences move to
+ * (0: no swapping).  Returns NULL for invalid arguments or when memory runs
+ * out. */
 pa_block_manager* pa_bm_create(int32_t num_blocks, int32_t block_size, int32_t num_host_blocks);
 void pa_bm_destroy(pa_block_manager* bm);
 
