@@ -604,6 +604,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="churned256")
     ap.add_argument("--partition-size", type=int, default=None)
+    ap.add_argument("--block-size", type=int, default=None, choices=[8, 16, 32],
+                    help="pool block size (default: the workload's, 16); the pool keeps its token capacity")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-graph", action="store_true", help="launch every step from the host (no CUDA graph)")
     ap.add_argument("--no-secondary", action="store_true")
@@ -637,7 +639,7 @@ def main():
     flush_write_only = lambda: flush_buf.zero_()
     use_graph = not args.no_graph
 
-    w = DeviceWorkload(args.workload, args.seed + rank, args.partition_size)
+    w = DeviceWorkload(args.workload, args.seed + rank, args.partition_size, block_size=args.block_size)
     clocks = ClockSampler(torch.cuda.current_device())
     step_ms, dec_ms = time_steps(w, args.steps, args.warmup, flush, use_graph)
     clk = clocks.stop()
@@ -754,7 +756,7 @@ def main():
             "pct_of_peak": round(100 * value / world / peak, 2),
             "seq_per_s": round(w.wl.num_seqs * world / (ms * 1e-3), 1),
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                         "frac": round(achieved / peak, 4), "traffic": profiled_traffic(c.name),
+                         "frac": round(achieved / peak, 4), "traffic": profiled_traffic(c.name if c.block_size == 16 else f"{c.name}_bs{c.block_size}"),
                          "algorithmic_bytes": w.kv_bytes,
                          "kernel": f"pa_decode call ({w.decode_launches} launch(es): [plan +] attention "
                                    "[+ reduce]), timed together; traffic = DRAM bytes of the attention kernel "
