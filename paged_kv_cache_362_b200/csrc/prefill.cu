@@ -16,7 +16,7 @@
 //
 // How: one CTA per (16-query tile, KV head, sequence), one warp per query
 // head of the GQA group, so each K/V block is loaded once into shared memory
-// (cp.async, double-buffered) for all G heads and 16 queries.  Per block a
+// (cp.async, a ring of kStages blocks) for all G heads and 16 queries.  Per block a
 // warp computes S = Q K^T (m16n8k16: 16 queries x 16 keys, two n-tiles), the
 // causal mask on the diagonal blocks, an online softmax per query row in fp32
 // (2^x on log2-scaled logits), and O += P V with the S accumulators reused as
@@ -31,6 +31,15 @@ namespace {
 
 constexpr float kNegInfP = -__builtin_huge_valf();
 constexpr int kQTile = 16;
+// K/V blocks in flight per CTA.  Registers hold a CTA of G <= 16 warps to
+// about 2 per SM, so each CTA hides its own load latency: a block is
+// requested kStages - 1 steps before it is used.
+constexpr int kStages = 4;
+
+template <int N>
+__device__ __forceinline__ void cp_async_wait_pending() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
 
 template <int D>
 struct PrefillCfg {
@@ -59,8 +68,8 @@ __global__ void __launch_bounds__(16 * 32) prefill_kernel(PrefillParams p) {
     const int kend = pos0 + rows;                    // keys [0, kend) are visible to some row
     const int nkb = ceil_div_i(kend, kChunk);
     uint8_t* qsm = smem;                                              // [G][16][kRow]
-    uint8_t* kv = smem + G * C::kQBytes;                              // [2 stages][K, V][16][kRow]
-    __shared__ int bad[2];                                            // the stage's block id was out of range
+    uint8_t* kv = smem + G * C::kQBytes;                              // [kStages][K, V][16][kRow]
+    __shared__ int bad[kStages];                                      // the stage's block id was out of range
     const T* q = static_cast<const T*>(p.q);
     const T* kc = static_cast<const T*>(p.key_cache);
     const T* vc = static_cast<const T*>(p.value_cache);
@@ -94,8 +103,10 @@ __global__ void __launch_bounds__(16 * 32) prefill_kernel(PrefillParams p) {
             else *reinterpret_cast<uint4*>(dst) = make_uint4(0, 0, 0, 0);
         }
     };
-    load_block(0, 0);
-    cp_async_commit();
+    for (int s = 0; s < kStages - 1; ++s) {
+        if (s < nkb) load_block(s, s);
+        cp_async_commit();
+    }
 
     const int h = warp;   // this warp's query head within the group
     const bool active = h < G;
@@ -110,10 +121,11 @@ __global__ void __launch_bounds__(16 * 32) prefill_kernel(PrefillParams p) {
     const float sl2 = p.scale_log2;
 
     for (int kb = 0; kb < nkb; ++kb) {
-        const int st = kb & 1;
-        if (kb + 1 < nkb) load_block(kb + 1, st ^ 1);
+        const int st = kb % kStages;
+        // the stage computed in the previous step takes block kb + kStages - 1
+        if (kb + kStages - 1 < nkb) load_block(kb + kStages - 1, (kb + kStages - 1) % kStages);
         cp_async_commit();
-        cp_async_wait_group1();
+        cp_async_wait_pending<kStages - 1>();   // block kb has landed
         __syncthreads();
         if (active) {
             const uint32_t kt = smem_u32(kv + (st * 2) * C::kTileBytes);
@@ -197,7 +209,7 @@ __global__ void __launch_bounds__(16 * 32) prefill_kernel(PrefillParams p) {
                 }
             }
         }
-        __syncthreads();   // the stage is loaded again two blocks later
+        __syncthreads();   // the next step refills this stage
     }
     if (!active) return;
     // ---- out = O / l for the tile's rows
@@ -225,7 +237,7 @@ template <typename T, int D>
 cudaError_t launch_prefill_t(const PrefillParams& p, cudaStream_t stream) {
     using C = PrefillCfg<D>;
     auto kernel = prefill_kernel<T, D>;
-    const size_t smem = (size_t)p.group * C::kQBytes + 4 * C::kTileBytes;
+    const size_t smem = (size_t)p.group * C::kQBytes + 2 * kStages * C::kTileBytes;
     static size_t attr = 0;
     if (smem > attr) {
         const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
