@@ -29,6 +29,7 @@ import os
 import shutil
 import statistics
 import subprocess
+import tempfile
 import sys
 import time
 
@@ -166,11 +167,10 @@ class ClockSampler:
 
     def __init__(self, gpu_index: int):
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{gpu_index}.csv")
+        self.path = os.path.join(tempfile.gettempdir(), f"pa_bench_clocks_gpu{gpu_index}_{os.getpid()}.csv")
         exe = shutil.which("nvidia-smi")
         if exe is None:
             return
-        os.makedirs(os.path.dirname(self.path), exist_ok=True)
         self.f = open(self.path, "w")
         self.proc = subprocess.Popen([exe, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
                                       "-i", str(gpu_index), "-lms", "50"], stdout=self.f,
@@ -199,6 +199,10 @@ class ClockSampler:
             for n, v in zip(names, parts[4:8]):
                 if v.lower() == "active":
                     reasons.add(n)
+        try:
+            os.remove(self.path)
+        except OSError:
+            pass
         if not sm:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
