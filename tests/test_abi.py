@@ -4,6 +4,7 @@ CPU only: every call here returns during host-side validation, before any CUDA c
 """
 
 import ctypes
+import glob
 import os
 import re
 
@@ -12,17 +13,23 @@ import pytest
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
-def _declared_functions():
-    src = open(os.path.join(ROOT, "include", "pa.h")).read()
-    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b(pa_[a-z_0-9]+)\s*\(", src)))
+def _declared_functions(header=None):
+    """Function names declared in include/*.h (or one header), comments stripped."""
+    names = set()
+    for h in sorted(glob.glob(os.path.join(ROOT, "include", header or "*.h"))):
+        src = re.sub(r"/\*.*?\*/", "", open(h).read(), flags=re.S)
+        names.update(re.findall(r"\b(pa_[a-z_0-9]+)\s*\(", src))
+    return sorted(names)
 
 
 def test_header_declares_the_boundary():
-    names = _declared_functions()
+    names = _declared_functions("pa.h")
     for n in ("pa_reshape_and_cache", "pa_decode", "pa_decode_workspace_size", "pa_copy_blocks",
-              "pa_get_error_string"):
+              "pa_get_error_string", "pa_swap_blocks", "pa_prefill"):
         assert n in names
+    bm = _declared_functions("pa_block_manager.h")
+    for n in ("pa_bm_create", "pa_bm_append_tokens", "pa_bm_fork", "pa_bm_swap_out", "pa_bm_block_tables"):
+        assert n in bm
 
 
 def test_library_exports_every_declared_symbol():
