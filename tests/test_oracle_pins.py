@@ -157,3 +157,25 @@ def test_oracle_never_reads_past_the_context(bs):
     after = c_oracle.decode(vh["q"], vh["key_cache"], vh["value_cache"], wl.block_tables, wl.context_lens,
                             cfg.scale, "f16", 2)
     assert np.isfinite(after).all() and np.array_equal(before, after)
+
+
+def test_unread_slots_keep_copy_sources_whole():
+    """A fork's clone is copied from a block no table names; its slots are still read (through the copy),
+    so poisoning unread slots must leave copy sources whole: the oracle's step is unchanged."""
+    from workloads import build_workload, get_config, host_values, poison_unread_slots, unread_slots
+    from parity import oracle_step
+
+    cfg = get_config("shared_prefix", num_heads=8, num_kv_heads=2, head_dim=64, num_blocks=4000)
+    wl = build_workload(cfg, seed=4, num_seqs=40)
+    assert wl.copy_pairs.size
+    blk, _ = unread_slots(wl)
+    assert not np.isin(wl.copy_pairs[:, 0], blk).any()
+    vh = host_values(wl)
+    sub = dict(q=vh["q"], key_cache=vh["key_cache"], value_cache=vh["value_cache"], block_tables=wl.block_tables,
+               context_lens=wl.context_lens, key=vh["key"], value=vh["value"], slot_mapping=wl.slot_mapping,
+               copy_pairs=wl.copy_pairs)
+    before = oracle_step(sub, cfg)
+    poison_unread_slots(wl, vh)
+    sub.update(key_cache=vh["key_cache"], value_cache=vh["value_cache"])
+    after = oracle_step(sub, cfg)
+    assert np.isfinite(after).all() and np.array_equal(before, after)
