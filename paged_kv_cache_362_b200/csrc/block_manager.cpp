@@ -292,14 +292,22 @@ pa_status pa_bm_block_tables(const pa_block_manager* bm, const int64_t* seq_ids,
                              int32_t max_blocks_per_seq, int32_t* block_tables, int32_t* context_lens) {
     if (!bm || n < 0 || max_blocks_per_seq <= 0) return PA_ERR_INVALID_ARG;
     if (n > 0 && (!seq_ids || !block_tables || !context_lens)) return PA_ERR_INVALID_ARG;
-    for (int32_t k = 0; k < n; ++k) {   // validate everything before writing anything
+    // validate everything before writing anything; each id is looked up once
+    std::vector<const Sequence*> seq;
+    try {
+        seq.resize(n);
+    } catch (...) {
+        return PA_ERR_INVALID_ARG;
+    }
+    for (int32_t k = 0; k < n; ++k) {
         auto it = bm->seqs.find(seq_ids[k]);
         if (it == bm->seqs.end() || it->second.swapped || (int64_t)it->second.blocks.size() > max_blocks_per_seq ||
             it->second.len > INT32_MAX)
             return PA_ERR_INVALID_ARG;
+        seq[k] = &it->second;
     }
     for (int32_t k = 0; k < n; ++k) {
-        const Sequence& s = bm->seqs.find(seq_ids[k])->second;
+        const Sequence& s = *seq[k];
         int32_t* row = block_tables + (size_t)k * max_blocks_per_seq;
         std::copy(s.blocks.begin(), s.blocks.end(), row);
         std::fill(row + s.blocks.size(), row + max_blocks_per_seq, -1);
