@@ -8,28 +8,35 @@ from workloads import CONFIGS, build_workload, get_config, host_values
 
 
 def _used_blocks(wl):
+    bs = wl.cfg.block_size
     out = []
     for b in range(wl.num_seqs):
-        n = -(-int(wl.context_lens[b]) // 16)
+        n = -(-int(wl.context_lens[b]) // bs)
         out.append(wl.block_tables[b, :n])
     return out
 
 
-@pytest.mark.parametrize("name", sorted(CONFIGS))
-def test_tables_slots_well_formed(name):
-    wl = build_workload(get_config(name), seed=0)
+def _check_well_formed(wl, name):
     cfg = wl.cfg
+    bs = cfg.block_size
     assert wl.context_lens.dtype == np.int32 and wl.block_tables.dtype == np.int32
     assert wl.slot_mapping.dtype == np.int64
     used = _used_blocks(wl)
     for b, blocks in enumerate(used):
         assert ((blocks >= 0) & (blocks < cfg.num_blocks)).all()
-        n = -(-int(wl.context_lens[b]) // 16)
+        n = -(-int(wl.context_lens[b]) // bs)
         assert (wl.block_tables[b, n:] == -1).all()
     # appended token b sits at position ctx-1 of sequence b
     for b in range(wl.num_seqs):
         pos = int(wl.context_lens[b]) - 1
-        assert wl.slot_mapping[b] == wl.block_tables[b, pos // 16] * 16 + pos % 16
+        assert wl.slot_mapping[b] == wl.block_tables[b, pos // bs] * bs + pos % bs
+    return used
+
+
+@pytest.mark.parametrize("name", sorted(CONFIGS))
+def test_tables_slots_well_formed(name):
+    wl = build_workload(get_config(name), seed=0)
+    used = _check_well_formed(wl, name)
     if name != "shared_prefix":
         flat = np.concatenate(used)
         assert len(np.unique(flat)) == len(flat), "private blocks must not be shared"
@@ -111,3 +118,19 @@ def test_seeded_generation_is_deterministic():
     assert np.array_equal(a.block_tables, b.block_tables) and np.array_equal(a.context_lens, b.context_lens)
     c = build_workload(get_config("churned256"), seed=8)
     assert not np.array_equal(a.context_lens, c.context_lens)
+
+
+@pytest.mark.parametrize("name", ["churned256", "long32k"])
+@pytest.mark.parametrize("bs", [8, 32])
+def test_block_size_variants_hold_the_same_sequences(name, bs):
+    """The block-size sweep compares like with like: the same context lengths, a pool of the same token
+    capacity, ceil(ctx / bs) private blocks per sequence, well-formed tables and slots."""
+    base = build_workload(get_config(name), seed=0)
+    c0 = get_config(name)
+    wl = build_workload(get_config(name, block_size=bs, num_blocks=c0.num_blocks * 16 // bs), seed=0)
+    assert np.array_equal(wl.context_lens, base.context_lens)
+    assert wl.num_blocks * bs == base.num_blocks * 16
+    used = _check_well_formed(wl, name)
+    flat = np.concatenate(used)
+    assert len(np.unique(flat)) == len(flat)
+    assert len(flat) == sum(-(-int(c) // bs) for c in wl.context_lens)
