@@ -117,9 +117,15 @@ size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_heads, int32_t num
  *     out[b][h][:] = sum_i softmax_i(scale * q[b][h][:] . K_i) V_i
  * computed in fp32 from the stored values and rounded to the element type.
  * n = 0 gives a zero row.  The context is split into partitions of
- * partition_size tokens that run in parallel; a second kernel merges them.
- * The merge is exact algebra, so the result does not depend on the split
- * beyond fp32 rounding, and it does not depend on where blocks live.
+ * partition_size tokens that run in parallel.  When no sequence spans more
+ * than 8 partitions (fp16/bf16, at most 16 query heads per KV head), the
+ * attention kernel merges a sequence's partitions itself: the CTA that
+ * finishes its last partition combines them, and no second kernel runs.
+ * Otherwise a reduce kernel merges them after the attention kernel.  The
+ * merge is exact algebra, so the result does not depend on the split beyond
+ * fp32 rounding, and it does not depend on where blocks live.  Scheduling
+ * alternatives (kernel shape, planner, split, order) are selectable through
+ * pa_decode_tuned (pa_tuning.h); this call always uses the defaults.
  *
  *   out                 [num_seqs][num_heads][head_dim], 16-byte aligned
  *   q                   [num_seqs][num_heads][head_dim], 16-byte aligned
@@ -253,7 +259,9 @@ pa_status pa_swap_blocks(const void* src_key_cache, const void* src_value_cache,
  * and enqueues nothing.  The first call made with a given device current
  * looks up the array's device address (cudaGetSymbolAddress), zero-fills it
  * on `stream` and waits for that (cudaStreamSynchronize); make that first
- * call before any stream capture begins.  No cudaMalloc or cudaFree is made.
+ * call before any stream capture begins (a first call on a stream that is
+ * being captured returns PA_ERR_INVALID_ARG and enqueues nothing).  No
+ * cudaMalloc or cudaFree is made.
  * All calls share the one array: calls whose kernels overlap on the GPU (two
  * streams, two host threads) race on it and give wrong results.  After a call
  * that reported PA_ERR_TIMEOUT, stop using this entry point in the process.

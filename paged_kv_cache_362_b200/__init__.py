@@ -16,6 +16,7 @@ from ._lib import (  # noqa: F401
     PA_ERR_UNSUPPORTED,
     PA_OK,
     BlockManager,
+    DecodeTuning,
     PagedAttentionError,
     check_copy_pairs,
     copy_blocks,
@@ -26,6 +27,8 @@ from ._lib import (  # noqa: F401
     make_workspace,
     prefill,
     reshape_and_cache,
+    set_default_tuning,
     swap_blocks,
+    tuning,
     version,
 )

@@ -33,12 +33,50 @@ class PagedAttentionError(RuntimeError):
         super().__init__(f"{where}: {error_string(code)} (status {code})")
 
 
+class DecodeTuning(ctypes.Structure):
+    """pa_decode_tuning (include/pa_tuning.h): scheduling alternatives and fault-path test hooks.
+
+    shape: 0 auto, 1 paired, 2 quad, 3 triple, 4 pair1; planner: 1 = always the planning kernel;
+    split: 1 = near-equal partitions; order: 1 = all items by size; wait_limit_ns: bound of every wait
+    in the attention kernel (0 = 2 s); stall_first_item: 1 = CTA 0 never publishes its first item.
+    """
+
+    _fields_ = [("shape", ctypes.c_int32), ("planner", ctypes.c_int32), ("split", ctypes.c_int32),
+                ("order", ctypes.c_int32), ("wait_limit_ns", ctypes.c_int64), ("stall_first_item", ctypes.c_int32),
+                ("reserved", ctypes.c_int32)]
+
+
+SHAPES = {"auto": 0, "paired": 1, "quad": 2, "triple": 3, "pair1": 4}
+
+
+def tuning(shape="auto", planner=0, split=0, order=0, wait_limit_ns=0, stall_first_item=0) -> DecodeTuning:
+    return DecodeTuning(SHAPES[shape] if isinstance(shape, str) else int(shape), int(planner), int(split), int(order),
+                        int(wait_limit_ns), int(stall_first_item), 0)
+
+
+# Options that decode() and decode_launch_count() use when the caller gives
+# none: None is the library's defaults.  The test suite sets it to run its
+# parity cases under each scheduling alternative; nothing else should.
+_default_tuning: DecodeTuning | None = None
+
+
+def set_default_tuning(t: DecodeTuning | None) -> None:
+    global _default_tuning
+    _default_tuning = t
+
+
+def _tuning_ptr(t):
+    t = _default_tuning if t is None else t
+    return None if t is None else ctypes.byref(t)
+
+
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"{LIB_PATH} is not built; run `python paged_kv_cache_362_b200/build.py`")
     lib = ctypes.CDLL(LIB_PATH)
     for sym in ("pa_reshape_and_cache", "pa_decode_workspace_size", "pa_decode", "pa_decode_launch_count",
-                "pa_copy_blocks", "pa_get_error_string", "pa_version", "pa_bm_create", "pa_bm_append_tokens", "pa_prefill", "pa_swap_blocks"):
+                "pa_copy_blocks", "pa_get_error_string", "pa_version", "pa_bm_create", "pa_bm_append_tokens",
+                "pa_prefill", "pa_swap_blocks", "pa_decode_tuned", "pa_decode_launch_count_tuned"):
         if not hasattr(lib, sym):
             raise ImportError(f"{LIB_PATH} lacks {sym} (stale build); run `python paged_kv_cache_362_b200/build.py`")
     p, i32, i64, f32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
@@ -51,6 +89,12 @@ def _load() -> ctypes.CDLL:
     lib.pa_decode.restype = ctypes.c_int
     lib.pa_decode_launch_count.argtypes = [i32, i32, i32, i32, i32, i32, ctypes.c_int]
     lib.pa_decode_launch_count.restype = i32
+    # scheduling options and fault-path test hooks (pa_tuning.h)
+    lib.pa_decode_tuned.argtypes = lib.pa_decode.argtypes + [ctypes.POINTER(DecodeTuning)]
+    lib.pa_decode_tuned.restype = ctypes.c_int
+    lib.pa_decode_launch_count_tuned.argtypes = [i32, i32, i32, i32, i32, i32, ctypes.c_int,
+                                                 ctypes.POINTER(DecodeTuning)]
+    lib.pa_decode_launch_count_tuned.restype = i32
     lib.pa_copy_blocks.argtypes = [p, p, p, i32, i32, i32, i32, i32, ctypes.c_int, p, p]
     lib.pa_copy_blocks.restype = ctypes.c_int
     # host block manager (pa_block_manager.h)
@@ -152,11 +196,11 @@ def decode_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, max_conte
 
 
 def decode_launch_count(num_seqs, num_heads, num_kv_heads, head_dim, max_context_len, partition_size=0,
-                        dtype="f16") -> int:
+                        dtype="f16", tuning=None) -> int:
     """Kernels one pa_decode call enqueues for these sizes on the current device."""
     code = {"f32": 0, "f16": 1, "bf16": 2}[dtype]
-    n = int(LIB.pa_decode_launch_count(num_seqs, num_heads, num_kv_heads, head_dim, max_context_len,
-                                       partition_size, code))
+    n = int(LIB.pa_decode_launch_count_tuned(num_seqs, num_heads, num_kv_heads, head_dim, max_context_len,
+                                             partition_size, code, _tuning_ptr(tuning)))
     if n < 0:
         raise PagedAttentionError(PA_ERR_INVALID_ARG, "pa_decode_launch_count")
     return n
@@ -171,10 +215,11 @@ def make_workspace(num_seqs, num_heads, num_kv_heads, head_dim, max_context_len,
 
 
 def decode(out, q, key_cache, value_cache, block_tables, context_lens, scale, max_context_len, workspace,
-           partition_size=0, status=None, stream=None):
+           partition_size=0, status=None, stream=None, tuning=None):
     """One decode step of paged attention (pa_decode); writes ``out`` [B, Hq, D].
 
-    The block size (8, 16 or 32 tokens) is the pools' dimension 2.
+    The block size (8, 16 or 32 tokens) is the pools' dimension 2.  ``tuning`` (a DecodeTuning) selects a
+    scheduling alternative or a test hook (pa_decode_tuned); None is the library's default schedule.
     """
     B, Hq, D = q.shape
     NB, Hkv, bs = key_cache.shape[0], key_cache.shape[1], key_cache.shape[2]
@@ -184,11 +229,11 @@ def decode(out, q, key_cache, value_cache, block_tables, context_lens, scale, ma
     assert block_tables.shape[0] == B and context_lens.shape == (B,)
     for t in (out, q, key_cache, value_cache, block_tables, context_lens, workspace):
         assert t.is_contiguous()
-    _check(LIB.pa_decode(_ptr(out), _ptr(q), _ptr(key_cache), _ptr(value_cache), _ptr(block_tables),
-                         block_tables.shape[1], _ptr(context_lens), B, Hq, Hkv, D, bs, NB, float(scale),
-                         int(max_context_len), int(partition_size), _ptr(workspace),
-                         workspace.numel() * workspace.element_size(), _dtype_code(q), _ptr(status),
-                         _stream(stream)),
+    _check(LIB.pa_decode_tuned(_ptr(out), _ptr(q), _ptr(key_cache), _ptr(value_cache), _ptr(block_tables),
+                               block_tables.shape[1], _ptr(context_lens), B, Hq, Hkv, D, bs, NB, float(scale),
+                               int(max_context_len), int(partition_size), _ptr(workspace),
+                               workspace.numel() * workspace.element_size(), _dtype_code(q), _ptr(status),
+                               _stream(stream), _tuning_ptr(tuning)),
            "pa_decode")
 
 

@@ -48,8 +48,6 @@
 //  3. reduce  -- (sequences over 8 partitions, or two-warp CTAs) rows of the
 //                multi-partition sequences: M = max m_p, L = sum l_p 2^(m_p - M),
 //                out = sum O_p 2^(m_p - M) / L.
-#include <cstdlib>
-#include <string>
 #include <type_traits>
 #include <utility>
 
@@ -67,7 +65,7 @@ constexpr float kNegInf = -__builtin_huge_valf();
 // Partitions.  A sequence of nblk blocks has n = max(1, ceil(nblk / PB))
 // partitions: partitions 0 .. nbig-1 hold `big` blocks, the others `small`.
 //  * full split (default): n - 1 partitions of PB blocks, then the remainder.
-//  * equal split (PA_SPLIT=equal, tuning): near-equal lengths, q + 1 blocks
+//  * equal split (pa_decode_tuning.split = 1): near-equal lengths, q + 1 blocks
 //    for the first r = nblk % n partitions and q = nblk / n for the rest.  It
 //    avoids small tail partitions, yet measured 1-6% slower on every workload.
 struct SeqParts {
@@ -508,6 +506,10 @@ __global__ void __launch_bounds__(TcCfg<D, NT, NCW, STAGES>::kThreads, TcCfg<D, 
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = p.group;
+    // every wait of the kernel is bounded (p.wait_limit_ns); on expiry the
+    // kernel reports PA_ERR_TIMEOUT, lets the copies it issued land and returns
+    const uint64_t wait_limit = p.wait_limit_ns;
+    auto wait_on = [wait_limit](uint64_t* bar, uint32_t parity) { return mbar_wait(bar, parity, wait_limit); };
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -562,7 +564,7 @@ __global__ void __launch_bounds__(TcCfg<D, NT, NCW, STAGES>::kThreads, TcCfg<D, 
             // finished and merges all their partitions, off the consumer's path.
             for (int t = 0;; ++t) {
                 const int qs = t % C::kQSlots;
-                if (!__all_sync(0xffffffffu, mbar_wait(&qfull[qs], (t / C::kQSlots) & 1)) || *abort_flag) {
+                if (!__all_sync(0xffffffffu, wait_on(&qfull[qs], (t / C::kQSlots) & 1)) || *abort_flag) {
                     *abort_flag = 1;
                     break;
                 }
@@ -673,7 +675,7 @@ __global__ void __launch_bounds__(TcCfg<D, NT, NCW, STAGES>::kThreads, TcCfg<D, 
         auto publish = [&](int it) -> int {
             const int islot = it % C::kISlots;
             int okw = 1;
-            if (lane == 0) okw = mbar_wait(&iempty[islot], ((it / C::kISlots) & 1) ^ 1);
+            if (lane == 0) okw = wait_on(&iempty[islot], ((it / C::kISlots) & 1) ^ 1);
             if (!__shfl_sync(0xffffffffu, okw, 0)) return -1;
             const DescSlot& dd = dsc[it % C::kDSlots];
             if (dd.rank >= n_items) {
@@ -683,6 +685,7 @@ __global__ void __launch_bounds__(TcCfg<D, NT, NCW, STAGES>::kThreads, TcCfg<D, 
                 }
                 return 0;
             }
+            if (p.stall_first_item && it == 0 && blockIdx.x == 0) return 1;   // test hook: never published
             if (lane == 0) {
                 const ItemGeom mm = item_geom(p, dd.e);
                 meta[islot] = ItemMeta{mm.b, mm.g, mm.p, mm.ctx, mm.j0, mm.nblk, mm.nparts, 0};
@@ -728,7 +731,7 @@ __global__ void __launch_bounds__(TcCfg<D, NT, NCW, STAGES>::kThreads, TcCfg<D, 
                 // (bitwise-reproducible results); the padding stages carry no data
                 for (; stage % NCW != 0; ++stage) {
                     const int s = stage % STAGES;
-                    if (!mbar_wait(&empty[s], ((stage / STAGES) & 1) ^ 1)) { okw = 0; break; }
+                    if (!wait_on(&empty[s], ((stage / STAGES) & 1) ^ 1)) { okw = 0; break; }
                     stage_bad[s] = 1;
                     mbar_arrive(&full[s]);
                 }
@@ -741,7 +744,7 @@ __global__ void __launch_bounds__(TcCfg<D, NT, NCW, STAGES>::kThreads, TcCfg<D, 
                     const bool has1 = bs < kChunk && 2 * c + 1 < nphys;
                     const int blk1 = has1 ? d.bt2[j] : 0;
                     const int s = stage % STAGES;
-                    if (!mbar_wait(&empty[s], ((stage / STAGES) & 1) ^ 1)) { okw = 0; break; }
+                    if (!wait_on(&empty[s], ((stage / STAGES) & 1) ^ 1)) { okw = 0; break; }
                     if (blk >= 0 && blk < p.num_blocks && blk1 >= 0 && blk1 < p.num_blocks) {
                         stage_bad[s] = 0;
                         const uint32_t kdst = smem_u32(stages + s * C::kStageBytes);
@@ -804,12 +807,12 @@ __global__ void __launch_bounds__(TcCfg<D, NT, NCW, STAGES>::kThreads, TcCfg<D, 
                 const uint32_t outstanding = stage < (uint32_t)STAGES ? stage : (uint32_t)STAGES;
                 for (uint32_t k = 1; k <= outstanding; ++k) {
                     const uint32_t n = stage - k;
-                    mbar_wait(&full[n % STAGES], (n / STAGES) & 1);
+                    wait_on(&full[n % STAGES], (n / STAGES) & 1);
                 }
                 const int qout = npub < C::kISlots ? npub : C::kISlots;
                 for (int k = 1; k <= qout; ++k) {
                     const int it = npub - k;
-                    mbar_wait(&ifull[it % C::kISlots], (it / C::kISlots) & 1);
+                    wait_on(&ifull[it % C::kISlots], (it / C::kISlots) & 1);
                 }
             }
         }
@@ -838,7 +841,7 @@ __global__ void __launch_bounds__(TcCfg<D, NT, NCW, STAGES>::kThreads, TcCfg<D, 
     for (int iter = 0;; ++iter) {
         const int islot = iter % C::kISlots;
         const uint32_t iph = (iter / C::kISlots) & 1;
-        if (!__all_sync(0xffffffffu, mbar_wait(&ifull[islot], iph)) || *abort_flag) {
+        if (!__all_sync(0xffffffffu, wait_on(&ifull[islot], iph)) || *abort_flag) {
             *abort_flag = 1;
             break;
         }
@@ -877,7 +880,7 @@ __global__ void __launch_bounds__(TcCfg<D, NT, NCW, STAGES>::kThreads, TcCfg<D, 
         const uint32_t item_base = (stage_base + NCW - 1) / NCW * NCW;
         for (uint32_t n = stage_base + (((uint32_t)cw + NCW - stage_base % NCW) % NCW); n < item_base; n += NCW) {
             const int s = n % STAGES;
-            if (!__all_sync(0xffffffffu, mbar_wait(&full[s], (n / STAGES) & 1)) || *abort_flag) {
+            if (!__all_sync(0xffffffffu, wait_on(&full[s], (n / STAGES) & 1)) || *abort_flag) {
                 *abort_flag = 1;
                 break;
             }
@@ -1013,7 +1016,7 @@ __global__ void __launch_bounds__(TcCfg<D, NT, NCW, STAGES>::kThreads, TcCfg<D, 
             return true;
         };
         auto wait_full = [&](uint32_t n) {
-            if (!__all_sync(0xffffffffu, mbar_wait(&full[n % STAGES], (n / STAGES) & 1)) || *abort_flag) {
+            if (!__all_sync(0xffffffffu, wait_on(&full[n % STAGES], (n / STAGES) & 1)) || *abort_flag) {
                 *abort_flag = 1;
                 return false;
             }
@@ -1116,7 +1119,7 @@ __global__ void __launch_bounds__(TcCfg<D, NT, NCW, STAGES>::kThreads, TcCfg<D, 
                 prev = __shfl_sync(0xffffffffu, prev, 0);
                 if (prev == m.nparts - 1) {
                     const int qs = nq % C::kQSlots;
-                    if (!__all_sync(0xffffffffu, mbar_wait(&qempty[qs], ((nq / C::kQSlots) & 1) ^ 1))) {
+                    if (!__all_sync(0xffffffffu, wait_on(&qempty[qs], ((nq / C::kQSlots) & 1) ^ 1))) {
                         *abort_flag = 1;
                         break;
                     }
@@ -1133,7 +1136,7 @@ __global__ void __launch_bounds__(TcCfg<D, NT, NCW, STAGES>::kThreads, TcCfg<D, 
         // ---- deposit this warp's state in merge buffer iter % 2 (no CTA-wide barrier)
         const int mslot = iter & 1;
         const uint32_t mph = (iter >> 1) & 1;
-        if (!__all_sync(0xffffffffu, mbar_wait(&mempty[mslot], mph ^ 1))) {
+        if (!__all_sync(0xffffffffu, wait_on(&mempty[mslot], mph ^ 1))) {
             *abort_flag = 1;
             break;
         }
@@ -1165,7 +1168,7 @@ __global__ void __launch_bounds__(TcCfg<D, NT, NCW, STAGES>::kThreads, TcCfg<D, 
 
         // ---- the item's merger (warp iter % NCW) combines the NCW states and writes the result
         if (cw == iter % NCW) {
-            if (!__all_sync(0xffffffffu, mbar_wait(&mfull[mslot], mph))) {
+            if (!__all_sync(0xffffffffu, wait_on(&mfull[mslot], mph))) {
                 *abort_flag = 1;
                 break;
             }
@@ -1211,7 +1214,7 @@ __global__ void __launch_bounds__(TcCfg<D, NT, NCW, STAGES>::kThreads, TcCfg<D, 
     if constexpr (NCW == 1) {
         // tell the merger warp there is nothing more
         const int qs = nq % C::kQSlots;
-        const bool okq = __all_sync(0xffffffffu, mbar_wait(&qempty[qs], ((nq / C::kQSlots) & 1) ^ 1));
+        const bool okq = __all_sync(0xffffffffu, wait_on(&qempty[qs], ((nq / C::kQSlots) & 1) ^ 1));
         if (lane == 0) {
             if (!okq) *abort_flag = 1;
             tasks[qs] = make_int4(-1, 0, 0, 0);
@@ -1382,19 +1385,17 @@ namespace {
 // The ring holds the bytes in flight that cover HBM latency; each consumer
 // warp holds two stages while it computes.  kQuad is the automatic choice
 // (measured best on every workload once consumers took two blocks per step);
-// PA_TC_SHAPE selects another (tuning).
+// the others are selectable through DecodeOptions (pa_tuning.h) for tuning
+// and for the tests.
 enum class TcShape { kAuto, kPaired, kQuad, kTriple, kPair1 };
-TcShape tc_shape() {
-    static const TcShape s = [] {
-        const char* e = getenv("PA_TC_SHAPE");
-        const std::string v = e ? e : "";
-        if (v == "paired") return TcShape::kPaired;
-        if (v == "quad") return TcShape::kQuad;
-        if (v == "triple") return TcShape::kTriple;
-        if (v == "pair1") return TcShape::kPair1;
-        return TcShape::kAuto;
-    }();
-    return s;
+TcShape tc_shape(const DecodeOptions& o) {
+    switch (o.shape) {
+        case PA_SHAPE_PAIRED: return TcShape::kPaired;
+        case PA_SHAPE_QUAD: return TcShape::kQuad;
+        case PA_SHAPE_TRIPLE: return TcShape::kTriple;
+        case PA_SHAPE_PAIR1: return TcShape::kPair1;
+        default: return TcShape::kAuto;
+    }
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
@@ -1447,15 +1448,6 @@ cudaError_t dispatch_shape(int group, TcShape sh, F&& f) {
 
 constexpr int kSelfPlanMaxSeqs = 256;
 
-// PA_SELF_PLAN=0 keeps the plan kernel for every shape (tuning and tests)
-bool self_plan_allowed() {
-    static const bool on = [] {
-        const char* e = getenv("PA_SELF_PLAN");
-        return !(e && std::string(e) == "0");
-    }();
-    return on;
-}
-
 // What launch_decode enqueues for a problem.
 struct DecodeChoice {
     bool tc = false;         // tensor-core partition kernel (else SIMT)
@@ -1469,16 +1461,13 @@ struct DecodeChoice {
 
 // grid of a tensor-core instance (one wave of resident CTAs) and whether it can self-plan
 template <typename T, int D, int NT, int NCW, int STAGES>
-cudaError_t tc_choice(const DecodeParams& p, long long max_items, DecodeChoice* c) {
+cudaError_t tc_choice(const DecodeParams& p, const DecodeOptions& o, long long max_items, DecodeChoice* c) {
     using Cfg = TcCfg<D, NT, NCW, STAGES>;
     auto kernel = decode_tc_kernel<T, D, NT, NCW, STAGES>;
-    static bool attr_done = false;
-    if (!attr_done) {
-        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
-        if (e != cudaSuccess) return e;
-        attr_done = true;
-    }
-    cudaError_t e = prefer_max_shared(reinterpret_cast<const void*>(kernel));
+    // the attribute is per device: set it on every call (a cheap host-side call)
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    e = prefer_max_shared(reinterpret_cast<const void*>(kernel));
     if (e != cudaSuccess) return e;
     DeviceInfo dev;
     e = device_info(&dev);
@@ -1494,20 +1483,20 @@ cudaError_t tc_choice(const DecodeParams& p, long long max_items, DecodeChoice* 
     // Each self-planning CTA scans all of context_lens; past a few hundred
     // sequences one plan kernel is cheaper (measured: equal at 256, the plan
     // kernel 3.6% faster at 1024, self-planning 2-11% faster at 8 and 32).
-    c->self_plan = self_plan_allowed() && p.num_seqs <= kSelfPlanMaxSeqs && p.num_seqs <= Cfg::kPlanSeqs &&
+    c->self_plan = !o.force_plan_kernel && p.num_seqs <= kSelfPlanMaxSeqs && p.num_seqs <= Cfg::kPlanSeqs &&
                    (long long)p.num_seqs * p.num_kv_heads <= kCounterSlots &&
                    (max_items + grid - 1) / grid <= Cfg::kMaxOwn;
     return cudaSuccess;
 }
 
 template <typename T, int D>
-cudaError_t choose(const DecodeParams& p, pa_dtype dtype, DecodeChoice* c) {
+cudaError_t choose(const DecodeParams& p, const DecodeOptions& o, pa_dtype dtype, DecodeChoice* c) {
     const long long max_items = (long long)p.num_seqs * p.max_parts * p.num_kv_heads;
     *c = DecodeChoice{};
     if constexpr (!std::is_same<T, float>::value) {
         if (decode_path(dtype, D, p.group) == DecodePath::kTensorCore) {
             c->tc = true;
-            TcShape sh = tc_shape();
+            TcShape sh = tc_shape(o);
             // Automatic: four single-warp CTAs per SM, which merge partitions
             // themselves when there are at most kFusedMaxParts of them.
             if (sh == TcShape::kAuto) sh = TcShape::kQuad;
@@ -1516,7 +1505,7 @@ cudaError_t choose(const DecodeParams& p, pa_dtype dtype, DecodeChoice* c) {
             c->fused = one_warp && p.max_parts > 1 && p.max_parts <= kFusedMaxParts;
             const cudaError_t e = dispatch_shape(p.group, sh, [&](auto tag) {
                 using Tg = decltype(tag);
-                return tc_choice<T, D, Tg::NT, Tg::NCW, Tg::ST>(p, max_items, c);
+                return tc_choice<T, D, Tg::NT, Tg::NCW, Tg::ST>(p, o, max_items, c);
             });
             if (e != cudaSuccess) return e;
         }
@@ -1552,9 +1541,9 @@ cudaError_t launch_simt(const DecodeParams& p, cudaStream_t stream, long long ma
 }
 
 template <typename T, int D>
-cudaError_t launch_all(DecodeParams p, pa_dtype dtype, cudaStream_t stream) {
+cudaError_t launch_all(DecodeParams p, const DecodeOptions& o, pa_dtype dtype, cudaStream_t stream) {
     DecodeChoice c;
-    cudaError_t e = choose<T, D>(p, dtype, &c);
+    cudaError_t e = choose<T, D>(p, o, dtype, &c);
     if (e != cudaSuccess) return e;
     p.fused_merge = c.fused ? 1 : 0;
     p.self_plan = c.self_plan ? 1 : 0;
@@ -1588,27 +1577,6 @@ cudaError_t launch_all(DecodeParams p, pa_dtype dtype, cudaStream_t stream) {
     return e;
 }
 
-// partition lengths: full partitions and the remainder last (measured best);
-// PA_SPLIT=equal gives near-equal lengths (tuning)
-int equal_split() {
-    static const int v = [] {
-        const char* e = getenv("PA_SPLIT");
-        return (e && std::string(e) == "equal") ? 1 : 0;
-    }();
-    return v;
-}
-
-int class_first_order() {
-    // item order: every item of the split sequences first, so that their
-    // merges happen early (measured best with the fused merge);
-    // PA_PLAN_ORDER=size orders all items by size alone (tuning)
-    static const int cf = [] {
-        const char* e = getenv("PA_PLAN_ORDER");
-        return (e && std::string(e) == "size") ? 0 : 1;
-    }();
-    return cf;
-}
-
 }  // namespace
 
 DecodePath decode_path(pa_dtype dtype, int head_dim, int group) {
@@ -1617,29 +1585,31 @@ DecodePath decode_path(pa_dtype dtype, int head_dim, int group) {
     return DecodePath::kTensorCore;
 }
 
-cudaError_t launch_decode(const DecodeParams& p_in, pa_dtype dtype, cudaStream_t stream) {
-    DecodeParams p = p_in;
-    p.class_first = class_first_order();
-    p.equal_split = equal_split();
+cudaError_t launch_decode(const DecodeParams& p, const DecodeOptions& o, pa_dtype dtype, cudaStream_t stream) {
     switch (dtype) {
-        case PA_F32: return p.head_dim == 64 ? launch_all<float, 64>(p, dtype, stream)
-                                             : launch_all<float, 128>(p, dtype, stream);
-        case PA_F16: return p.head_dim == 64 ? launch_all<__half, 64>(p, dtype, stream)
-                                             : launch_all<__half, 128>(p, dtype, stream);
-        case PA_BF16: return p.head_dim == 64 ? launch_all<__nv_bfloat16, 64>(p, dtype, stream)
-                                              : launch_all<__nv_bfloat16, 128>(p, dtype, stream);
+        case PA_F32: return p.head_dim == 64 ? launch_all<float, 64>(p, o, dtype, stream)
+                                             : launch_all<float, 128>(p, o, dtype, stream);
+        case PA_F16: return p.head_dim == 64 ? launch_all<__half, 64>(p, o, dtype, stream)
+                                             : launch_all<__half, 128>(p, o, dtype, stream);
+        case PA_BF16: return p.head_dim == 64 ? launch_all<__nv_bfloat16, 64>(p, o, dtype, stream)
+                                              : launch_all<__nv_bfloat16, 128>(p, o, dtype, stream);
     }
     return cudaErrorInvalidValue;
 }
 
-cudaError_t decode_launch_count(const DecodeParams& p, pa_dtype dtype, int* launches) {
+cudaError_t decode_launch_count(const DecodeParams& p, const DecodeOptions& o, pa_dtype dtype, int* launches) {
     DecodeChoice c;
     cudaError_t e = cudaErrorInvalidValue;
     switch (dtype) {
-        case PA_F32: e = p.head_dim == 64 ? choose<float, 64>(p, dtype, &c) : choose<float, 128>(p, dtype, &c); break;
-        case PA_F16: e = p.head_dim == 64 ? choose<__half, 64>(p, dtype, &c) : choose<__half, 128>(p, dtype, &c); break;
+        case PA_F32:
+            e = p.head_dim == 64 ? choose<float, 64>(p, o, dtype, &c) : choose<float, 128>(p, o, dtype, &c);
+            break;
+        case PA_F16:
+            e = p.head_dim == 64 ? choose<__half, 64>(p, o, dtype, &c) : choose<__half, 128>(p, o, dtype, &c);
+            break;
         case PA_BF16:
-            e = p.head_dim == 64 ? choose<__nv_bfloat16, 64>(p, dtype, &c) : choose<__nv_bfloat16, 128>(p, dtype, &c);
+            e = p.head_dim == 64 ? choose<__nv_bfloat16, 64>(p, o, dtype, &c)
+                                 : choose<__nv_bfloat16, 128>(p, o, dtype, &c);
             break;
     }
     if (e == cudaSuccess) *launches = c.launches;

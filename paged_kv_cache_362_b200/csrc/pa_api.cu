@@ -60,17 +60,48 @@ int64_t ceil_div64(int64_t a, int64_t b) { return (a + b - 1) / b; }
 // size that stays within that limit is taken instead, provided it still
 // fills one wave of CTAs (4 per SM): one launch instead of an extra reduce
 // kernel, measured 6% faster for 32 sequences of up to 2048 tokens.
+//
+// The SM count is the current device's (148 on a B200, also the value taken
+// when no device can be queried); pa_decode_workspace_size and pa_decode
+// therefore agree as long as they are called with the same device current.
+int64_t current_sm_count() {
+    DeviceInfo d;
+    return device_info(&d) == cudaSuccess && d.sm_count > 0 ? d.sm_count : 148;
+}
+
 int auto_partition_size(int64_t num_seqs, int64_t num_kv_heads, int64_t max_context_len) {
+    const int64_t sms = current_sm_count();
     auto items = [&](int P) { return num_seqs * num_kv_heads * ceil_div64(max_context_len, P); };
     int P = 512;
-    while (P > 64 && items(P) < 8 * 148) P /= 2;
+    while (P > 64 && items(P) < 8 * sms) P /= 2;
     const int64_t fused = decode_fused_max_parts();
     if (ceil_div64(max_context_len, P) > fused) {
         int Pf = P;
         while (Pf < 512 && ceil_div64(max_context_len, Pf) > fused) Pf *= 2;
-        if (ceil_div64(max_context_len, Pf) <= fused && items(Pf) >= 4 * 148) P = Pf;
+        if (ceil_div64(max_context_len, Pf) <= fused && items(Pf) >= 4 * sms) P = Pf;
     }
     return P;
+}
+
+// Options of pa_decode_tuned: NULL (or all zero) gives the defaults.
+bool decode_options(const pa_decode_tuning* t, DecodeOptions* o, int* equal_split, int* class_first,
+                    uint64_t* wait_limit_ns, int* stall) {
+    *o = DecodeOptions{};
+    *equal_split = 0;
+    *class_first = 1;
+    *wait_limit_ns = kWaitLimitNs;
+    *stall = 0;
+    if (t == nullptr) return true;
+    if (t->shape < PA_SHAPE_AUTO || t->shape > PA_SHAPE_PAIR1) return false;
+    if ((t->planner | t->split | t->order | t->stall_first_item) & ~1) return false;
+    if (t->wait_limit_ns < 0) return false;
+    o->shape = t->shape;
+    o->force_plan_kernel = t->planner == 1;
+    *equal_split = t->split;
+    *class_first = t->order == 0 ? 1 : 0;
+    if (t->wait_limit_ns > 0) *wait_limit_ns = (uint64_t)t->wait_limit_ns;
+    *stall = t->stall_first_item;
+    return true;
 }
 
 // Workspace: a 256-byte header (the plan kernel's list length), the merge
@@ -143,6 +174,21 @@ pa_status pa_decode(void* out, const void* q, const void* key_cache, const void*
                     int32_t block_size, int32_t num_blocks, float scale, int32_t max_context_len,
                     int32_t partition_size, void* workspace, size_t workspace_bytes, pa_dtype dtype,
                     int32_t* status, pa_stream_t stream) {
+    return pa_decode_tuned(out, q, key_cache, value_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs,
+                           num_heads, num_kv_heads, head_dim, block_size, num_blocks, scale, max_context_len,
+                           partition_size, workspace, workspace_bytes, dtype, status, stream, nullptr);
+}
+
+pa_status pa_decode_tuned(void* out, const void* q, const void* key_cache, const void* value_cache,
+                          const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* context_lens,
+                          int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads, int32_t head_dim,
+                          int32_t block_size, int32_t num_blocks, float scale, int32_t max_context_len,
+                          int32_t partition_size, void* workspace, size_t workspace_bytes, pa_dtype dtype,
+                          int32_t* status, pa_stream_t stream, const pa_decode_tuning* tuning) {
+    DecodeOptions opt;
+    int equal_split = 0, class_first = 1, stall = 0;
+    uint64_t wait_limit = kWaitLimitNs;
+    if (!decode_options(tuning, &opt, &equal_split, &class_first, &wait_limit, &stall)) return PA_ERR_INVALID_ARG;
     if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || num_blocks <= 0 ||
         max_blocks_per_seq <= 0 || max_context_len < 0)
         return PA_ERR_INVALID_ARG;
@@ -193,12 +239,27 @@ pa_status pa_decode(void* out, const void* q, const void* key_cache, const void*
     p.part_m = reinterpret_cast<float*>(ws + w.off_m);
     p.part_l = reinterpret_cast<float*>(ws + w.off_l);
     p.part_o = reinterpret_cast<float*>(ws + w.off_o);
-    const cudaError_t e = launch_decode(p, dtype, reinterpret_cast<cudaStream_t>(stream));
+    p.equal_split = equal_split;
+    p.class_first = class_first;
+    p.wait_limit_ns = wait_limit;
+    p.stall_first_item = stall;
+    const cudaError_t e = launch_decode(p, opt, dtype, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 int32_t pa_decode_launch_count(int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads, int32_t head_dim,
                                int32_t max_context_len, int32_t partition_size, pa_dtype dtype) {
+    return pa_decode_launch_count_tuned(num_seqs, num_heads, num_kv_heads, head_dim, max_context_len, partition_size,
+                                        dtype, nullptr);
+}
+
+int32_t pa_decode_launch_count_tuned(int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads, int32_t head_dim,
+                                     int32_t max_context_len, int32_t partition_size, pa_dtype dtype,
+                                     const pa_decode_tuning* tuning) {
+    DecodeOptions opt;
+    int equal_split = 0, class_first = 1, stall = 0;
+    uint64_t wait_limit = kWaitLimitNs;
+    if (!decode_options(tuning, &opt, &equal_split, &class_first, &wait_limit, &stall)) return -1;
     if (num_seqs <= 0 || num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads != 0) return -1;
     if (!valid_dtype(dtype) || (head_dim != 64 && head_dim != 128) || num_kv_heads > 255) return -1;
     WsLayout w;
@@ -213,7 +274,7 @@ int32_t pa_decode_launch_count(int32_t num_seqs, int32_t num_heads, int32_t num_
     p.part_blocks = w.partition_size / kChunk;
     p.max_parts = w.max_parts;
     int n = 0;
-    return decode_launch_count(p, dtype, &n) == cudaSuccess ? n : -1;
+    return decode_launch_count(p, opt, dtype, &n) == cudaSuccess ? n : -1;
 }
 
 pa_status pa_copy_blocks(void* key_cache, void* value_cache, const int64_t* block_pairs, int32_t num_pairs,

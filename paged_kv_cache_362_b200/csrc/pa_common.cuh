@@ -117,12 +117,12 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // reached through a logic error; it turns a hang into an error status).
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 15u) == 0 && global_timer_ns() - t0 > kWaitLimitNs) return false;
+        if ((i & 15u) == 0 && global_timer_ns() - t0 > limit_ns) return false;
     }
 }
 
@@ -254,6 +254,8 @@ struct DecodeParams {
     int class_first;              // item order: 1 = multi-partition sequences' items first
     int self_plan;                // 1: each partition-kernel CTA derives its own items (no plan kernel)
     int equal_split;              // 1: a sequence's partitions have near-equal lengths (else full + remainder)
+    int stall_first_item;         // test hook: CTA 0 never publishes its first item (its waits run out)
+    uint64_t wait_limit_ns;       // bound of every wait in the attention kernel
     int4* items;                  // [max_items]: (b, (p << 8) | g, clamped ctx, 0), largest first (plan kernel)
     float* part_m;                // [B, Hq, NP_max]   max logit (log2 units)
     float* part_l;                // [B, Hq, NP_max]   sum of 2^(s - m)

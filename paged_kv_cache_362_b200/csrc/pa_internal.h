@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 
 #include "pa_common.cuh"
+#include "pa_tuning.h"
 
 namespace pa {
 
@@ -41,12 +42,18 @@ DecodePath decode_path(pa_dtype dtype, int head_dim, int group);
 // zeroes the counters it uses.
 constexpr int kCounterSlots = 16384;
 
+// Host-side scheduling choices of a decode call (pa_decode_tuning).
+struct DecodeOptions {
+    int shape = PA_SHAPE_AUTO;       // pa_decode_shape
+    bool force_plan_kernel = false;  // the planning kernel even where attention CTAs could plan
+};
+
 // [plan] + partition kernel + (if sequences span several partitions and the
 // partition kernel does not merge them) reduce.
-cudaError_t launch_decode(const DecodeParams& p, pa_dtype dtype, cudaStream_t stream);
+cudaError_t launch_decode(const DecodeParams& p, const DecodeOptions& o, pa_dtype dtype, cudaStream_t stream);
 
 // Number of kernels launch_decode enqueues for these sizes (p's pointers unused).
-cudaError_t decode_launch_count(const DecodeParams& p, pa_dtype dtype, int* launches);
+cudaError_t decode_launch_count(const DecodeParams& p, const DecodeOptions& o, pa_dtype dtype, int* launches);
 
 // Most partitions per sequence that the attention kernel merges itself (more
 // take the reduce kernel).

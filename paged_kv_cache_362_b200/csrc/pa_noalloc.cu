@@ -35,25 +35,31 @@ void* g_scratch_addr[kMaxDevices] = {};
 // Device address of g_decode_scratch on the current device, resolved on the
 // first call made with that device current.  That first call also zero-fills
 // the array on `stream` and waits for it, so the state pa_decode expects of a
-// fresh workspace does not rest on how the module was loaded.
-cudaError_t scratch_address(void** out, cudaStream_t stream) {
+// fresh workspace does not rest on how the module was loaded.  A first call
+// on a stream that is being captured into a graph could neither wait nor
+// leave the fill out of the graph: it is refused (PA_ERR_INVALID_ARG) before
+// anything is enqueued.
+pa_status scratch_address(void** out, cudaStream_t stream) {
     int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return PA_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_mu);
     if (g_scratch_addr[dev] == nullptr) {
+        cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+        if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) return PA_ERR_CUDA;
+        if (cs != cudaStreamCaptureStatusNone) return PA_ERR_INVALID_ARG;
+        cudaError_t e;
         void* p = nullptr;
         e = cudaGetSymbolAddress(&p, g_decode_scratch);
-        if (e != cudaSuccess) return e;
+        if (e != cudaSuccess) return PA_ERR_CUDA;
         e = cudaMemsetAsync(p, 0, kStaticScratchBytes, stream);
-        if (e != cudaSuccess) return e;
+        if (e != cudaSuccess) return PA_ERR_CUDA;
         e = cudaStreamSynchronize(stream);
-        if (e != cudaSuccess) return e;
+        if (e != cudaSuccess) return PA_ERR_CUDA;
         g_scratch_addr[dev] = p;
     }
     *out = g_scratch_addr[dev];
-    return cudaSuccess;
+    return PA_OK;
 }
 
 }  // namespace
@@ -70,7 +76,8 @@ extern "C" pa_status pa_decode_noalloc(void* out, const void* q, const void* key
     if (need == 0) return PA_ERR_INVALID_ARG;
     if (need > kStaticScratchBytes) return PA_ERR_UNSUPPORTED;  // problem too large for the fixed scratch
     void* scratch = nullptr;
-    if (scratch_address(&scratch, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return PA_ERR_CUDA;
+    const pa_status st = scratch_address(&scratch, reinterpret_cast<cudaStream_t>(stream));
+    if (st != PA_OK) return st;
     return pa_decode(out, q, key_cache, value_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs,
                      num_heads, num_kv_heads, head_dim, block_size, num_blocks, scale, max_context_len,
                      partition_size, scratch, kStaticScratchBytes, dtype, status, stream);

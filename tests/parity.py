@@ -72,6 +72,74 @@ def compare(gpu: np.ndarray, ref: np.ndarray, dtype: str, what: str = ""):
     return float(err.max()), raw_rel
 
 
+def round_to_storage_bits(ref: np.ndarray, dtype: str) -> np.ndarray:
+    """The fp64 oracle rounded to the storage dtype, round-to-nearest-even, as raw uint16 bits.
+
+    f16 uses NumPy's conversion (correctly rounded from float64).  bf16 takes the
+    candidate from float32 and its two neighbours and keeps the nearest in fp64
+    (ties to the even pattern), so no double rounding creeps in.
+    """
+    ref = np.asarray(ref, dtype=np.float64)
+    if dtype == "f16":
+        return ref.astype(np.float16).view(np.uint16)
+    assert dtype == "bf16"
+    b32 = ref.astype(np.float32).view(np.uint32).astype(np.int64)
+    cand = (b32 + 0x7FFF + ((b32 >> 16) & 1)) >> 16
+    best, best_err = cand.copy(), None
+    for d in (-1, 0, 1):
+        c = (cand + d) & 0xFFFF
+        v = (c.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+        err = np.abs(v - ref)
+        if best_err is None:
+            best, best_err = c, err
+        else:
+            take = (err < best_err) | ((err == best_err) & ((c & 1) == 0))
+            best = np.where(take, c, best)
+            best_err = np.where(take, err, best_err)
+    return best.astype(np.uint16)
+
+
+def _ordered(bits: np.ndarray) -> np.ndarray:
+    """16-bit sign-magnitude patterns -> integers in value order (adjacent values differ by 1)."""
+    b = bits.astype(np.int64)
+    return np.where(b & 0x8000, -(b & 0x7FFF), b)
+
+
+def ulp_distance(gpu_bits: np.ndarray, ref: np.ndarray, dtype: str) -> np.ndarray:
+    """How many representable steps of the storage dtype lie between the GPU output and RNE(oracle)."""
+    return np.abs(_ordered(np.asarray(gpu_bits).view(np.uint16)) - _ordered(round_to_storage_bits(ref, dtype)))
+
+
+# Sharper check than the tolerance (16-bit outputs), next to compare().  Every
+# element must be within ULP_MAX[dtype] representable steps of the oracle
+# rounded to the storage dtype, unless its absolute error is below
+# ULP_FLOOR[dtype] (outputs near zero, where a step is far smaller than fp32
+# accumulation error).  bf16: the kernels carry P as a hi + lo pair (about 16
+# significant bits), so beyond fp32 rounding the only error is the final
+# rounding: 1 step.  f16: decode rounds P to f16 (11 bits) before the PV
+# product; that error is about a third of an output step on typical rows and
+# its tails reach a few steps, so f16 is held to 4 steps or 2^-14 absolute.
+ULP_MAX = {"bf16": 1, "f16": 4}
+ULP_FLOOR = {"bf16": 2.0 ** -20, "f16": 2.0 ** -14}
+
+
+def ulp_check(gpu_t, ref: np.ndarray, dtype: str, what: str = "") -> dict:
+    """Assert the 1-step check above on a device tensor of 16-bit outputs; return its statistics."""
+    import torch
+
+    if dtype not in ULP_MAX:
+        return {}
+    gbits = gpu_t.view(torch.int16).cpu().numpy().view(np.uint16).reshape(ref.shape)
+    gval = gpu_t.to(torch.float64).cpu().numpy().reshape(ref.shape)
+    dist = ulp_distance(gbits, ref, dtype)
+    err = np.abs(gval - ref)
+    bad = (dist > ULP_MAX[dtype]) & (err > ULP_FLOOR[dtype])
+    assert not bad.any(), (f"{what}: {int(bad.sum())} elements beyond {ULP_MAX[dtype]} step(s) of RNE(oracle), "
+                           f"max {int(dist[bad].max())} steps, abs error {float(err[bad].max()):.3e}")
+    return {"max_abs": float(err.max()), "over_2e-3": int((err > 2e-3).sum()), "max_steps": int(dist.max()),
+            "within_1_step": float((dist <= 1).mean()), "elements": int(dist.size)}
+
+
 class DeviceCase:
     """A workload's tensors on the device plus host copies taken before any kernel ran."""
 

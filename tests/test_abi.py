@@ -136,6 +136,28 @@ def test_decode_validation():
     assert _dec(B=0) == pa.PA_OK
 
 
+def test_decode_tuned_validation():
+    """pa_decode_tuned checks its options on the host before anything else; NULL options are pa_decode."""
+    import paged_kv_cache_362_b200 as pa
+
+    f = pa._lib.LIB.pa_decode_tuned
+
+    def dec_t(t, **o):
+        a = [o.get("out", FAKE), FAKE, FAKE, FAKE, FAKE, 4, FAKE, o.get("B", 2), 4, 2, 64, 16, 8,
+             ctypes.c_float(0.125), 64, 0, P(0x100000), 1 << 20, 1, None, None, None if t is None else ctypes.byref(t)]
+        return f(*a)
+
+    for bad in (pa.tuning(shape=5), pa.tuning(shape=-1), pa.tuning(planner=2), pa.tuning(split=-1),
+                pa.tuning(order=3), pa.tuning(wait_limit_ns=-5), pa.tuning(stall_first_item=2)):
+        assert dec_t(bad) == pa.PA_ERR_INVALID_ARG
+    # valid options fall through to pa_decode's own checks
+    assert dec_t(pa.tuning(shape="paired"), out=P(0)) == pa.PA_ERR_INVALID_ARG
+    assert dec_t(None, B=0) == pa.PA_OK
+    assert dec_t(pa.tuning(shape="pair1", planner=1, split=1, order=1, wait_limit_ns=1000), B=0) == pa.PA_OK
+    lc = pa._lib.LIB.pa_decode_launch_count_tuned
+    assert lc(8, 28, 4, 128, 4096, 512, 1, ctypes.byref(pa.tuning(shape=7))) == -1
+
+
 def test_copy_blocks_validation():
     import paged_kv_cache_362_b200 as pa
 

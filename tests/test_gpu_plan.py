@@ -125,20 +125,20 @@ def test_launch_counts():
 
 
 @pytest.mark.parametrize("env", [
-    {"PA_SELF_PLAN": "0"},          # the planning kernel writes the list
-    {"PA_PLAN_ORDER": "size"},      # all items by size alone
-    {"PA_SPLIT": "equal"},          # partitions of near-equal length
-    {"PA_TC_SHAPE": "paired"},      # 2 CTAs per SM, two consumer warps, 10-stage ring, reduce kernel
-    {"PA_TC_SHAPE": "triple"},      # 3 CTAs per SM, 8-stage ring
-    {"PA_TC_SHAPE": "pair1"},       # 2 CTAs per SM, 13-stage ring
-], ids=lambda e: ",".join(f"{k}={v}" for k, v in e.items()))
+    {"PA_TEST_DECODE_TUNING": "planner=1"},       # the planning kernel writes the list
+    {"PA_TEST_DECODE_TUNING": "order=1"},         # all items by size alone
+    {"PA_TEST_DECODE_TUNING": "split=1"},         # partitions of near-equal length
+    {"PA_TEST_DECODE_TUNING": "shape=paired"},    # 2 CTAs per SM, two consumer warps, 10-stage ring, reduce kernel
+    {"PA_TEST_DECODE_TUNING": "shape=triple"},    # 3 CTAs per SM, 8-stage ring
+    {"PA_TEST_DECODE_TUNING": "shape=pair1"},     # 2 CTAs per SM, 13-stage ring
+], ids=lambda e: ",".join(f"{v}" for v in e.values()))
 def test_scheduling_variants_in_subprocess(env):
-    """The same parity cases under the library's scheduling variants and kernel shapes (read once per process),
-    block sizes 8/16/32 with NaN in the unread slots included."""
+    """The same parity cases under the library's scheduling alternatives and kernel shapes (pa_decode_tuned,
+    set for the whole child test process), block sizes 8/16/32 with NaN in the unread slots included."""
     cmd = [sys.executable, "-m", "pytest", "-q", "-m", "gpu", "-p", "no:cacheprovider",
            os.path.join(ROOT, "tests", "test_gpu_decode.py"), os.path.join(ROOT, "tests", "test_gpu_plan.py"),
            os.path.join(ROOT, "tests", "test_gpu_block_sizes.py"),
-           "-k", "(small_cases_every_element and (28x4 or 16x2)) or full_size_step_sampled or bitwise "
+           "-k", "(small_cases_every_element and (28x4 or 16x2)) or full_size_step_every_sequence or bitwise "
                  "or planners_match_oracle or one_workspace or (every_element_nan and (28x4 or 32x2)) "
                  "or long_contexts or bad_block_drops"]
     r = subprocess.run(cmd, cwd=ROOT, env=dict(os.environ, **env), capture_output=True, text=True, timeout=900)

@@ -89,6 +89,38 @@ def test_noalloc_matches_workspace_decode_two_calls_in_a_row():
         compare(out_f64(got), oracle, c.dtype, f"noalloc call {k}")
 
 
+def test_noalloc_fused_merge_two_calls_in_a_row():
+    """Two problems of different shape whose long sequences split into 2 to 8 partitions, which the attention
+    kernel merges itself through per-(sequence, KV head) counters kept in the shared scratch: one launch per call
+    (checked), so the second call only gives the right bits if the first left those counters at zero."""
+    import torch
+
+    pa, _ = _lib()
+    cases = [
+        (get_config("qwen_layer", dtype="f16", num_blocks=700, ctx_kind="fixed",
+                    ctx_args=(2048, 700, 1500, 33, 1025, 256, 1800)), 256),
+        (get_config("qwen_layer", dtype="bf16", num_heads=16, num_kv_heads=2, num_blocks=600, ctx_kind="fixed",
+                    ctx_args=(1900, 512, 1300, 17, 2000)), 256),
+    ]
+    for k, (cfg, P_) in enumerate(cases):
+        wl = build_workload(cfg, seed=60 + k)
+        c = wl.cfg
+        parts = -(-wl.max_context_len // P_)
+        assert 2 <= parts <= 8
+        assert pa.decode_launch_count(wl.num_seqs, c.num_heads, c.num_kv_heads, c.head_dim, wl.max_context_len, P_,
+                                      c.dtype) == 1
+        vh = host_values(wl)
+        case = DeviceCase(wl, vh)
+        got = _noalloc(case, P_)
+        ref = _with_workspace(case, P_)   # a fresh, zeroed workspace
+        torch.cuda.synchronize()
+        assert int(case.status.item()) == 0
+        assert torch.equal(got.view(torch.int16), ref.view(torch.int16)), f"fused call {k}"
+        oracle = parity.c_oracle.decode(vh["q"], vh["key_cache"], vh["value_cache"], wl.block_tables,
+                                        wl.context_lens, c.scale, c.dtype, c.num_kv_heads)
+        compare(out_f64(got), oracle, c.dtype, f"noalloc fused call {k}")
+
+
 def test_noalloc_rejects_problems_beyond_the_fixed_scratch():
     pa, f = _lib()
     # 1024 sequences x 28 heads x 64 partitions x (128 + 2) floats is far above 32 MiB
