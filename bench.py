@@ -517,8 +517,10 @@ def prefill_throughput(seed: int, reps: int = 20):
     flops = 4 * Hq * D * B * sum(past + i + 1 for i in range(chunk))
     tf = flops / (ms * 1e-3) / 1e12
     peak, _ = measured_bf16_peak()
+    kernel = "tcgen05 (prefill_tc_kernel)" if chunk * (Hq // Hkv) >= 32 else "mma.sync (prefill_kernel)"
     return {"workload": f"{B} sequences x ({chunk} new on {past} cached tokens), 28/4 heads, D 128, bf16",
-            "ms": round(ms, 4), "tflops": round(tf, 1), "peak_tflops": peak, "frac": round(tf / peak, 4)}
+            "kernel": kernel, "ms": round(ms, 4), "tflops": round(tf, 1), "peak_tflops": peak,
+            "frac": round(tf / peak, 4)}
 
 
 def measured_bf16_peak():

@@ -1374,31 +1374,7 @@ __global__ void __launch_bounds__(128) decode_reduce_kernel(const DecodeParams p
 // ===========================================================================
 // host side
 // ===========================================================================
-namespace {
-
-// Shapes of the tensor-core partition kernel (consumer warps x ring stages; CTAs per SM
-// at D = 128 and a GQA group of at most 8, as shared memory allows):
-//   kPaired: 2 x 10 (80 KB ring), 2 CTAs per SM, warps merge through shared memory
-//   kQuad:   1 x 6  (48 KB ring), 4 CTAs per SM, one warp per item, no merge
-//   kTriple: 1 x 8  (64 KB ring), 3 CTAs per SM
-//   kPair1:  1 x 13 (104 KB ring), 2 CTAs per SM
-// The ring holds the bytes in flight that cover HBM latency; each consumer
-// warp holds two stages while it computes.  kQuad is the automatic choice
-// (measured best on every workload once consumers took two blocks per step);
-// the others are selectable through DecodeOptions (pa_tuning.h) for tuning
-// and for the tests.
-enum class TcShape { kAuto, kPaired, kQuad, kTriple, kPair1 };
-TcShape tc_shape(const DecodeOptions& o) {
-    switch (o.shape) {
-        case PA_SHAPE_PAIRED: return TcShape::kPaired;
-        case PA_SHAPE_QUAD: return TcShape::kQuad;
-        case PA_SHAPE_TRIPLE: return TcShape::kTriple;
-        case PA_SHAPE_PAIR1: return TcShape::kPair1;
-        default: return TcShape::kAuto;
-    }
-}
-
-PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+static PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
         void* f = nullptr;
         cudaDriverEntryPointQueryResult q;
@@ -1427,6 +1403,30 @@ cudaError_t make_pool_map(CUtensorMap* map, const void* pool, pa_dtype dtype, in
                               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+namespace {
+
+// Shapes of the tensor-core partition kernel (consumer warps x ring stages; CTAs per SM
+// at D = 128 and a GQA group of at most 8, as shared memory allows):
+//   kPaired: 2 x 10 (80 KB ring), 2 CTAs per SM, warps merge through shared memory
+//   kQuad:   1 x 6  (48 KB ring), 4 CTAs per SM, one warp per item, no merge
+//   kTriple: 1 x 8  (64 KB ring), 3 CTAs per SM
+//   kPair1:  1 x 13 (104 KB ring), 2 CTAs per SM
+// The ring holds the bytes in flight that cover HBM latency; each consumer
+// warp holds two stages while it computes.  kQuad is the automatic choice
+// (measured best on every workload once consumers took two blocks per step);
+// the others are selectable through DecodeOptions (pa_tuning.h) for tuning
+// and for the tests.
+enum class TcShape { kAuto, kPaired, kQuad, kTriple, kPair1 };
+TcShape tc_shape(const DecodeOptions& o) {
+    switch (o.shape) {
+        case PA_SHAPE_PAIRED: return TcShape::kPaired;
+        case PA_SHAPE_QUAD: return TcShape::kQuad;
+        case PA_SHAPE_TRIPLE: return TcShape::kTriple;
+        case PA_SHAPE_PAIR1: return TcShape::kPair1;
+        default: return TcShape::kAuto;
+    }
 }
 
 template <int NT_, int NCW_, int ST_>

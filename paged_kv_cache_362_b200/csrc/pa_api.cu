@@ -304,7 +304,8 @@ pa_status pa_prefill(void* out, const void* q, const void* key_cache, const void
     if (block_size != kChunk || (head_dim != 64 && head_dim != 128) || dtype == PA_F32 ||
         num_heads / num_kv_heads > 16)
         return PA_ERR_UNSUPPORTED;
-    if ((int64_t)num_blocks * num_kv_heads * kChunk * head_dim > INT64_MAX / 4) return PA_ERR_UNSUPPORTED;
+    // pool rows (blocks x KV heads x 16) index the tensor copies in int32
+    if ((int64_t)num_blocks * num_kv_heads * kChunk > INT32_MAX) return PA_ERR_UNSUPPORTED;
     if (num_seqs == 0 || max_query_len == 0) return PA_OK;
     if (!out || !q || !key_cache || !value_cache || !block_tables || !query_start || !context_lens)
         return PA_ERR_INVALID_ARG;

@@ -30,8 +30,18 @@ cudaError_t launch_swap_blocks(const void* src_key, const void* src_value, void*
                                int32_t dst_num_blocks, int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
                                int elt_bytes, int32_t* status, cudaStream_t stream);
 
-// Causal attention of each sequence's new query tokens over its paged cache.
+// Causal attention of each sequence's new query tokens over its paged cache:
+// the tcgen05 kernel where prefill_tc_serves() (chunks that fill its 128-row
+// tiles), else the mma.sync kernel.
 cudaError_t launch_prefill(const PrefillParams& p, pa_dtype dtype, cudaStream_t stream);
+bool prefill_tc_serves(const PrefillParams& p);
+cudaError_t launch_prefill_tc(const PrefillParams& p, pa_dtype dtype, cudaStream_t stream);
+
+// TMA descriptor of a K or V pool viewed as 2-D: rows of head_dim elements,
+// one row per (block, KV head, slot); a box is 16 rows (8 for 8-token blocks)
+// x 64 elements (128 B), 128-byte swizzled in shared memory.
+cudaError_t make_pool_map(CUtensorMap* map, const void* pool, pa_dtype dtype, int num_blocks, int num_kv_heads,
+                          int head_dim, int block_size);
 
 // Which main decode kernel serves a shape.
 enum class DecodePath { kTensorCore, kSimt };

@@ -238,12 +238,9 @@ cudaError_t launch_prefill_t(const PrefillParams& p, cudaStream_t stream) {
     using C = PrefillCfg<D>;
     auto kernel = prefill_kernel<T, D>;
     const size_t smem = (size_t)p.group * C::kQBytes + 2 * kStages * C::kTileBytes;
-    static size_t attr = 0;
-    if (smem > attr) {
-        const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-        attr = smem;
-    }
+    // the attribute is per device: set it on every call (a cheap host-side call)
+    const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
     const dim3 grid((p.max_query_len + kQTile - 1) / kQTile, p.num_kv_heads, p.num_seqs);
     return launch_pdl(kernel, grid, dim3(32 * p.group), smem, stream, p);
 }
@@ -251,6 +248,7 @@ cudaError_t launch_prefill_t(const PrefillParams& p, cudaStream_t stream) {
 }  // namespace
 
 cudaError_t launch_prefill(const PrefillParams& p, pa_dtype dtype, cudaStream_t stream) {
+    if (prefill_tc_serves(p)) return launch_prefill_tc(p, dtype, stream);
     if (dtype == PA_F16) return p.head_dim == 64 ? launch_prefill_t<__half, 64>(p, stream)
                                                  : launch_prefill_t<__half, 128>(p, stream);
     if (dtype == PA_BF16) return p.head_dim == 64 ? launch_prefill_t<__nv_bfloat16, 64>(p, stream)

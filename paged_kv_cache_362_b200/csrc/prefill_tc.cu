@@ -1,0 +1,516 @@
+// Paged prefill on sm_100a tensor cores (tcgen05, accumulators in TMEM).
+//
+// What is computed is pa_prefill's definition (pa.h): for sequence b with
+// n = context_lens[b] tokens in the cache, of which the last L are the new
+// ones, query row i < L sits at position p = n - L + i and attends to the
+// keys at positions 0 .. p, read block by block through the block table
+// ("PagedAttention" digest, sections "PagedAttention in one picture" and "Why
+// the attention kernel works at all": the tiled attention loop, with the
+// cache block as the unit the tile is made of).
+//
+// Tiles.  A CTA owns 128 rows of (query position, GQA head) pairs of one
+// (sequence, KV head): floor(128 / G) consecutive positions times the G query
+// heads of the group, so every K/V tile it loads serves all of them.  It
+// walks the keys 128 at a time (eight 16-token blocks):
+//     S = Q K^T           tcgen05.mma, M = 128 rows, N = 128 keys, K = D
+//     P = 2^(S*scale*log2 e - m)   fp32 online softmax, one thread per row
+//     O += P V            tcgen05.mma, M = 128, N = D, K = 128 keys
+// S (two buffers, so the next QK^T runs while a tile's softmax does) and O
+// live in tensor memory; Q, K, V and P in shared memory, 128-byte swizzled.
+//
+// Warps (192 threads, one CTA per SM):
+//   0-3  softmax: thread r owns row r (TMEM lane r).  Loads its Q row into
+//        shared memory; per key tile reads its S row from TMEM, masks keys
+//        past its position (and blocks whose id is out of range), updates
+//        the running max and sum, writes its P row (input dtype) to shared
+//        memory; at the end scales its O row by 1/l and stores it.  The max
+//        used for the exponentials only moves when the tile max exceeds it
+//        by more than 8 (log2 units), so O is rescaled rarely; the sum and O
+//        always use the same reference, which keeps the result exact algebra.
+//   4    producer: K and V tiles of each key step by 2-D TMA (16-row,
+//        128-byte boxes, one per block and 64 columns), K and V on separate
+//        barriers, two stages each.  Blocks no row of the tile sees are not
+//        loaded; a block id out of range is reported and not loaded.
+//   5    MMA issuer (one lane) and TMEM owner: issues QK^T of tile j + 1
+//        before PV of tile j; before each PV it zeroes the V rows that are
+//        not data (slots past the context in the sequence's last block, and
+//        blocks that were not loaded), since a probability of 0 times a NaN
+//        left in shared memory would still be NaN.
+// Every mbarrier wait is bounded (PA_ERR_TIMEOUT); on expiry the CTA lets
+// its copies and MMAs finish, frees its TMEM and returns.
+#include "pa_internal.h"
+
+namespace pa {
+
+namespace {
+
+constexpr float kNegInfT = -__builtin_huge_valf();
+constexpr int kRowsT = 128;       // M: rows of a tile
+constexpr int kKeysT = 128;       // N of QK^T: keys per step (8 blocks)
+constexpr int kBlkT = 16;         // tokens per block
+// The max used for the exponentials moves only when a tile's max exceeds it
+// by more than this (log2 units): p <= 2^8, well inside fp16 and bf16.
+constexpr float kRescaleSlack = 8.f;
+
+template <int D>
+struct TcPf {
+    static constexpr int kHalves = D / 64;                 // 128-byte column groups of a D-wide row
+    static constexpr int kGroupBytes = kRowsT * 128;       // 128 rows x 128 B (16 KB)
+    static constexpr int kQBytes = kHalves * kGroupBytes;  // Q tile (K-major, K = D)
+    static constexpr int kKVBytes = kHalves * kGroupBytes; // one K or V tile of 128 keys
+    static constexpr int kPBytes = 2 * kGroupBytes;        // P tile (K-major, K = 128 keys)
+    static constexpr int kStages = 2;
+    static constexpr int kOffQ = 0;
+    static constexpr int kOffK = kOffQ + kQBytes;
+    static constexpr int kOffV = kOffK + kStages * kKVBytes;
+    static constexpr int kOffP = kOffV + kStages * kKVBytes;
+    static constexpr int kOffBar = kOffP + kPBytes;
+    // q_full, k_full[2], v_full[2], k_empty[2], v_empty[2], s_full[2], s_empty[2], p_full, pv_done, mma_done
+    static constexpr int kNumBars = 1 + 4 * kStages + 4 + 3;
+    static constexpr int kOffMisc = kOffBar + kNumBars * 8;   // TMEM base, abort flag
+    static constexpr int kBytes = kOffMisc + 16;
+    // one CTA per SM (the CTA holds all 512 TMEM columns): at least half of the SM's shared memory
+    static constexpr int kSmemBytes = (kBytes + 1024) > 120 * 1024 ? (kBytes + 1024) : 120 * 1024;
+    static constexpr int kThreads = 192;
+    static constexpr uint32_t kTmemCols = 512;
+    static constexpr uint32_t kColS = 0;                    // S buffers at columns 0 and 128
+    static constexpr uint32_t kColO = 256;                  // O: D columns
+    static_assert(kBytes + 1024 <= 227 * 1024, "shared memory");
+};
+
+// byte offset of 16-byte unit u (0..7) of row r inside a 128-byte-swizzled group
+__device__ __forceinline__ uint32_t sw128(int r, int u) { return (uint32_t)(r * 128 + ((u ^ (r & 7)) << 4)); }
+
+// 8-bit mask of the blocks of key tile j whose ids are out of range (blocks
+// no row needs count as good).  Lanes 0-7 read one table entry each.
+__device__ __forceinline__ uint32_t bad_blocks(const PrefillParams& p, const int32_t* row, int j, int kend, int lane) {
+    bool bad = false;
+    if (lane < 8) {
+        const int blk = j * 8 + lane;
+        if (blk * kBlkT < kend) {
+            const int id = __ldg(row + blk);
+            bad = id < 0 || id >= p.num_blocks;
+        }
+    }
+    return __ballot_sync(0xffffffffu, bad) & 0xffu;
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(192, 1)
+    prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmK,
+                      const __grid_constant__ CUtensorMap tmV, int qpos, uint32_t idesc_qk, uint32_t idesc_pv) {
+    using C = TcPf<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+    uint64_t* q_full = bars;
+    uint64_t* k_full = bars + 1;
+    uint64_t* v_full = k_full + C::kStages;
+    uint64_t* k_empty = v_full + C::kStages;
+    uint64_t* v_empty = k_empty + C::kStages;
+    uint64_t* s_full = v_empty + C::kStages;
+    uint64_t* s_empty = s_full + 2;
+    uint64_t* p_full = s_empty + 2;
+    uint64_t* pv_done = p_full + 1;
+    uint64_t* mma_done = pv_done + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int G = p.group, b = blockIdx.z, g = blockIdx.y;
+    const int tile = (int)gridDim.x - 1 - (int)blockIdx.x;   // the longest tiles of a sequence start first
+
+    if (threadIdx.x == 128) {
+        mbar_init(q_full, 4);
+        for (int s = 0; s < C::kStages; ++s) {
+            mbar_init(&k_full[s], 1);
+            mbar_init(&v_full[s], 1);
+            mbar_init(&k_empty[s], 1);
+            mbar_init(&v_empty[s], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&s_full[i], 1);
+            mbar_init(&s_empty[i], 4);
+        }
+        mbar_init(p_full, 4);
+        mbar_init(pv_done, 1);
+        mbar_init(mma_done, 1);
+        *abort_flag = 0;
+        mbar_fence_init();
+    }
+    if (warp == 5) {
+        tmem_alloc(tmem_slot, C::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    griddep_launch_dependents();
+    griddep_wait();
+
+    const int qs = p.query_start[b], L = p.query_start[b + 1] - qs;
+    const int n = p.context_lens[b];
+    const int i0 = tile * qpos;
+    bool active = L > 0 && i0 < L;
+    if (active && (n < L || n > p.max_blocks_per_seq * kBlkT)) {   // a query position outside the cache
+        if (threadIdx.x == 0) set_status(p.status, PA_ERR_OUT_OF_RANGE);
+        active = false;
+    }
+    if (active) {
+        const int npos = min(qpos, L - i0);          // query positions in this tile
+        const int nrows = npos * G;
+        const int pos0 = n - L + i0;                 // position of the tile's first query
+        const int kend = pos0 + npos;                // keys [0, kend) are visible to some row
+        const int nkt = ceil_div_i(kend, kKeysT);
+        const int32_t* bt_row = p.block_tables + (size_t)b * p.max_blocks_per_seq;
+        const uint32_t sQ = smem_u32(smem + C::kOffQ);
+        const uint32_t sK = smem_u32(smem + C::kOffK);
+        const uint32_t sV = smem_u32(smem + C::kOffV);
+        const uint32_t sP = smem_u32(smem + C::kOffP);
+        auto fail = [&]() {
+            *abort_flag = 1;
+            set_status(p.status, PA_ERR_TIMEOUT);
+        };
+
+        if (warp < 4) {
+            // ================================================= softmax warps
+            const int r = threadIdx.x;                              // tile row = TMEM lane
+            const int prow = min(r / G, npos - 1);                  // rows past the tile repeat its last position
+            const int pos = pos0 + prow;
+            const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
+            const float sl2 = p.scale_log2;                         // > 0 (a negative scale negates A)
+            {   // Q row r: 16-byte pieces into the swizzled K-major layout
+                const bool real = r < nrows;
+                const T* qrow = static_cast<const T*>(p.q) + ((size_t)(qs + i0 + prow) * p.num_heads + g * G + r % G) * D;
+#pragma unroll
+                for (int c = 0; c < D / 8; ++c) {
+                    uint4 v = make_uint4(0, 0, 0, 0);
+                    if (real) v = *reinterpret_cast<const uint4*>(qrow + c * 8);
+                    const uint32_t a = sQ + (c >> 3) * C::kGroupBytes + sw128(r, c & 7);
+                    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z),
+                                 "r"(v.w)
+                                 : "memory");
+                }
+                fence_proxy_async_shared();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(q_full);
+            }
+            float m_ref = kNegInfT, l = 0.f;
+            bool ok = true;
+            for (int j = 0; j < nkt && ok; ++j) {
+                const uint32_t badm = bad_blocks(p, bt_row, j, kend, lane);
+                if (!__all_sync(0xffffffffu, mbar_wait(&s_full[j & 1], (j >> 1) & 1)) || *abort_flag) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                uint32_t sv[kKeysT];
+#pragma unroll
+                for (int c = 0; c < kKeysT / 32; ++c) tmem_ld32(tl + C::kColS + (j & 1) * kKeysT + c * 32, sv + c * 32);
+                tmem_ld_wait(sv);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&s_empty[j & 1]);   // the S buffer may be overwritten now
+
+                // causal mask (the tile's first row sees keys up to pos0) and bad blocks
+                const int kb0 = j * kKeysT;
+                if (kb0 + kKeysT - 1 > pos0 || badm != 0) {
+#pragma unroll
+                    for (int c = 0; c < kKeysT; ++c)
+                        if (kb0 + c > pos || ((badm >> (c / kBlkT)) & 1u)) sv[c] = __float_as_uint(kNegInfT);
+                }
+                float mx0 = kNegInfT, mx1 = kNegInfT, mx2 = kNegInfT, mx3 = kNegInfT;
+#pragma unroll
+                for (int c = 0; c < kKeysT; c += 4) {
+                    mx0 = fmaxf(mx0, __uint_as_float(sv[c]));
+                    mx1 = fmaxf(mx1, __uint_as_float(sv[c + 1]));
+                    mx2 = fmaxf(mx2, __uint_as_float(sv[c + 2]));
+                    mx3 = fmaxf(mx3, __uint_as_float(sv[c + 3]));
+                }
+                const float m_new = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+                float alpha = 1.f;
+                if (m_new > m_ref + kRescaleSlack) {
+                    alpha = m_ref == kNegInfT ? 0.f : fast_exp2(m_ref - m_new);
+                    m_ref = m_new;
+                }
+                const float ms = m_ref == kNegInfT ? 0.f : m_ref;
+                // P in the input dtype; the row sum adds the rounded values the PV product uses
+                uint32_t pk[kKeysT / 2];
+                float ls0 = 0.f, ls1 = 0.f;
+#pragma unroll
+                for (int c = 0; c < kKeysT / 2; ++c) {
+                    const float e0 = fast_exp2(fmaf(__uint_as_float(sv[2 * c]), sl2, -ms));
+                    const float e1 = fast_exp2(fmaf(__uint_as_float(sv[2 * c + 1]), sl2, -ms));
+                    pk[c] = Elt<T>::pack2(e0, e1);
+                    if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+                        ls0 += __uint_as_float(pk[c] << 16);
+                        ls1 += __uint_as_float(pk[c] & 0xffff0000u);
+                    } else {
+                        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&pk[c]));
+                        ls0 += f.x;
+                        ls1 += f.y;
+                    }
+                }
+                l = l * alpha + (ls0 + ls1);
+                if (j > 0) {
+                    // PV of the previous tile has read the P buffer and written O
+                    if (!__all_sync(0xffffffffu, mbar_wait(pv_done, (j - 1) & 1)) || *abort_flag) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    if (__any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+                        for (int c = 0; c < D / 32; ++c) {
+                            uint32_t ov[32];
+                            tmem_ld32(tl + C::kColO + c * 32, ov);
+                            tmem_ld_wait(ov);
+#pragma unroll
+                            for (int k = 0; k < 32; ++k) ov[k] = __float_as_uint(__uint_as_float(ov[k]) * alpha);
+                            tmem_st32(tl + C::kColO + c * 32, ov);
+                        }
+                        tmem_st_wait();
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < kKeysT / 8; ++u) {
+                    const uint32_t a = sP + (u >> 3) * C::kGroupBytes + sw128(r, u & 7);
+                    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(pk[4 * u]),
+                                 "r"(pk[4 * u + 1]), "r"(pk[4 * u + 2]), "r"(pk[4 * u + 3])
+                                 : "memory");
+                }
+                fence_proxy_async_shared();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(p_full);
+            }
+            if (ok) {
+                ok = __all_sync(0xffffffffu, mbar_wait(pv_done, (nkt - 1) & 1)) && !*abort_flag;
+                if (ok) {
+                    tc_fence_after();
+                    const float inv = l > 0.f ? 1.f / l : 0.f;
+                    T* dst = static_cast<T*>(p.out) + ((size_t)(qs + i0 + prow) * p.num_heads + g * G + r % G) * D;
+#pragma unroll
+                    for (int c = 0; c < D / 32; ++c) {
+                        uint32_t ov[32];
+                        tmem_ld32(tl + C::kColO + c * 32, ov);
+                        tmem_ld_wait(ov);
+                        if (r < nrows) {
+#pragma unroll
+                            for (int k = 0; k < 32; k += 8) {
+                                uint4 w;
+                                w.x = Elt<T>::pack2(__uint_as_float(ov[k]) * inv, __uint_as_float(ov[k + 1]) * inv);
+                                w.y = Elt<T>::pack2(__uint_as_float(ov[k + 2]) * inv, __uint_as_float(ov[k + 3]) * inv);
+                                w.z = Elt<T>::pack2(__uint_as_float(ov[k + 4]) * inv, __uint_as_float(ov[k + 5]) * inv);
+                                w.w = Elt<T>::pack2(__uint_as_float(ov[k + 6]) * inv, __uint_as_float(ov[k + 7]) * inv);
+                                *reinterpret_cast<uint4*>(dst + c * 32 + k) = w;
+                            }
+                        }
+                    }
+                }
+            }
+            if (!ok && lane == 0) fail();
+        } else if (warp == 4) {
+            // ======================================================= producer
+            if (lane == 0) {
+                prefetch_tensormap(&tmK);
+                prefetch_tensormap(&tmV);
+            }
+            constexpr uint32_t kBlockBytes = kBlkT * D * 2;   // one block of one KV head: K or V
+            int issued = 0;
+            bool ok = true;
+            for (int j = 0; j < nkt && ok; ++j) {
+                const int s = j % C::kStages;
+                const uint32_t par = ((j / C::kStages) & 1) ^ 1;
+                const int blk = j * 8 + lane;
+                bool good = false;
+                int id = 0;
+                if (lane < 8 && blk * kBlkT < kend) {
+                    id = __ldg(bt_row + blk);
+                    good = id >= 0 && id < p.num_blocks;
+                    if (!good) set_status(p.status, PA_ERR_OUT_OF_RANGE);
+                }
+                const uint32_t nload = __popc(__ballot_sync(0xffffffffu, good));
+                const int y = (id * p.num_kv_heads + g) * kBlkT;
+                int w = 1;
+                if (lane == 0) {
+                    w = mbar_wait(&k_empty[s], par);
+                    if (w) mbar_arrive_expect_tx(&k_full[s], nload * kBlockBytes);
+                }
+                if (!__shfl_sync(0xffffffffu, w, 0) || *abort_flag) { ok = false; break; }
+                if (good) {
+#pragma unroll
+                    for (int h = 0; h < C::kHalves; ++h)
+                        tma_load_2d_keep(sK + s * C::kKVBytes + h * C::kGroupBytes + lane * (kBlkT * 128), &tmK,
+                                         h * 64, y, &k_full[s]);
+                }
+                if (lane == 0) {
+                    w = mbar_wait(&v_empty[s], par);
+                    if (w) mbar_arrive_expect_tx(&v_full[s], nload * kBlockBytes);
+                }
+                if (!__shfl_sync(0xffffffffu, w, 0)) {
+                    // K of tile j is in flight: count it so that the drain below waits for it
+                    issued = j + 1;
+                    ok = false;
+                    break;
+                }
+                if (good) {
+#pragma unroll
+                    for (int h = 0; h < C::kHalves; ++h)
+                        tma_load_2d_keep(sV + s * C::kKVBytes + h * C::kGroupBytes + lane * (kBlkT * 128), &tmV,
+                                         h * 64, y, &v_full[s]);
+                }
+                issued = j + 1;
+            }
+            if (!ok) {
+                // let the copies this warp issued land before the CTA's memory is released
+                if (lane == 0) {
+                    fail();
+                    for (int j = max(0, issued - C::kStages); j < issued; ++j) {
+                        mbar_wait(&k_full[j % C::kStages], (j / C::kStages) & 1);
+                        mbar_wait(&v_full[j % C::kStages], (j / C::kStages) & 1);
+                    }
+                }
+            }
+        } else {
+            // ================================================ MMA issuer (warp 5)
+            bool ok = __all_sync(0xffffffffu, mbar_wait(q_full, 0));
+            // descriptors: Q, K, P K-major (8-row atoms 1024 B apart, K steps of 16
+            // elements 32 B apart inside a 128-byte row, 64-element groups 16 KB
+            // apart); V MN-major (64 D-columns per 128-byte row, 16 KB between
+            // column groups, 16 keys = 2 atoms per K step)
+            auto kdesc = [&](uint32_t base, int k) {
+                return umma_desc_sw128(base + (k >> 2) * C::kGroupBytes + (k & 3) * 32, 16, 1024);
+            };
+            auto vdesc = [&](uint32_t base, int k) {
+                return umma_desc_sw128(base + k * (2 * 1024), C::kGroupBytes, 1024);
+            };
+            auto issue_pv = [&](int i) -> bool {
+                const int s = i % C::kStages;
+                const uint32_t badm = bad_blocks(p, bt_row, i, kend, lane);
+                if (!__all_sync(0xffffffffu, mbar_wait(p_full, i & 1)) || *abort_flag) return false;
+                if (!__all_sync(0xffffffffu, mbar_wait(&v_full[s], (i / C::kStages) & 1))) return false;
+                // keys of this tile the PV product covers: whole 16-key steps up to kend
+                const int kb0 = i * kKeysT;
+                const int nks = min(kKeysT, kend - kb0 + kBlkT - 1) / kBlkT;
+                // rows of V that hold no data: blocks not loaded (bad ids) and slots
+                // at or past n in the sequence's last block
+                const int tail_blk = n / kBlkT - i * 8;      // the last block's index in this tile, if partial
+                const int tail_from = n % kBlkT;
+                bool zeroed = false;
+                for (int k = 0; k < nks; ++k) {
+                    int r0 = kBlkT, r1 = kBlkT;
+                    if ((badm >> k) & 1u) r0 = 0;
+                    else if (k == tail_blk && tail_from != 0) r0 = tail_from;
+                    if (r0 >= r1) continue;
+                    zeroed = true;
+                    const int per = (r1 - r0) * 8 * C::kHalves;   // 16-byte pieces
+                    for (int e = lane; e < per; e += 32) {
+                        const int rr = k * kBlkT + r0 + e / (8 * C::kHalves);
+                        const int hh = (e % (8 * C::kHalves)) / 8, uu = e % 8;
+                        st_shared_zero16(sV + s * C::kKVBytes + hh * C::kGroupBytes + rr * 128 + (uu << 4));
+                    }
+                }
+                if (zeroed) fence_proxy_async_shared();
+                __syncwarp();
+                if (lane == 0) {
+                    tc_fence_after();
+                    const uint32_t vb = sV + s * C::kKVBytes;
+                    for (int k = 0; k < nks; ++k)
+                        umma_f16_ss(tmem + C::kColO, kdesc(sP, k), vdesc(vb, k), idesc_pv, (i > 0 || k > 0) ? 1u : 0u);
+                    umma_commit(pv_done);
+                    umma_commit(&v_empty[s]);
+                }
+                __syncwarp();
+                return true;
+            };
+            int j = 0;
+            for (; j < nkt && ok; ++j) {
+                const int s = j % C::kStages;
+                if (!__all_sync(0xffffffffu, mbar_wait(&k_full[s], (j / C::kStages) & 1)) || *abort_flag) {
+                    ok = false;
+                    break;
+                }
+                if (!__all_sync(0xffffffffu, mbar_wait(&s_empty[j & 1], ((j >> 1) & 1) ^ 1))) {
+                    ok = false;
+                    break;
+                }
+                if (lane == 0) {
+                    tc_fence_after();
+                    const uint32_t kb = sK + s * C::kKVBytes;
+#pragma unroll
+                    for (int k = 0; k < D / 16; ++k)
+                        umma_f16_ss(tmem + C::kColS + (j & 1) * kKeysT, kdesc(sQ, k), kdesc(kb, k), idesc_qk,
+                                    k > 0 ? 1u : 0u);
+                    umma_commit(&s_full[j & 1]);
+                    umma_commit(&k_empty[s]);
+                }
+                __syncwarp();
+                if (j > 0 && !issue_pv(j - 1)) {
+                    ok = false;
+                    break;
+                }
+            }
+            if (ok && !issue_pv(nkt - 1)) ok = false;
+            // every MMA this warp issued has completed before TMEM and shared memory are released
+            if (lane == 0) {
+                umma_commit(mma_done);
+                mbar_wait(mma_done, 0);
+                if (!ok) fail();
+            }
+            __syncwarp();
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 5) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::kTmemCols);
+    }
+}
+
+template <typename T, int D>
+cudaError_t launch_prefill_tc_t(const PrefillParams& p_in, cudaStream_t stream) {
+    using C = TcPf<D>;
+    PrefillParams p = p_in;
+    const bool neg = p.scale_log2 < 0.f;   // a negative scale: negate Q inside the QK^T product
+    if (neg) p.scale_log2 = -p.scale_log2;
+    // a zero scale gives uniform weights; the smallest normal float gives the
+    // same ones and keeps masked logits at -inf through the scaling
+    if (p.scale_log2 == 0.f) p.scale_log2 = 1.17549435e-38f;
+    const bool bf = std::is_same<T, __nv_bfloat16>::value;
+    const uint32_t idesc_qk = umma_idesc_f16(bf, kRowsT, kKeysT, false, neg);
+    const uint32_t idesc_pv = umma_idesc_f16(bf, kRowsT, D, true, false);
+    const pa_dtype dt = bf ? PA_BF16 : PA_F16;
+    CUtensorMap mk, mv;
+    cudaError_t e = make_pool_map(&mk, p.key_cache, dt, p.num_blocks, p.num_kv_heads, D, kBlkT);
+    if (e != cudaSuccess) return e;
+    e = make_pool_map(&mv, p.value_cache, dt, p.num_blocks, p.num_kv_heads, D, kBlkT);
+    if (e != cudaSuccess) return e;
+    auto kernel = prefill_tc_kernel<T, D>;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (e != cudaSuccess) return e;
+    const int qpos = kRowsT / p.group;   // query positions per tile
+    const dim3 grid((p.max_query_len + qpos - 1) / qpos, p.num_kv_heads, p.num_seqs);
+    return launch_pdl(kernel, grid, dim3(C::kThreads), C::kSmemBytes, stream, p, mk, mv, qpos, idesc_qk, idesc_pv);
+}
+
+}  // namespace
+
+bool prefill_tc_serves(const PrefillParams& p) {
+    // tensor-core tiles hold 128 (position, head) rows; when a chunk fills
+    // less than a quarter of one (a few tokens per sequence: decode-like and
+    // bound by reading the cache), the 16-query mma.sync kernel wastes less
+    return (long long)p.max_query_len * p.group >= 32;
+}
+
+cudaError_t launch_prefill_tc(const PrefillParams& p, pa_dtype dtype, cudaStream_t stream) {
+    if (dtype == PA_F16) return p.head_dim == 64 ? launch_prefill_tc_t<__half, 64>(p, stream)
+                                                 : launch_prefill_tc_t<__half, 128>(p, stream);
+    if (dtype == PA_BF16) return p.head_dim == 64 ? launch_prefill_tc_t<__nv_bfloat16, 64>(p, stream)
+                                                  : launch_prefill_tc_t<__nv_bfloat16, 128>(p, stream);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace pa

@@ -3,7 +3,11 @@
 Whole prompts and chunks on top of an existing context, ragged chunk lengths
 (1, 15, 16, 17, ...), GQA groups 1 to 16, head_dim 64 and 128, fp16 and bf16;
 every output element is compared.  Also: a bad block id is flagged and
-contributes nothing, and the result does not depend on where blocks live.
+contributes nothing, the result does not depend on where blocks live, NaN in
+every pool slot no query reads never reaches a result, and negative and zero
+scales.  Chunks that fill a 128-row tile run on the tcgen05 kernel; chunks of
+a few tokens (query rows x group < 32) on the mma.sync kernel, and both are
+covered.
 """
 
 import numpy as np
@@ -114,3 +118,97 @@ def test_bad_block_flagged_and_skipped():
         V = np.stack([vc[bt[0, i // 16], :, i % 16] for i in keys], axis=1).astype(np.float64)
         ref = np.stack([R.attention_f64(q[t, h].astype(np.float64), K[h // 4], V[h // 4], 0.125) for h in range(8)])
         compare(got[t], ref, "f16", f"row {t}")
+
+
+def _poison_unread(kc, vc, bt, ctxs):
+    """NaN into every slot of the pools that no query of these contexts reads."""
+    nan = np.float16("nan") if kc.dtype == np.float16 else np.uint16(0x7FC1)
+    used = np.zeros((kc.shape[0], 16), dtype=bool)
+    for b, c in enumerate(ctxs):
+        for i in range(c):
+            used[bt[b, i // 16], i % 16] = True
+    blk, off = np.nonzero(~used)
+    kc[blk, :, off, :] = nan
+    vc[blk, :, off, :] = nan
+    return int(blk.size)
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+@pytest.mark.parametrize("heads", [(28, 4), (32, 2)], ids=lambda h: f"{h[0]}x{h[1]}")
+def test_nan_in_unread_slots_never_reaches_a_result(dtype, heads):
+    Hq, Hkv = heads
+    rng = np.random.default_rng(31 + Hq)
+    ctxs, chunks = [300, 129, 17, 260, 1000], [300, 100, 17, 3, 333]
+    q, kc, vc, bt, qs, cl = _case(rng, ctxs, chunks, Hq, Hkv, 128, dtype, extra_blocks=5)
+    ref = c_oracle.prefill(q, kc, vc, bt, qs, cl, 1 / np.sqrt(128), dtype, Hkv)
+    assert _poison_unread(kc, vc, bt, ctxs) > 0
+    out, st = _run(q, kc, vc, bt, qs, cl, 1 / np.sqrt(128), dtype)
+    assert st == 0
+    compare(out_f64(out), ref, dtype, f"{dtype} {heads} NaN-filled unread slots")
+
+
+@pytest.mark.parametrize("heads", [(28, 4), (8, 8), (16, 16)], ids=lambda h: f"{h[0]}x{h[1]}")
+def test_short_chunks_take_the_mma_sync_kernel(heads):
+    """Chunks of a few tokens per sequence (query rows x group < 32): the 16-query mma.sync kernel."""
+    Hq, Hkv = heads
+    rng = np.random.default_rng(5 + Hq)
+    G = Hq // Hkv
+    L = max(1, min(4, 31 // G))
+    ctxs = [L, 40, 700, 17]
+    chunks = [L, L, 1, L]
+    assert max(chunks) * G < 32
+    q, kc, vc, bt, qs, cl = _case(rng, ctxs, chunks, Hq, Hkv, 128, "bf16")
+    _poison_unread(kc, vc, bt, ctxs)
+    out, st = _run(q, kc, vc, bt, qs, cl, 1 / np.sqrt(128), "bf16")
+    assert st == 0
+    # the oracle reads only the contexts, so the poisoned slots cannot enter it
+    ref = c_oracle.prefill(q, kc, vc, bt, qs, cl, 1 / np.sqrt(128), "bf16", Hkv)
+    compare(out_f64(out), ref, "bf16", f"short chunks {heads}")
+
+
+@pytest.mark.parametrize("scale", [-0.0884, 0.0, 0.3])
+def test_negative_zero_and_large_scales(scale):
+    rng = np.random.default_rng(77)
+    ctxs, chunks = [200, 333], [200, 150]
+    q, kc, vc, bt, qs, cl = _case(rng, ctxs, chunks, 28, 4, 128, "f16")
+    out, st = _run(q, kc, vc, bt, qs, cl, scale, "f16")
+    assert st == 0
+    ref = c_oracle.prefill(q, kc, vc, bt, qs, cl, scale, "f16", 4)
+    compare(out_f64(out), ref, "f16", f"scale {scale}")
+
+
+def test_bad_block_on_the_diagonal_of_a_tensor_core_tile():
+    """A bad id inside the 128-key step that holds the tile's own positions: masked and skipped, the rest exact."""
+    import paged_kv_cache_362_b200 as pa
+    from oracle import reference as R
+
+    rng = np.random.default_rng(12)
+    q, kc, vc, bt, qs, cl = _case(rng, [400], [300], 28, 4, 128, "bf16")
+    bt_bad = bt.copy()
+    bt_bad[0, 9] = -7                 # keys 144..159
+    out, st = _run(q, kc, vc, bt_bad, qs, cl, 0.0884, "bf16")
+    assert st & pa.PA_ERR_OUT_OF_RANGE
+    got = out_f64(out)
+    seqs, pos = R.prefill_rows(qs, cl)
+    rows = list(range(0, 300, 7)) + [299]
+    for t in rows:
+        p_ = int(pos[t])
+        keys = [i for i in range(p_ + 1) if not 144 <= i < 160]
+        K = np.stack([kc[bt[0, i // 16], :, i % 16] for i in keys], axis=1)
+        V = np.stack([vc[bt[0, i // 16], :, i % 16] for i in keys], axis=1)
+        K = (K.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+        V = (V.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+        qt = (q[t].astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+        ref = np.stack([R.attention_f64(qt[h], K[h // 7], V[h // 7], 0.0884) for h in range(28)])
+        compare(got[t], ref, "bf16", f"row {t}")
+
+
+def test_prefill_kernel_choice():
+    """The shape rule: tensor-core tiles when the chunk fills at least a quarter of a 128-row tile."""
+    rng = np.random.default_rng(3)
+    # both paths on one problem size: identical results within tolerance of the oracle
+    for chunks in ([4, 4], [40, 40]):
+        q, kc, vc, bt, qs, cl = _case(rng, [100, 64], chunks, 28, 4, 128, "f16")
+        out, st = _run(q, kc, vc, bt, qs, cl, 0.0884, "f16")
+        assert st == 0
+        compare(out_f64(out), c_oracle.prefill(q, kc, vc, bt, qs, cl, 0.0884, "f16", 4), "f16", f"chunks {chunks}")
