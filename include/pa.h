@@ -138,6 +138,13 @@ size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_heads, int32_t num
  *                       nothing (with 8-token blocks that includes the other
  *                       block of the tile; with 32-token blocks, both tiles
  *                       of the block)
+ *                       (with context_lens: read-only here, and possibly read
+ *                       before this call's kernels wait for kernels enqueued
+ *                       earlier with programmatic dependent launch, i.e.
+ *                       kernels that signal their dependents before they end;
+ *                       no kernel of this library writes either array, and a
+ *                       kernel without that signal has ended before this call
+ *                       starts)
  *   context_lens        int32 [num_seqs]; a value outside
  *                       [0, min(max_context_len, max_blocks_per_seq * BS)] is
  *                       clamped into that range and sets PA_ERR_OUT_OF_RANGE

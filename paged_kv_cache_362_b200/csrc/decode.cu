@@ -538,10 +538,14 @@ __global__ void __launch_bounds__(TcCfg<D, NT, NCW, STAGES>::kThreads, TcCfg<D, 
     __syncthreads();
 
     griddep_launch_dependents();
-    griddep_wait();
     const int PB = p.part_blocks;
     int4* own = reinterpret_cast<int4*>(smem + C::kOffOwn);
     int* s_plan = const_cast<int*>(abort_flag) + 1;   // [0] list length, [1] own items (self-planning)
+    // Self-planning reads only context_lens and block_tables, which no kernel
+    // of this library writes, so it runs before the wait for the preceding
+    // kernel (the append of the same step, chained by programmatic dependent
+    // launch); everything that kernel may write -- the pools, q, out, the
+    // workspace -- is touched only after griddep_wait() below.
     if (p.self_plan) {
         {   // warm L2 with this CTA's share of the block tables: the rows are read right after planning
             const char* bt = reinterpret_cast<const char*>(p.block_tables);
@@ -556,6 +560,7 @@ __global__ void __launch_bounds__(TcCfg<D, NT, NCW, STAGES>::kThreads, TcCfg<D, 
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         __syncthreads();
     }
+    griddep_wait();
 
     if constexpr (NCW == 1) {
         if (warp == NCW + 1) {

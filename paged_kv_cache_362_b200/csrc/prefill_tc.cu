@@ -52,13 +52,15 @@ constexpr int kBlkT = 16;         // tokens per block
 // by more than this (log2 units): p <= 2^8, well inside fp16 and bf16.
 constexpr float kRescaleSlack = 8.f;
 
-template <int D>
+template <int D, bool kPTmem, bool kSplitP>
 struct TcPf {
     static constexpr int kHalves = D / 64;                 // 128-byte column groups of a D-wide row
     static constexpr int kGroupBytes = kRowsT * 128;       // 128 rows x 128 B (16 KB)
     static constexpr int kQBytes = kHalves * kGroupBytes;  // Q tile (K-major, K = D)
     static constexpr int kKVBytes = kHalves * kGroupBytes; // one K or V tile of 128 keys
-    static constexpr int kPBytes = 2 * kGroupBytes;        // P tile (K-major, K = 128 keys)
+    // P tile(s) in shared memory (K-major, K = 128 keys): hi, and with kSplitP also lo
+    static constexpr int kPTile = 2 * kGroupBytes;
+    static constexpr int kPBytes = kPTmem ? 0 : (kSplitP ? 2 : 1) * kPTile;
     static constexpr int kStages = 2;
     static constexpr int kOffQ = 0;
     static constexpr int kOffK = kOffQ + kQBytes;
@@ -75,6 +77,8 @@ struct TcPf {
     static constexpr uint32_t kTmemCols = 512;
     static constexpr uint32_t kColS = 0;                    // S buffers at columns 0 and 128
     static constexpr uint32_t kColO = 256;                  // O: D columns
+    static constexpr uint32_t kColP = 384;                  // P in tensor memory: 64 columns of 16-bit pairs
+    static constexpr uint32_t kColPLo = 448;                // and its lo part (kSplitP)
     static_assert(kBytes + 1024 <= 227 * 1024, "shared memory");
 };
 
@@ -95,11 +99,16 @@ __device__ __forceinline__ uint32_t bad_blocks(const PrefillParams& p, const int
     return __ballot_sync(0xffffffffu, bad) & 0xffu;
 }
 
-template <typename T, int D>
+template <typename T, int D, bool kPTmem>
 __global__ void __launch_bounds__(192, 1)
     prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, int qpos, uint32_t idesc_qk, uint32_t idesc_pv) {
-    using C = TcPf<D>;
+    // bf16 P (8-bit significand) would perturb the softmax weights by up to
+    // 2^-8, which on rows with a few comparable keys moves the output by up
+    // to ~1e-2; it is carried as hi + lo (two bf16 parts, ~16 bits) and the PV
+    // product runs once per part.  fp16 P (11 bits) is used as is.
+    constexpr bool kSplitP = std::is_same<T, __nv_bfloat16>::value;
+    using C = TcPf<D, kPTmem, kSplitP>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
@@ -235,17 +244,20 @@ __global__ void __launch_bounds__(192, 1)
                     m_ref = m_new;
                 }
                 const float ms = m_ref == kNegInfT ? 0.f : m_ref;
-                // P in the input dtype; the row sum adds the rounded values the PV product uses
+                // P in the input dtype (bf16: hi + lo); the row sum adds what the PV products
+                // use: the rounded fp16 values, or the fp32 values hi + lo carry to ~16 bits
                 uint32_t pk[kKeysT / 2];
+                uint32_t pl[kSplitP ? kKeysT / 2 : 1];
                 float ls0 = 0.f, ls1 = 0.f;
 #pragma unroll
                 for (int c = 0; c < kKeysT / 2; ++c) {
                     const float e0 = fast_exp2(fmaf(__uint_as_float(sv[2 * c]), sl2, -ms));
                     const float e1 = fast_exp2(fmaf(__uint_as_float(sv[2 * c + 1]), sl2, -ms));
                     pk[c] = Elt<T>::pack2(e0, e1);
-                    if constexpr (std::is_same<T, __nv_bfloat16>::value) {
-                        ls0 += __uint_as_float(pk[c] << 16);
-                        ls1 += __uint_as_float(pk[c] & 0xffff0000u);
+                    if constexpr (kSplitP) {
+                        pl[c] = Elt<T>::pack2(e0 - __uint_as_float(pk[c] << 16), e1 - __uint_as_float(pk[c] & 0xffff0000u));
+                        ls0 += e0;
+                        ls1 += e1;
                     } else {
                         const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&pk[c]));
                         ls0 += f.x;
@@ -273,14 +285,29 @@ __global__ void __launch_bounds__(192, 1)
                         tmem_st_wait();
                     }
                 }
+                if constexpr (kPTmem) {
+                    // P row r into TMEM lane r, keys 2c and 2c + 1 in column c
+                    tmem_st32(tl + C::kColP, pk);
+                    tmem_st32(tl + C::kColP + 32, pk + 32);
+                    if constexpr (kSplitP) {
+                        tmem_st32(tl + C::kColPLo, pl);
+                        tmem_st32(tl + C::kColPLo + 32, pl + 32);
+                    }
+                    tmem_st_wait();
+                } else {
 #pragma unroll
-                for (int u = 0; u < kKeysT / 8; ++u) {
-                    const uint32_t a = sP + (u >> 3) * C::kGroupBytes + sw128(r, u & 7);
-                    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(pk[4 * u]),
-                                 "r"(pk[4 * u + 1]), "r"(pk[4 * u + 2]), "r"(pk[4 * u + 3])
-                                 : "memory");
+                    for (int u = 0; u < kKeysT / 8; ++u) {
+                        const uint32_t a = sP + (u >> 3) * C::kGroupBytes + sw128(r, u & 7);
+                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(pk[4 * u]),
+                                     "r"(pk[4 * u + 1]), "r"(pk[4 * u + 2]), "r"(pk[4 * u + 3])
+                                     : "memory");
+                        if constexpr (kSplitP)
+                            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a + C::kPTile),
+                                         "r"(pl[4 * u]), "r"(pl[4 * u + 1]), "r"(pl[4 * u + 2]), "r"(pl[4 * u + 3])
+                                         : "memory");
+                    }
+                    fence_proxy_async_shared();
                 }
-                fence_proxy_async_shared();
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(p_full);
@@ -417,8 +444,22 @@ __global__ void __launch_bounds__(192, 1)
                 if (lane == 0) {
                     tc_fence_after();
                     const uint32_t vb = sV + s * C::kKVBytes;
-                    for (int k = 0; k < nks; ++k)
-                        umma_f16_ss(tmem + C::kColO, kdesc(sP, k), vdesc(vb, k), idesc_pv, (i > 0 || k > 0) ? 1u : 0u);
+                    for (int k = 0; k < nks; ++k) {
+                        if constexpr (kPTmem)
+                            umma_f16_ts(tmem + C::kColO, tmem + C::kColP + k * 8, vdesc(vb, k), idesc_pv,
+                                        (i > 0 || k > 0) ? 1u : 0u);
+                        else
+                            umma_f16_ss(tmem + C::kColO, kdesc(sP, k), vdesc(vb, k), idesc_pv,
+                                        (i > 0 || k > 0) ? 1u : 0u);
+                    }
+                    if constexpr (kSplitP) {
+                        for (int k = 0; k < nks; ++k) {
+                            if constexpr (kPTmem)
+                                umma_f16_ts(tmem + C::kColO, tmem + C::kColPLo + k * 8, vdesc(vb, k), idesc_pv, 1u);
+                            else
+                                umma_f16_ss(tmem + C::kColO, kdesc(sP + C::kPTile, k), vdesc(vb, k), idesc_pv, 1u);
+                        }
+                    }
                     umma_commit(pv_done);
                     umma_commit(&v_empty[s]);
                 }
@@ -470,9 +511,12 @@ __global__ void __launch_bounds__(192, 1)
     }
 }
 
+// P in shared memory (SS products) or in tensor memory (TS form of PV)
+constexpr bool kPrefillPInTmem = false;
+
 template <typename T, int D>
 cudaError_t launch_prefill_tc_t(const PrefillParams& p_in, cudaStream_t stream) {
-    using C = TcPf<D>;
+    using C = TcPf<D, kPrefillPInTmem, std::is_same<T, __nv_bfloat16>::value>;
     PrefillParams p = p_in;
     const bool neg = p.scale_log2 < 0.f;   // a negative scale: negate Q inside the QK^T product
     if (neg) p.scale_log2 = -p.scale_log2;
@@ -488,7 +532,7 @@ cudaError_t launch_prefill_tc_t(const PrefillParams& p_in, cudaStream_t stream) 
     if (e != cudaSuccess) return e;
     e = make_pool_map(&mv, p.value_cache, dt, p.num_blocks, p.num_kv_heads, D, kBlkT);
     if (e != cudaSuccess) return e;
-    auto kernel = prefill_tc_kernel<T, D>;
+    auto kernel = prefill_tc_kernel<T, D, kPrefillPInTmem>;
     e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
     const int qpos = kRowsT / p.group;   // query positions per tile

@@ -110,34 +110,55 @@ def ulp_distance(gpu_bits: np.ndarray, ref: np.ndarray, dtype: str) -> np.ndarra
     return np.abs(_ordered(np.asarray(gpu_bits).view(np.uint16)) - _ordered(round_to_storage_bits(ref, dtype)))
 
 
-# Sharper check than the tolerance (16-bit outputs), next to compare().  Every
-# element must be within ULP_MAX[dtype] representable steps of the oracle
-# rounded to the storage dtype, unless its absolute error is below
-# ULP_FLOOR[dtype] (outputs near zero, where a step is far smaller than fp32
-# accumulation error).  bf16: the kernels carry P as a hi + lo pair (about 16
+def abs_values(arr: np.ndarray, dtype: str) -> np.ndarray:
+    """|x| of a host array in the oracle's storage convention (bf16 as uint16 bits)."""
+    return (arr & np.uint16(0x7FFF)) if dtype == "bf16" else np.abs(arr)
+
+
+# Sharper checks than the tolerance (16-bit outputs), next to compare().
+#
+# bf16: the decode kernel carries P as a hi + lo pair of bf16 (about 16
 # significant bits), so beyond fp32 rounding the only error is the final
-# rounding: 1 step.  f16: decode rounds P to f16 (11 bits) before the PV
-# product; that error is about a third of an output step on typical rows and
-# its tails reach a few steps, so f16 is held to 4 steps or 2^-14 absolute.
-ULP_MAX = {"bf16": 1, "f16": 4}
-ULP_FLOOR = {"bf16": 2.0 ** -20, "f16": 2.0 ** -14}
+# rounding to bf16.  Every element must be within 1 representable step of the
+# oracle rounded to bf16 (round-to-nearest-even), unless its absolute error is
+# below 2^-20 (outputs near zero, where a step is far smaller than the fp32
+# accumulation error).
+#
+# f16: the decode kernel rounds each p to f16 (relative error <= 2^-11) before
+# the PV product and sums l from the unrounded p, so
+#     |out - oracle| <= 2^-11 * sum_i p_i |v_i| / sum_i p_i   (P rounding)
+#                     + 2^-11 * |oracle|                      (output rounding)
+# where the first sum is the oracle's own result with |V| in place of V.
+# Every element must meet that bound (times 1.01, plus 2^-16 for fp32
+# accumulation and f16 subnormal p); its rows with few comparable keys reach
+# several output steps, so a step count is reported, not asserted.
+BF16_FLOOR = 2.0 ** -20
 
 
-def ulp_check(gpu_t, ref: np.ndarray, dtype: str, what: str = "") -> dict:
-    """Assert the 1-step check above on a device tensor of 16-bit outputs; return its statistics."""
+def sharp_check(gpu_t, ref: np.ndarray, dtype: str, ref_absv: np.ndarray | None = None, what: str = "") -> dict:
+    """Assert the check above for a device tensor of 16-bit outputs; return its statistics."""
     import torch
 
-    if dtype not in ULP_MAX:
+    if dtype not in ("bf16", "f16"):
         return {}
     gbits = gpu_t.view(torch.int16).cpu().numpy().view(np.uint16).reshape(ref.shape)
     gval = gpu_t.to(torch.float64).cpu().numpy().reshape(ref.shape)
     dist = ulp_distance(gbits, ref, dtype)
     err = np.abs(gval - ref)
-    bad = (dist > ULP_MAX[dtype]) & (err > ULP_FLOOR[dtype])
-    assert not bad.any(), (f"{what}: {int(bad.sum())} elements beyond {ULP_MAX[dtype]} step(s) of RNE(oracle), "
-                           f"max {int(dist[bad].max())} steps, abs error {float(err[bad].max()):.3e}")
+    if dtype == "bf16":
+        bad = (dist > 1) & (err > BF16_FLOOR)
+        assert not bad.any(), (f"{what}: {int(bad.sum())} elements beyond 1 step of RNE(oracle), "
+                               f"max {int(dist[bad].max())} steps, abs error {float(err[bad].max()):.3e}")
+        worst = None
+    else:
+        assert ref_absv is not None
+        bound = 1.01 * 2.0 ** -11 * (ref_absv.reshape(ref.shape) + np.abs(ref)) + 2.0 ** -16
+        bad = err > bound
+        assert not bad.any(), (f"{what}: {int(bad.sum())} elements beyond the P-rounding bound, "
+                               f"worst error/bound {float((err / bound).max()):.3f}")
+        worst = float((err / bound).max())
     return {"max_abs": float(err.max()), "over_2e-3": int((err > 2e-3).sum()), "max_steps": int(dist.max()),
-            "within_1_step": float((dist <= 1).mean()), "elements": int(dist.size)}
+            "within_1_step": float((dist <= 1).mean()), "worst_err_over_bound": worst, "elements": int(dist.size)}
 
 
 class DeviceCase:

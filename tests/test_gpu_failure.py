@@ -30,7 +30,7 @@ LIMIT_NS = 20_000_000   # 20 ms per wait
 
 
 def _case(seed):
-    cfg = get_config("qwen_layer", dtype="f16", num_blocks=400, ctx_kind="fixed",
+    cfg = get_config("qwen_layer", dtype="f16", num_blocks=600, ctx_kind="fixed",
                      ctx_args=(1500, 300, 17, 2048, 777, 64, 1200, 905))
     wl = build_workload(cfg, seed=seed)
     vh = host_values(wl)
