@@ -337,22 +337,34 @@ struct DescSlot {
 // per-sequence item counts.  Scratch lives in the tile ring, which is free
 // until the first copy.
 //
+// Scratch layout (ints): key counts, key offsets, then per sequence its
+// clamped context length, nbig, partition count and keys.
+constexpr int kPlanCtxOff = 2 * kMaxKeys + 2;
+
+// First step of self-planning, issued at the very start of the kernel so that
+// its latency overlaps the prologue: context_lens into the scratch, one
+// cp.async group per thread (plan_own_items waits for it).
+__device__ __forceinline__ void plan_load_ctx(const DecodeParams& p, int* scratch) {
+    int* s_ctx = scratch + kPlanCtxOff;
+    for (int b = threadIdx.x; b < p.num_seqs; b += blockDim.x) cp_async_4(smem_u32(&s_ctx[b]), p.context_lens + b);
+    cp_async_commit();
+}
+
 // Fills own[0 .. n_own) with this CTA's items (ranks c, 2C-1-c, 2C+c, ...);
-// s_list[0] = list length, s_list[1] = n_own.  Called by every thread of the CTA.
+// s_list[0] = list length, s_list[1] = n_own.  Called by every thread of the
+// CTA, after plan_load_ctx.
 template <int kMaxOwn>
 __device__ void plan_own_items(const DecodeParams& p, int* scratch, int4* own, int* s_list) {
     const int tid = threadIdx.x, nthr = blockDim.x, lane = tid & 31, wid = tid >> 5, nwarps = nthr >> 5;
     const int B = p.num_seqs;
     int* s_cnt = scratch;                        // [kMaxKeys]
     int* s_off = s_cnt + kMaxKeys;               // [kMaxKeys + 1]
-    int* s_ctx = s_off + kMaxKeys + 2;           // [B] clamped context lengths
+    int* s_ctx = scratch + kPlanCtxOff;          // [B] clamped context lengths
     int* s_r = s_ctx + B;                        // [B] partitions of the longer length (nbig)
     int* s_np = s_r + B;                         // [B] partitions
     int* s_key = s_np + B;                       // [B] kbig | ksmall << 8
     const PlanKeys K{p.part_blocks, p.part_blocks + 1, p.num_kv_heads, p.class_first};
     const int nkeys = K.nkeys();
-    for (int b = tid; b < B; b += nthr) cp_async_4(smem_u32(&s_ctx[b]), p.context_lens + b);
-    cp_async_commit();
     for (int i = tid; i < nkeys; i += nthr) s_cnt[i] = 0;
     cp_async_wait_all();
     __syncthreads();
@@ -506,6 +518,7 @@ __global__ void __launch_bounds__(TcCfg<D, NT, NCW, STAGES>::kThreads, TcCfg<D, 
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = p.group;
+    if (p.self_plan) plan_load_ctx(p, reinterpret_cast<int*>(stages));
     // every wait of the kernel is bounded (p.wait_limit_ns); on expiry the
     // kernel reports PA_ERR_TIMEOUT, lets the copies it issued land and returns
     const uint64_t wait_limit = p.wait_limit_ns;

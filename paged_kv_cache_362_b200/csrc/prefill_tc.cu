@@ -85,18 +85,16 @@ struct TcPf {
 // byte offset of 16-byte unit u (0..7) of row r inside a 128-byte-swizzled group
 __device__ __forceinline__ uint32_t sw128(int r, int u) { return (uint32_t)(r * 128 + ((u ^ (r & 7)) << 4)); }
 
-// 8-bit mask of the blocks of key tile j whose ids are out of range (blocks
-// no row needs count as good).  Lanes 0-7 read one table entry each.
-__device__ __forceinline__ uint32_t bad_blocks(const PrefillParams& p, const int32_t* row, int j, int kend, int lane) {
-    bool bad = false;
-    if (lane < 8) {
-        const int blk = j * 8 + lane;
-        if (blk * kBlkT < kend) {
-            const int id = __ldg(row + blk);
-            bad = id < 0 || id >= p.num_blocks;
-        }
-    }
-    return __ballot_sync(0xffffffffu, bad) & 0xffu;
+// Block ids of key tile j: lane l < 8 reads the table entry of block 8j + l
+// if some row of the tile needs it (else 0, a valid id).  Issued a tile ahead
+// of its use, so no global-memory latency sits in front of an MMA issue.
+__device__ __forceinline__ int tile_block_id(const int32_t* row, int j, int nkt, int kend, int lane) {
+    const int blk = j * 8 + lane;
+    return (j < nkt && lane < 8 && blk * kBlkT < kend) ? __ldg(row + blk) : 0;
+}
+// 8-bit mask of the blocks of a key tile whose ids are out of range
+__device__ __forceinline__ uint32_t bad_mask(const PrefillParams& p, int id) {
+    return __ballot_sync(0xffffffffu, id < 0 || id >= p.num_blocks) & 0xffu;
 }
 
 template <typename T, int D, bool kPTmem>
@@ -207,8 +205,10 @@ __global__ void __launch_bounds__(192, 1)
             }
             float m_ref = kNegInfT, l = 0.f;
             bool ok = true;
+            int id_next = tile_block_id(bt_row, 0, nkt, kend, lane);
             for (int j = 0; j < nkt && ok; ++j) {
-                const uint32_t badm = bad_blocks(p, bt_row, j, kend, lane);
+                const int id_cur = id_next;
+                id_next = tile_block_id(bt_row, j + 1, nkt, kend, lane);
                 if (!__all_sync(0xffffffffu, mbar_wait(&s_full[j & 1], (j >> 1) & 1)) || *abort_flag) {
                     ok = false;
                     break;
@@ -221,6 +221,7 @@ __global__ void __launch_bounds__(192, 1)
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&s_empty[j & 1]);   // the S buffer may be overwritten now
+                const uint32_t badm = bad_mask(p, id_cur);
 
                 // causal mask (the tile's first row sees keys up to pos0) and bad blocks
                 const int kb0 = j * kKeysT;
@@ -347,17 +348,15 @@ __global__ void __launch_bounds__(192, 1)
             constexpr uint32_t kBlockBytes = kBlkT * D * 2;   // one block of one KV head: K or V
             int issued = 0;
             bool ok = true;
+            int id_next = tile_block_id(bt_row, 0, nkt, kend, lane);
             for (int j = 0; j < nkt && ok; ++j) {
                 const int s = j % C::kStages;
                 const uint32_t par = ((j / C::kStages) & 1) ^ 1;
-                const int blk = j * 8 + lane;
-                bool good = false;
-                int id = 0;
-                if (lane < 8 && blk * kBlkT < kend) {
-                    id = __ldg(bt_row + blk);
-                    good = id >= 0 && id < p.num_blocks;
-                    if (!good) set_status(p.status, PA_ERR_OUT_OF_RANGE);
-                }
+                const int id = id_next;
+                id_next = tile_block_id(bt_row, j + 1, nkt, kend, lane);
+                const bool need = lane < 8 && (j * 8 + lane) * kBlkT < kend;
+                const bool good = need && id >= 0 && id < p.num_blocks;
+                if (need && !good) set_status(p.status, PA_ERR_OUT_OF_RANGE);
                 const uint32_t nload = __popc(__ballot_sync(0xffffffffu, good));
                 const int y = (id * p.num_kv_heads + g) * kBlkT;
                 int w = 1;
@@ -413,9 +412,9 @@ __global__ void __launch_bounds__(192, 1)
             auto vdesc = [&](uint32_t base, int k) {
                 return umma_desc_sw128(base + k * (2 * 1024), C::kGroupBytes, 1024);
             };
-            auto issue_pv = [&](int i) -> bool {
+            auto issue_pv = [&](int i, int ids) -> bool {
                 const int s = i % C::kStages;
-                const uint32_t badm = bad_blocks(p, bt_row, i, kend, lane);
+                const uint32_t badm = bad_mask(p, ids);
                 if (!__all_sync(0xffffffffu, mbar_wait(p_full, i & 1)) || *abort_flag) return false;
                 if (!__all_sync(0xffffffffu, mbar_wait(&v_full[s], (i / C::kStages) & 1))) return false;
                 // keys of this tile the PV product covers: whole 16-key steps up to kend
@@ -467,6 +466,7 @@ __global__ void __launch_bounds__(192, 1)
                 return true;
             };
             int j = 0;
+            int id_prev = 0, id_cur = tile_block_id(bt_row, 0, nkt, kend, lane);   // ids of tiles j - 1 and j
             for (; j < nkt && ok; ++j) {
                 const int s = j % C::kStages;
                 if (!__all_sync(0xffffffffu, mbar_wait(&k_full[s], (j / C::kStages) & 1)) || *abort_flag) {
@@ -488,12 +488,15 @@ __global__ void __launch_bounds__(192, 1)
                     umma_commit(&k_empty[s]);
                 }
                 __syncwarp();
-                if (j > 0 && !issue_pv(j - 1)) {
+                const int id_pv = id_prev;
+                id_prev = id_cur;
+                id_cur = tile_block_id(bt_row, j + 1, nkt, kend, lane);
+                if (j > 0 && !issue_pv(j - 1, id_pv)) {
                     ok = false;
                     break;
                 }
             }
-            if (ok && !issue_pv(nkt - 1)) ok = false;
+            if (ok && !issue_pv(nkt - 1, id_prev)) ok = false;
             // every MMA this warp issued has completed before TMEM and shared memory are released
             if (lane == 0) {
                 umma_commit(mma_done);
@@ -512,7 +515,7 @@ __global__ void __launch_bounds__(192, 1)
 }
 
 // P in shared memory (SS products) or in tensor memory (TS form of PV)
-constexpr bool kPrefillPInTmem = false;
+constexpr bool kPrefillPInTmem = true;
 
 template <typename T, int D>
 cudaError_t launch_prefill_tc_t(const PrefillParams& p_in, cudaStream_t stream) {
