@@ -214,7 +214,7 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 class DeviceWorkload:
     def __init__(self, name: str, seed: int, partition_size: int | None = None, placement: str | None = None,
-                 block_size: int | None = None):
+                 block_size: int | None = None, layers: int = 1):
         import torch
 
         import paged_kv_cache_362_b200 as pa
@@ -232,6 +232,11 @@ class DeviceWorkload:
         v = device_values(self.wl, dev)
         self.q, self.key, self.value = v["q"], v["key"], v["value"]
         self.kc, self.vc = v["key_cache"], v["value_cache"]
+        # one K/V pool per model layer; block tables, context lengths and q are
+        # shared by the layers of a step, as in a serving engine
+        self.kcs = [self.kc] + [self.kc.clone() for _ in range(layers - 1)]
+        self.vcs = [self.vc] + [self.vc.clone() for _ in range(layers - 1)]
+        self.layers = layers
         wl = self.wl
         self.bt = torch.from_numpy(wl.block_tables).to(dev)
         self.cl = torch.from_numpy(wl.context_lens).to(dev)
@@ -249,15 +254,16 @@ class DeviceWorkload:
                                                       self.max_ctx, self.P, c.dtype)
         self.launches_per_step = (1 if self.has_copy else 0) + 1 + self.decode_launches
 
-    def pre(self):
+    def pre(self, layer: int = 0):
+        kc, vc = self.kcs[layer], self.vcs[layer]
         if self.has_copy:
-            self.pa.copy_blocks(self.kc, self.vc, self.pairs, status=self.status)
-        self.pa.reshape_and_cache(self.key, self.value, self.kc, self.vc, self.slots, status=self.status)
+            self.pa.copy_blocks(kc, vc, self.pairs, status=self.status)
+        self.pa.reshape_and_cache(self.key, self.value, kc, vc, self.slots, status=self.status)
 
-    def decode(self):
+    def decode(self, layer: int = 0):
         c = self.cfg
-        self.pa.decode(self.out, self.q, self.kc, self.vc, self.bt, self.cl, c.scale, self.max_ctx, self.ws,
-                       partition_size=self.P, status=self.status)
+        self.pa.decode(self.out, self.q, self.kcs[layer], self.vcs[layer], self.bt, self.cl, c.scale, self.max_ctx,
+                       self.ws, partition_size=self.P, status=self.status)
 
 
 def unique_kv_bytes(wl) -> int:
@@ -347,6 +353,72 @@ def time_steps(w: DeviceWorkload, steps: int, warmup: int, flush, use_graph: boo
         run_pre()
         e0.record(stream)
         run_dec()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    dist_barrier()
+    dec_ms = [e0.elapsed_time(e1) for e0, e1 in ev]
+    return step_ms, dec_ms
+
+
+def time_steps_layers(w: DeviceWorkload, steps: int, warmup: int):
+    """Per-step CUDA-event times (ms) of consecutive steps that go to different layers' K/V pools.
+
+    A serving engine runs the decode once per layer, each layer on its own
+    pool, while block tables, context lengths and the kernels' code stay hot.
+    Step k here is layer k mod L of the workload (L pools of the workload's
+    size each, together far larger than L2), so no step finds in L2 the K/V
+    it reads: the step two layers back read other data of the same size.  No
+    flush runs between steps.  Whole steps (graphs of copy + append + decode)
+    and the decode alone (after an untimed append) are timed in two passes.
+    """
+    import torch
+
+    stream = torch.cuda.current_stream()
+    L = w.layers
+    for l in range(L):
+        for _ in range(2):
+            w.pre(l)
+            w.decode(l)
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    s.wait_stream(stream)
+    g_step, g_pre, g_dec = [], [], []
+    with torch.cuda.stream(s):
+        for l in range(L):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=s):
+                w.pre(l)
+                w.decode(l)
+            g_step.append(g)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=s):
+                w.pre(l)
+            g_pre.append(g)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=s):
+                w.decode(l)
+            g_dec.append(g)
+    stream.wait_stream(s)
+    torch.cuda.synchronize()
+    for k in range(max(warmup, 3) * L):
+        g_step[k % L].replay()
+    torch.cuda.synchronize()
+    dist_barrier()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for k, (e0, e1) in enumerate(ev):
+        e0.record(stream)
+        g_step[k % L].replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    dist_barrier()
+    step_ms = [e0.elapsed_time(e1) for e0, e1 in ev]
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for k, (e0, e1) in enumerate(ev):
+        g_pre[k % L].replay()
+        e0.record(stream)
+        g_dec[k % L].replay()
         e1.record(stream)
     torch.cuda.synchronize()
     dist_barrier()
@@ -618,6 +690,8 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of CPU oracle timing")
     ap.add_argument("--cpu-seqs", type=int, default=64)
     ap.add_argument("--ref-total-s", type=float, default=90.0, help="CPU seconds the reference arm may take")
+    ap.add_argument("--layers", type=int, default=4,
+                    help="K/V pools (model layers) the layer-rotation measurement cycles through")
     args = ap.parse_args()
 
     if args.impl == "reference":
@@ -645,9 +719,17 @@ def main():
     flush_write_only = lambda: flush_buf.zero_()
     use_graph = not args.no_graph
 
-    w = DeviceWorkload(args.workload, args.seed + rank, args.partition_size, block_size=args.block_size)
+    w = DeviceWorkload(args.workload, args.seed + rank, args.partition_size, block_size=args.block_size,
+                       layers=args.layers)
+    # Timed steps: consecutive steps decode different layers' K/V pools (the
+    # layer rotation of a serving engine: K/V cold, block tables and code hot);
+    # without graphs or with one layer, an L2 flush before every step instead
+    rotation = use_graph and w.layers > 1
     clocks = ClockSampler(torch.cuda.current_device())
-    step_ms, dec_ms = time_steps(w, args.steps, args.warmup, flush, use_graph)
+    if rotation:
+        step_ms, dec_ms = time_steps_layers(w, args.steps, args.warmup)
+    else:
+        step_ms, dec_ms = time_steps(w, args.steps, args.warmup, flush, use_graph)
     clk = clocks.stop()
     torch.cuda.synchronize()
     status = int(w.status.item())
@@ -658,6 +740,9 @@ def main():
     total_bytes = dist_sum(float(w.kv_bytes))
     dec = dist_max(float(np.mean(dec_ms)))
     achieved = w.kv_bytes / (dec * 1e-3) / 1e9
+    # the same steps after an L2 flush each (K/V, tables and the kernels' code all cold)
+    f_step, f_dec = time_steps(w, args.steps, args.warmup, flush, use_graph) if rotation else (step_ms, dec_ms)
+    f_s, f_d = dist_max(float(np.mean(f_step))), dist_max(float(np.mean(f_dec)))
 
     e2e_ms, h2d, d2h = time_e2e(w, max(50, args.steps // 10), args.warmup, flush)
     e2e = dist_max(float(np.mean(e2e_ms)))
@@ -665,6 +750,11 @@ def main():
     # writing back up to an L2 of the flush's dirty lines
     _, wo_dec = time_steps(w, max(50, args.steps // 10), args.warmup, flush_write_only, use_graph)
     wo = dist_max(float(np.mean(wo_dec)))
+    flushed = {"step_ms": round(f_s, 5), "decode_ms": round(f_d, 5),
+               "step_kv_gbs": round(w.kv_bytes / (f_s * 1e-3) / 1e9, 1),
+               "achieved": round(w.kv_bytes / (f_d * 1e-3) / 1e9, 1),
+               "frac": round(w.kv_bytes / (f_d * 1e-3) / 1e9 / peak, 4),
+               "decode_ms_p10_p50_p90": pct3(f_dec)}
 
     secondary = {}
     placement = {}
@@ -672,10 +762,15 @@ def main():
         for name in ("long32k", "qwen_layer", "shared_prefix"):
             if name == args.workload:
                 continue
-            sw = DeviceWorkload(name, args.seed + rank)
-            s_step, s_dec = time_steps(sw, max(50, args.steps // 10), args.warmup, flush, use_graph)
+            sw = DeviceWorkload(name, args.seed + rank, layers=args.layers if rotation else 1)
+            if rotation:
+                s_step, s_dec = time_steps_layers(sw, max(50, args.steps // 10), args.warmup)
+            else:
+                s_step, s_dec = time_steps(sw, max(50, args.steps // 10), args.warmup, flush, use_graph)
+            _, sf_dec = time_steps(sw, max(50, args.steps // 10), args.warmup, flush, use_graph)
             sd = dist_max(float(np.mean(s_dec)))
             ss = dist_max(float(np.mean(s_step)))
+            sfd = dist_max(float(np.mean(sf_dec)))
             if name == "shared_prefix":
                 ub = unique_kv_bytes(sw.wl)
                 unique_note = {"unique_kv_bytes": ub, "decode_unique_gbs": round(ub / (sd * 1e-3) / 1e9, 1)}
@@ -685,6 +780,7 @@ def main():
                 "decode_ms": round(sd, 5), "step_ms": round(ss, 5),
                 "decode_kv_gbs": round(sw.kv_bytes / (sd * 1e-3) / 1e9, 1),
                 "decode_frac_of_peak": round(sw.kv_bytes / (sd * 1e-3) / 1e9 / peak, 4),
+                "decode_kv_gbs_flushed_every_step": round(sw.kv_bytes / (sfd * 1e-3) / 1e9, 1),
                 "kv_bytes": sw.kv_bytes, "seq_per_s": round(sw.wl.num_seqs / (ss * 1e-3), 1),
                 "decode_launches": sw.decode_launches,
             }
@@ -753,9 +849,14 @@ def main():
                        "num_blocks": c.num_blocks, "mean_context": float(np.mean(w.wl.context_lens)),
                        "max_context": w.max_ctx, "partition_size": w.P or "auto",
                        "parallelism": f"replicas x{world}",
-                       "l2": "flushed before every timed step, outside its events: a 256 MiB write, then a "
-                             "256 MiB read of another buffer (so the flush's dirty lines are written back before "
-                             "the step)",
+                       "l2": (f"no flush: consecutive timed steps decode {w.layers} different layers' K/V pools "
+                              "(each larger than L2, so no step finds the K/V it reads in L2), while block tables, "
+                              "context lengths, q and the kernels' code stay L2-resident as in a serving engine; "
+                              "roofline.flushed_every_step repeats the steps after a 256 MiB write + 256 MiB read "
+                              "flush each") if rotation else
+                             ("flushed before every timed step, outside its events: a 256 MiB write, then a "
+                              "256 MiB read of another buffer (so the flush's dirty lines are written back before "
+                              "the step)"),
                        "cuda_graph": ("one graph per step (copy + append + decode, PDL-chained); the decode "
                                       "alone timed as its own graph") if use_graph else False,
                        "step": ("copy_blocks + " if w.has_copy else "") + "reshape_and_cache + decode"},
@@ -768,6 +869,7 @@ def main():
                                    "[+ reduce]), timed together; traffic = DRAM bytes of the attention kernel "
                                    "from profiles/traffic.json",
                          "peak_kind": peak_kind,
+                         "flushed_every_step": flushed,
                          "after_write_only_flush": {"decode_ms": round(wo, 5),
                                                     "achieved": round(w.kv_bytes / (wo * 1e-3) / 1e9, 1),
                                                     "frac": round(w.kv_bytes / (wo * 1e-3) / 1e9 / peak, 4)}},

@@ -126,6 +126,39 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64
     }
 }
 
+// Non-suspending variant for waits on the critical path of a pipeline (a
+// thread that issues tensor-core work): mbarrier.test_wait in a spin, so the
+// thread resumes as soon as the phase completes, bounded like mbar_wait.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ bool mbar_spin_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns = kWaitLimitNs) {
+    if (mbar_test_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_test_wait(bar, parity)) return true;
+        if ((i & 1023u) == 0 && global_timer_ns() - t0 > limit_ns) return false;
+    }
+}
+// A warp waits: lane 0 spins, then every lane observes the completed phase
+// itself (its own acquire of what the phase released).  Returns false on
+// expiry, for every lane.
+__device__ __forceinline__ bool warp_spin_wait(uint64_t* bar, uint32_t parity, int lane) {
+    int ok = 1;
+    if (lane == 0) ok = mbar_spin_wait(bar, parity);
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    if (ok) mbar_test_wait(bar, parity);
+    return ok != 0;
+}
+
 // ---------------------------------------------------------------------------
 // TMA (bulk async copies into shared memory, completion counted on an mbarrier)
 // ---------------------------------------------------------------------------

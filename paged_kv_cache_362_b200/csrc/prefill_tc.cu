@@ -14,23 +14,24 @@
 // walks the keys 128 at a time (eight 16-token blocks):
 //     S = Q K^T           tcgen05.mma, M = 128 rows, N = 128 keys, K = D
 //     P = 2^(S*scale*log2 e - m)   fp32 online softmax, one thread per row
-//     O += P V            tcgen05.mma, M = 128, N = D, K = 128 keys
-// S (two buffers, so the next QK^T runs while a tile's softmax does) and O
-// live in tensor memory; Q, K, V and P in shared memory, 128-byte swizzled.
+//     O += P V            tcgen05.mma with P in tensor memory, M = 128, N = D,
+//                         K = 128 keys (bf16: once for P's hi part, once for lo)
+// S (two buffers, so the next QK^T runs while a tile's softmax does), O and P
+// live in tensor memory; Q, K and V in shared memory, 128-byte swizzled.
 //
-// Warps (192 threads, one CTA per SM):
+// Warps (224 threads, one CTA per SM):
 //   0-3  softmax: thread r owns row r (TMEM lane r).  Loads its Q row into
 //        shared memory; per key tile reads its S row from TMEM, masks keys
 //        past its position (and blocks whose id is out of range), updates
-//        the running max and sum, writes its P row (input dtype) to shared
-//        memory; at the end scales its O row by 1/l and stores it.  The max
-//        used for the exponentials only moves when the tile max exceeds it
-//        by more than 8 (log2 units), so O is rescaled rarely; the sum and O
-//        always use the same reference, which keeps the result exact algebra.
-//   4    producer: K and V tiles of each key step by 2-D TMA (16-row,
-//        128-byte boxes, one per block and 64 columns), K and V on separate
-//        barriers, two stages each.  Blocks no row of the tile sees are not
-//        loaded; a block id out of range is reported and not loaded.
+//        the running max and sum, writes its P row to tensor memory; at the
+//        end scales its O row by 1/l and stores it.  The max used for the
+//        exponentials only moves when the tile max exceeds it by more than 8
+//        (log2 units), so O is rescaled rarely; the sum and O always use the
+//        same reference, which keeps the result exact algebra.
+//   4, 6 producers of K (warp 4) and V (warp 6): 2-D TMA of each block of the
+//        key step (16-row, 128-byte boxes, one per 64 columns), two stages
+//        each.  Blocks no row of the tile sees are not loaded; a block id out
+//        of range is reported and not loaded.
 //   5    MMA issuer (one lane) and TMEM owner: issues QK^T of tile j + 1
 //        before PV of tile j; before each PV it zeroes the V rows that are
 //        not data (slots past the context in the sequence's last block, and
@@ -69,11 +70,11 @@ struct TcPf {
     static constexpr int kOffBar = kOffP + kPBytes;
     // q_full, k_full[2], v_full[2], k_empty[2], v_empty[2], s_full[2], s_empty[2], p_full, pv_done, mma_done
     static constexpr int kNumBars = 1 + 4 * kStages + 4 + 3;
-    static constexpr int kOffMisc = kOffBar + kNumBars * 8;   // TMEM base, abort flag
-    static constexpr int kBytes = kOffMisc + 16;
+    static constexpr int kOffMisc = kOffBar + kNumBars * 8;   // TMEM base, abort flag, per-stage bad-block masks
+    static constexpr int kBytes = kOffMisc + 16 + 4 * kStages;
     // one CTA per SM (the CTA holds all 512 TMEM columns): at least half of the SM's shared memory
     static constexpr int kSmemBytes = (kBytes + 1024) > 120 * 1024 ? (kBytes + 1024) : 120 * 1024;
-    static constexpr int kThreads = 192;
+    static constexpr int kThreads = 224;   // 4 softmax warps, K producer, MMA issuer, V producer
     static constexpr uint32_t kTmemCols = 512;
     static constexpr uint32_t kColS = 0;                    // S buffers at columns 0 and 128
     static constexpr uint32_t kColO = 256;                  // O: D columns
@@ -98,7 +99,7 @@ __device__ __forceinline__ uint32_t bad_mask(const PrefillParams& p, int id) {
 }
 
 template <typename T, int D, bool kPTmem>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(224, 1)
     prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, int qpos, uint32_t idesc_qk, uint32_t idesc_pv) {
     // bf16 P (8-bit significand) would perturb the softmax weights by up to
@@ -122,6 +123,9 @@ __global__ void __launch_bounds__(192, 1)
     uint64_t* mma_done = pv_done + 1;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+    // the V stage's blocks with an out-of-range id (written by the V producer before the stage's
+    // arrival, read by the MMA issuer after it)
+    volatile uint32_t* stage_bad = reinterpret_cast<volatile uint32_t*>(smem + C::kOffMisc + 16);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = p.group, b = blockIdx.z, g = blockIdx.y;
@@ -209,7 +213,7 @@ __global__ void __launch_bounds__(192, 1)
             for (int j = 0; j < nkt && ok; ++j) {
                 const int id_cur = id_next;
                 id_next = tile_block_id(bt_row, j + 1, nkt, kend, lane);
-                if (!__all_sync(0xffffffffu, mbar_wait(&s_full[j & 1], (j >> 1) & 1)) || *abort_flag) {
+                if (!warp_spin_wait(&s_full[j & 1], (j >> 1) & 1, lane) || *abort_flag) {
                     ok = false;
                     break;
                 }
@@ -246,7 +250,7 @@ __global__ void __launch_bounds__(192, 1)
                 }
                 const float ms = m_ref == kNegInfT ? 0.f : m_ref;
                 // P in the input dtype (bf16: hi + lo); the row sum adds what the PV products
-                // use: the rounded fp16 values, or the fp32 values hi + lo carry to ~16 bits
+                // use: the rounded fp16 values, or the fp32 values hi + lo carry
                 uint32_t pk[kKeysT / 2];
                 uint32_t pl[kSplitP ? kKeysT / 2 : 1];
                 float ls0 = 0.f, ls1 = 0.f;
@@ -254,12 +258,20 @@ __global__ void __launch_bounds__(192, 1)
                 for (int c = 0; c < kKeysT / 2; ++c) {
                     const float e0 = fast_exp2(fmaf(__uint_as_float(sv[2 * c]), sl2, -ms));
                     const float e1 = fast_exp2(fmaf(__uint_as_float(sv[2 * c + 1]), sl2, -ms));
-                    pk[c] = Elt<T>::pack2(e0, e1);
                     if constexpr (kSplitP) {
-                        pl[c] = Elt<T>::pack2(e0 - __uint_as_float(pk[c] << 16), e1 - __uint_as_float(pk[c] & 0xffff0000u));
+                        // hi = p truncated to bf16 (its upper 16 bits), lo = p - hi (exact in fp32)
+                        // truncated likewise: hi + lo is p to within 2^-15 relative.  Integer
+                        // ops only: the transcendental pipe that computes 2^x is the softmax's
+                        // bottleneck, and a float -> bf16 conversion would run on it too.
+                        const uint32_t u0 = __float_as_uint(e0), u1 = __float_as_uint(e1);
+                        pk[c] = __byte_perm(u0, u1, 0x7632);
+                        const float r0 = e0 - __uint_as_float(u0 & 0xffff0000u);
+                        const float r1 = e1 - __uint_as_float(u1 & 0xffff0000u);
+                        pl[c] = __byte_perm(__float_as_uint(r0), __float_as_uint(r1), 0x7632);
                         ls0 += e0;
                         ls1 += e1;
                     } else {
+                        pk[c] = Elt<T>::pack2(e0, e1);
                         const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&pk[c]));
                         ls0 += f.x;
                         ls1 += f.y;
@@ -268,7 +280,7 @@ __global__ void __launch_bounds__(192, 1)
                 l = l * alpha + (ls0 + ls1);
                 if (j > 0) {
                     // PV of the previous tile has read the P buffer and written O
-                    if (!__all_sync(0xffffffffu, mbar_wait(pv_done, (j - 1) & 1)) || *abort_flag) {
+                    if (!warp_spin_wait(pv_done, (j - 1) & 1, lane) || *abort_flag) {
                         ok = false;
                         break;
                     }
@@ -314,7 +326,7 @@ __global__ void __launch_bounds__(192, 1)
                 if (lane == 0) mbar_arrive(p_full);
             }
             if (ok) {
-                ok = __all_sync(0xffffffffu, mbar_wait(pv_done, (nkt - 1) & 1)) && !*abort_flag;
+                ok = warp_spin_wait(pv_done, (nkt - 1) & 1, lane) && !*abort_flag;
                 if (ok) {
                     tc_fence_after();
                     const float inv = l > 0.f ? 1.f / l : 0.f;
@@ -339,12 +351,16 @@ __global__ void __launch_bounds__(192, 1)
                 }
             }
             if (!ok && lane == 0) fail();
-        } else if (warp == 4) {
-            // ======================================================= producer
-            if (lane == 0) {
-                prefetch_tensormap(&tmK);
-                prefetch_tensormap(&tmV);
-            }
+        } else if (warp == 4 || warp == 6) {
+            // ============================== producers: warp 4 loads K, warp 6 loads V
+            // (separately, so that a K stage is refilled as soon as its QK^T is done,
+            // not after the previous tile's PV has freed a V stage)
+            const bool is_k = warp == 4;
+            const CUtensorMap* map = is_k ? &tmK : &tmV;
+            uint64_t* fullb = is_k ? k_full : v_full;
+            uint64_t* emptyb = is_k ? k_empty : v_empty;
+            const uint32_t base = is_k ? sK : sV;
+            if (lane == 0) prefetch_tensormap(map);
             constexpr uint32_t kBlockBytes = kBlkT * D * 2;   // one block of one KV head: K or V
             int issued = 0;
             bool ok = true;
@@ -356,149 +372,130 @@ __global__ void __launch_bounds__(192, 1)
                 id_next = tile_block_id(bt_row, j + 1, nkt, kend, lane);
                 const bool need = lane < 8 && (j * 8 + lane) * kBlkT < kend;
                 const bool good = need && id >= 0 && id < p.num_blocks;
-                if (need && !good) set_status(p.status, PA_ERR_OUT_OF_RANGE);
+                if (is_k && need && !good) set_status(p.status, PA_ERR_OUT_OF_RANGE);
                 const uint32_t nload = __popc(__ballot_sync(0xffffffffu, good));
                 const int y = (id * p.num_kv_heads + g) * kBlkT;
+                const uint32_t badm = __ballot_sync(0xffffffffu, need && !good) & 0xffu;
                 int w = 1;
                 if (lane == 0) {
-                    w = mbar_wait(&k_empty[s], par);
-                    if (w) mbar_arrive_expect_tx(&k_full[s], nload * kBlockBytes);
+                    w = mbar_wait(&emptyb[s], par);
+                    if (w && !is_k) stage_bad[s] = badm;
+                    if (w) mbar_arrive_expect_tx(&fullb[s], nload * kBlockBytes);
                 }
                 if (!__shfl_sync(0xffffffffu, w, 0) || *abort_flag) { ok = false; break; }
                 if (good) {
 #pragma unroll
                     for (int h = 0; h < C::kHalves; ++h)
-                        tma_load_2d_keep(sK + s * C::kKVBytes + h * C::kGroupBytes + lane * (kBlkT * 128), &tmK,
-                                         h * 64, y, &k_full[s]);
-                }
-                if (lane == 0) {
-                    w = mbar_wait(&v_empty[s], par);
-                    if (w) mbar_arrive_expect_tx(&v_full[s], nload * kBlockBytes);
-                }
-                if (!__shfl_sync(0xffffffffu, w, 0)) {
-                    // K of tile j is in flight: count it so that the drain below waits for it
-                    issued = j + 1;
-                    ok = false;
-                    break;
-                }
-                if (good) {
-#pragma unroll
-                    for (int h = 0; h < C::kHalves; ++h)
-                        tma_load_2d_keep(sV + s * C::kKVBytes + h * C::kGroupBytes + lane * (kBlkT * 128), &tmV,
-                                         h * 64, y, &v_full[s]);
+                        tma_load_2d_keep(base + s * C::kKVBytes + h * C::kGroupBytes + lane * (kBlkT * 128), map,
+                                         h * 64, y, &fullb[s]);
                 }
                 issued = j + 1;
             }
-            if (!ok) {
+            if (!ok && lane == 0) {
                 // let the copies this warp issued land before the CTA's memory is released
-                if (lane == 0) {
-                    fail();
-                    for (int j = max(0, issued - C::kStages); j < issued; ++j) {
-                        mbar_wait(&k_full[j % C::kStages], (j / C::kStages) & 1);
-                        mbar_wait(&v_full[j % C::kStages], (j / C::kStages) & 1);
-                    }
-                }
+                fail();
+                for (int j = max(0, issued - C::kStages); j < issued; ++j)
+                    mbar_wait(&fullb[j % C::kStages], (j / C::kStages) & 1);
             }
         } else {
             // ================================================ MMA issuer (warp 5)
-            bool ok = __all_sync(0xffffffffu, mbar_wait(q_full, 0));
+            bool ok = true;
             // descriptors: Q, K, P K-major (8-row atoms 1024 B apart, K steps of 16
             // elements 32 B apart inside a 128-byte row, 64-element groups 16 KB
             // apart); V MN-major (64 D-columns per 128-byte row, 16 KB between
             // column groups, 16 keys = 2 atoms per K step)
+            //
+            // The issuing thread shares its scheduler with a softmax warp that
+            // always has work, so its own instruction count between MMAs is what
+            // the tensor core waits on: descriptors are built once, and a K step
+            // only adds a constant to the start-address field (bits 0-13, in
+            // 16-byte units) of the step-0 descriptor.
             auto kdesc = [&](uint32_t base, int k) {
                 return umma_desc_sw128(base + (k >> 2) * C::kGroupBytes + (k & 3) * 32, 16, 1024);
             };
             auto vdesc = [&](uint32_t base, int k) {
                 return umma_desc_sw128(base + k * (2 * 1024), C::kGroupBytes, 1024);
             };
-            auto issue_pv = [&](int i, int ids) -> bool {
+            const uint64_t dQ = kdesc(sQ, 0);
+            const uint64_t dK0 = kdesc(sK, 0), dV0 = vdesc(sV, 0);
+            constexpr uint64_t kStageStep = (uint64_t)(C::kKVBytes >> 4);    // one K or V stage
+            auto kstep = [](int k) { return (uint64_t)(((k >> 2) * C::kGroupBytes + (k & 3) * 32) >> 4); };
+            constexpr uint64_t kVStep = (2 * 1024) >> 4;                      // 16 keys of V
+            // One lane issues everything; the other lanes of the warp only meet it at
+            // the end.  Waits spin (bounded) on the mbarriers.
+            auto issue_pv = [&](int i) -> bool {
                 const int s = i % C::kStages;
-                const uint32_t badm = bad_mask(p, ids);
-                if (!__all_sync(0xffffffffu, mbar_wait(p_full, i & 1)) || *abort_flag) return false;
-                if (!__all_sync(0xffffffffu, mbar_wait(&v_full[s], (i / C::kStages) & 1))) return false;
+                if (!mbar_spin_wait(p_full, i & 1) || *abort_flag) return false;
+                if (!mbar_spin_wait(&v_full[s], (i / C::kStages) & 1)) return false;
+                const uint32_t badm = stage_bad[s];
                 // keys of this tile the PV product covers: whole 16-key steps up to kend
-                const int kb0 = i * kKeysT;
-                const int nks = min(kKeysT, kend - kb0 + kBlkT - 1) / kBlkT;
+                const int nks = min(kKeysT, kend - i * kKeysT + kBlkT - 1) / kBlkT;
                 // rows of V that hold no data: blocks not loaded (bad ids) and slots
-                // at or past n in the sequence's last block
+                // at or past n in the sequence's last block (only the sequence's last
+                // tile has those; a tile with neither skips the scan)
                 const int tail_blk = n / kBlkT - i * 8;      // the last block's index in this tile, if partial
                 const int tail_from = n % kBlkT;
-                bool zeroed = false;
-                for (int k = 0; k < nks; ++k) {
-                    int r0 = kBlkT, r1 = kBlkT;
-                    if ((badm >> k) & 1u) r0 = 0;
-                    else if (k == tail_blk && tail_from != 0) r0 = tail_from;
-                    if (r0 >= r1) continue;
-                    zeroed = true;
-                    const int per = (r1 - r0) * 8 * C::kHalves;   // 16-byte pieces
-                    for (int e = lane; e < per; e += 32) {
-                        const int rr = k * kBlkT + r0 + e / (8 * C::kHalves);
-                        const int hh = (e % (8 * C::kHalves)) / 8, uu = e % 8;
-                        st_shared_zero16(sV + s * C::kKVBytes + hh * C::kGroupBytes + rr * 128 + (uu << 4));
+                if (badm != 0 || (tail_from != 0 && tail_blk < nks)) {
+                    for (int k = 0; k < nks; ++k) {
+                        const int r0 = ((badm >> k) & 1u) ? 0 : (k == tail_blk ? tail_from : kBlkT);
+                        for (int rr = k * kBlkT + r0; rr < (k + 1) * kBlkT; ++rr)
+#pragma unroll
+                            for (int hh = 0; hh < C::kHalves; ++hh)
+#pragma unroll
+                                for (int uu = 0; uu < 8; ++uu)
+                                    st_shared_zero16(sV + s * C::kKVBytes + hh * C::kGroupBytes + rr * 128 + (uu << 4));
+                    }
+                    fence_proxy_async_shared();
+                }
+                tc_fence_after();
+                const uint64_t dv = dV0 + (uint64_t)s * kStageStep;
+                const uint32_t acc0 = i > 0 ? 1u : 0u;
+#pragma unroll
+                for (int k = 0; k < kKeysT / kBlkT; ++k) {
+                    if (k < nks) {
+                        if constexpr (kPTmem)
+                            umma_f16_ts(tmem + C::kColO, tmem + C::kColP + k * 8, dv + k * kVStep, idesc_pv,
+                                        k > 0 ? 1u : acc0);
+                        else
+                            umma_f16_ss(tmem + C::kColO, kdesc(sP, k), dv + k * kVStep, idesc_pv, k > 0 ? 1u : acc0);
                     }
                 }
-                if (zeroed) fence_proxy_async_shared();
-                __syncwarp();
-                if (lane == 0) {
-                    tc_fence_after();
-                    const uint32_t vb = sV + s * C::kKVBytes;
-                    for (int k = 0; k < nks; ++k) {
-                        if constexpr (kPTmem)
-                            umma_f16_ts(tmem + C::kColO, tmem + C::kColP + k * 8, vdesc(vb, k), idesc_pv,
-                                        (i > 0 || k > 0) ? 1u : 0u);
-                        else
-                            umma_f16_ss(tmem + C::kColO, kdesc(sP, k), vdesc(vb, k), idesc_pv,
-                                        (i > 0 || k > 0) ? 1u : 0u);
-                    }
-                    if constexpr (kSplitP) {
-                        for (int k = 0; k < nks; ++k) {
+                if constexpr (kSplitP) {
+#pragma unroll
+                    for (int k = 0; k < kKeysT / kBlkT; ++k) {
+                        if (k < nks) {
                             if constexpr (kPTmem)
-                                umma_f16_ts(tmem + C::kColO, tmem + C::kColPLo + k * 8, vdesc(vb, k), idesc_pv, 1u);
+                                umma_f16_ts(tmem + C::kColO, tmem + C::kColPLo + k * 8, dv + k * kVStep, idesc_pv, 1u);
                             else
-                                umma_f16_ss(tmem + C::kColO, kdesc(sP + C::kPTile, k), vdesc(vb, k), idesc_pv, 1u);
+                                umma_f16_ss(tmem + C::kColO, kdesc(sP + C::kPTile, k), dv + k * kVStep, idesc_pv, 1u);
                         }
                     }
-                    umma_commit(pv_done);
-                    umma_commit(&v_empty[s]);
                 }
-                __syncwarp();
+                umma_commit(pv_done);
+                umma_commit(&v_empty[s]);
                 return true;
             };
-            int j = 0;
-            int id_prev = 0, id_cur = tile_block_id(bt_row, 0, nkt, kend, lane);   // ids of tiles j - 1 and j
-            for (; j < nkt && ok; ++j) {
-                const int s = j % C::kStages;
-                if (!__all_sync(0xffffffffu, mbar_wait(&k_full[s], (j / C::kStages) & 1)) || *abort_flag) {
-                    ok = false;
-                    break;
-                }
-                if (!__all_sync(0xffffffffu, mbar_wait(&s_empty[j & 1], ((j >> 1) & 1) ^ 1))) {
-                    ok = false;
-                    break;
-                }
-                if (lane == 0) {
+            if (lane == 0) {
+                ok = mbar_spin_wait(q_full, 0);
+                for (int j = 0; j < nkt && ok; ++j) {
+                    const int s = j % C::kStages;
+                    if (!mbar_spin_wait(&k_full[s], (j / C::kStages) & 1) || *abort_flag ||
+                        !mbar_spin_wait(&s_empty[j & 1], ((j >> 1) & 1) ^ 1)) {
+                        ok = false;
+                        break;
+                    }
                     tc_fence_after();
-                    const uint32_t kb = sK + s * C::kKVBytes;
+                    const uint64_t dk = dK0 + (uint64_t)s * kStageStep;
+                    const uint32_t dS = tmem + C::kColS + (j & 1) * kKeysT;
 #pragma unroll
                     for (int k = 0; k < D / 16; ++k)
-                        umma_f16_ss(tmem + C::kColS + (j & 1) * kKeysT, kdesc(sQ, k), kdesc(kb, k), idesc_qk,
-                                    k > 0 ? 1u : 0u);
+                        umma_f16_ss(dS, dQ + kstep(k), dk + kstep(k), idesc_qk, k > 0 ? 1u : 0u);
                     umma_commit(&s_full[j & 1]);
                     umma_commit(&k_empty[s]);
+                    if (j > 0 && !issue_pv(j - 1)) ok = false;
                 }
-                __syncwarp();
-                const int id_pv = id_prev;
-                id_prev = id_cur;
-                id_cur = tile_block_id(bt_row, j + 1, nkt, kend, lane);
-                if (j > 0 && !issue_pv(j - 1, id_pv)) {
-                    ok = false;
-                    break;
-                }
-            }
-            if (ok && !issue_pv(nkt - 1, id_prev)) ok = false;
-            // every MMA this warp issued has completed before TMEM and shared memory are released
-            if (lane == 0) {
+                if (ok && !issue_pv(nkt - 1)) ok = false;
+                // every MMA issued has completed before TMEM and shared memory are released
                 umma_commit(mma_done);
                 mbar_wait(mma_done, 0);
                 if (!ok) fail();
