@@ -16,27 +16,34 @@
 //     P = 2^(S*scale*log2 e - m)   fp32 online softmax, one thread per row
 //     O += P V            tcgen05.mma with P in tensor memory, M = 128, N = D,
 //                         K = 128 keys (bf16: once for P's hi part, once for lo)
-// S (two buffers, so the next QK^T runs while a tile's softmax does), O and P
-// live in tensor memory; Q, K and V in shared memory, 128-byte swizzled.
+// S has three buffers in tensor memory; the softmax writes a tile's P over
+// its scores in place (16-bit pairs: hi in the buffer's first 64 columns, lo
+// in the next 64), so QK^T runs up to three tiles ahead and the softmax never
+// waits for the previous PV product except to rescale O.  O also lives in
+// tensor memory (columns 384..511); Q, K and V in shared memory, 128-byte
+// swizzled.
 //
 // Warps (224 threads, one CTA per SM):
 //   0-3  softmax: thread r owns row r (TMEM lane r).  Loads its Q row into
 //        shared memory; per key tile reads its S row from TMEM, masks keys
 //        past its position (and blocks whose id is out of range), updates
-//        the running max and sum, writes its P row to tensor memory; at the
-//        end scales its O row by 1/l and stores it.  The max used for the
-//        exponentials only moves when the tile max exceeds it by more than 8
-//        (log2 units), so O is rescaled rarely; the sum and O always use the
-//        same reference, which keeps the result exact algebra.
+//        the running max and sum, writes its P row back in a quarter of the
+//        tile at a time; at the end scales its O row by 1/l and stores it.
+//        The max used for the exponentials only moves when the tile max
+//        exceeds it by more than 8 (log2 units), so O is rescaled rarely; the
+//        sum and O always use the same reference, which keeps the result
+//        exact algebra.
 //   4, 6 producers of K (warp 4) and V (warp 6): 2-D TMA of each block of the
 //        key step (16-row, 128-byte boxes, one per 64 columns), two stages
 //        each.  Blocks no row of the tile sees are not loaded; a block id out
-//        of range is reported and not loaded.
-//   5    MMA issuer (one lane) and TMEM owner: issues QK^T of tile j + 1
-//        before PV of tile j; before each PV it zeroes the V rows that are
-//        not data (slots past the context in the sequence's last block, and
-//        blocks that were not loaded), since a probability of 0 times a NaN
-//        left in shared memory would still be NaN.
+//        of range is reported and not loaded (the V producer hands the mask
+//        of such blocks to the MMA warp with the stage).
+//   5    MMA issuer and TMEM owner: QK^T of tiles 0-2, then per tile j the PV
+//        product of j and the QK^T of j + 3.  The warp runs the loop in
+//        lockstep and an elected lane issues.  Before a PV product it zeroes
+//        the V rows that are not data (slots past the context in the
+//        sequence's last block, and blocks that were not loaded), since a
+//        probability of 0 times a NaN left in shared memory would still be NaN.
 // Every mbarrier wait is bounded (PA_ERR_TIMEOUT); on expiry the CTA lets
 // its copies and MMAs finish, frees its TMEM and returns.
 #include "pa_internal.h"
@@ -53,33 +60,31 @@ constexpr int kBlkT = 16;         // tokens per block
 // by more than this (log2 units): p <= 2^8, well inside fp16 and bf16.
 constexpr float kRescaleSlack = 8.f;
 
-template <int D, bool kPTmem, bool kSplitP>
+template <int D>
 struct TcPf {
     static constexpr int kHalves = D / 64;                 // 128-byte column groups of a D-wide row
     static constexpr int kGroupBytes = kRowsT * 128;       // 128 rows x 128 B (16 KB)
     static constexpr int kQBytes = kHalves * kGroupBytes;  // Q tile (K-major, K = D)
     static constexpr int kKVBytes = kHalves * kGroupBytes; // one K or V tile of 128 keys
-    // P tile(s) in shared memory (K-major, K = 128 keys): hi, and with kSplitP also lo
-    static constexpr int kPTile = 2 * kGroupBytes;
-    static constexpr int kPBytes = kPTmem ? 0 : (kSplitP ? 2 : 1) * kPTile;
-    static constexpr int kStages = 2;
+    static constexpr int kStages = 2;                      // K and V stages
+    static constexpr int kSBufs = 3;                       // S (then P) buffers in tensor memory
     static constexpr int kOffQ = 0;
     static constexpr int kOffK = kOffQ + kQBytes;
     static constexpr int kOffV = kOffK + kStages * kKVBytes;
-    static constexpr int kOffP = kOffV + kStages * kKVBytes;
-    static constexpr int kOffBar = kOffP + kPBytes;
-    // q_full, k_full[2], v_full[2], k_empty[2], v_empty[2], s_full[2], s_empty[2], p_full, pv_done, mma_done
-    static constexpr int kNumBars = 1 + 4 * kStages + 4 + 3;
+    static constexpr int kOffBar = kOffV + kStages * kKVBytes;
+    // q_full, k_full[2], v_full[2], k_empty[2], v_empty[2], s_full[3], p_full[3], pv_done[3], mma_done
+    static constexpr int kNumBars = 1 + 4 * kStages + 3 * kSBufs + 1;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;   // TMEM base, abort flag, per-stage bad-block masks
     static constexpr int kBytes = kOffMisc + 16 + 4 * kStages;
     // one CTA per SM (the CTA holds all 512 TMEM columns): at least half of the SM's shared memory
     static constexpr int kSmemBytes = (kBytes + 1024) > 120 * 1024 ? (kBytes + 1024) : 120 * 1024;
     static constexpr int kThreads = 224;   // 4 softmax warps, K producer, MMA issuer, V producer
     static constexpr uint32_t kTmemCols = 512;
-    static constexpr uint32_t kColS = 0;                    // S buffers at columns 0 and 128
-    static constexpr uint32_t kColO = 256;                  // O: D columns
-    static constexpr uint32_t kColP = 384;                  // P in tensor memory: 64 columns of 16-bit pairs
-    static constexpr uint32_t kColPLo = 448;                // and its lo part (kSplitP)
+    // S buffer b at columns 128b: the fp32 scores of a 128-key tile, then, in
+    // place, P as 16-bit pairs: columns 0-63 (hi) and 64-127 (lo, bf16 only)
+    static constexpr uint32_t kColS = 0;
+    static constexpr uint32_t kColPLo = 64;                 // lo part, relative to the buffer
+    static constexpr uint32_t kColO = 384;                  // O: D columns
     static_assert(kBytes + 1024 <= 227 * 1024, "shared memory");
 };
 
@@ -98,7 +103,7 @@ __device__ __forceinline__ uint32_t bad_mask(const PrefillParams& p, int id) {
     return __ballot_sync(0xffffffffu, id < 0 || id >= p.num_blocks) & 0xffu;
 }
 
-template <typename T, int D, bool kPTmem>
+template <typename T, int D>
 __global__ void __launch_bounds__(224, 1)
     prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, int qpos, uint32_t idesc_qk, uint32_t idesc_pv) {
@@ -107,7 +112,7 @@ __global__ void __launch_bounds__(224, 1)
     // to ~1e-2; it is carried as hi + lo (two bf16 parts, ~16 bits) and the PV
     // product runs once per part.  fp16 P (11 bits) is used as is.
     constexpr bool kSplitP = std::is_same<T, __nv_bfloat16>::value;
-    using C = TcPf<D, kPTmem, kSplitP>;
+    using C = TcPf<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
@@ -116,11 +121,13 @@ __global__ void __launch_bounds__(224, 1)
     uint64_t* v_full = k_full + C::kStages;
     uint64_t* k_empty = v_full + C::kStages;
     uint64_t* v_empty = k_empty + C::kStages;
+    // per S buffer b (key tiles j = b mod 3): scores written, P written, PV done.
+    // One buffer's barrier completes once per three tiles and a waiter is never
+    // more than one phase behind it.
     uint64_t* s_full = v_empty + C::kStages;
-    uint64_t* s_empty = s_full + 2;
-    uint64_t* p_full = s_empty + 2;
-    uint64_t* pv_done = p_full + 1;
-    uint64_t* mma_done = pv_done + 1;
+    uint64_t* p_full = s_full + C::kSBufs;
+    uint64_t* pv_done = p_full + C::kSBufs;
+    uint64_t* mma_done = pv_done + C::kSBufs;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
     // the V stage's blocks with an out-of-range id (written by the V producer before the stage's
@@ -139,12 +146,11 @@ __global__ void __launch_bounds__(224, 1)
             mbar_init(&k_empty[s], 1);
             mbar_init(&v_empty[s], 1);
         }
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < C::kSBufs; ++i) {
             mbar_init(&s_full[i], 1);
-            mbar_init(&s_empty[i], 4);
+            mbar_init(&p_full[i], 4);
+            mbar_init(&pv_done[i], 1);
         }
-        mbar_init(p_full, 4);
-        mbar_init(pv_done, 1);
         mbar_init(mma_done, 1);
         *abort_flag = 0;
         mbar_fence_init();
@@ -178,7 +184,6 @@ __global__ void __launch_bounds__(224, 1)
         const uint32_t sQ = smem_u32(smem + C::kOffQ);
         const uint32_t sK = smem_u32(smem + C::kOffK);
         const uint32_t sV = smem_u32(smem + C::kOffV);
-        const uint32_t sP = smem_u32(smem + C::kOffP);
         auto fail = [&]() {
             *abort_flag = 1;
             set_status(p.status, PA_ERR_TIMEOUT);
@@ -213,18 +218,18 @@ __global__ void __launch_bounds__(224, 1)
             for (int j = 0; j < nkt && ok; ++j) {
                 const int id_cur = id_next;
                 id_next = tile_block_id(bt_row, j + 1, nkt, kend, lane);
-                if (!warp_spin_wait(&s_full[j & 1], (j >> 1) & 1, lane) || *abort_flag) {
+                const int sb = j % C::kSBufs;
+                const uint32_t sph = (uint32_t)(j / C::kSBufs) & 1u;
+                if (!warp_spin_wait(&s_full[sb], sph, lane) || *abort_flag) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
+                const uint32_t tS = tl + C::kColS + sb * kKeysT;
                 uint32_t sv[kKeysT];
 #pragma unroll
-                for (int c = 0; c < kKeysT / 32; ++c) tmem_ld32(tl + C::kColS + (j & 1) * kKeysT + c * 32, sv + c * 32);
+                for (int c = 0; c < kKeysT / 32; ++c) tmem_ld32(tS + c * 32, sv + c * 32);
                 tmem_ld_wait(sv);
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&s_empty[j & 1]);   // the S buffer may be overwritten now
                 const uint32_t badm = bad_mask(p, id_cur);
 
                 // causal mask (the tile's first row sees keys up to pos0) and bad blocks
@@ -236,13 +241,13 @@ __global__ void __launch_bounds__(224, 1)
                 }
                 float mx0 = kNegInfT, mx1 = kNegInfT, mx2 = kNegInfT, mx3 = kNegInfT;
 #pragma unroll
-                for (int c = 0; c < kKeysT; c += 4) {
-                    mx0 = fmaxf(mx0, __uint_as_float(sv[c]));
-                    mx1 = fmaxf(mx1, __uint_as_float(sv[c + 1]));
-                    mx2 = fmaxf(mx2, __uint_as_float(sv[c + 2]));
-                    mx3 = fmaxf(mx3, __uint_as_float(sv[c + 3]));
+                for (int c = 0; c < kKeysT; c += 8) {
+                    mx0 = fmax3(mx0, __uint_as_float(sv[c]), __uint_as_float(sv[c + 1]));
+                    mx1 = fmax3(mx1, __uint_as_float(sv[c + 2]), __uint_as_float(sv[c + 3]));
+                    mx2 = fmax3(mx2, __uint_as_float(sv[c + 4]), __uint_as_float(sv[c + 5]));
+                    mx3 = fmax3(mx3, __uint_as_float(sv[c + 6]), __uint_as_float(sv[c + 7]));
                 }
-                const float m_new = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+                const float m_new = fmax3(mx0, mx1, fmaxf(mx2, mx3)) * sl2;
                 float alpha = 1.f;
                 if (m_new > m_ref + kRescaleSlack) {
                     alpha = m_ref == kNegInfT ? 0.f : fast_exp2(m_ref - m_new);
@@ -250,83 +255,76 @@ __global__ void __launch_bounds__(224, 1)
                 }
                 const float ms = m_ref == kNegInfT ? 0.f : m_ref;
                 // P in the input dtype (bf16: hi + lo); the row sum adds what the PV products
-                // use: the rounded fp16 values, or the fp32 values hi + lo carry
-                uint32_t pk[kKeysT / 2];
-                uint32_t pl[kSplitP ? kKeysT / 2 : 1];
-                float ls0 = 0.f, ls1 = 0.f;
+                // use: the rounded fp16 values, or the fp32 values hi + lo carry.  P row r
+                // goes over the scores just read (TMEM lane r, keys 2c and 2c + 1 in column
+                // c), a quarter of the tile at a time so that the stores overlap the
+                // exponentials of the next quarter.  The PV product of this tile is issued
+                // before the QK^T product that next writes this buffer, and the tensor
+                // core runs them in that order.  Pairs of keys go through the packed
+                // fp32x2 add and fma.
+                const float2 sl2v = make_float2(sl2, sl2), nms = make_float2(-ms, -ms);
+                float2 lsa = make_float2(0.f, 0.f), lsb = make_float2(0.f, 0.f);
 #pragma unroll
-                for (int c = 0; c < kKeysT / 2; ++c) {
-                    const float e0 = fast_exp2(fmaf(__uint_as_float(sv[2 * c]), sl2, -ms));
-                    const float e1 = fast_exp2(fmaf(__uint_as_float(sv[2 * c + 1]), sl2, -ms));
-                    if constexpr (kSplitP) {
-                        // hi = p truncated to bf16 (its upper 16 bits), lo = p - hi (exact in fp32)
-                        // truncated likewise: hi + lo is p to within 2^-15 relative.  Integer
-                        // ops only: the transcendental pipe that computes 2^x is the softmax's
-                        // bottleneck, and a float -> bf16 conversion would run on it too.
-                        const uint32_t u0 = __float_as_uint(e0), u1 = __float_as_uint(e1);
-                        pk[c] = __byte_perm(u0, u1, 0x7632);
-                        const float r0 = e0 - __uint_as_float(u0 & 0xffff0000u);
-                        const float r1 = e1 - __uint_as_float(u1 & 0xffff0000u);
-                        pl[c] = __byte_perm(__float_as_uint(r0), __float_as_uint(r1), 0x7632);
-                        ls0 += e0;
-                        ls1 += e1;
-                    } else {
-                        pk[c] = Elt<T>::pack2(e0, e1);
-                        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&pk[c]));
-                        ls0 += f.x;
-                        ls1 += f.y;
+                for (int qt = 0; qt < kKeysT / 32; ++qt) {
+                    uint32_t pk[16];
+                    uint32_t pl[kSplitP ? 16 : 1];
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) {
+                        const int k0 = qt * 32 + 2 * c;
+                        const float2 x = __ffma2_rn(make_float2(__uint_as_float(sv[k0]), __uint_as_float(sv[k0 + 1])),
+                                                    sl2v, nms);
+                        const float e0 = fast_exp2(x.x), e1 = fast_exp2(x.y);
+                        float2& ls = (c & 1) ? lsb : lsa;
+                        if constexpr (kSplitP) {
+                            // hi = p truncated to bf16 (its upper 16 bits), lo = p - hi (exact in
+                            // fp32) truncated likewise: hi + lo is p to within 2^-15 relative.
+                            // Integer ops only: the transcendental pipe that computes 2^x is the
+                            // softmax's bottleneck, and a float -> bf16 conversion would run on it too.
+                            const uint32_t u0 = __float_as_uint(e0), u1 = __float_as_uint(e1);
+                            pk[c] = __byte_perm(u0, u1, 0x7632);
+                            const float2 r = __fadd2_rn(make_float2(e0, e1),
+                                                        make_float2(__uint_as_float((u0 & 0xffff0000u) ^ 0x80000000u),
+                                                                    __uint_as_float((u1 & 0xffff0000u) ^ 0x80000000u)));
+                            pl[c] = __byte_perm(__float_as_uint(r.x), __float_as_uint(r.y), 0x7632);
+                            ls = __fadd2_rn(ls, make_float2(e0, e1));
+                        } else {
+                            pk[c] = Elt<T>::pack2(e0, e1);
+                            ls = __fadd2_rn(ls, __half22float2(*reinterpret_cast<const __half2*>(&pk[c])));
+                        }
                     }
+                    tmem_st16(tS + qt * 16, pk);
+                    if constexpr (kSplitP) tmem_st16(tS + C::kColPLo + qt * 16, pl);
                 }
-                l = l * alpha + (ls0 + ls1);
-                if (j > 0) {
-                    // PV of the previous tile has read the P buffer and written O
-                    if (!warp_spin_wait(pv_done, (j - 1) & 1, lane) || *abort_flag) {
+                l = l * alpha + ((lsa.x + lsb.x) + (lsa.y + lsb.y));
+                // O is rescaled only when some row's reference max moved: that needs
+                // the previous tiles' PV products complete.  The PV of tile j - 1
+                // signals buffer (j - 1) mod 3, whose previous signal (tile j - 4)
+                // preceded this tile's scores, so the parity names one phase.
+                if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+                    const int pb = (j - 1) % C::kSBufs;
+                    if (!warp_spin_wait(&pv_done[pb], (uint32_t)((j - 1) / C::kSBufs) & 1u, lane) || *abort_flag) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    if (__any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
-                        for (int c = 0; c < D / 32; ++c) {
-                            uint32_t ov[32];
-                            tmem_ld32(tl + C::kColO + c * 32, ov);
-                            tmem_ld_wait(ov);
+                    for (int c = 0; c < D / 32; ++c) {
+                        uint32_t ov[32];
+                        tmem_ld32(tl + C::kColO + c * 32, ov);
+                        tmem_ld_wait(ov);
 #pragma unroll
-                            for (int k = 0; k < 32; ++k) ov[k] = __float_as_uint(__uint_as_float(ov[k]) * alpha);
-                            tmem_st32(tl + C::kColO + c * 32, ov);
-                        }
-                        tmem_st_wait();
+                        for (int k = 0; k < 32; ++k) ov[k] = __float_as_uint(__uint_as_float(ov[k]) * alpha);
+                        tmem_st32(tl + C::kColO + c * 32, ov);
                     }
                 }
-                if constexpr (kPTmem) {
-                    // P row r into TMEM lane r, keys 2c and 2c + 1 in column c
-                    tmem_st32(tl + C::kColP, pk);
-                    tmem_st32(tl + C::kColP + 32, pk + 32);
-                    if constexpr (kSplitP) {
-                        tmem_st32(tl + C::kColPLo, pl);
-                        tmem_st32(tl + C::kColPLo + 32, pl + 32);
-                    }
-                    tmem_st_wait();
-                } else {
-#pragma unroll
-                    for (int u = 0; u < kKeysT / 8; ++u) {
-                        const uint32_t a = sP + (u >> 3) * C::kGroupBytes + sw128(r, u & 7);
-                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(pk[4 * u]),
-                                     "r"(pk[4 * u + 1]), "r"(pk[4 * u + 2]), "r"(pk[4 * u + 3])
-                                     : "memory");
-                        if constexpr (kSplitP)
-                            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a + C::kPTile),
-                                         "r"(pl[4 * u]), "r"(pl[4 * u + 1]), "r"(pl[4 * u + 2]), "r"(pl[4 * u + 3])
-                                         : "memory");
-                    }
-                    fence_proxy_async_shared();
-                }
+                tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(p_full);
+                if (lane == 0) mbar_arrive(&p_full[sb]);
             }
             if (ok) {
-                ok = warp_spin_wait(pv_done, (nkt - 1) & 1, lane) && !*abort_flag;
+                ok = warp_spin_wait(&pv_done[(nkt - 1) % C::kSBufs], (uint32_t)((nkt - 1) / C::kSBufs) & 1u, lane) &&
+                     !*abort_flag;
                 if (ok) {
                     tc_fence_after();
                     const float inv = l > 0.f ? 1.f / l : 0.f;
@@ -421,13 +419,34 @@ __global__ void __launch_bounds__(224, 1)
             constexpr uint64_t kStageStep = (uint64_t)(C::kKVBytes >> 4);    // one K or V stage
             auto kstep = [](int k) { return (uint64_t)(((k >> 2) * C::kGroupBytes + (k & 3) * 32) >> 4); };
             constexpr uint64_t kVStep = (2 * 1024) >> 4;                      // 16 keys of V
-            // One lane issues everything; the other lanes of the warp only meet it at
-            // the end.  Waits spin (bounded) on the mbarriers.
+            // The whole warp runs the issue loop (warp-uniform control flow: the
+            // descriptors stay in uniform registers) and one elected lane issues
+            // each product; waits spin (bounded) and end for all lanes together.
+            // (Suspending in mbarrier.try_wait measured slower: the wake-up
+            // latency lands on the tensor core's critical path.)
+            auto wait_all = [&](uint64_t* bar, uint32_t par) -> bool {
+                return __all_sync(0xffffffffu, mbar_spin_wait(bar, par) && !*abort_flag);
+            };
+            auto issue_qk = [&](int j) -> bool {
+                const int s = j % C::kStages;
+                if (!wait_all(&k_full[s], (j / C::kStages) & 1)) return false;
+                tc_fence_after();
+                const uint64_t dk = dK0 + (uint64_t)s * kStageStep;
+                const int sb = j % C::kSBufs;
+                const uint32_t dS = tmem + C::kColS + sb * kKeysT;
+#pragma unroll
+                for (int k = 0; k < D / 16; ++k)
+                    umma_f16_ss_warp(dS, dQ + kstep(k), dk + kstep(k), idesc_qk, k > 0 ? 1u : 0u);
+                umma_commit_warp(&s_full[sb]);
+                umma_commit_warp(&k_empty[s]);
+                return true;
+            };
             auto issue_pv = [&](int i) -> bool {
                 const int s = i % C::kStages;
-                if (!mbar_spin_wait(p_full, i & 1) || *abort_flag) return false;
-                if (!mbar_spin_wait(&v_full[s], (i / C::kStages) & 1)) return false;
-                const uint32_t badm = stage_bad[s];
+                const int sb = i % C::kSBufs;
+                if (!wait_all(&p_full[sb], (uint32_t)(i / C::kSBufs) & 1u)) return false;
+                if (!wait_all(&v_full[s], (i / C::kStages) & 1)) return false;
+                const uint32_t badm = __shfl_sync(0xffffffffu, stage_bad[s], 0);
                 // keys of this tile the PV product covers: whole 16-key steps up to kend
                 const int nks = min(kKeysT, kend - i * kKeysT + kBlkT - 1) / kBlkT;
                 // rows of V that hold no data: blocks not loaded (bad ids) and slots
@@ -436,69 +455,50 @@ __global__ void __launch_bounds__(224, 1)
                 const int tail_blk = n / kBlkT - i * 8;      // the last block's index in this tile, if partial
                 const int tail_from = n % kBlkT;
                 if (badm != 0 || (tail_from != 0 && tail_blk < nks)) {
+                    // 16-byte pieces of the rows to clear, spread over the warp
                     for (int k = 0; k < nks; ++k) {
                         const int r0 = ((badm >> k) & 1u) ? 0 : (k == tail_blk ? tail_from : kBlkT);
-                        for (int rr = k * kBlkT + r0; rr < (k + 1) * kBlkT; ++rr)
-#pragma unroll
-                            for (int hh = 0; hh < C::kHalves; ++hh)
-#pragma unroll
-                                for (int uu = 0; uu < 8; ++uu)
-                                    st_shared_zero16(sV + s * C::kKVBytes + hh * C::kGroupBytes + rr * 128 + (uu << 4));
+                        for (int u = (k * kBlkT + r0) * 8 * C::kHalves + lane; u < (k + 1) * kBlkT * 8 * C::kHalves;
+                             u += 32) {
+                            const int rr = u / (8 * C::kHalves), hh = (u / 8) % C::kHalves, uu = u % 8;
+                            st_shared_zero16(sV + s * C::kKVBytes + hh * C::kGroupBytes + rr * 128 + (uu << 4));
+                        }
                     }
                     fence_proxy_async_shared();
+                    __syncwarp();
                 }
                 tc_fence_after();
                 const uint64_t dv = dV0 + (uint64_t)s * kStageStep;
+                const uint32_t tP = tmem + C::kColS + sb * kKeysT;
                 const uint32_t acc0 = i > 0 ? 1u : 0u;
 #pragma unroll
-                for (int k = 0; k < kKeysT / kBlkT; ++k) {
-                    if (k < nks) {
-                        if constexpr (kPTmem)
-                            umma_f16_ts(tmem + C::kColO, tmem + C::kColP + k * 8, dv + k * kVStep, idesc_pv,
-                                        k > 0 ? 1u : acc0);
-                        else
-                            umma_f16_ss(tmem + C::kColO, kdesc(sP, k), dv + k * kVStep, idesc_pv, k > 0 ? 1u : acc0);
-                    }
-                }
+                for (int k = 0; k < kKeysT / kBlkT; ++k)
+                    if (k < nks)
+                        umma_f16_ts_warp(tmem + C::kColO, tP + k * 8, dv + k * kVStep, idesc_pv, k > 0 ? 1u : acc0);
                 if constexpr (kSplitP) {
 #pragma unroll
-                    for (int k = 0; k < kKeysT / kBlkT; ++k) {
-                        if (k < nks) {
-                            if constexpr (kPTmem)
-                                umma_f16_ts(tmem + C::kColO, tmem + C::kColPLo + k * 8, dv + k * kVStep, idesc_pv, 1u);
-                            else
-                                umma_f16_ss(tmem + C::kColO, kdesc(sP + C::kPTile, k), dv + k * kVStep, idesc_pv, 1u);
-                        }
-                    }
+                    for (int k = 0; k < kKeysT / kBlkT; ++k)
+                        if (k < nks)
+                            umma_f16_ts_warp(tmem + C::kColO, tP + C::kColPLo + k * 8, dv + k * kVStep, idesc_pv, 1u);
                 }
-                umma_commit(pv_done);
-                umma_commit(&v_empty[s]);
+                umma_commit_warp(&pv_done[sb]);
+                umma_commit_warp(&v_empty[s]);
                 return true;
             };
-            if (lane == 0) {
-                ok = mbar_spin_wait(q_full, 0);
+            {
+                // QK^T runs up to three tiles ahead (one per S buffer); the QK^T
+                // product of tile j + 3 follows the PV product of tile j, which
+                // reads the P that shares its buffer
+                ok = wait_all(q_full, 0);
+                for (int j = 0; j < min(nkt, C::kSBufs) && ok; ++j) ok = issue_qk(j);
                 for (int j = 0; j < nkt && ok; ++j) {
-                    const int s = j % C::kStages;
-                    if (!mbar_spin_wait(&k_full[s], (j / C::kStages) & 1) || *abort_flag ||
-                        !mbar_spin_wait(&s_empty[j & 1], ((j >> 1) & 1) ^ 1)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint64_t dk = dK0 + (uint64_t)s * kStageStep;
-                    const uint32_t dS = tmem + C::kColS + (j & 1) * kKeysT;
-#pragma unroll
-                    for (int k = 0; k < D / 16; ++k)
-                        umma_f16_ss(dS, dQ + kstep(k), dk + kstep(k), idesc_qk, k > 0 ? 1u : 0u);
-                    umma_commit(&s_full[j & 1]);
-                    umma_commit(&k_empty[s]);
-                    if (j > 0 && !issue_pv(j - 1)) ok = false;
+                    ok = issue_pv(j);
+                    if (ok && j + C::kSBufs < nkt) ok = issue_qk(j + C::kSBufs);
                 }
-                if (ok && !issue_pv(nkt - 1)) ok = false;
                 // every MMA issued has completed before TMEM and shared memory are released
-                umma_commit(mma_done);
+                umma_commit_warp(mma_done);
                 mbar_wait(mma_done, 0);
-                if (!ok) fail();
+                if (!ok && lane == 0) fail();
             }
             __syncwarp();
         }
@@ -511,12 +511,9 @@ __global__ void __launch_bounds__(224, 1)
     }
 }
 
-// P in shared memory (SS products) or in tensor memory (TS form of PV)
-constexpr bool kPrefillPInTmem = true;
-
 template <typename T, int D>
 cudaError_t launch_prefill_tc_t(const PrefillParams& p_in, cudaStream_t stream) {
-    using C = TcPf<D, kPrefillPInTmem, std::is_same<T, __nv_bfloat16>::value>;
+    using C = TcPf<D>;
     PrefillParams p = p_in;
     const bool neg = p.scale_log2 < 0.f;   // a negative scale: negate Q inside the QK^T product
     if (neg) p.scale_log2 = -p.scale_log2;
@@ -532,7 +529,7 @@ cudaError_t launch_prefill_tc_t(const PrefillParams& p_in, cudaStream_t stream) 
     if (e != cudaSuccess) return e;
     e = make_pool_map(&mv, p.value_cache, dt, p.num_blocks, p.num_kv_heads, D, kBlkT);
     if (e != cudaSuccess) return e;
-    auto kernel = prefill_tc_kernel<T, D, kPrefillPInTmem>;
+    auto kernel = prefill_tc_kernel<T, D>;
     e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
     const int qpos = kRowsT / p.group;   // query positions per tile
