@@ -558,7 +558,9 @@ def swap_bandwidth(w, nblocks: int = 4096, reps: int = 5):
 
 def prefill_throughput(seed: int, reps: int = 20):
     """pa_prefill on chunked prompts (4 sequences: 512 new tokens on 3,584 cached ones, Qwen-shaped
-    heads, bf16): causal attention TFLOP/s against the measured bf16 tensor peak."""
+    heads, bf16): causal attention TFLOP/s against the measured bf16 tensor peak.  Each timed call
+    follows an L2 flush (the 34 MB of K/V would otherwise stay L2-resident between calls) and is
+    timed alone with CUDA events; the median is reported."""
     import torch
 
     import paged_kv_cache_362_b200 as pa
@@ -576,23 +578,38 @@ def prefill_throughput(seed: int, reps: int = 20):
     qs = torch.arange(0, B * chunk + 1, chunk, dtype=torch.int32, device="cuda")
     cl = torch.full((B,), ctx, dtype=torch.int32, device="cuda")
     args = (out, q, kc, vc, bt, qs, cl, 1 / D ** 0.5, chunk)
+    flush_w = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
     for _ in range(3):
         pa.prefill(*args)
     torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
+    times = []
     for _ in range(reps):
+        flush_w.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
         pa.prefill(*args)
-    e1.record()
-    torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / reps
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    ms = float(np.median(times))
     flops = 4 * Hq * D * B * sum(past + i + 1 for i in range(chunk))
     tf = flops / (ms * 1e-3) / 1e12
-    peak, _ = measured_bf16_peak()
-    kernel = "tcgen05 (prefill_tc_kernel)" if chunk * (Hq // Hkv) >= 32 else "mma.sync (prefill_kernel)"
+    peak, peak_kind = measured_bf16_peak()
+    tc = chunk * (Hq // Hkv) >= 32
+    kernel = "tcgen05 (prefill_tc_kernel)" if tc else "mma.sync (prefill_kernel)"
+    # tensor-core work issued per 128-key step of a 128-row tile: QK^T (K = D) and, for bf16, PV
+    # twice (P's hi and lo parts); the useful flops count each PV once
+    issued = 1.5 if tc else 1.0
     return {"workload": f"{B} sequences x ({chunk} new on {past} cached tokens), 28/4 heads, D 128, bf16",
-            "kernel": kernel, "ms": round(ms, 4), "tflops": round(tf, 1), "peak_tflops": peak,
-            "frac": round(tf / peak, 4)}
+            "kernel": kernel, "ms": round(ms, 4), "ms_p10_p50_p90": pct3(times), "tflops": round(tf, 1),
+            "peak_tflops": peak, "peak_kind": peak_kind, "frac": round(tf / peak, 4),
+            "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": peak, "unit": "TFLOP/s",
+                         "frac": round(tf / peak, 4),
+                         "issued_tflops": round(tf * issued, 1),
+                         "note": "achieved counts causal attention flops (4 x D per query-key pair); the "
+                                 "kernel issues 1.5x that on the tensor cores (bf16 P as hi + lo)"},
+            "l2": "flushed before every timed call (256 MiB write), each call timed alone; median of "
+                  f"{reps}"}
 
 
 def measured_bf16_peak():
@@ -692,6 +709,8 @@ def main():
     ap.add_argument("--ref-total-s", type=float, default=90.0, help="CPU seconds the reference arm may take")
     ap.add_argument("--layers", type=int, default=4,
                     help="K/V pools (model layers) the layer-rotation measurement cycles through")
+    ap.add_argument("--prefill-only", action="store_true",
+                    help="time pa_prefill on its chunked-prompt workload, print its JSON line and exit")
     args = ap.parse_args()
 
     if args.impl == "reference":
@@ -704,6 +723,11 @@ def main():
 
     if not torch.cuda.is_available():
         raise SystemExit("bench.py needs a CUDA device")
+    if args.prefill_only:
+        if rank == 0:
+            print(json.dumps(prefill_throughput(args.seed)), flush=True)
+        dist_done()
+        return
     peak, peak_kind = measured_hbm_peak()
     # L2 flush before every timed step: write 256 MiB (twice the L2), then read
     # another 256 MiB so that the write's dirty lines are written back during
