@@ -59,6 +59,11 @@ constexpr int kBlkT = 16;         // tokens per block
 // The max used for the exponentials moves only when a tile's max exceeds it
 // by more than this (log2 units): p <= 2^8, well inside fp16 and bf16.
 constexpr float kRescaleSlack = 8.f;
+// Waiting warps sleep this long between polls of an mbarrier: the softmax warps
+// and the MMA warp share schedulers, and a tight poll takes the issue slots the
+// warp being waited for needs (1.5% of the kernel's time on the bench workload;
+// suspending in mbarrier.try_wait instead cost 3.5%).
+constexpr uint32_t kPollNs = 20;
 
 template <int D>
 struct TcPf {
@@ -87,6 +92,29 @@ struct TcPf {
     static constexpr uint32_t kColO = 384;                  // O: D columns
     static_assert(kBytes + 1024 <= 227 * 1024, "shared memory");
 };
+
+// Spin with a short sleep between polls (bounded like mbar_wait): a waiting
+// warp then leaves most issue slots to the warps that share its scheduler,
+// and still resumes within tens of nanoseconds of the phase completing.
+__device__ __forceinline__ bool mbar_sleep_wait(uint64_t* bar, uint32_t parity, uint32_t sleep_ns,
+                                                uint64_t limit_ns = kWaitLimitNs) {
+    if (mbar_test_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (;;) {
+        __nanosleep(sleep_ns);
+        if (mbar_test_wait(bar, parity)) return true;
+        if (global_timer_ns() - t0 > limit_ns) return false;
+    }
+}
+// The same for a warp: lane 0 polls, then every lane observes the completed
+// phase itself.  Returns false on expiry, for every lane.
+__device__ __forceinline__ bool warp_sleep_wait(uint64_t* bar, uint32_t parity, int lane, uint32_t sleep_ns) {
+    int ok = 1;
+    if (lane == 0) ok = mbar_sleep_wait(bar, parity, sleep_ns);
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    if (ok) mbar_test_wait(bar, parity);
+    return ok != 0;
+}
 
 // byte offset of 16-byte unit u (0..7) of row r inside a 128-byte-swizzled group
 __device__ __forceinline__ uint32_t sw128(int r, int u) { return (uint32_t)(r * 128 + ((u ^ (r & 7)) << 4)); }
@@ -220,7 +248,7 @@ __global__ void __launch_bounds__(224, 1)
                 id_next = tile_block_id(bt_row, j + 1, nkt, kend, lane);
                 const int sb = j % C::kSBufs;
                 const uint32_t sph = (uint32_t)(j / C::kSBufs) & 1u;
-                if (!warp_spin_wait(&s_full[sb], sph, lane) || *abort_flag) {
+                if (!warp_sleep_wait(&s_full[sb], sph, lane, kPollNs) || *abort_flag) {
                     ok = false;
                     break;
                 }
@@ -302,7 +330,7 @@ __global__ void __launch_bounds__(224, 1)
                 // preceded this tile's scores, so the parity names one phase.
                 if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
                     const int pb = (j - 1) % C::kSBufs;
-                    if (!warp_spin_wait(&pv_done[pb], (uint32_t)((j - 1) / C::kSBufs) & 1u, lane) || *abort_flag) {
+                    if (!warp_sleep_wait(&pv_done[pb], (uint32_t)((j - 1) / C::kSBufs) & 1u, lane, kPollNs) || *abort_flag) {
                         ok = false;
                         break;
                     }
@@ -323,7 +351,7 @@ __global__ void __launch_bounds__(224, 1)
                 if (lane == 0) mbar_arrive(&p_full[sb]);
             }
             if (ok) {
-                ok = warp_spin_wait(&pv_done[(nkt - 1) % C::kSBufs], (uint32_t)((nkt - 1) / C::kSBufs) & 1u, lane) &&
+                ok = warp_sleep_wait(&pv_done[(nkt - 1) % C::kSBufs], (uint32_t)((nkt - 1) / C::kSBufs) & 1u, lane, kPollNs) &&
                      !*abort_flag;
                 if (ok) {
                     tc_fence_after();
@@ -421,11 +449,10 @@ __global__ void __launch_bounds__(224, 1)
             constexpr uint64_t kVStep = (2 * 1024) >> 4;                      // 16 keys of V
             // The whole warp runs the issue loop (warp-uniform control flow: the
             // descriptors stay in uniform registers) and one elected lane issues
-            // each product; waits spin (bounded) and end for all lanes together.
-            // (Suspending in mbarrier.try_wait measured slower: the wake-up
-            // latency lands on the tensor core's critical path.)
+            // each product; waits poll with a short sleep (bounded) and end for
+            // all lanes together.
             auto wait_all = [&](uint64_t* bar, uint32_t par) -> bool {
-                return __all_sync(0xffffffffu, mbar_spin_wait(bar, par) && !*abort_flag);
+                return __all_sync(0xffffffffu, mbar_sleep_wait(bar, par, kPollNs) && !*abort_flag);
             };
             auto issue_qk = [&](int j) -> bool {
                 const int s = j % C::kStages;
