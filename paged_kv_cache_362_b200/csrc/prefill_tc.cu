@@ -9,9 +9,10 @@
 // cache block as the unit the tile is made of).
 //
 // Tiles.  A CTA owns 128 rows of (query position, GQA head) pairs of one
-// (sequence, KV head): floor(128 / G) consecutive positions times the G query
-// heads of the group, so every K/V tile it loads serves all of them.  It
-// walks the keys 128 at a time (eight 16-token blocks):
+// (sequence, KV head), in the order position * G + head, so every K/V tile it
+// loads serves the whole group and no row is left empty except at the end of
+// a chunk (a tile may begin and end inside a position's group).  It walks the
+// keys 128 at a time (eight 16-token blocks):
 //     S = Q K^T           tcgen05.mma, M = 128 rows, N = 128 keys, K = D
 //     P = 2^(S*scale*log2 e - m)   fp32 online softmax, one thread per row
 //     O += P V            tcgen05.mma with P in tensor memory, M = 128, N = D,
@@ -134,7 +135,7 @@ __device__ __forceinline__ uint32_t bad_mask(const PrefillParams& p, int id) {
 template <typename T, int D>
 __global__ void __launch_bounds__(224, 1)
     prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmK,
-                      const __grid_constant__ CUtensorMap tmV, int qpos, uint32_t idesc_qk, uint32_t idesc_pv) {
+                      const __grid_constant__ CUtensorMap tmV, uint32_t idesc_qk, uint32_t idesc_pv) {
     // bf16 P (8-bit significand) would perturb the softmax weights by up to
     // 2^-8, which on rows with a few comparable keys moves the output by up
     // to ~1e-2; it is carried as hi + lo (two bf16 parts, ~16 bits) and the PV
@@ -196,17 +197,20 @@ __global__ void __launch_bounds__(224, 1)
 
     const int qs = p.query_start[b], L = p.query_start[b + 1] - qs;
     const int n = p.context_lens[b];
-    const int i0 = tile * qpos;
-    bool active = L > 0 && i0 < L;
+    // The chunk's query rows are (position i, head k of the group) pairs in
+    // the order i * G + k; tile t holds rows 128t .. 128t + 127, so a tile may
+    // start and end in the middle of a position's group.
+    const int R0 = tile * kRowsT;                    // the tile's first row
+    bool active = L > 0 && R0 < L * G;
     if (active && (n < L || n > p.max_blocks_per_seq * kBlkT)) {   // a query position outside the cache
         if (threadIdx.x == 0) set_status(p.status, PA_ERR_OUT_OF_RANGE);
         active = false;
     }
     if (active) {
-        const int npos = min(qpos, L - i0);          // query positions in this tile
-        const int nrows = npos * G;
-        const int pos0 = n - L + i0;                 // position of the tile's first query
-        const int kend = pos0 + npos;                // keys [0, kend) are visible to some row
+        const int nrows = min(kRowsT, L * G - R0);   // rows of this tile that hold a query
+        const int i0 = R0 / G;                       // query index of the tile's first row
+        const int pos0 = n - L + i0;                 // its position in the sequence
+        const int kend = n - L + (R0 + nrows - 1) / G + 1;   // keys [0, kend) are visible to some row
         const int nkt = ceil_div_i(kend, kKeysT);
         const int32_t* bt_row = p.block_tables + (size_t)b * p.max_blocks_per_seq;
         const uint32_t sQ = smem_u32(smem + C::kOffQ);
@@ -220,13 +224,14 @@ __global__ void __launch_bounds__(224, 1)
         if (warp < 4) {
             // ================================================= softmax warps
             const int r = threadIdx.x;                              // tile row = TMEM lane
-            const int prow = min(r / G, npos - 1);                  // rows past the tile repeat its last position
-            const int pos = pos0 + prow;
+            const int rq = R0 + min(r, nrows - 1);                  // rows past the chunk repeat its last row
+            const int qi = rq / G, qk = rq - qi * G;                // query index and head of the row
+            const int pos = n - L + qi;
             const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
             const float sl2 = p.scale_log2;                         // > 0 (a negative scale negates A)
             {   // Q row r: 16-byte pieces into the swizzled K-major layout
                 const bool real = r < nrows;
-                const T* qrow = static_cast<const T*>(p.q) + ((size_t)(qs + i0 + prow) * p.num_heads + g * G + r % G) * D;
+                const T* qrow = static_cast<const T*>(p.q) + ((size_t)(qs + qi) * p.num_heads + g * G + qk) * D;
 #pragma unroll
                 for (int c = 0; c < D / 8; ++c) {
                     uint4 v = make_uint4(0, 0, 0, 0);
@@ -356,7 +361,7 @@ __global__ void __launch_bounds__(224, 1)
                 if (ok) {
                     tc_fence_after();
                     const float inv = l > 0.f ? 1.f / l : 0.f;
-                    T* dst = static_cast<T*>(p.out) + ((size_t)(qs + i0 + prow) * p.num_heads + g * G + r % G) * D;
+                    T* dst = static_cast<T*>(p.out) + ((size_t)(qs + qi) * p.num_heads + g * G + qk) * D;
 #pragma unroll
                     for (int c = 0; c < D / 32; ++c) {
                         uint32_t ov[32];
@@ -559,9 +564,9 @@ cudaError_t launch_prefill_tc_t(const PrefillParams& p_in, cudaStream_t stream) 
     auto kernel = prefill_tc_kernel<T, D>;
     e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
-    const int qpos = kRowsT / p.group;   // query positions per tile
-    const dim3 grid((p.max_query_len + qpos - 1) / qpos, p.num_kv_heads, p.num_seqs);
-    return launch_pdl(kernel, grid, dim3(C::kThreads), C::kSmemBytes, stream, p, mk, mv, qpos, idesc_qk, idesc_pv);
+    // 128-row tiles over the (position, head) rows of the longest chunk
+    const dim3 grid((unsigned)(((long long)p.max_query_len * p.group + kRowsT - 1) / kRowsT), p.num_kv_heads, p.num_seqs);
+    return launch_pdl(kernel, grid, dim3(C::kThreads), C::kSmemBytes, stream, p, mk, mv, idesc_qk, idesc_pv);
 }
 
 }  // namespace
