@@ -226,6 +226,41 @@ pa_status pa_prefill(void* out, const void* q, const void* key_cache, const void
                      pa_dtype dtype, int32_t* status, pa_stream_t stream);
 
 /*
+ * pa_prefill_ws -- pa_prefill with a workspace, which lets the tensor-core
+ * kernel balance its last wave.  That kernel runs one CTA per SM on 128-row
+ * tiles; when the tiles do not fill whole waves, each tile of the last,
+ * partial wave is split by key range into pieces (up to 8) that run on the
+ * SMs the wave would leave idle.  Each piece writes its rows' unnormalised
+ * partial output, reference max and sum to the workspace, and a second
+ * kernel, chained to the first, merges them (exact algebra: out = sum_q
+ * 2^(m_q - m) O_q / sum_q 2^(m_q - m) l_q).  The result is the same function
+ * as pa_prefill's, up to fp32 rounding.
+ *
+ *   workspace        device memory of at least pa_prefill_workspace_size()
+ *                    bytes for these sizes, 16-byte aligned; scratch only (no
+ *                    contents carry from one call to the next).  May be NULL
+ *                    when the size is 0.
+ *   workspace_bytes  its size; smaller than required: PA_ERR_INVALID_ARG
+ * Calls that share a workspace must not run concurrently.  Everything else is
+ * as pa_prefill.
+ */
+pa_status pa_prefill_ws(void* out, const void* q, const void* key_cache, const void* value_cache,
+                        const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* query_start,
+                        const int32_t* context_lens, int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads,
+                        int32_t head_dim, int32_t block_size, int32_t num_blocks, float scale, int32_t max_query_len,
+                        void* workspace, size_t workspace_bytes, pa_dtype dtype, int32_t* status,
+                        pa_stream_t stream);
+
+/*
+ * pa_prefill_workspace_size -- the workspace pa_prefill_ws needs for these
+ * sizes on the current device (the split depends on its SM count; 0 when the
+ * tiles fill whole waves or the chunk is served by the mma.sync kernel).
+ * Invalid sizes: the error pa_prefill would return.
+ */
+pa_status pa_prefill_workspace_size(int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads, int32_t head_dim,
+                                    int32_t max_query_len, pa_dtype dtype, size_t* bytes);
+
+/*
  * pa_swap_blocks -- copy whole blocks from one pool to another of the same
  * shape, for evicting blocks to CPU memory and bringing them back
  * ("PagedAttention, Visualized", Part 3: the operating-system table, where

@@ -26,6 +26,7 @@ from ._lib import (  # noqa: F401
     error_string,
     make_workspace,
     prefill,
+    prefill_workspace_size,
     reshape_and_cache,
     set_default_tuning,
     swap_blocks,

@@ -76,7 +76,8 @@ def _load() -> ctypes.CDLL:
     lib = ctypes.CDLL(LIB_PATH)
     for sym in ("pa_reshape_and_cache", "pa_decode_workspace_size", "pa_decode", "pa_decode_launch_count",
                 "pa_copy_blocks", "pa_get_error_string", "pa_version", "pa_bm_create", "pa_bm_append_tokens",
-                "pa_prefill", "pa_swap_blocks", "pa_decode_tuned", "pa_decode_launch_count_tuned"):
+                "pa_prefill", "pa_swap_blocks", "pa_decode_tuned", "pa_decode_launch_count_tuned", "pa_prefill_ws",
+                "pa_prefill_workspace_size"):
         if not hasattr(lib, sym):
             raise ImportError(f"{LIB_PATH} lacks {sym} (stale build); run `python paged_kv_cache_362_b200/build.py`")
     p, i32, i64, f32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
@@ -122,6 +123,11 @@ def _load() -> ctypes.CDLL:
     lib.pa_bm_is_swapped.restype = i32
     lib.pa_prefill.argtypes = [p, p, p, p, p, i32, p, p, i32, i32, i32, i32, i32, i32, f32, i32, ctypes.c_int, p, p]
     lib.pa_prefill.restype = ctypes.c_int
+    lib.pa_prefill_ws.argtypes = [p, p, p, p, p, i32, p, p, i32, i32, i32, i32, i32, i32, f32, i32, p, sz,
+                                  ctypes.c_int, p, p]
+    lib.pa_prefill_ws.restype = ctypes.c_int
+    lib.pa_prefill_workspace_size.argtypes = [i32, i32, i32, i32, i32, ctypes.c_int, ctypes.POINTER(sz)]
+    lib.pa_prefill_workspace_size.restype = ctypes.c_int
     lib.pa_swap_blocks.argtypes = [p, p, p, p, p, i32, i32, i32, i32, i32, i32, ctypes.c_int, p, p]
     lib.pa_swap_blocks.restype = ctypes.c_int
     lib.pa_bm_block_tables.argtypes = [p, p, i32, i32, p, p]
@@ -237,12 +243,28 @@ def decode(out, q, key_cache, value_cache, block_tables, context_lens, scale, ma
            "pa_decode")
 
 
+def prefill_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, max_query_len, dtype="bf16") -> int:
+    """Bytes of workspace pa_prefill_ws needs for these sizes on the current device (may be 0)."""
+    n = ctypes.c_size_t(0)
+    if isinstance(dtype, str):
+        code = {"f32": PA_F32, "f16": PA_F16, "bf16": PA_BF16}[dtype]
+    else:
+        import torch
+
+        code = {torch.float32: PA_F32, torch.float16: PA_F16, torch.bfloat16: PA_BF16}[dtype]
+    _check(LIB.pa_prefill_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, max_query_len, code,
+                                         ctypes.byref(n)), "pa_prefill_workspace_size")
+    return int(n.value)
+
+
 def prefill(out, q, key_cache, value_cache, block_tables, query_start, context_lens, scale, max_query_len,
-            status=None, stream=None):
+            status=None, stream=None, workspace=None):
     """Causal attention of each sequence's new query rows over its paged cache (pa_prefill).
 
     q, out [T, Hq, D]; query_start int32 [B + 1]; context_lens int32 [B] (the new tokens included,
-    already written with reshape_and_cache).
+    already written with reshape_and_cache).  With a workspace (a uint8 device tensor of at least
+    prefill_workspace_size(...) bytes, scratch) the call is pa_prefill_ws, which splits the tensor-core
+    kernel's last partial wave.
     """
     T, Hq, D = q.shape
     NB, Hkv, bs = key_cache.shape[0], key_cache.shape[1], key_cache.shape[2]
@@ -253,10 +275,19 @@ def prefill(out, q, key_cache, value_cache, block_tables, query_start, context_l
     assert query_start.shape == (B + 1,) and block_tables.shape[0] == B
     for t in (out, q, key_cache, value_cache, block_tables, query_start, context_lens):
         assert t.is_contiguous()
-    _check(LIB.pa_prefill(_ptr(out), _ptr(q), _ptr(key_cache), _ptr(value_cache), _ptr(block_tables),
-                          block_tables.shape[1], _ptr(query_start), _ptr(context_lens), B, Hq, Hkv, D, bs, NB,
-                          float(scale), int(max_query_len), _dtype_code(q), _ptr(status), _stream(stream)),
-           "pa_prefill")
+    if workspace is None:
+        _check(LIB.pa_prefill(_ptr(out), _ptr(q), _ptr(key_cache), _ptr(value_cache), _ptr(block_tables),
+                              block_tables.shape[1], _ptr(query_start), _ptr(context_lens), B, Hq, Hkv, D, bs, NB,
+                              float(scale), int(max_query_len), _dtype_code(q), _ptr(status), _stream(stream)),
+               "pa_prefill")
+        return
+    assert workspace.is_contiguous()
+    _check(LIB.pa_prefill_ws(_ptr(out), _ptr(q), _ptr(key_cache), _ptr(value_cache), _ptr(block_tables),
+                             block_tables.shape[1], _ptr(query_start), _ptr(context_lens), B, Hq, Hkv, D, bs, NB,
+                             float(scale), int(max_query_len), _ptr(workspace),
+                             workspace.numel() * workspace.element_size(), _dtype_code(q), _ptr(status),
+                             _stream(stream)),
+           "pa_prefill_ws")
 
 
 def copy_blocks(key_cache, value_cache, block_pairs, status=None, stream=None):

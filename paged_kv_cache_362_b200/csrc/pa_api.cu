@@ -292,11 +292,12 @@ pa_status pa_copy_blocks(void* key_cache, void* value_cache, const int64_t* bloc
     return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
-pa_status pa_prefill(void* out, const void* q, const void* key_cache, const void* value_cache,
-                     const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* query_start,
-                     const int32_t* context_lens, int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads,
-                     int32_t head_dim, int32_t block_size, int32_t num_blocks, float scale, int32_t max_query_len,
-                     pa_dtype dtype, int32_t* status, pa_stream_t stream) {
+namespace {
+// Validates pa_prefill's sizes and fills the kernel parameters (pointers are
+// checked by the callers, which know whether the call has work to do).
+pa_status prefill_params(PrefillParams* p, int32_t max_blocks_per_seq, int32_t num_seqs, int32_t num_heads,
+                         int32_t num_kv_heads, int32_t head_dim, int32_t block_size, int32_t num_blocks, float scale,
+                         int32_t max_query_len, pa_dtype dtype) {
     if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || num_blocks <= 0 ||
         max_blocks_per_seq <= 0 || max_query_len < 0)
         return PA_ERR_INVALID_ARG;
@@ -306,12 +307,38 @@ pa_status pa_prefill(void* out, const void* q, const void* key_cache, const void
         return PA_ERR_UNSUPPORTED;
     // pool rows (blocks x KV heads x 16) index the tensor copies in int32
     if ((int64_t)num_blocks * num_kv_heads * kChunk > INT32_MAX) return PA_ERR_UNSUPPORTED;
+    *p = PrefillParams{};
+    p->num_seqs = num_seqs;
+    p->num_heads = num_heads;
+    p->num_kv_heads = num_kv_heads;
+    p->head_dim = head_dim;
+    p->group = num_heads / num_kv_heads;
+    p->max_blocks_per_seq = max_blocks_per_seq;
+    p->num_blocks = num_blocks;
+    p->max_query_len = max_query_len;
+    p->scale_log2 = scale * 1.4426950408889634f;  // log2(e)
+    return PA_OK;
+}
+
+pa_status prefill_impl(void* out, const void* q, const void* key_cache, const void* value_cache,
+                       const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* query_start,
+                       const int32_t* context_lens, int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads,
+                       int32_t head_dim, int32_t block_size, int32_t num_blocks, float scale, int32_t max_query_len,
+                       bool with_ws, void* workspace, size_t workspace_bytes, pa_dtype dtype, int32_t* status,
+                       pa_stream_t stream) {
+    PrefillParams p;
+    const pa_status v = prefill_params(&p, max_blocks_per_seq, num_seqs, num_heads, num_kv_heads, head_dim,
+                                       block_size, num_blocks, scale, max_query_len, dtype);
+    if (v != PA_OK) return v;
     if (num_seqs == 0 || max_query_len == 0) return PA_OK;
     if (!out || !q || !key_cache || !value_cache || !block_tables || !query_start || !context_lens)
         return PA_ERR_INVALID_ARG;
     if (!aligned16(out) || !aligned16(q) || !aligned16(key_cache) || !aligned16(value_cache))
         return PA_ERR_INVALID_ARG;
-    PrefillParams p{};
+    if (with_ws) {
+        const size_t need = prefill_workspace_bytes(p);
+        if (need > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace))) return PA_ERR_INVALID_ARG;
+    }
     p.out = out;
     p.q = q;
     p.key_cache = key_cache;
@@ -320,17 +347,42 @@ pa_status pa_prefill(void* out, const void* q, const void* key_cache, const void
     p.query_start = query_start;
     p.context_lens = context_lens;
     p.status = status;
-    p.num_seqs = num_seqs;
-    p.num_heads = num_heads;
-    p.num_kv_heads = num_kv_heads;
-    p.head_dim = head_dim;
-    p.group = num_heads / num_kv_heads;
-    p.max_blocks_per_seq = max_blocks_per_seq;
-    p.num_blocks = num_blocks;
-    p.max_query_len = max_query_len;
-    p.scale_log2 = scale * 1.4426950408889634f;  // log2(e)
-    const cudaError_t e = launch_prefill(p, dtype, reinterpret_cast<cudaStream_t>(stream));
+    const cudaError_t e = launch_prefill(p, with_ws ? workspace : nullptr, with_ws ? workspace_bytes : 0, dtype,
+                                         reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+}  // namespace
+
+pa_status pa_prefill(void* out, const void* q, const void* key_cache, const void* value_cache,
+                     const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* query_start,
+                     const int32_t* context_lens, int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads,
+                     int32_t head_dim, int32_t block_size, int32_t num_blocks, float scale, int32_t max_query_len,
+                     pa_dtype dtype, int32_t* status, pa_stream_t stream) {
+    return prefill_impl(out, q, key_cache, value_cache, block_tables, max_blocks_per_seq, query_start, context_lens,
+                        num_seqs, num_heads, num_kv_heads, head_dim, block_size, num_blocks, scale, max_query_len,
+                        false, nullptr, 0, dtype, status, stream);
+}
+
+pa_status pa_prefill_workspace_size(int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads, int32_t head_dim,
+                                    int32_t max_query_len, pa_dtype dtype, size_t* bytes) {
+    if (!bytes) return PA_ERR_INVALID_ARG;
+    PrefillParams p;
+    const pa_status v = prefill_params(&p, 1, num_seqs, num_heads, num_kv_heads, head_dim, kChunk, 1, 1.f,
+                                       max_query_len, dtype);
+    if (v != PA_OK) return v;
+    *bytes = (num_seqs == 0 || max_query_len == 0) ? 0 : prefill_workspace_bytes(p);
+    return PA_OK;
+}
+
+pa_status pa_prefill_ws(void* out, const void* q, const void* key_cache, const void* value_cache,
+                        const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* query_start,
+                        const int32_t* context_lens, int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads,
+                        int32_t head_dim, int32_t block_size, int32_t num_blocks, float scale, int32_t max_query_len,
+                        void* workspace, size_t workspace_bytes, pa_dtype dtype, int32_t* status,
+                        pa_stream_t stream) {
+    return prefill_impl(out, q, key_cache, value_cache, block_tables, max_blocks_per_seq, query_start, context_lens,
+                        num_seqs, num_heads, num_kv_heads, head_dim, block_size, num_blocks, scale, max_query_len,
+                        true, workspace, workspace_bytes, dtype, status, stream);
 }
 
 pa_status pa_swap_blocks(const void* src_key_cache, const void* src_value_cache, void* dst_key_cache,

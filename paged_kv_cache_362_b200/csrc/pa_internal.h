@@ -33,9 +33,14 @@ cudaError_t launch_swap_blocks(const void* src_key, const void* src_value, void*
 // Causal attention of each sequence's new query tokens over its paged cache:
 // the tcgen05 kernel where prefill_tc_serves() (chunks that fill its 128-row
 // tiles), else the mma.sync kernel.
-cudaError_t launch_prefill(const PrefillParams& p, pa_dtype dtype, cudaStream_t stream);
+// With a workspace of prefill_workspace_bytes(p) bytes (scratch), the tcgen05
+// kernel splits the items of its last, partial wave by key range and a second
+// kernel merges the pieces.
+cudaError_t launch_prefill(const PrefillParams& p, void* ws, size_t ws_bytes, pa_dtype dtype, cudaStream_t stream);
+size_t prefill_workspace_bytes(const PrefillParams& p);
 bool prefill_tc_serves(const PrefillParams& p);
-cudaError_t launch_prefill_tc(const PrefillParams& p, pa_dtype dtype, cudaStream_t stream);
+size_t prefill_tc_workspace_bytes(const PrefillParams& p);
+cudaError_t launch_prefill_tc(const PrefillParams& p, void* ws, size_t ws_bytes, pa_dtype dtype, cudaStream_t stream);
 
 // TMA descriptor of a K or V pool viewed as 2-D: rows of head_dim elements,
 // one row per (block, KV head, slot); a box is 16 rows (8 for 8-token blocks)

@@ -247,8 +247,10 @@ cudaError_t launch_prefill_t(const PrefillParams& p, cudaStream_t stream) {
 
 }  // namespace
 
-cudaError_t launch_prefill(const PrefillParams& p, pa_dtype dtype, cudaStream_t stream) {
-    if (prefill_tc_serves(p)) return launch_prefill_tc(p, dtype, stream);
+size_t prefill_workspace_bytes(const PrefillParams& p) { return prefill_tc_workspace_bytes(p); }
+
+cudaError_t launch_prefill(const PrefillParams& p, void* ws, size_t ws_bytes, pa_dtype dtype, cudaStream_t stream) {
+    if (prefill_tc_serves(p)) return launch_prefill_tc(p, ws, ws_bytes, dtype, stream);
     if (dtype == PA_F16) return p.head_dim == 64 ? launch_prefill_t<__half, 64>(p, stream)
                                                  : launch_prefill_t<__half, 128>(p, stream);
     if (dtype == PA_BF16) return p.head_dim == 64 ? launch_prefill_t<__nv_bfloat16, 64>(p, stream)

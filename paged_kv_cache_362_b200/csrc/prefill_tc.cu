@@ -47,6 +47,8 @@
 //        probability of 0 times a NaN left in shared memory would still be NaN.
 // Every mbarrier wait is bounded (PA_ERR_TIMEOUT); on expiry the CTA lets
 // its copies and MMAs finish, frees its TMEM and returns.
+#include <algorithm>
+
 #include "pa_internal.h"
 
 namespace pa {
@@ -132,10 +134,28 @@ __device__ __forceinline__ uint32_t bad_mask(const PrefillParams& p, int id) {
     return __ballot_sync(0xffffffffu, id < 0 || id >= p.num_blocks) & 0xffu;
 }
 
+// The grid: tx tiles per (sequence, KV head); work item i is tile
+// tx - 1 - (i mod tx) of KV head (i / tx) mod Hkv of sequence i / (tx Hkv)
+// (a sequence's longest tiles first).  Items 0 .. nfull - 1 are whole CTAs;
+// each item after them (the grid's last, partial wave) is split by key range
+// into ksplit pieces, one CTA each, whose partial results (O unnormalised,
+// the reference max and the sum, per row) go to `part`; prefill_merge_kernel,
+// launched next, combines them.
+struct PrefillGrid {
+    int tx, nfull, ksplit;
+    float* part;   // [tail items][ksplit][128 rows][D + 4]: O, then m and l (and 2 floats of padding)
+};
+// At most this many pieces per split item: more would shorten the last wave
+// further but make the merge read more partial rows.
+constexpr int kMaxSplit = 8;
+// floats per partial row: 16-byte aligned rows for the vector stores and loads
+__host__ __device__ constexpr int part_row_floats(int d) { return d + 4; }
+
 template <typename T, int D>
 __global__ void __launch_bounds__(224, 1)
     prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmK,
-                      const __grid_constant__ CUtensorMap tmV, uint32_t idesc_qk, uint32_t idesc_pv) {
+                      const __grid_constant__ CUtensorMap tmV, uint32_t idesc_qk, uint32_t idesc_pv,
+                      const PrefillGrid pg) {
     // bf16 P (8-bit significand) would perturb the softmax weights by up to
     // 2^-8, which on rows with a few comparable keys moves the output by up
     // to ~1e-2; it is carried as hi + lo (two bf16 parts, ~16 bits) and the PV
@@ -164,8 +184,16 @@ __global__ void __launch_bounds__(224, 1)
     volatile uint32_t* stage_bad = reinterpret_cast<volatile uint32_t*>(smem + C::kOffMisc + 16);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int G = p.group, b = blockIdx.z, g = blockIdx.y;
-    const int tile = (int)gridDim.x - 1 - (int)blockIdx.x;   // the longest tiles of a sequence start first
+    const int G = p.group;
+    int item = (int)blockIdx.x, piece = 0, npieces = 1;
+    if (item >= pg.nfull) {
+        const int t = item - pg.nfull;
+        item = pg.nfull + t / pg.ksplit;
+        piece = t % pg.ksplit;
+        npieces = pg.ksplit;
+    }
+    const int g = (item / pg.tx) % p.num_kv_heads, b = item / (pg.tx * p.num_kv_heads);
+    const int tile = pg.tx - 1 - item % pg.tx;   // the longest tiles of a sequence start first
 
     if (threadIdx.x == 128) {
         mbar_init(q_full, 4);
@@ -212,6 +240,10 @@ __global__ void __launch_bounds__(224, 1)
         const int pos0 = n - L + i0;                 // its position in the sequence
         const int kend = n - L + (R0 + nrows - 1) / G + 1;   // keys [0, kend) are visible to some row
         const int nkt = ceil_div_i(kend, kKeysT);
+        // this CTA's key tiles: all of them, or its piece of the range
+        const int kt_lo = (int)((long long)nkt * piece / npieces);
+        const int kt_hi = (int)((long long)nkt * (piece + 1) / npieces);
+        const int nloc = kt_hi - kt_lo;
         const int32_t* bt_row = p.block_tables + (size_t)b * p.max_blocks_per_seq;
         const uint32_t sQ = smem_u32(smem + C::kOffQ);
         const uint32_t sK = smem_u32(smem + C::kOffK);
@@ -247,12 +279,13 @@ __global__ void __launch_bounds__(224, 1)
             }
             float m_ref = kNegInfT, l = 0.f;
             bool ok = true;
-            int id_next = tile_block_id(bt_row, 0, nkt, kend, lane);
-            for (int j = 0; j < nkt && ok; ++j) {
+            int id_next = tile_block_id(bt_row, kt_lo, kt_hi, kend, lane);
+            for (int j = kt_lo; j < kt_hi && ok; ++j) {
+                const int jj = j - kt_lo;                       // local index: buffers and phases
                 const int id_cur = id_next;
-                id_next = tile_block_id(bt_row, j + 1, nkt, kend, lane);
-                const int sb = j % C::kSBufs;
-                const uint32_t sph = (uint32_t)(j / C::kSBufs) & 1u;
+                id_next = tile_block_id(bt_row, j + 1, kt_hi, kend, lane);
+                const int sb = jj % C::kSBufs;
+                const uint32_t sph = (uint32_t)(jj / C::kSBufs) & 1u;
                 if (!warp_sleep_wait(&s_full[sb], sph, lane, kPollNs) || *abort_flag) {
                     ok = false;
                     break;
@@ -333,9 +366,10 @@ __global__ void __launch_bounds__(224, 1)
                 // the previous tiles' PV products complete.  The PV of tile j - 1
                 // signals buffer (j - 1) mod 3, whose previous signal (tile j - 4)
                 // preceded this tile's scores, so the parity names one phase.
-                if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-                    const int pb = (j - 1) % C::kSBufs;
-                    if (!warp_sleep_wait(&pv_done[pb], (uint32_t)((j - 1) / C::kSBufs) & 1u, lane, kPollNs) || *abort_flag) {
+                if (jj > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+                    const int pb = (jj - 1) % C::kSBufs;
+                    if (!warp_sleep_wait(&pv_done[pb], (uint32_t)((jj - 1) / C::kSBufs) & 1u, lane, kPollNs) ||
+                        *abort_flag) {
                         ok = false;
                         break;
                     }
@@ -355,31 +389,55 @@ __global__ void __launch_bounds__(224, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&p_full[sb]);
             }
-            if (ok) {
-                ok = warp_sleep_wait(&pv_done[(nkt - 1) % C::kSBufs], (uint32_t)((nkt - 1) / C::kSBufs) & 1u, lane, kPollNs) &&
+            // every PV product of this CTA has completed (a piece with no key tile has none)
+            if (ok && nloc > 0)
+                ok = warp_sleep_wait(&pv_done[(nloc - 1) % C::kSBufs], (uint32_t)((nloc - 1) / C::kSBufs) & 1u, lane,
+                                     kPollNs) &&
                      !*abort_flag;
-                if (ok) {
-                    tc_fence_after();
-                    const float inv = l > 0.f ? 1.f / l : 0.f;
-                    T* dst = static_cast<T*>(p.out) + ((size_t)(qs + qi) * p.num_heads + g * G + qk) * D;
+            if (ok) tc_fence_after();
+            T* dst = static_cast<T*>(p.out) + ((size_t)(qs + qi) * p.num_heads + g * G + qk) * D;
+            auto store_row = [&](const float* v, int c0) {   // 32 output elements from column c0
 #pragma unroll
-                    for (int c = 0; c < D / 32; ++c) {
-                        uint32_t ov[32];
-                        tmem_ld32(tl + C::kColO + c * 32, ov);
-                        tmem_ld_wait(ov);
-                        if (r < nrows) {
-#pragma unroll
-                            for (int k = 0; k < 32; k += 8) {
-                                uint4 w;
-                                w.x = Elt<T>::pack2(__uint_as_float(ov[k]) * inv, __uint_as_float(ov[k + 1]) * inv);
-                                w.y = Elt<T>::pack2(__uint_as_float(ov[k + 2]) * inv, __uint_as_float(ov[k + 3]) * inv);
-                                w.z = Elt<T>::pack2(__uint_as_float(ov[k + 4]) * inv, __uint_as_float(ov[k + 5]) * inv);
-                                w.w = Elt<T>::pack2(__uint_as_float(ov[k + 6]) * inv, __uint_as_float(ov[k + 7]) * inv);
-                                *reinterpret_cast<uint4*>(dst + c * 32 + k) = w;
-                            }
-                        }
-                    }
+                for (int k = 0; k < 32; k += 8) {
+                    uint4 w;
+                    w.x = Elt<T>::pack2(v[k], v[k + 1]);
+                    w.y = Elt<T>::pack2(v[k + 2], v[k + 3]);
+                    w.z = Elt<T>::pack2(v[k + 4], v[k + 5]);
+                    w.w = Elt<T>::pack2(v[k + 6], v[k + 7]);
+                    *reinterpret_cast<uint4*>(dst + c0 + k) = w;
                 }
+            };
+            if (ok && npieces == 1) {
+                const float inv = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t ov[32];
+                    tmem_ld32(tl + C::kColO + c * 32, ov);
+                    tmem_ld_wait(ov);
+                    float v[32];
+#pragma unroll
+                    for (int k = 0; k < 32; ++k) v[k] = __uint_as_float(ov[k]) * inv;
+                    if (r < nrows) store_row(v, c * 32);
+                }
+            } else if (ok) {
+                // A piece of a split item: its row's O (unnormalised, relative to
+                // m_ref), m_ref and l go to the workspace for prefill_merge_kernel
+                // (a piece that saw no key leaves l = 0 and an O the merge ignores).
+                constexpr int kRow = part_row_floats(D);
+                float* mine = pg.part + (((size_t)(item - pg.nfull) * npieces + piece) * kRowsT + r) * kRow;
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t ov[32];
+                    tmem_ld32(tl + C::kColO + c * 32, ov);
+                    tmem_ld_wait(ov);
+#pragma unroll
+                    for (int k = 0; k < 32; k += 4)
+                        *reinterpret_cast<float4*>(mine + c * 32 + k) =
+                            make_float4(__uint_as_float(ov[k]), __uint_as_float(ov[k + 1]), __uint_as_float(ov[k + 2]),
+                                        __uint_as_float(ov[k + 3]));
+                }
+                mine[D] = m_ref;
+                mine[D + 1] = l;
             }
             if (!ok && lane == 0) fail();
         } else if (warp == 4 || warp == 6) {
@@ -395,12 +453,13 @@ __global__ void __launch_bounds__(224, 1)
             constexpr uint32_t kBlockBytes = kBlkT * D * 2;   // one block of one KV head: K or V
             int issued = 0;
             bool ok = true;
-            int id_next = tile_block_id(bt_row, 0, nkt, kend, lane);
-            for (int j = 0; j < nkt && ok; ++j) {
-                const int s = j % C::kStages;
-                const uint32_t par = ((j / C::kStages) & 1) ^ 1;
+            int id_next = tile_block_id(bt_row, kt_lo, kt_hi, kend, lane);
+            for (int j = kt_lo; j < kt_hi && ok; ++j) {
+                const int jj = j - kt_lo;                     // local index: stages and phases
+                const int s = jj % C::kStages;
+                const uint32_t par = ((jj / C::kStages) & 1) ^ 1;
                 const int id = id_next;
-                id_next = tile_block_id(bt_row, j + 1, nkt, kend, lane);
+                id_next = tile_block_id(bt_row, j + 1, kt_hi, kend, lane);
                 const bool need = lane < 8 && (j * 8 + lane) * kBlkT < kend;
                 const bool good = need && id >= 0 && id < p.num_blocks;
                 if (is_k && need && !good) set_status(p.status, PA_ERR_OUT_OF_RANGE);
@@ -420,7 +479,7 @@ __global__ void __launch_bounds__(224, 1)
                         tma_load_2d_keep(base + s * C::kKVBytes + h * C::kGroupBytes + lane * (kBlkT * 128), map,
                                          h * 64, y, &fullb[s]);
                 }
-                issued = j + 1;
+                issued = jj + 1;
             }
             if (!ok && lane == 0) {
                 // let the copies this warp issued land before the CTA's memory is released
@@ -459,12 +518,15 @@ __global__ void __launch_bounds__(224, 1)
             auto wait_all = [&](uint64_t* bar, uint32_t par) -> bool {
                 return __all_sync(0xffffffffu, mbar_sleep_wait(bar, par, kPollNs) && !*abort_flag);
             };
+            // key tile j of the item; stages, buffers and phases follow this CTA's
+            // local index j - kt_lo
             auto issue_qk = [&](int j) -> bool {
-                const int s = j % C::kStages;
-                if (!wait_all(&k_full[s], (j / C::kStages) & 1)) return false;
+                const int jj = j - kt_lo;
+                const int s = jj % C::kStages;
+                if (!wait_all(&k_full[s], (jj / C::kStages) & 1)) return false;
                 tc_fence_after();
                 const uint64_t dk = dK0 + (uint64_t)s * kStageStep;
-                const int sb = j % C::kSBufs;
+                const int sb = jj % C::kSBufs;
                 const uint32_t dS = tmem + C::kColS + sb * kKeysT;
 #pragma unroll
                 for (int k = 0; k < D / 16; ++k)
@@ -474,10 +536,11 @@ __global__ void __launch_bounds__(224, 1)
                 return true;
             };
             auto issue_pv = [&](int i) -> bool {
-                const int s = i % C::kStages;
-                const int sb = i % C::kSBufs;
-                if (!wait_all(&p_full[sb], (uint32_t)(i / C::kSBufs) & 1u)) return false;
-                if (!wait_all(&v_full[s], (i / C::kStages) & 1)) return false;
+                const int ii = i - kt_lo;
+                const int s = ii % C::kStages;
+                const int sb = ii % C::kSBufs;
+                if (!wait_all(&p_full[sb], (uint32_t)(ii / C::kSBufs) & 1u)) return false;
+                if (!wait_all(&v_full[s], (ii / C::kStages) & 1)) return false;
                 const uint32_t badm = __shfl_sync(0xffffffffu, stage_bad[s], 0);
                 // keys of this tile the PV product covers: whole 16-key steps up to kend
                 const int nks = min(kKeysT, kend - i * kKeysT + kBlkT - 1) / kBlkT;
@@ -502,7 +565,7 @@ __global__ void __launch_bounds__(224, 1)
                 tc_fence_after();
                 const uint64_t dv = dV0 + (uint64_t)s * kStageStep;
                 const uint32_t tP = tmem + C::kColS + sb * kKeysT;
-                const uint32_t acc0 = i > 0 ? 1u : 0u;
+                const uint32_t acc0 = ii > 0 ? 1u : 0u;
 #pragma unroll
                 for (int k = 0; k < kKeysT / kBlkT; ++k)
                     if (k < nks)
@@ -522,10 +585,10 @@ __global__ void __launch_bounds__(224, 1)
                 // product of tile j + 3 follows the PV product of tile j, which
                 // reads the P that shares its buffer
                 ok = wait_all(q_full, 0);
-                for (int j = 0; j < min(nkt, C::kSBufs) && ok; ++j) ok = issue_qk(j);
-                for (int j = 0; j < nkt && ok; ++j) {
+                for (int j = kt_lo; j < min(kt_hi, kt_lo + C::kSBufs) && ok; ++j) ok = issue_qk(j);
+                for (int j = kt_lo; j < kt_hi && ok; ++j) {
                     ok = issue_pv(j);
-                    if (ok && j + C::kSBufs < nkt) ok = issue_qk(j + C::kSBufs);
+                    if (ok && j + C::kSBufs < kt_hi) ok = issue_qk(j + C::kSBufs);
                 }
                 // every MMA issued has completed before TMEM and shared memory are released
                 umma_commit_warp(mma_done);
@@ -543,8 +606,93 @@ __global__ void __launch_bounds__(224, 1)
     }
 }
 
+
+// The grid for one CTA per SM: tx tiles per (sequence, KV head), and the
+// items of the last, partial wave split into ksplit pieces when that leaves
+// at least two pieces per item.
+struct SplitPlan {
+    int tx = 0;
+    long long items = 0;
+    int tail = 0, ksplit = 1;
+    size_t bytes = 0;   // workspace: the split items' partial rows
+};
+SplitPlan split_plan(const PrefillParams& p, int sm_count) {
+    SplitPlan s;
+    s.tx = (int)(((long long)p.max_query_len * p.group + kRowsT - 1) / kRowsT);
+    s.items = (long long)s.tx * p.num_kv_heads * p.num_seqs;
+    if (sm_count > 0 && s.items > sm_count) {
+        const int tail = (int)(s.items % sm_count);
+        const int k = tail > 0 ? std::min(kMaxSplit, sm_count / tail) : 1;
+        if (k >= 2) {
+            s.tail = tail;
+            s.ksplit = k;
+            s.bytes = (size_t)tail * k * kRowsT * part_row_floats(p.head_dim) * sizeof(float);
+        }
+    }
+    return s;
+}
+int sm_count_now() {
+    DeviceInfo d;
+    return device_info(&d) == cudaSuccess && d.sm_count > 0 ? d.sm_count : 148;
+}
+
+// Combines the pieces of the split items: one warp per (item, row), lanes
+// over the row's columns (4 each), the pieces' maxima and sums combined with
+// warp shuffles:
+//     out = sum_q 2^(m_q - m) O_q / sum_q 2^(m_q - m) l_q,  m = max_q m_q,
+// over the pieces that saw a key (l_q > 0).  Runs after the attention kernel
+// (programmatic dependent launch: it waits for that grid's completion).
 template <typename T, int D>
-cudaError_t launch_prefill_tc_t(const PrefillParams& p_in, cudaStream_t stream) {
+__global__ void __launch_bounds__(128) prefill_merge_kernel(const PrefillParams p, const PrefillGrid pg, int tail) {
+    griddep_wait();
+    const int lane = threadIdx.x & 31;
+    const long long gw = (long long)blockIdx.x * 4 + (threadIdx.x >> 5);
+    const int ti = (int)(gw / kRowsT), r = (int)(gw % kRowsT);
+    if (ti >= tail) return;
+    const int G = p.group, item = pg.nfull + ti;
+    const int g = (item / pg.tx) % p.num_kv_heads, b = item / (pg.tx * p.num_kv_heads);
+    const int tile = pg.tx - 1 - item % pg.tx;
+    const int qs = p.query_start[b], L = p.query_start[b + 1] - qs, n = p.context_lens[b];
+    const int R = tile * kRowsT + r;
+    // the rows the attention kernel computed (its sequence checks, and rows that hold a query)
+    if (L <= 0 || R >= L * G || n < L || n > p.max_blocks_per_seq * kBlkT) return;
+    constexpr int kRow = part_row_floats(D);
+    const float* rows = pg.part + ((size_t)ti * pg.ksplit * kRowsT + r) * kRow;
+    const size_t pstride = (size_t)kRowsT * kRow;
+    float mq = kNegInfT, lq = 0.f;
+    if (lane < pg.ksplit) {
+        mq = __ldcg(rows + lane * pstride + D);
+        lq = __ldcg(rows + lane * pstride + D + 1);
+    }
+    float m = lq > 0.f ? mq : kNegInfT;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    const float w = lq > 0.f ? fast_exp2(mq - m) : 0.f;
+    float lt = w * lq;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) lt += __shfl_xor_sync(0xffffffffu, lt, o);
+    const float inv = lt > 0.f ? 1.f / lt : 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int q = 0; q < kMaxSplit; ++q) {
+        const float f = __shfl_sync(0xffffffffu, w, q) * inv;
+        if (q < pg.ksplit && f != 0.f && lane * 4 < D) {
+            const float4 o = __ldcg(reinterpret_cast<const float4*>(rows + q * pstride) + lane);
+            acc.x += f * o.x;
+            acc.y += f * o.y;
+            acc.z += f * o.z;
+            acc.w += f * o.w;
+        }
+    }
+    if (lane * 4 < D) {
+        const int qi = R / G, qk = R - (R / G) * G;
+        T* dst = static_cast<T*>(p.out) + ((size_t)(qs + qi) * p.num_heads + g * G + qk) * D + lane * 4;
+        *reinterpret_cast<uint2*>(dst) = make_uint2(Elt<T>::pack2(acc.x, acc.y), Elt<T>::pack2(acc.z, acc.w));
+    }
+}
+
+template <typename T, int D>
+cudaError_t launch_prefill_tc_t(const PrefillParams& p_in, void* ws, size_t ws_bytes, cudaStream_t stream) {
     using C = TcPf<D>;
     PrefillParams p = p_in;
     const bool neg = p.scale_log2 < 0.f;   // a negative scale: negate Q inside the QK^T product
@@ -564,9 +712,25 @@ cudaError_t launch_prefill_tc_t(const PrefillParams& p_in, cudaStream_t stream) 
     auto kernel = prefill_tc_kernel<T, D>;
     e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return e;
-    // 128-row tiles over the (position, head) rows of the longest chunk
-    const dim3 grid((unsigned)(((long long)p.max_query_len * p.group + kRowsT - 1) / kRowsT), p.num_kv_heads, p.num_seqs);
-    return launch_pdl(kernel, grid, dim3(C::kThreads), C::kSmemBytes, stream, p, mk, mv, idesc_qk, idesc_pv);
+    // 128-row tiles over the (position, head) rows of the longest chunk, one
+    // work item per (tile, KV head, sequence); with a workspace, the last
+    // partial wave's items are split by key range
+    const SplitPlan sp = split_plan(p, sm_count_now());
+    PrefillGrid pg{sp.tx, (int)sp.items, 1, nullptr};
+    const bool split = ws && sp.tail > 0 && ws_bytes >= sp.bytes;
+    if (split) {
+        pg.nfull = (int)(sp.items - sp.tail);
+        pg.ksplit = sp.ksplit;
+        pg.part = static_cast<float*>(ws);
+    }
+    const long long ctas = pg.nfull + (sp.items - pg.nfull) * pg.ksplit;
+    if (ctas > INT32_MAX) return cudaErrorInvalidValue;
+    e = launch_pdl(kernel, dim3((unsigned)ctas), dim3(C::kThreads), C::kSmemBytes, stream, p, mk, mv, idesc_qk,
+                   idesc_pv, pg);
+    if (e != cudaSuccess || !split) return e;
+    // one warp per row of the split items
+    return launch_pdl(prefill_merge_kernel<T, D>, dim3((unsigned)(sp.tail * kRowsT / 4)), dim3(128), 0, stream, p,
+                      pg, sp.tail);
 }
 
 }  // namespace
@@ -578,11 +742,15 @@ bool prefill_tc_serves(const PrefillParams& p) {
     return (long long)p.max_query_len * p.group >= 32;
 }
 
-cudaError_t launch_prefill_tc(const PrefillParams& p, pa_dtype dtype, cudaStream_t stream) {
-    if (dtype == PA_F16) return p.head_dim == 64 ? launch_prefill_tc_t<__half, 64>(p, stream)
-                                                 : launch_prefill_tc_t<__half, 128>(p, stream);
-    if (dtype == PA_BF16) return p.head_dim == 64 ? launch_prefill_tc_t<__nv_bfloat16, 64>(p, stream)
-                                                  : launch_prefill_tc_t<__nv_bfloat16, 128>(p, stream);
+size_t prefill_tc_workspace_bytes(const PrefillParams& p) {
+    return prefill_tc_serves(p) ? split_plan(p, sm_count_now()).bytes : 0;
+}
+
+cudaError_t launch_prefill_tc(const PrefillParams& p, void* ws, size_t ws_bytes, pa_dtype dtype, cudaStream_t stream) {
+    if (dtype == PA_F16) return p.head_dim == 64 ? launch_prefill_tc_t<__half, 64>(p, ws, ws_bytes, stream)
+                                                 : launch_prefill_tc_t<__half, 128>(p, ws, ws_bytes, stream);
+    if (dtype == PA_BF16) return p.head_dim == 64 ? launch_prefill_tc_t<__nv_bfloat16, 64>(p, ws, ws_bytes, stream)
+                                                  : launch_prefill_tc_t<__nv_bfloat16, 128>(p, ws, ws_bytes, stream);
     return cudaErrorInvalidValue;
 }
 

@@ -185,6 +185,35 @@ def test_prefill_and_swap_validation():
         assert sw(bs, n=0) == pa.PA_OK
 
 
+def test_prefill_workspace_size_and_validation():
+    """pa_prefill_ws's workspace: the tiles of the last, partial wave (one CTA per SM; 148 SMs when no
+    device can be queried) split into up to 16 pieces; none when the tiles fill whole waves."""
+    import paged_kv_cache_362_b200 as pa
+
+    lib = pa._lib.LIB
+    n = ctypes.c_size_t(0)
+
+    def size(B, Hq, Hkv, D, L, dt=2):
+        rc = lib.pa_prefill_workspace_size(B, Hq, Hkv, D, L, dt, ctypes.byref(n))
+        return rc, n.value
+
+    # 4 x 512 queries, 28/4 heads, D 128: 28 tiles x 4 KV heads x 4 = 448 items = 3 x 148 + 4;
+    # the 4 are split 8 ways: 4 x 8 x 128 partial rows of 128 + 4 floats
+    assert size(4, 28, 4, 128, 512) == (pa.PA_OK, 4 * 8 * 128 * 132 * 4)
+    assert size(1, 28, 4, 128, 512)[1] == 0          # 112 items: one wave
+    assert size(2, 28, 4, 128, 676)[1] == 0          # 37 tiles x 8 = 296 items: two whole waves
+    assert size(4, 28, 4, 128, 4)[1] == 0            # 4 x 7 rows < 32: the mma.sync kernel
+    assert size(0, 28, 4, 128, 512) == (pa.PA_OK, 0)
+    assert size(4, 28, 4, 96, 512)[0] == pa.PA_ERR_UNSUPPORTED
+    assert size(4, 28, 4, 128, 512, dt=0)[0] == pa.PA_ERR_UNSUPPORTED
+    assert lib.pa_prefill_workspace_size(4, 28, 4, 128, 512, 2, None) == pa.PA_ERR_INVALID_ARG
+    need = size(4, 28, 4, 128, 512)[1]
+    ws = lambda wsp, nbytes: lib.pa_prefill_ws(FAKE, FAKE, FAKE, FAKE, FAKE, 256, FAKE, FAKE, 4, 28, 4, 128, 16, 1000,
+                                                ctypes.c_float(0.088), 512, wsp, nbytes, 2, None, None)
+    assert ws(None, 0) == pa.PA_ERR_INVALID_ARG              # a workspace is needed for these sizes
+    assert ws(FAKE, need - 1) == pa.PA_ERR_INVALID_ARG       # too small
+
+
 def test_host_copy_pair_checker():
     import numpy as np
 

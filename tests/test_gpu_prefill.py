@@ -43,7 +43,7 @@ def _case(rng, ctxs, chunks, Hq, Hkv, D, dtype, extra_blocks=3):
     return q, kc, vc, bt, qs, np.array(ctxs, dtype=np.int32)
 
 
-def _run(q, kc, vc, bt, qs, cl, scale, dtype, status=None):
+def _run(q, kc, vc, bt, qs, cl, scale, dtype, status=None, workspace=None):
     import torch
 
     import paged_kv_cache_362_b200 as pa
@@ -52,7 +52,8 @@ def _run(q, kc, vc, bt, qs, cl, scale, dtype, status=None):
                      device="cuda")
     st = torch.zeros(1, dtype=torch.int32, device="cuda") if status is None else status
     pa.prefill(out, to_device(q, dtype), to_device(kc, dtype), to_device(vc, dtype), torch.from_numpy(bt).cuda(),
-               torch.from_numpy(qs).cuda(), torch.from_numpy(cl).cuda(), scale, int(np.diff(qs).max()), status=st)
+               torch.from_numpy(qs).cuda(), torch.from_numpy(cl).cuda(), scale, int(np.diff(qs).max()), status=st,
+               workspace=workspace)
     torch.cuda.synchronize()
     return out, int(st.item())
 
@@ -212,3 +213,55 @@ def test_prefill_kernel_choice():
         out, st = _run(q, kc, vc, bt, qs, cl, 0.0884, "f16")
         assert st == 0
         compare(out_f64(out), c_oracle.prefill(q, kc, vc, bt, qs, cl, 0.0884, "f16", 4), "f16", f"chunks {chunks}")
+
+
+def _sm_count():
+    import torch
+
+    return torch.cuda.get_device_properties(0).multi_processor_count
+
+
+@pytest.mark.parametrize("ctx_last", [620, 3000], ids=["pieces-mostly-empty", "pieces-of-2-3-tiles"])
+def test_split_last_wave_every_element(ctx_last):
+    """pa_prefill_ws: 4 chunks of 512 rows x 7 heads = 448 tiles, 3 waves of 148 and 4 tiles split by key
+    range into pieces whose partial rows a second kernel merges.  With a short last context most pieces
+    hold no key tile (the merge must skip them); with a long one each holds two or three.  Two calls in a
+    row on the same workspace, every element against the oracle, the two results bit-identical, and the
+    call without a workspace agrees within the tolerance."""
+    import torch
+
+    import paged_kv_cache_362_b200 as pa
+
+    rng = np.random.default_rng(ctx_last)
+    ctxs, chunks = [1500, 900, 2100, ctx_last], [512, 512, 512, 512]
+    q, kc, vc, bt, qs, cl = _case(rng, ctxs, chunks, 28, 4, 128, "bf16")
+    need = pa.prefill_workspace_size(4, 28, 4, 128, 512, "bf16")
+    if _sm_count() != 148:
+        pytest.skip("the split sizes here assume 148 SMs")
+    assert need == 4 * 8 * 128 * 132 * 4
+    ws = torch.full((need,), 0xFF, dtype=torch.uint8, device="cuda")   # scratch: any contents
+    scale = 1.0 / np.sqrt(128)
+    ref = c_oracle.prefill(q, kc, vc, bt, qs, cl, scale, "bf16", 4)
+    out1, st1 = _run(q, kc, vc, bt, qs, cl, scale, "bf16", workspace=ws)
+    out2, st2 = _run(q, kc, vc, bt, qs, cl, scale, "bf16", workspace=ws)
+    assert st1 == 0 and st2 == 0
+    compare(out_f64(out1), ref, "bf16", f"split, last context {ctx_last}")
+    assert torch.equal(out1.view(torch.int16), out2.view(torch.int16))
+    out0, st0 = _run(q, kc, vc, bt, qs, cl, scale, "bf16")
+    assert st0 == 0
+    compare(out_f64(out0), ref, "bf16", f"unsplit, last context {ctx_last}")
+
+
+def test_split_workspace_too_small_is_rejected():
+    import torch
+
+    import paged_kv_cache_362_b200 as pa
+
+    if _sm_count() != 148:
+        pytest.skip("the split sizes here assume 148 SMs")
+    rng = np.random.default_rng(5)
+    q, kc, vc, bt, qs, cl = _case(rng, [600] * 4, [512] * 4, 28, 4, 128, "bf16")
+    need = pa.prefill_workspace_size(4, 28, 4, 128, 512, "bf16")
+    ws = torch.zeros(need - 16, dtype=torch.uint8, device="cuda")
+    with pytest.raises(pa.PagedAttentionError):
+        _run(q, kc, vc, bt, qs, cl, 0.088, "bf16", workspace=ws)
