@@ -229,7 +229,7 @@ pa_status pa_prefill(void* out, const void* q, const void* key_cache, const void
  * pa_prefill_ws -- pa_prefill with a workspace, which lets the tensor-core
  * kernel balance its last wave.  That kernel runs one CTA per SM on 128-row
  * tiles; when the tiles do not fill whole waves, each tile of the last,
- * partial wave is split by key range into pieces (up to 8) that run on the
+ * partial wave is split by key range into pieces (up to 16) that run on the
  * SMs the wave would leave idle.  Each piece writes its rows' unnormalised
  * partial output, reference max and sum to the workspace, and a second
  * kernel, chained to the first, merges them (exact algebra: out = sum_q

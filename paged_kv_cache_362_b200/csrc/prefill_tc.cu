@@ -135,8 +135,11 @@ __device__ __forceinline__ uint32_t bad_mask(const PrefillParams& p, int id) {
 }
 
 // The grid: tx tiles per (sequence, KV head); work item i is tile
-// tx - 1 - (i mod tx) of KV head (i / tx) mod Hkv of sequence i / (tx Hkv)
-// (a sequence's longest tiles first).  Items 0 .. nfull - 1 are whole CTAs;
+// tx - 1 - i / (Hkv B) of KV head (i mod Hkv B) mod Hkv of sequence
+// (i mod Hkv B) / Hkv: every (sequence, KV head)'s last tile first, then
+// every one's second-last, ..., so that the grid runs longest tiles first
+// (a tile's keys grow with its last query position) and each SM's share of
+// whole tiles evens out.  Items 0 .. nfull - 1 are whole CTAs;
 // each item after them (the grid's last, partial wave) is split by key range
 // into ksplit pieces, one CTA each, whose partial results (O unnormalised,
 // the reference max and the sum, per row) go to `part`; prefill_merge_kernel,
@@ -147,7 +150,7 @@ struct PrefillGrid {
 };
 // At most this many pieces per split item: more would shorten the last wave
 // further but make the merge read more partial rows.
-constexpr int kMaxSplit = 8;
+constexpr int kMaxSplit = 16;
 // floats per partial row: 16-byte aligned rows for the vector stores and loads
 __host__ __device__ constexpr int part_row_floats(int d) { return d + 4; }
 
@@ -192,8 +195,9 @@ __global__ void __launch_bounds__(224, 1)
         piece = t % pg.ksplit;
         npieces = pg.ksplit;
     }
-    const int g = (item / pg.tx) % p.num_kv_heads, b = item / (pg.tx * p.num_kv_heads);
-    const int tile = pg.tx - 1 - item % pg.tx;   // the longest tiles of a sequence start first
+    const int pairs = p.num_kv_heads * p.num_seqs;
+    const int g = (item % pairs) % p.num_kv_heads, b = (item % pairs) / p.num_kv_heads;
+    const int tile = pg.tx - 1 - item / pairs;   // the longest tiles start first
 
     if (threadIdx.x == 128) {
         mbar_init(q_full, 4);
@@ -650,8 +654,9 @@ __global__ void __launch_bounds__(128) prefill_merge_kernel(const PrefillParams 
     const int ti = (int)(gw / kRowsT), r = (int)(gw % kRowsT);
     if (ti >= tail) return;
     const int G = p.group, item = pg.nfull + ti;
-    const int g = (item / pg.tx) % p.num_kv_heads, b = item / (pg.tx * p.num_kv_heads);
-    const int tile = pg.tx - 1 - item % pg.tx;
+    const int pairs = p.num_kv_heads * p.num_seqs;
+    const int g = (item % pairs) % p.num_kv_heads, b = (item % pairs) / p.num_kv_heads;
+    const int tile = pg.tx - 1 - item / pairs;
     const int qs = p.query_start[b], L = p.query_start[b + 1] - qs, n = p.context_lens[b];
     const int R = tile * kRowsT + r;
     // the rows the attention kernel computed (its sequence checks, and rows that hold a query)

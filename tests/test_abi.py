@@ -198,8 +198,8 @@ def test_prefill_workspace_size_and_validation():
         return rc, n.value
 
     # 4 x 512 queries, 28/4 heads, D 128: 28 tiles x 4 KV heads x 4 = 448 items = 3 x 148 + 4;
-    # the 4 are split 8 ways: 4 x 8 x 128 partial rows of 128 + 4 floats
-    assert size(4, 28, 4, 128, 512) == (pa.PA_OK, 4 * 8 * 128 * 132 * 4)
+    # the 4 are split 16 ways: 4 x 16 x 128 partial rows of 128 + 4 floats
+    assert size(4, 28, 4, 128, 512) == (pa.PA_OK, 4 * 16 * 128 * 132 * 4)
     assert size(1, 28, 4, 128, 512)[1] == 0          # 112 items: one wave
     assert size(2, 28, 4, 128, 676)[1] == 0          # 37 tiles x 8 = 296 items: two whole waves
     assert size(4, 28, 4, 128, 4)[1] == 0            # 4 x 7 rows < 32: the mma.sync kernel
