@@ -80,13 +80,16 @@ struct TcPf {
     static constexpr int kOffK = kOffQ + kQBytes;
     static constexpr int kOffV = kOffK + kStages * kKVBytes;
     static constexpr int kOffBar = kOffV + kStages * kKVBytes;
-    // q_full, k_full[2], v_full[2], k_empty[2], v_empty[2], s_full[3], p_full[3], pv_done[3], mma_done
-    static constexpr int kNumBars = 1 + 4 * kStages + 3 * kSBufs + 1;
+    // q_full, k_full[2], v_full[2], k_empty[2], v_empty[2], s_full[3], p_full[3], pv_done[3], qk_done, pv_all
+    static constexpr int kNumBars = 1 + 4 * kStages + 3 * kSBufs + 2;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;   // TMEM base, abort flag, per-stage bad-block masks
     static constexpr int kBytes = kOffMisc + 16 + 4 * kStages;
     // one CTA per SM (the CTA holds all 512 TMEM columns): at least half of the SM's shared memory
     static constexpr int kSmemBytes = (kBytes + 1024) > 120 * 1024 ? (kBytes + 1024) : 120 * 1024;
-    static constexpr int kThreads = 224;   // 4 softmax warps, K producer, MMA issuer, V producer
+    // 4 softmax warps, K producer, QK^T issuer, V producer, PV issuer: the two
+    // issuers sit on different schedulers (warps 5 and 7), each beside one
+    // softmax warp, so each of those two takes half the issuing's share
+    static constexpr int kThreads = 256;
     static constexpr uint32_t kTmemCols = 512;
     // S buffer b at columns 128b: the fp32 scores of a 128-key tile, then, in
     // place, P as 16-bit pairs: columns 0-63 (hi) and 64-127 (lo, bf16 only)
@@ -155,7 +158,7 @@ constexpr int kMaxSplit = 16;
 __host__ __device__ constexpr int part_row_floats(int d) { return d + 4; }
 
 template <typename T, int D>
-__global__ void __launch_bounds__(224, 1)
+__global__ void __launch_bounds__(256, 1)
     prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, uint32_t idesc_qk, uint32_t idesc_pv,
                       const PrefillGrid pg) {
@@ -179,7 +182,8 @@ __global__ void __launch_bounds__(224, 1)
     uint64_t* s_full = v_empty + C::kStages;
     uint64_t* p_full = s_full + C::kSBufs;
     uint64_t* pv_done = p_full + C::kSBufs;
-    uint64_t* mma_done = pv_done + C::kSBufs;
+    uint64_t* qk_done = pv_done + C::kSBufs;   // every QK^T product has completed
+    uint64_t* pv_all = qk_done + 1;             // every PV product has completed
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
     // the V stage's blocks with an out-of-range id (written by the V producer before the stage's
@@ -212,7 +216,8 @@ __global__ void __launch_bounds__(224, 1)
             mbar_init(&p_full[i], 4);
             mbar_init(&pv_done[i], 1);
         }
-        mbar_init(mma_done, 1);
+        mbar_init(qk_done, 1);
+        mbar_init(pv_all, 1);
         *abort_flag = 0;
         mbar_fence_init();
     }
@@ -492,7 +497,7 @@ __global__ void __launch_bounds__(224, 1)
                     mbar_wait(&fullb[j % C::kStages], (j / C::kStages) & 1);
             }
         } else {
-            // ================================================ MMA issuer (warp 5)
+            // ============================= MMA issuers: QK^T (warp 5), PV (warp 7)
             bool ok = true;
             // descriptors: Q, K, P K-major (8-row atoms 1024 B apart, K steps of 16
             // elements 32 B apart inside a 128-byte row, 64-element groups 16 KB
@@ -584,21 +589,31 @@ __global__ void __launch_bounds__(224, 1)
                 umma_commit_warp(&v_empty[s]);
                 return true;
             };
-            {
-                // QK^T runs up to three tiles ahead (one per S buffer); the QK^T
-                // product of tile j + 3 follows the PV product of tile j, which
-                // reads the P that shares its buffer
+            if (warp == 5) {
+                // QK^T runs up to three tiles ahead (one per S buffer).  Buffer
+                // j mod 3 holds the P of tile j - 3, which the other issuer's PV
+                // product reads: the QK^T of tile j waits for that product to
+                // complete (products of different threads are not ordered).
                 ok = wait_all(q_full, 0);
-                for (int j = kt_lo; j < min(kt_hi, kt_lo + C::kSBufs) && ok; ++j) ok = issue_qk(j);
                 for (int j = kt_lo; j < kt_hi && ok; ++j) {
-                    ok = issue_pv(j);
-                    if (ok && j + C::kSBufs < kt_hi) ok = issue_qk(j + C::kSBufs);
+                    const int jj = j - kt_lo;
+                    if (jj >= C::kSBufs &&
+                        !wait_all(&pv_done[(jj - C::kSBufs) % C::kSBufs], (uint32_t)((jj - C::kSBufs) / C::kSBufs) & 1u)) {
+                        ok = false;
+                        break;
+                    }
+                    ok = issue_qk(j);
                 }
-                // every MMA issued has completed before TMEM and shared memory are released
-                umma_commit_warp(mma_done);
-                mbar_wait(mma_done, 0);
-                if (!ok && lane == 0) fail();
+                // every product this warp issued has completed before TMEM and
+                // shared memory are released
+                umma_commit_warp(qk_done);
+                mbar_wait(qk_done, 0);
+            } else {
+                for (int j = kt_lo; j < kt_hi && ok; ++j) ok = issue_pv(j);
+                umma_commit_warp(pv_all);
+                mbar_wait(pv_all, 0);
             }
+            if (!ok && lane == 0) fail();
             __syncwarp();
         }
     }
