@@ -14,7 +14,7 @@
 // a chunk (a tile may begin and end inside a position's group).  It walks the
 // keys 128 at a time (eight 16-token blocks):
 //     S = Q K^T           tcgen05.mma, M = 128 rows, N = 128 keys, K = D
-//     P = 2^(S*scale*log2 e - m)   fp32 online softmax, one thread per row
+//     P = 2^(S*scale*log2 e - m)   fp32 online softmax, four threads per row
 //     O += P V            tcgen05.mma with P in tensor memory, M = 128, N = D,
 //                         K = 128 keys (bf16: once for P's hi part, once for lo)
 // S has three buffers in tensor memory; the softmax writes a tile's P over
@@ -24,27 +24,33 @@
 // tensor memory (columns 384..511); Q, K and V in shared memory, 128-byte
 // swizzled.
 //
-// Warps (224 threads, one CTA per SM):
-//   0-3  softmax: thread r owns row r (TMEM lane r).  Loads its Q row into
-//        shared memory; per key tile reads its S row from TMEM, masks keys
-//        past its position (and blocks whose id is out of range), updates
-//        the running max and sum, writes its P row back in a quarter of the
-//        tile at a time; at the end scales its O row by 1/l and stores it.
-//        The max used for the exponentials only moves when the tile max
-//        exceeds it by more than 8 (log2 units), so O is rescaled rarely; the
-//        sum and O always use the same reference, which keeps the result
-//        exact algebra.
-//   4, 6 producers of K (warp 4) and V (warp 6): 2-D TMA of each block of the
-//        key step (16-row, 128-byte boxes, one per 64 columns), two stages
-//        each.  Blocks no row of the tile sees are not loaded; a block id out
-//        of range is reported and not loaded (the V producer hands the mask
-//        of such blocks to the MMA warp with the stage).
-//   5    MMA issuer and TMEM owner: QK^T of tiles 0-2, then per tile j the PV
-//        product of j and the QK^T of j + 3.  The warp runs the loop in
-//        lockstep and an elected lane issues.  Before a PV product it zeroes
-//        the V rows that are not data (slots past the context in the
-//        sequence's last block, and blocks that were not loaded), since a
-//        probability of 0 times a NaN left in shared memory would still be NaN.
+// Warps (384 threads, one CTA per SM):
+//   0-7  softmax, two warps per scheduler: warp w owns the first (w < 4) or
+//        last 16 TMEM lanes of quarter w mod 4, each thread two rows (lanes
+//        L and L + 8) and a quarter of each 8-key group, read and written
+//        through the 16-lane tcgen05.ld/st shapes; the row max and sum are
+//        combined over a row's four threads with shuffles.  The warps load Q
+//        into shared memory; per key tile they read S, mask keys past each
+//        row's position (and blocks whose id is out of range), update the
+//        running max and sum, write P back a quarter of the tile at a time;
+//        at the end they scale O by 1/l and store it.  The max used for the
+//        exponentials only moves when the tile max exceeds it by more than 8
+//        (log2 units), so O is rescaled rarely; the sum and O always use the
+//        same reference, which keeps the result exact algebra.
+//   8, 10 producers of K (warp 8) and V (warp 10): 2-D TMA of each block of
+//        the key step (16-row, 128-byte boxes, one per 64 columns), two
+//        stages each.  Blocks no row of the tile sees are not loaded; a block
+//        id out of range is reported and not loaded (the V producer hands the
+//        mask of such blocks to the PV issuer with the stage).
+//   9    QK^T issuer and TMEM owner: QK^T of tile j once the PV product of
+//        tile j - 3 (which reads the same buffer) has completed.
+//   11   PV issuer: per tile, once its P is written, the PV product(s).  Before
+//        one it zeroes the V rows that are not data (slots past the context
+//        in the sequence's last block, and blocks that were not loaded),
+//        since a probability of 0 times a NaN left in shared memory would
+//        still be NaN.
+// The issuers run their loops as whole warps (an elected lane issues), each on
+// a scheduler of its own beside two softmax warps.
 // Every mbarrier wait is bounded (PA_ERR_TIMEOUT); on expiry the CTA lets
 // its copies and MMAs finish, frees its TMEM and returns.
 #include <algorithm>
@@ -86,10 +92,10 @@ struct TcPf {
     static constexpr int kBytes = kOffMisc + 16 + 4 * kStages;
     // one CTA per SM (the CTA holds all 512 TMEM columns): at least half of the SM's shared memory
     static constexpr int kSmemBytes = (kBytes + 1024) > 120 * 1024 ? (kBytes + 1024) : 120 * 1024;
-    // 4 softmax warps, K producer, QK^T issuer, V producer, PV issuer: the two
-    // issuers sit on different schedulers (warps 5 and 7), each beside one
-    // softmax warp, so each of those two takes half the issuing's share
-    static constexpr int kThreads = 256;
+    // softmax warps 0-7 (two per scheduler: warps w and w + 4 own the first and
+    // the last 16 lanes of quarter w), then on the four schedulers the K
+    // producer (8), the QK^T issuer (9), the V producer (10), the PV issuer (11)
+    static constexpr int kThreads = 384;
     static constexpr uint32_t kTmemCols = 512;
     // S buffer b at columns 128b: the fp32 scores of a 128-key tile, then, in
     // place, P as 16-bit pairs: columns 0-63 (hi) and 64-127 (lo, bf16 only)
@@ -120,6 +126,41 @@ __device__ __forceinline__ bool warp_sleep_wait(uint64_t* bar, uint32_t parity, 
     ok = __shfl_sync(0xffffffffu, ok, 0);
     if (ok) mbar_test_wait(bar, parity);
     return ok != 0;
+}
+
+// Tensor-memory loads and stores in the 16-lane shapes, for a warp that owns
+// 16 of its quarter's 32 lanes (the address carries the first lane).  Thread
+// t holds lanes L = first + (t >> 2) and L + 8:
+//   .16x256b, repetition r: registers 4r, 4r + 1 are lane L, columns
+//       8r + 2(t & 3) and 8r + 2(t & 3) + 1; 4r + 2, 4r + 3 the same for L + 8;
+//   .16x128b, repetition r: registers 2r, 2r + 1 are lanes L, L + 8 at column
+//       4r + (t & 3).
+// (Measured: each lane's values written through the 32x32b shape and read
+// back through these.)
+__device__ __forceinline__ void tmem_ld_16x256b_x8(uint32_t taddr, uint32_t* r) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x256b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st_16x256b_x8(uint32_t taddr, const uint32_t* r) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.16x256b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]),
+        "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]),
+        "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_st_16x128b_x4(uint32_t taddr, const uint32_t* r) {
+    asm volatile("tcgen05.st.sync.aligned.16x128b.x4.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+                 "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+                 : "memory");
 }
 
 // byte offset of 16-byte unit u (0..7) of row r inside a 128-byte-swizzled group
@@ -158,7 +199,7 @@ constexpr int kMaxSplit = 16;
 __host__ __device__ constexpr int part_row_floats(int d) { return d + 4; }
 
 template <typename T, int D>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(384, 1)
     prefill_tc_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, uint32_t idesc_qk, uint32_t idesc_pv,
                       const PrefillGrid pg) {
@@ -203,8 +244,8 @@ __global__ void __launch_bounds__(256, 1)
     const int g = (item % pairs) % p.num_kv_heads, b = (item % pairs) / p.num_kv_heads;
     const int tile = pg.tx - 1 - item / pairs;   // the longest tiles start first
 
-    if (threadIdx.x == 128) {
-        mbar_init(q_full, 4);
+    if (threadIdx.x == 256) {
+        mbar_init(q_full, 8);
         for (int s = 0; s < C::kStages; ++s) {
             mbar_init(&k_full[s], 1);
             mbar_init(&v_full[s], 1);
@@ -213,7 +254,7 @@ __global__ void __launch_bounds__(256, 1)
         }
         for (int i = 0; i < C::kSBufs; ++i) {
             mbar_init(&s_full[i], 1);
-            mbar_init(&p_full[i], 4);
+            mbar_init(&p_full[i], 8);
             mbar_init(&pv_done[i], 1);
         }
         mbar_init(qk_done, 1);
@@ -221,7 +262,7 @@ __global__ void __launch_bounds__(256, 1)
         *abort_flag = 0;
         mbar_fence_init();
     }
-    if (warp == 5) {
+    if (warp == 9) {
         tmem_alloc(tmem_slot, C::kTmemCols);
         tmem_relinquish();
     }
@@ -262,19 +303,31 @@ __global__ void __launch_bounds__(256, 1)
             set_status(p.status, PA_ERR_TIMEOUT);
         };
 
-        if (warp < 4) {
+        if (warp < 8) {
             // ================================================= softmax warps
-            const int r = threadIdx.x;                              // tile row = TMEM lane
-            const int rq = R0 + min(r, nrows - 1);                  // rows past the chunk repeat its last row
-            const int qi = rq / G, qk = rq - qi * G;                // query index and head of the row
-            const int pos = n - L + qi;
-            const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
+            // Warp w owns TMEM lanes 32(w mod 4) + 16(w / 4) .. + 15 (its
+            // quarter's first or last 16 lanes); thread t of it holds rows
+            // rA = that base + t / 4 and rB = rA + 8, and in each 8-key group of
+            // a tile the keys 2(t mod 4) and 2(t mod 4) + 1.  A row's four
+            // threads are lanes 4k .. 4k + 3 of the warp.
+            const int cg = lane & 3;
+            const int lbase = 32 * (warp & 3) + 16 * (warp >> 2);
+            const int rA = lbase + (lane >> 2), rB = rA + 8;
+            const int rqA = R0 + min(rA, nrows - 1), rqB = R0 + min(rB, nrows - 1);   // rows past the chunk
+            const int qiA = rqA / G, qkA = rqA - qiA * G;                             // repeat its last row
+            const int qiB = rqB / G, qkB = rqB - qiB * G;
+            const int posA = n - L + qiA, posB = n - L + qiB;
+            const uint32_t tl = tmem + ((uint32_t)lbase << 16);
             const float sl2 = p.scale_log2;                         // > 0 (a negative scale negates A)
-            {   // Q row r: 16-byte pieces into the swizzled K-major layout
+            {   // Q: thread i loads half i mod 2 of row i / 2 (16-byte pieces into the
+                // swizzled K-major layout)
+                const int r = threadIdx.x >> 1, hq = threadIdx.x & 1;
                 const bool real = r < nrows;
+                const int rq = R0 + min(r, nrows - 1), qi = rq / G, qk = rq - qi * G;
                 const T* qrow = static_cast<const T*>(p.q) + ((size_t)(qs + qi) * p.num_heads + g * G + qk) * D;
 #pragma unroll
-                for (int c = 0; c < D / 8; ++c) {
+                for (int cc = 0; cc < D / 16; ++cc) {
+                    const int c = hq * (D / 16) + cc;
                     uint4 v = make_uint4(0, 0, 0, 0);
                     if (real) v = *reinterpret_cast<const uint4*>(qrow + c * 8);
                     const uint32_t a = sQ + (c >> 3) * C::kGroupBytes + sw128(r, c & 7);
@@ -286,7 +339,9 @@ __global__ void __launch_bounds__(256, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(q_full);
             }
-            float m_ref = kNegInfT, l = 0.f;
+            // per row: the reference max (equal in the row's four threads) and this
+            // thread's share of the sum
+            float mA = kNegInfT, mB = kNegInfT, lA = 0.f, lB = 0.f;
             bool ok = true;
             int id_next = tile_block_id(bt_row, kt_lo, kt_hi, kend, lane);
             for (int j = kt_lo; j < kt_hi && ok; ++j) {
@@ -301,9 +356,10 @@ __global__ void __launch_bounds__(256, 1)
                 }
                 tc_fence_after();
                 const uint32_t tS = tl + C::kColS + sb * kKeysT;
-                uint32_t sv[kKeysT];
-#pragma unroll
-                for (int c = 0; c < kKeysT / 32; ++c) tmem_ld32(tS + c * 32, sv + c * 32);
+                // sv[4e + 0, 1]: row A, keys 8e + 2cg, + 1; sv[4e + 2, 3]: row B, the same keys
+                uint32_t sv[kKeysT / 2];
+                tmem_ld_16x256b_x8(tS, sv);
+                tmem_ld_16x256b_x8(tS + 64, sv + 32);
                 tmem_ld_wait(sv);
                 const uint32_t badm = bad_mask(p, id_cur);
 
@@ -311,71 +367,94 @@ __global__ void __launch_bounds__(256, 1)
                 const int kb0 = j * kKeysT;
                 if (kb0 + kKeysT - 1 > pos0 || badm != 0) {
 #pragma unroll
-                    for (int c = 0; c < kKeysT; ++c)
-                        if (kb0 + c > pos || ((badm >> (c / kBlkT)) & 1u)) sv[c] = __float_as_uint(kNegInfT);
+                    for (int e = 0; e < kKeysT / 8; ++e) {
+                        const bool bad = (badm >> (e >> 1)) & 1u;
+                        const int key = kb0 + 8 * e + 2 * cg;
+                        if (bad || key > posA) sv[4 * e] = __float_as_uint(kNegInfT);
+                        if (bad || key + 1 > posA) sv[4 * e + 1] = __float_as_uint(kNegInfT);
+                        if (bad || key > posB) sv[4 * e + 2] = __float_as_uint(kNegInfT);
+                        if (bad || key + 1 > posB) sv[4 * e + 3] = __float_as_uint(kNegInfT);
+                    }
                 }
-                float mx0 = kNegInfT, mx1 = kNegInfT, mx2 = kNegInfT, mx3 = kNegInfT;
+                float xa0 = kNegInfT, xa1 = kNegInfT, xb0 = kNegInfT, xb1 = kNegInfT;
 #pragma unroll
-                for (int c = 0; c < kKeysT; c += 8) {
-                    mx0 = fmax3(mx0, __uint_as_float(sv[c]), __uint_as_float(sv[c + 1]));
-                    mx1 = fmax3(mx1, __uint_as_float(sv[c + 2]), __uint_as_float(sv[c + 3]));
-                    mx2 = fmax3(mx2, __uint_as_float(sv[c + 4]), __uint_as_float(sv[c + 5]));
-                    mx3 = fmax3(mx3, __uint_as_float(sv[c + 6]), __uint_as_float(sv[c + 7]));
+                for (int e = 0; e < kKeysT / 8; e += 2) {
+                    xa0 = fmax3(xa0, __uint_as_float(sv[4 * e]), __uint_as_float(sv[4 * e + 1]));
+                    xb0 = fmax3(xb0, __uint_as_float(sv[4 * e + 2]), __uint_as_float(sv[4 * e + 3]));
+                    xa1 = fmax3(xa1, __uint_as_float(sv[4 * e + 4]), __uint_as_float(sv[4 * e + 5]));
+                    xb1 = fmax3(xb1, __uint_as_float(sv[4 * e + 6]), __uint_as_float(sv[4 * e + 7]));
                 }
-                const float m_new = fmax3(mx0, mx1, fmaxf(mx2, mx3)) * sl2;
-                float alpha = 1.f;
-                if (m_new > m_ref + kRescaleSlack) {
-                    alpha = m_ref == kNegInfT ? 0.f : fast_exp2(m_ref - m_new);
-                    m_ref = m_new;
+                // the row maxima over the row's four threads
+                float mxA = fmaxf(xa0, xa1), mxB = fmaxf(xb0, xb1);
+                mxA = fmaxf(mxA, __shfl_xor_sync(0xffffffffu, mxA, 1));
+                mxB = fmaxf(mxB, __shfl_xor_sync(0xffffffffu, mxB, 1));
+                mxA = fmaxf(mxA, __shfl_xor_sync(0xffffffffu, mxA, 2));
+                mxB = fmaxf(mxB, __shfl_xor_sync(0xffffffffu, mxB, 2));
+                const float mnA = mxA * sl2, mnB = mxB * sl2;
+                float alphaA = 1.f, alphaB = 1.f;
+                if (mnA > mA + kRescaleSlack) {
+                    alphaA = mA == kNegInfT ? 0.f : fast_exp2(mA - mnA);
+                    mA = mnA;
                 }
-                const float ms = m_ref == kNegInfT ? 0.f : m_ref;
-                // P in the input dtype (bf16: hi + lo); the row sum adds what the PV products
-                // use: the rounded fp16 values, or the fp32 values hi + lo carry.  P row r
-                // goes over the scores just read (TMEM lane r, keys 2c and 2c + 1 in column
-                // c), a quarter of the tile at a time so that the stores overlap the
-                // exponentials of the next quarter.  The PV product of this tile is issued
-                // before the QK^T product that next writes this buffer, and the tensor
-                // core runs them in that order.  Pairs of keys go through the packed
-                // fp32x2 add and fma.
-                const float2 sl2v = make_float2(sl2, sl2), nms = make_float2(-ms, -ms);
-                float2 lsa = make_float2(0.f, 0.f), lsb = make_float2(0.f, 0.f);
+                if (mnB > mB + kRescaleSlack) {
+                    alphaB = mB == kNegInfT ? 0.f : fast_exp2(mB - mnB);
+                    mB = mnB;
+                }
+                const float msA = mA == kNegInfT ? 0.f : mA, msB = mB == kNegInfT ? 0.f : mB;
+                // P in the input dtype (bf16: hi + lo); the row sums add what the PV
+                // products use: the rounded fp16 values, or the fp32 values hi + lo
+                // carry.  The pair of keys 8e + 2cg, + 1 of a row goes to P column
+                // 4e + cg of its lane (the buffer's scores are overwritten in place),
+                // a quarter of the tile at a time so that the stores overlap the
+                // exponentials of the next quarter.  The PV product of this tile is
+                // issued before the QK^T product that next writes this buffer, and
+                // the QK^T issuer waits for it.
+                const float2 sl2v = make_float2(sl2, sl2), nmA = make_float2(-msA, -msA), nmB = make_float2(-msB, -msB);
+                float2 lsA = make_float2(0.f, 0.f), lsB = make_float2(0.f, 0.f);
 #pragma unroll
-                for (int qt = 0; qt < kKeysT / 32; ++qt) {
-                    uint32_t pk[16];
-                    uint32_t pl[kSplitP ? 16 : 1];
+                for (int qt = 0; qt < 4; ++qt) {
+                    // 16x128b repetition i of this quarter: P column 4(4qt + i) + cg, rows A, B
+                    uint32_t pk[8];
+                    uint32_t pl[kSplitP ? 8 : 1];
 #pragma unroll
-                    for (int c = 0; c < 16; ++c) {
-                        const int k0 = qt * 32 + 2 * c;
-                        const float2 x = __ffma2_rn(make_float2(__uint_as_float(sv[k0]), __uint_as_float(sv[k0 + 1])),
-                                                    sl2v, nms);
-                        const float e0 = fast_exp2(x.x), e1 = fast_exp2(x.y);
-                        float2& ls = (c & 1) ? lsb : lsa;
-                        if constexpr (kSplitP) {
-                            // hi = p truncated to bf16 (its upper 16 bits), lo = p - hi (exact in
-                            // fp32) truncated likewise: hi + lo is p to within 2^-15 relative.
-                            // Integer ops only: the transcendental pipe that computes 2^x is the
-                            // softmax's bottleneck, and a float -> bf16 conversion would run on it too.
-                            const uint32_t u0 = __float_as_uint(e0), u1 = __float_as_uint(e1);
-                            pk[c] = __byte_perm(u0, u1, 0x7632);
-                            const float2 r = __fadd2_rn(make_float2(e0, e1),
-                                                        make_float2(__uint_as_float((u0 & 0xffff0000u) ^ 0x80000000u),
-                                                                    __uint_as_float((u1 & 0xffff0000u) ^ 0x80000000u)));
-                            pl[c] = __byte_perm(__float_as_uint(r.x), __float_as_uint(r.y), 0x7632);
-                            ls = __fadd2_rn(ls, make_float2(e0, e1));
-                        } else {
-                            pk[c] = Elt<T>::pack2(e0, e1);
-                            ls = __fadd2_rn(ls, __half22float2(*reinterpret_cast<const __half2*>(&pk[c])));
+                    for (int i = 0; i < 4; ++i) {
+                        const int e = 4 * qt + i;
+#pragma unroll
+                        for (int rb = 0; rb < 2; ++rb) {
+                            const float2 x = __ffma2_rn(
+                                make_float2(__uint_as_float(sv[4 * e + 2 * rb]), __uint_as_float(sv[4 * e + 2 * rb + 1])),
+                                sl2v, rb ? nmB : nmA);
+                            const float e0 = fast_exp2(x.x), e1 = fast_exp2(x.y);
+                            float2& ls = rb ? lsB : lsA;
+                            if constexpr (kSplitP) {
+                                // hi = p truncated to bf16 (its upper 16 bits), lo = p - hi (exact
+                                // in fp32) truncated likewise: hi + lo is p to within 2^-15
+                                // relative.  Integer ops only: the transcendental pipe that
+                                // computes 2^x is the softmax's bottleneck, and a float -> bf16
+                                // conversion would run on it too.
+                                const uint32_t u0 = __float_as_uint(e0), u1 = __float_as_uint(e1);
+                                pk[2 * i + rb] = __byte_perm(u0, u1, 0x7632);
+                                const float2 rr = __fadd2_rn(
+                                    make_float2(e0, e1), make_float2(__uint_as_float((u0 & 0xffff0000u) ^ 0x80000000u),
+                                                                     __uint_as_float((u1 & 0xffff0000u) ^ 0x80000000u)));
+                                pl[2 * i + rb] = __byte_perm(__float_as_uint(rr.x), __float_as_uint(rr.y), 0x7632);
+                                ls = __fadd2_rn(ls, make_float2(e0, e1));
+                            } else {
+                                pk[2 * i + rb] = Elt<T>::pack2(e0, e1);
+                                ls = __fadd2_rn(ls, __half22float2(*reinterpret_cast<const __half2*>(&pk[2 * i + rb])));
+                            }
                         }
                     }
-                    tmem_st16(tS + qt * 16, pk);
-                    if constexpr (kSplitP) tmem_st16(tS + C::kColPLo + qt * 16, pl);
+                    tmem_st_16x128b_x4(tS + qt * 16, pk);
+                    if constexpr (kSplitP) tmem_st_16x128b_x4(tS + C::kColPLo + qt * 16, pl);
                 }
-                l = l * alpha + ((lsa.x + lsb.x) + (lsa.y + lsb.y));
+                lA = lA * alphaA + (lsA.x + lsA.y);
+                lB = lB * alphaB + (lsB.x + lsB.y);
                 // O is rescaled only when some row's reference max moved: that needs
                 // the previous tiles' PV products complete.  The PV of tile j - 1
                 // signals buffer (j - 1) mod 3, whose previous signal (tile j - 4)
                 // preceded this tile's scores, so the parity names one phase.
-                if (jj > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+                if (jj > 0 && __any_sync(0xffffffffu, alphaA != 1.f || alphaB != 1.f)) {
                     const int pb = (jj - 1) % C::kSBufs;
                     if (!warp_sleep_wait(&pv_done[pb], (uint32_t)((jj - 1) / C::kSBufs) & 1u, lane, kPollNs) ||
                         *abort_flag) {
@@ -384,13 +463,14 @@ __global__ void __launch_bounds__(256, 1)
                     }
                     tc_fence_after();
 #pragma unroll
-                    for (int c = 0; c < D / 32; ++c) {
+                    for (int c = 0; c < D / 64; ++c) {
                         uint32_t ov[32];
-                        tmem_ld32(tl + C::kColO + c * 32, ov);
+                        tmem_ld_16x256b_x8(tl + C::kColO + c * 64, ov);
                         tmem_ld_wait(ov);
 #pragma unroll
-                        for (int k = 0; k < 32; ++k) ov[k] = __float_as_uint(__uint_as_float(ov[k]) * alpha);
-                        tmem_st32(tl + C::kColO + c * 32, ov);
+                        for (int k = 0; k < 32; ++k)
+                            ov[k] = __float_as_uint(__uint_as_float(ov[k]) * ((k & 2) ? alphaB : alphaA));
+                        tmem_st_16x256b_x8(tl + C::kColO + c * 64, ov);
                     }
                 }
                 tmem_st_wait();
@@ -404,56 +484,67 @@ __global__ void __launch_bounds__(256, 1)
                                      kPollNs) &&
                      !*abort_flag;
             if (ok) tc_fence_after();
-            T* dst = static_cast<T*>(p.out) + ((size_t)(qs + qi) * p.num_heads + g * G + qk) * D;
-            auto store_row = [&](const float* v, int c0) {   // 32 output elements from column c0
-#pragma unroll
-                for (int k = 0; k < 32; k += 8) {
-                    uint4 w;
-                    w.x = Elt<T>::pack2(v[k], v[k + 1]);
-                    w.y = Elt<T>::pack2(v[k + 2], v[k + 3]);
-                    w.z = Elt<T>::pack2(v[k + 4], v[k + 5]);
-                    w.w = Elt<T>::pack2(v[k + 6], v[k + 7]);
-                    *reinterpret_cast<uint4*>(dst + c0 + k) = w;
-                }
-            };
+            // the rows' sums: the four threads' shares
+            lA += __shfl_xor_sync(0xffffffffu, lA, 1);
+            lA += __shfl_xor_sync(0xffffffffu, lA, 2);
+            lB += __shfl_xor_sync(0xffffffffu, lB, 1);
+            lB += __shfl_xor_sync(0xffffffffu, lB, 2);
             if (ok && npieces == 1) {
-                const float inv = l > 0.f ? 1.f / l : 0.f;
+                const float invA = lA > 0.f ? 1.f / lA : 0.f, invB = lB > 0.f ? 1.f / lB : 0.f;
+                T* dA = static_cast<T*>(p.out) + ((size_t)(qs + qiA) * p.num_heads + g * G + qkA) * D + 2 * cg;
+                T* dB = static_cast<T*>(p.out) + ((size_t)(qs + qiB) * p.num_heads + g * G + qkB) * D + 2 * cg;
 #pragma unroll
-                for (int c = 0; c < D / 32; ++c) {
+                for (int c = 0; c < D / 64; ++c) {
                     uint32_t ov[32];
-                    tmem_ld32(tl + C::kColO + c * 32, ov);
+                    tmem_ld_16x256b_x8(tl + C::kColO + c * 64, ov);
                     tmem_ld_wait(ov);
-                    float v[32];
 #pragma unroll
-                    for (int k = 0; k < 32; ++k) v[k] = __uint_as_float(ov[k]) * inv;
-                    if (r < nrows) store_row(v, c * 32);
+                    for (int e = 0; e < 8; ++e) {
+                        const int col = c * 64 + 8 * e;
+                        if (rA < nrows)
+                            *reinterpret_cast<uint32_t*>(dA + col) =
+                                Elt<T>::pack2(__uint_as_float(ov[4 * e]) * invA, __uint_as_float(ov[4 * e + 1]) * invA);
+                        if (rB < nrows)
+                            *reinterpret_cast<uint32_t*>(dB + col) = Elt<T>::pack2(
+                                __uint_as_float(ov[4 * e + 2]) * invB, __uint_as_float(ov[4 * e + 3]) * invB);
+                    }
                 }
             } else if (ok) {
-                // A piece of a split item: its row's O (unnormalised, relative to
-                // m_ref), m_ref and l go to the workspace for prefill_merge_kernel
-                // (a piece that saw no key leaves l = 0 and an O the merge ignores).
+                // A piece of a split item: its rows' O (unnormalised, relative to the
+                // reference max), the max and the sum go to the workspace for
+                // prefill_merge_kernel (a piece that saw no key leaves l = 0 and an O
+                // the merge ignores).
                 constexpr int kRow = part_row_floats(D);
-                float* mine = pg.part + (((size_t)(item - pg.nfull) * npieces + piece) * kRowsT + r) * kRow;
+                float* base = pg.part + ((size_t)(item - pg.nfull) * npieces + piece) * kRowsT * kRow;
+                float* mineA = base + (size_t)rA * kRow;
+                float* mineB = base + (size_t)rB * kRow;
 #pragma unroll
-                for (int c = 0; c < D / 32; ++c) {
+                for (int c = 0; c < D / 64; ++c) {
                     uint32_t ov[32];
-                    tmem_ld32(tl + C::kColO + c * 32, ov);
+                    tmem_ld_16x256b_x8(tl + C::kColO + c * 64, ov);
                     tmem_ld_wait(ov);
 #pragma unroll
-                    for (int k = 0; k < 32; k += 4)
-                        *reinterpret_cast<float4*>(mine + c * 32 + k) =
-                            make_float4(__uint_as_float(ov[k]), __uint_as_float(ov[k + 1]), __uint_as_float(ov[k + 2]),
-                                        __uint_as_float(ov[k + 3]));
+                    for (int e = 0; e < 8; ++e) {
+                        const int col = c * 64 + 8 * e + 2 * cg;
+                        *reinterpret_cast<float2*>(mineA + col) =
+                            make_float2(__uint_as_float(ov[4 * e]), __uint_as_float(ov[4 * e + 1]));
+                        *reinterpret_cast<float2*>(mineB + col) =
+                            make_float2(__uint_as_float(ov[4 * e + 2]), __uint_as_float(ov[4 * e + 3]));
+                    }
                 }
-                mine[D] = m_ref;
-                mine[D + 1] = l;
+                if (cg == 0) {
+                    mineA[D] = mA;
+                    mineA[D + 1] = lA;
+                    mineB[D] = mB;
+                    mineB[D + 1] = lB;
+                }
             }
             if (!ok && lane == 0) fail();
-        } else if (warp == 4 || warp == 6) {
-            // ============================== producers: warp 4 loads K, warp 6 loads V
+        } else if (warp == 8 || warp == 10) {
+            // ============================== producers: warp 8 loads K, warp 10 loads V
             // (separately, so that a K stage is refilled as soon as its QK^T is done,
             // not after the previous tile's PV has freed a V stage)
-            const bool is_k = warp == 4;
+            const bool is_k = warp == 8;
             const CUtensorMap* map = is_k ? &tmK : &tmV;
             uint64_t* fullb = is_k ? k_full : v_full;
             uint64_t* emptyb = is_k ? k_empty : v_empty;
@@ -497,7 +588,7 @@ __global__ void __launch_bounds__(256, 1)
                     mbar_wait(&fullb[j % C::kStages], (j / C::kStages) & 1);
             }
         } else {
-            // ============================= MMA issuers: QK^T (warp 5), PV (warp 7)
+            // ============================= MMA issuers: QK^T (warp 9), PV (warp 11)
             bool ok = true;
             // descriptors: Q, K, P K-major (8-row atoms 1024 B apart, K steps of 16
             // elements 32 B apart inside a 128-byte row, 64-element groups 16 KB
@@ -589,7 +680,7 @@ __global__ void __launch_bounds__(256, 1)
                 umma_commit_warp(&v_empty[s]);
                 return true;
             };
-            if (warp == 5) {
+            if (warp == 9) {
                 // QK^T runs up to three tiles ahead (one per S buffer).  Buffer
                 // j mod 3 holds the P of tile j - 3, which the other issuer's PV
                 // product reads: the QK^T of tile j waits for that product to
@@ -619,7 +710,7 @@ __global__ void __launch_bounds__(256, 1)
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == 9) {
         tc_fence_after();
         tmem_dealloc(tmem, C::kTmemCols);
     }
