@@ -244,6 +244,47 @@ __global__ void __launch_bounds__(384, 1)
     const int g = (item % pairs) % p.num_kv_heads, b = (item % pairs) / p.num_kv_heads;
     const int tile = pg.tx - 1 - item / pairs;   // the longest tiles start first
 
+    griddep_launch_dependents();
+    // query_start, context_lens, the block table and Q may be written by the
+    // preceding kernel: read only once it has completed
+    griddep_wait();
+    const int qs = p.query_start[b], L = p.query_start[b + 1] - qs;
+    const int n = p.context_lens[b];
+    // The chunk's query rows are (position i, head k of the group) pairs in
+    // the order i * G + k; tile t holds rows 128t .. 128t + 127, so a tile may
+    // start and end in the middle of a position's group.
+    const int R0 = tile * kRowsT;                    // the tile's first row
+    bool active = L > 0 && R0 < L * G;
+    if (active && (n < L || n > p.max_blocks_per_seq * kBlkT)) {   // a query position outside the cache
+        if (threadIdx.x == 0) set_status(p.status, PA_ERR_OUT_OF_RANGE);
+        active = false;
+    }
+    const int nrows = active ? min(kRowsT, L * G - R0) : 1;   // rows of this tile that hold a query
+    const int i0 = R0 / G;                                     // query index of the tile's first row
+    const int pos0 = n - L + i0;                               // its position in the sequence
+    const int kend = n - L + (R0 + nrows - 1) / G + 1;         // keys [0, kend) are visible to some row
+    const int nkt = ceil_div_i(kend, kKeysT);
+    // this CTA's key tiles: all of them, or its piece of the range
+    const int kt_lo = (int)((long long)nkt * piece / npieces);
+    const int kt_hi = (int)((long long)nkt * (piece + 1) / npieces);
+    const int nloc = kt_hi - kt_lo;
+    const int32_t* bt_row = p.block_tables + (size_t)b * p.max_blocks_per_seq;
+    // Issued before the CTA's setup, so that their latency overlaps it: the
+    // first key tile's block ids and, in the softmax warps, the thread's half
+    // of a Q row (all its pieces at once: one round trip, not one per piece).
+    const int id_first = active ? tile_block_id(bt_row, kt_lo, kt_hi, kend, lane) : 0;
+    uint4 qv[D / 16];
+    const int q_r = threadIdx.x >> 1, q_h = threadIdx.x & 1;   // Q row and half (softmax warps)
+    if (active && warp < 8) {
+        const bool real = q_r < nrows;
+        const int rq = R0 + min(q_r, nrows - 1), qi = rq / G, qk = rq - qi * G;
+        const uint4* qrow = reinterpret_cast<const uint4*>(static_cast<const T*>(p.q) +
+                                                           ((size_t)(qs + qi) * p.num_heads + g * G + qk) * D) +
+                            q_h * (D / 16);
+#pragma unroll
+        for (int cc = 0; cc < D / 16; ++cc) qv[cc] = real ? qrow[cc] : make_uint4(0, 0, 0, 0);
+    }
+
     if (threadIdx.x == 256) {
         mbar_init(q_full, 8);
         for (int s = 0; s < C::kStages; ++s) {
@@ -270,31 +311,8 @@ __global__ void __launch_bounds__(384, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    griddep_launch_dependents();
-    griddep_wait();
 
-    const int qs = p.query_start[b], L = p.query_start[b + 1] - qs;
-    const int n = p.context_lens[b];
-    // The chunk's query rows are (position i, head k of the group) pairs in
-    // the order i * G + k; tile t holds rows 128t .. 128t + 127, so a tile may
-    // start and end in the middle of a position's group.
-    const int R0 = tile * kRowsT;                    // the tile's first row
-    bool active = L > 0 && R0 < L * G;
-    if (active && (n < L || n > p.max_blocks_per_seq * kBlkT)) {   // a query position outside the cache
-        if (threadIdx.x == 0) set_status(p.status, PA_ERR_OUT_OF_RANGE);
-        active = false;
-    }
     if (active) {
-        const int nrows = min(kRowsT, L * G - R0);   // rows of this tile that hold a query
-        const int i0 = R0 / G;                       // query index of the tile's first row
-        const int pos0 = n - L + i0;                 // its position in the sequence
-        const int kend = n - L + (R0 + nrows - 1) / G + 1;   // keys [0, kend) are visible to some row
-        const int nkt = ceil_div_i(kend, kKeysT);
-        // this CTA's key tiles: all of them, or its piece of the range
-        const int kt_lo = (int)((long long)nkt * piece / npieces);
-        const int kt_hi = (int)((long long)nkt * (piece + 1) / npieces);
-        const int nloc = kt_hi - kt_lo;
-        const int32_t* bt_row = p.block_tables + (size_t)b * p.max_blocks_per_seq;
         const uint32_t sQ = smem_u32(smem + C::kOffQ);
         const uint32_t sK = smem_u32(smem + C::kOffK);
         const uint32_t sV = smem_u32(smem + C::kOffV);
@@ -319,20 +337,14 @@ __global__ void __launch_bounds__(384, 1)
             const int posA = n - L + qiA, posB = n - L + qiB;
             const uint32_t tl = tmem + ((uint32_t)lbase << 16);
             const float sl2 = p.scale_log2;                         // > 0 (a negative scale negates A)
-            {   // Q: thread i loads half i mod 2 of row i / 2 (16-byte pieces into the
-                // swizzled K-major layout)
-                const int r = threadIdx.x >> 1, hq = threadIdx.x & 1;
-                const bool real = r < nrows;
-                const int rq = R0 + min(r, nrows - 1), qi = rq / G, qk = rq - qi * G;
-                const T* qrow = static_cast<const T*>(p.q) + ((size_t)(qs + qi) * p.num_heads + g * G + qk) * D;
+            {   // Q: thread i stores half i mod 2 of row i / 2, loaded above (16-byte
+                // pieces into the swizzled K-major layout)
 #pragma unroll
                 for (int cc = 0; cc < D / 16; ++cc) {
-                    const int c = hq * (D / 16) + cc;
-                    uint4 v = make_uint4(0, 0, 0, 0);
-                    if (real) v = *reinterpret_cast<const uint4*>(qrow + c * 8);
-                    const uint32_t a = sQ + (c >> 3) * C::kGroupBytes + sw128(r, c & 7);
-                    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z),
-                                 "r"(v.w)
+                    const int c = q_h * (D / 16) + cc;
+                    const uint32_t a = sQ + (c >> 3) * C::kGroupBytes + sw128(q_r, c & 7);
+                    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(qv[cc].x), "r"(qv[cc].y),
+                                 "r"(qv[cc].z), "r"(qv[cc].w)
                                  : "memory");
                 }
                 fence_proxy_async_shared();
@@ -343,7 +355,7 @@ __global__ void __launch_bounds__(384, 1)
             // thread's share of the sum
             float mA = kNegInfT, mB = kNegInfT, lA = 0.f, lB = 0.f;
             bool ok = true;
-            int id_next = tile_block_id(bt_row, kt_lo, kt_hi, kend, lane);
+            int id_next = id_first;
             for (int j = kt_lo; j < kt_hi && ok; ++j) {
                 const int jj = j - kt_lo;                       // local index: buffers and phases
                 const int id_cur = id_next;
@@ -408,7 +420,8 @@ __global__ void __launch_bounds__(384, 1)
                 // a quarter of the tile at a time so that the stores overlap the
                 // exponentials of the next quarter.  The PV product of this tile is
                 // issued before the QK^T product that next writes this buffer, and
-                // the QK^T issuer waits for it.
+                // the QK^T issuer waits for it.  Pairs of keys go through the packed
+                // fp32x2 add and fma.
                 const float2 sl2v = make_float2(sl2, sl2), nmA = make_float2(-msA, -msA), nmB = make_float2(-msB, -msB);
                 float2 lsA = make_float2(0.f, 0.f), lsB = make_float2(0.f, 0.f);
 #pragma unroll
@@ -429,9 +442,8 @@ __global__ void __launch_bounds__(384, 1)
                             if constexpr (kSplitP) {
                                 // hi = p truncated to bf16 (its upper 16 bits), lo = p - hi (exact
                                 // in fp32) truncated likewise: hi + lo is p to within 2^-15
-                                // relative.  Integer ops only: the transcendental pipe that
-                                // computes 2^x is the softmax's bottleneck, and a float -> bf16
-                                // conversion would run on it too.
+                                // relative.  Integer ops only: a float -> bf16 conversion would
+                                // run on the transcendental pipe that computes 2^x.
                                 const uint32_t u0 = __float_as_uint(e0), u1 = __float_as_uint(e1);
                                 pk[2 * i + rb] = __byte_perm(u0, u1, 0x7632);
                                 const float2 rr = __fadd2_rn(
@@ -553,7 +565,7 @@ __global__ void __launch_bounds__(384, 1)
             constexpr uint32_t kBlockBytes = kBlkT * D * 2;   // one block of one KV head: K or V
             int issued = 0;
             bool ok = true;
-            int id_next = tile_block_id(bt_row, kt_lo, kt_hi, kend, lane);
+            int id_next = id_first;
             for (int j = kt_lo; j < kt_hi && ok; ++j) {
                 const int jj = j - kt_lo;                     // local index: stages and phases
                 const int s = jj % C::kStages;
