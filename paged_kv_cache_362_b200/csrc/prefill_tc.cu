@@ -442,13 +442,17 @@ __global__ void __launch_bounds__(384, 1)
                             if constexpr (kSplitP) {
                                 // hi = p truncated to bf16 (its upper 16 bits), lo = p - hi (exact
                                 // in fp32) truncated likewise: hi + lo is p to within 2^-15
-                                // relative.  Integer ops only: a float -> bf16 conversion would
-                                // run on the transcendental pipe that computes 2^x.
-                                const uint32_t u0 = __float_as_uint(e0), u1 = __float_as_uint(e1);
-                                pk[2 * i + rb] = __byte_perm(u0, u1, 0x7632);
-                                const float2 rr = __fadd2_rn(
-                                    make_float2(e0, e1), make_float2(__uint_as_float((u0 & 0xffff0000u) ^ 0x80000000u),
-                                                                     __uint_as_float((u1 & 0xffff0000u) ^ 0x80000000u)));
+                                // relative.  No float -> bf16 conversion: it would run on the
+                                // transcendental pipe that computes 2^x.  The pair's hi parts are
+                                // one byte permute; back as floats, one is a shift of it and the
+                                // other a mask, and lo is one packed fma (hi * -1 + p): the
+                                // integer pipe, the busiest here after the tensor core, gets
+                                // three operations per pair.
+                                const uint32_t hp = __byte_perm(__float_as_uint(e0), __float_as_uint(e1), 0x7632);
+                                pk[2 * i + rb] = hp;
+                                const float2 rr =
+                                    __ffma2_rn(make_float2(__uint_as_float(hp << 16), __uint_as_float(hp & 0xffff0000u)),
+                                               make_float2(-1.f, -1.f), make_float2(e0, e1));
                                 pl[2 * i + rb] = __byte_perm(__float_as_uint(rr.x), __float_as_uint(rr.y), 0x7632);
                                 ls = __fadd2_rn(ls, make_float2(e0, e1));
                             } else {
