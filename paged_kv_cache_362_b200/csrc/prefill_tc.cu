@@ -157,10 +157,15 @@ __device__ __forceinline__ void tmem_st_16x256b_x8(uint32_t taddr, const uint32_
         "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
         : "memory");
 }
-__device__ __forceinline__ void tmem_st_16x128b_x4(uint32_t taddr, const uint32_t* r) {
-    asm volatile("tcgen05.st.sync.aligned.16x128b.x4.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
-                 "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
-                 : "memory");
+__device__ __forceinline__ void tmem_st_16x128b_x16(uint32_t taddr, const uint32_t* r) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.16x128b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]),
+        "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]),
+        "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
 }
 
 // byte offset of 16-byte unit u (0..7) of row r inside a 128-byte-swizzled group
@@ -417,21 +422,19 @@ __global__ void __launch_bounds__(384, 1)
                 // products use: the rounded fp16 values, or the fp32 values hi + lo
                 // carry.  The pair of keys 8e + 2cg, + 1 of a row goes to P column
                 // 4e + cg of its lane (the buffer's scores are overwritten in place),
-                // a quarter of the tile at a time so that the stores overlap the
-                // exponentials of the next quarter.  The PV product of this tile is
-                // issued before the QK^T product that next writes this buffer, and
-                // the QK^T issuer waits for it.  Pairs of keys go through the packed
-                // fp32x2 add and fma.
+                // one store per part for the whole tile (fewer, wider tensor-memory
+                // stores measured faster than a quarter at a time).  The PV product of
+                // this tile is issued before the QK^T product that next writes this
+                // buffer, and the QK^T issuer waits for it.  Pairs of keys go through
+                // the packed fp32x2 add and fma.
                 const float2 sl2v = make_float2(sl2, sl2), nmA = make_float2(-msA, -msA), nmB = make_float2(-msB, -msB);
                 float2 lsA = make_float2(0.f, 0.f), lsB = make_float2(0.f, 0.f);
+                {
+                    // 16x128b repetition e: P column 4e + cg, rows A, B
+                    uint32_t pk[kKeysT / 4];
+                    uint32_t pl[kSplitP ? kKeysT / 4 : 1];
 #pragma unroll
-                for (int qt = 0; qt < 4; ++qt) {
-                    // 16x128b repetition i of this quarter: P column 4(4qt + i) + cg, rows A, B
-                    uint32_t pk[8];
-                    uint32_t pl[kSplitP ? 8 : 1];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int e = 4 * qt + i;
+                    for (int e = 0; e < kKeysT / 8; ++e) {
 #pragma unroll
                         for (int rb = 0; rb < 2; ++rb) {
                             const float2 x = __ffma2_rn(
@@ -449,20 +452,20 @@ __global__ void __launch_bounds__(384, 1)
                                 // integer pipe, the busiest here after the tensor core, gets
                                 // three operations per pair.
                                 const uint32_t hp = __byte_perm(__float_as_uint(e0), __float_as_uint(e1), 0x7632);
-                                pk[2 * i + rb] = hp;
+                                pk[2 * e + rb] = hp;
                                 const float2 rr =
                                     __ffma2_rn(make_float2(__uint_as_float(hp << 16), __uint_as_float(hp & 0xffff0000u)),
                                                make_float2(-1.f, -1.f), make_float2(e0, e1));
-                                pl[2 * i + rb] = __byte_perm(__float_as_uint(rr.x), __float_as_uint(rr.y), 0x7632);
+                                pl[2 * e + rb] = __byte_perm(__float_as_uint(rr.x), __float_as_uint(rr.y), 0x7632);
                                 ls = __fadd2_rn(ls, make_float2(e0, e1));
                             } else {
-                                pk[2 * i + rb] = Elt<T>::pack2(e0, e1);
-                                ls = __fadd2_rn(ls, __half22float2(*reinterpret_cast<const __half2*>(&pk[2 * i + rb])));
+                                pk[2 * e + rb] = Elt<T>::pack2(e0, e1);
+                                ls = __fadd2_rn(ls, __half22float2(*reinterpret_cast<const __half2*>(&pk[2 * e + rb])));
                             }
                         }
                     }
-                    tmem_st_16x128b_x4(tS + qt * 16, pk);
-                    if constexpr (kSplitP) tmem_st_16x128b_x4(tS + C::kColPLo + qt * 16, pl);
+                    tmem_st_16x128b_x16(tS, pk);
+                    if constexpr (kSplitP) tmem_st_16x128b_x16(tS + C::kColPLo, pl);
                 }
                 lA = lA * alphaA + (lsA.x + lsA.y);
                 lB = lB * alphaB + (lsB.x + lsB.y);
