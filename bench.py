@@ -39,6 +39,10 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "paged decode attention: achieved KV-read HBM GB/s (% of peak), seq/s"
+# Layers of one model step in the layer rotation: the decode's plan (pa_decode_plan) is made once per
+# this many layers, as a serving engine makes it once per step for all layers.  28 is the layer count
+# of Qwen2.5-7B, whose attention shape (28 query heads, 4 KV heads, head_dim 128) the workloads use.
+MODEL_LAYERS = 28
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -253,6 +257,9 @@ class DeviceWorkload:
         self.decode_launches = pa.decode_launch_count(wl.num_seqs, c.num_heads, c.num_kv_heads, c.head_dim,
                                                       self.max_ctx, self.P, c.dtype)
         self.launches_per_step = (1 if self.has_copy else 0) + 1 + self.decode_launches
+        # with a plan made once per step of the model (pa_decode_plan) and one planned decode per layer
+        self.planned_launches = pa.decode_launch_count(wl.num_seqs, c.num_heads, c.num_kv_heads, c.head_dim,
+                                                       self.max_ctx, self.P, c.dtype, planned=True)
 
     def pre(self, layer: int = 0):
         kc, vc = self.kcs[layer], self.vcs[layer]
@@ -260,10 +267,23 @@ class DeviceWorkload:
             self.pa.copy_blocks(kc, vc, self.pairs, status=self.status)
         self.pa.reshape_and_cache(self.key, self.value, kc, vc, self.slots, status=self.status)
 
-    def decode(self, layer: int = 0):
+    def decode(self, layer: int = 0, planned: bool = False):
         c = self.cfg
         self.pa.decode(self.out, self.q, self.kcs[layer], self.vcs[layer], self.bt, self.cl, c.scale, self.max_ctx,
-                       self.ws, partition_size=self.P, status=self.status)
+                       self.ws, partition_size=self.P, status=self.status, planned=planned)
+
+    def plan(self):
+        """The step's work list into the workspace (pa_decode_plan): shared by every layer's planned decode."""
+        c = self.cfg
+        self.pa.decode_plan(self.bt, self.cl, c.num_heads, c.num_kv_heads, c.head_dim, c.block_size, self.max_ctx,
+                            self.ws, partition_size=self.P, status=self.status)
+
+    def layer_decode(self, layer: int):
+        """Decode of model layer ``layer`` (on pool layer mod the pools): the step's first layer makes the plan
+        that every layer of the step decodes with."""
+        if layer % MODEL_LAYERS == 0:
+            self.plan()
+        self.decode(layer % self.layers, planned=True)
 
 
 def unique_kv_bytes(wl) -> int:
@@ -370,15 +390,20 @@ def time_steps_layers(w: DeviceWorkload, steps: int, warmup: int):
     it reads: the step two layers back read other data of the same size.  No
     flush runs between steps.  Whole steps (graphs of copy + append + decode)
     and the decode alone (after an untimed append) are timed in two passes.
+    As in a serving engine, the decode's work list depends only on the context
+    lengths, which the layers of a model step share: the first layer of every
+    MODEL_LAYERS makes it (pa_decode_plan) and every layer decodes with it
+    (pa_decode_planned), so the plan's time is in the timed steps once per
+    model step.  Layer m decodes pool m mod L.
     """
     import torch
 
     stream = torch.cuda.current_stream()
-    L = w.layers
+    L = MODEL_LAYERS   # graphs per model step; layer m uses pool m mod w.layers
     for l in range(L):
         for _ in range(2):
-            w.pre(l)
-            w.decode(l)
+            w.pre(l % w.layers)
+            w.layer_decode(l)
     torch.cuda.synchronize()
     s = torch.cuda.Stream()
     s.wait_stream(stream)
@@ -387,20 +412,20 @@ def time_steps_layers(w: DeviceWorkload, steps: int, warmup: int):
         for l in range(L):
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=s):
-                w.pre(l)
-                w.decode(l)
+                w.pre(l % w.layers)
+                w.layer_decode(l)
             g_step.append(g)
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=s):
-                w.pre(l)
+                w.pre(l % w.layers)
             g_pre.append(g)
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=s):
-                w.decode(l)
+                w.layer_decode(l)
             g_dec.append(g)
     stream.wait_stream(s)
     torch.cuda.synchronize()
-    for k in range(max(warmup, 3) * L):
+    for k in range(max(warmup, 3) * w.layers):
         g_step[k % L].replay()
     torch.cuda.synchronize()
     dist_barrier()
@@ -811,7 +836,8 @@ def main():
                 "decode_frac_of_peak": round(sw.kv_bytes / (sd * 1e-3) / 1e9 / peak, 4),
                 "decode_kv_gbs_flushed_every_step": round(sw.kv_bytes / (sfd * 1e-3) / 1e9, 1),
                 "kv_bytes": sw.kv_bytes, "seq_per_s": round(sw.wl.num_seqs / (ss * 1e-3), 1),
-                "decode_launches": sw.decode_launches,
+                "decode_launches": (f"{sw.planned_launches} per layer + 1 plan per {MODEL_LAYERS} layers"
+                                    if rotation else sw.decode_launches),
             }
             del sw
             torch.cuda.empty_cache()
@@ -888,15 +914,25 @@ def main():
                               "the step)"),
                        "cuda_graph": ("one graph per step (copy + append + decode, PDL-chained); the decode "
                                       "alone timed as its own graph") if use_graph else False,
-                       "step": ("copy_blocks + " if w.has_copy else "") + "reshape_and_cache + decode"},
+                       "step": ("copy_blocks + " if w.has_copy else "") + "reshape_and_cache + decode" + (
+                           f" (pa_decode_planned; the first of every {MODEL_LAYERS} layers, one model step of "
+                           "a 28-layer model, also makes the step's plan, pa_decode_plan)" if rotation
+                           else " (pa_decode)")},
             "pct_of_peak": round(100 * value / world / peak, 2),
             "seq_per_s": round(w.wl.num_seqs * world / (ms * 1e-3), 1),
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4), "traffic": profiled_traffic(c.name if c.block_size == 16 else f"{c.name}_bs{c.block_size}"),
                          "algorithmic_bytes": w.kv_bytes,
-                         "kernel": f"pa_decode call ({w.decode_launches} launch(es): [plan +] attention "
-                                   "[+ reduce]), timed together; traffic = DRAM bytes of the attention kernel "
-                                   "from profiles/traffic.json",
+                         "kernel": ((f"pa_decode_planned per layer ({w.planned_launches} launch(es): attention "
+                                     f"[+ reduce]), plus pa_decode_plan (1 launch) once per {MODEL_LAYERS} layers "
+                                     f"(a model step): the mean per layer, plan included, over consecutive timed "
+                                     f"steps")
+                                    if rotation else
+                                    f"pa_decode call ({w.decode_launches} launch(es): [plan +] attention "
+                                    "[+ reduce]), timed together") +
+                                   "; traffic = DRAM bytes of the attention kernel from profiles/traffic.json; "
+                                   "flushed_every_step and after_write_only_flush time pa_decode (a plan in "
+                                   "every call)",
                          "peak_kind": peak_kind,
                          "flushed_every_step": flushed,
                          "after_write_only_flush": {"decode_ms": round(wo, 5),
@@ -911,7 +947,8 @@ def main():
             "block_manager": bm_step,
             "swap": swap,
             "prefill": prefill_res,
-            "gpu_launches": w.launches_per_step * args.steps,
+            "gpu_launches": ((w.launches_per_step - w.decode_launches + w.planned_launches) * args.steps
+                             + -(-args.steps // MODEL_LAYERS)) if rotation else w.launches_per_step * args.steps,
             "clocks": clk,
             "secondary": secondary,
         }

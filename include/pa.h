@@ -178,6 +178,52 @@ int32_t pa_decode_launch_count(int32_t num_seqs, int32_t num_heads, int32_t num_
                                int32_t max_context_len, int32_t partition_size, pa_dtype dtype);
 
 /*
+ * pa_decode_plan, pa_decode_planned -- pa_decode split into a plan, made once
+ * per step, and one planned decode per model layer.
+ *
+ * The work of a decode step is a list of (sequence, partition, KV head) items
+ * that depends only on context_lens and the sizes (the partitioning of
+ * "PagedAttention" digest, "Why the attention kernel works at all"); every
+ * layer of a model decodes the same step over its own pools.  pa_decode_plan
+ * writes that list into `workspace` (one small kernel); each
+ * pa_decode_planned call then decodes without making it.  pa_decode_planned
+ * computes exactly what pa_decode computes (the same kernels, the same
+ * result bits) provided that:
+ *   - the workspace was last planned by pa_decode_plan with this call's
+ *     context_lens values, num_seqs, num_heads, num_kv_heads, head_dim,
+ *     block_size, max_blocks_per_seq, max_context_len and partition_size;
+ *   - the plan is ordered before the call: the same stream (the library's
+ *     kernels complete in stream order), or an event or synchronization
+ *     between streams;
+ *   - no call on the workspace has since reported an error (after
+ *     PA_ERR_TIMEOUT, zero the workspace and plan again).
+ * A plan stays valid for any number of planned calls.  pa_decode (or
+ * pa_decode_tuned) on the same workspace may replace it: plan again after one.
+ *
+ * pa_decode_plan's arguments mean what they mean for pa_decode (status and
+ * stream too: a length outside [0, min(max_context_len, max_blocks_per_seq *
+ * block_size)] is clamped and reported as PA_ERR_OUT_OF_RANGE); it reads only
+ * context_lens, and its validation and errors are pa_decode's for those
+ * arguments.  It enqueues one kernel.  pa_decode_planned takes pa_decode's
+ * arguments and enqueues pa_decode_planned_launch_count() kernels (the
+ * attention kernel, and the reduce kernel when a sequence spans more
+ * partitions than the attention kernel merges).
+ */
+pa_status pa_decode_plan(const int32_t* context_lens, int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads,
+                         int32_t head_dim, int32_t block_size, int32_t max_blocks_per_seq, int32_t max_context_len,
+                         int32_t partition_size, void* workspace, size_t workspace_bytes, int32_t* status,
+                         pa_stream_t stream);
+pa_status pa_decode_planned(void* out, const void* q, const void* key_cache, const void* value_cache,
+                            const int32_t* block_tables, int32_t max_blocks_per_seq,
+                            const int32_t* context_lens, int32_t num_seqs, int32_t num_heads,
+                            int32_t num_kv_heads, int32_t head_dim, int32_t block_size, int32_t num_blocks,
+                            float scale, int32_t max_context_len, int32_t partition_size, void* workspace,
+                            size_t workspace_bytes, pa_dtype dtype, int32_t* status, pa_stream_t stream);
+int32_t pa_decode_planned_launch_count(int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads,
+                                       int32_t head_dim, int32_t max_context_len, int32_t partition_size,
+                                       pa_dtype dtype);
+
+/*
  * pa_copy_blocks -- copy-on-write clone of whole blocks, in both pools.
  *
  * For each pair k < num_pairs with (src, dst) = (block_pairs[2k], block_pairs[2k+1]):

@@ -22,6 +22,7 @@ from ._lib import (  # noqa: F401
     copy_blocks,
     decode,
     decode_launch_count,
+    decode_plan,
     decode_workspace_size,
     error_string,
     make_workspace,

@@ -77,7 +77,7 @@ def _load() -> ctypes.CDLL:
     for sym in ("pa_reshape_and_cache", "pa_decode_workspace_size", "pa_decode", "pa_decode_launch_count",
                 "pa_copy_blocks", "pa_get_error_string", "pa_version", "pa_bm_create", "pa_bm_append_tokens",
                 "pa_prefill", "pa_swap_blocks", "pa_decode_tuned", "pa_decode_launch_count_tuned", "pa_prefill_ws",
-                "pa_prefill_workspace_size"):
+                "pa_prefill_workspace_size", "pa_decode_plan", "pa_decode_planned", "pa_decode_planned_launch_count"):
         if not hasattr(lib, sym):
             raise ImportError(f"{LIB_PATH} lacks {sym} (stale build); run `python paged_kv_cache_362_b200/build.py`")
     p, i32, i64, f32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
@@ -93,6 +93,12 @@ def _load() -> ctypes.CDLL:
     # scheduling options and fault-path test hooks (pa_tuning.h)
     lib.pa_decode_tuned.argtypes = lib.pa_decode.argtypes + [ctypes.POINTER(DecodeTuning)]
     lib.pa_decode_tuned.restype = ctypes.c_int
+    lib.pa_decode_planned.argtypes = lib.pa_decode.argtypes
+    lib.pa_decode_planned.restype = ctypes.c_int
+    lib.pa_decode_plan.argtypes = [p, i32, i32, i32, i32, i32, i32, i32, i32, p, sz, p, p]
+    lib.pa_decode_plan.restype = ctypes.c_int
+    lib.pa_decode_planned_launch_count.argtypes = [i32, i32, i32, i32, i32, i32, ctypes.c_int]
+    lib.pa_decode_planned_launch_count.restype = i32
     lib.pa_decode_launch_count_tuned.argtypes = [i32, i32, i32, i32, i32, i32, ctypes.c_int,
                                                  ctypes.POINTER(DecodeTuning)]
     lib.pa_decode_launch_count_tuned.restype = i32
@@ -202,11 +208,16 @@ def decode_workspace_size(num_seqs, num_heads, num_kv_heads, head_dim, max_conte
 
 
 def decode_launch_count(num_seqs, num_heads, num_kv_heads, head_dim, max_context_len, partition_size=0,
-                        dtype="f16", tuning=None) -> int:
-    """Kernels one pa_decode call enqueues for these sizes on the current device."""
+                        dtype="f16", tuning=None, planned=False) -> int:
+    """Kernels one pa_decode (planned: pa_decode_planned) call enqueues for these sizes on the current device."""
     code = {"f32": 0, "f16": 1, "bf16": 2}[dtype]
-    n = int(LIB.pa_decode_launch_count_tuned(num_seqs, num_heads, num_kv_heads, head_dim, max_context_len,
-                                             partition_size, code, _tuning_ptr(tuning)))
+    if planned:
+        assert tuning is None, "a planned decode takes no tuning"
+        n = int(LIB.pa_decode_planned_launch_count(num_seqs, num_heads, num_kv_heads, head_dim, max_context_len,
+                                                   partition_size, code))
+    else:
+        n = int(LIB.pa_decode_launch_count_tuned(num_seqs, num_heads, num_kv_heads, head_dim, max_context_len,
+                                                 partition_size, code, _tuning_ptr(tuning)))
     if n < 0:
         raise PagedAttentionError(PA_ERR_INVALID_ARG, "pa_decode_launch_count")
     return n
@@ -220,12 +231,29 @@ def make_workspace(num_seqs, num_heads, num_kv_heads, head_dim, max_context_len,
     return torch.zeros(n, dtype=torch.uint8, device=device or "cuda")
 
 
+def decode_plan(block_tables, context_lens, num_heads, num_kv_heads, head_dim, block_size, max_context_len,
+                workspace, partition_size=0, status=None, stream=None):
+    """The work list of a decode step into ``workspace`` (pa_decode_plan), for ``decode(..., planned=True)``.
+
+    Sizes are those the planned decodes will pass: B = context_lens.shape[0] sequences, block_tables
+    [B, max_blocks_per_seq].  Only context_lens is read.
+    """
+    assert context_lens.dtype.itemsize == 4 and context_lens.is_contiguous() and workspace.is_contiguous()
+    B = context_lens.shape[0]
+    assert block_tables.shape[0] == B
+    _check(LIB.pa_decode_plan(_ptr(context_lens), B, num_heads, num_kv_heads, head_dim, block_size,
+                              block_tables.shape[1], int(max_context_len), int(partition_size), _ptr(workspace),
+                              workspace.numel() * workspace.element_size(), _ptr(status), _stream(stream)),
+           "pa_decode_plan")
+
+
 def decode(out, q, key_cache, value_cache, block_tables, context_lens, scale, max_context_len, workspace,
-           partition_size=0, status=None, stream=None, tuning=None):
+           partition_size=0, status=None, stream=None, tuning=None, planned=False):
     """One decode step of paged attention (pa_decode); writes ``out`` [B, Hq, D].
 
     The block size (8, 16 or 32 tokens) is the pools' dimension 2.  ``tuning`` (a DecodeTuning) selects a
     scheduling alternative or a test hook (pa_decode_tuned); None is the library's default schedule.
+    ``planned`` decodes with the plan decode_plan left in ``workspace`` (pa_decode_planned; no tuning).
     """
     B, Hq, D = q.shape
     NB, Hkv, bs = key_cache.shape[0], key_cache.shape[1], key_cache.shape[2]
@@ -235,6 +263,15 @@ def decode(out, q, key_cache, value_cache, block_tables, context_lens, scale, ma
     assert block_tables.shape[0] == B and context_lens.shape == (B,)
     for t in (out, q, key_cache, value_cache, block_tables, context_lens, workspace):
         assert t.is_contiguous()
+    if planned:
+        assert tuning is None, "a planned decode takes no tuning"
+        _check(LIB.pa_decode_planned(_ptr(out), _ptr(q), _ptr(key_cache), _ptr(value_cache), _ptr(block_tables),
+                                     block_tables.shape[1], _ptr(context_lens), B, Hq, Hkv, D, bs, NB, float(scale),
+                                     int(max_context_len), int(partition_size), _ptr(workspace),
+                                     workspace.numel() * workspace.element_size(), _dtype_code(q), _ptr(status),
+                                     _stream(stream)),
+               "pa_decode_planned")
+        return
     _check(LIB.pa_decode_tuned(_ptr(out), _ptr(q), _ptr(key_cache), _ptr(value_cache), _ptr(block_tables),
                                block_tables.shape[1], _ptr(context_lens), B, Hq, Hkv, D, bs, NB, float(scale),
                                int(max_context_len), int(partition_size), _ptr(workspace),

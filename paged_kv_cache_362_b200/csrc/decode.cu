@@ -1501,7 +1501,7 @@ cudaError_t tc_choice(const DecodeParams& p, const DecodeOptions& o, long long m
     // Each self-planning CTA scans all of context_lens; past a few hundred
     // sequences one plan kernel is cheaper (measured: equal at 256, the plan
     // kernel 3.6% faster at 1024, self-planning 2-11% faster at 8 and 32).
-    c->self_plan = !o.force_plan_kernel && p.num_seqs <= kSelfPlanMaxSeqs && p.num_seqs <= Cfg::kPlanSeqs &&
+    c->self_plan = !o.force_plan_kernel && !o.planned && p.num_seqs <= kSelfPlanMaxSeqs && p.num_seqs <= Cfg::kPlanSeqs &&
                    (long long)p.num_seqs * p.num_kv_heads <= kCounterSlots &&
                    (max_items + grid - 1) / grid <= Cfg::kMaxOwn;
     return cudaSuccess;
@@ -1529,7 +1529,7 @@ cudaError_t choose(const DecodeParams& p, const DecodeOptions& o, pa_dtype dtype
         }
     }
     c->reduce = p.max_parts > 1 && !c->fused;
-    c->launches = (c->self_plan ? 0 : 1) + 1 + (c->reduce ? 1 : 0);
+    c->launches = ((c->self_plan || o.planned) ? 0 : 1) + 1 + (c->reduce ? 1 : 0);
     return cudaSuccess;
 }
 
@@ -1558,6 +1558,12 @@ cudaError_t launch_simt(const DecodeParams& p, cudaStream_t stream, long long ma
     return launch_pdl(decode_simt_kernel<T, D, NW>, dim3(grid), dim3(NW * 32), 0, stream, p);
 }
 
+// plan: one CTA; 256 threads cover typical batches in one pass, 1024 large ones
+cudaError_t launch_plan(const DecodeParams& p, cudaStream_t stream) {
+    return p.num_seqs <= 256 ? launch_pdl(decode_plan_kernel<256>, dim3(1), dim3(256), 0, stream, p)
+                             : launch_pdl(decode_plan_kernel<1024>, dim3(1), dim3(1024), 0, stream, p);
+}
+
 template <typename T, int D>
 cudaError_t launch_all(DecodeParams p, const DecodeOptions& o, pa_dtype dtype, cudaStream_t stream) {
     DecodeChoice c;
@@ -1565,10 +1571,9 @@ cudaError_t launch_all(DecodeParams p, const DecodeOptions& o, pa_dtype dtype, c
     if (e != cudaSuccess) return e;
     p.fused_merge = c.fused ? 1 : 0;
     p.self_plan = c.self_plan ? 1 : 0;
-    if (!c.self_plan) {
-        // plan: one CTA; 256 threads cover typical batches in one pass, 1024 large ones
-        e = p.num_seqs <= 256 ? launch_pdl(decode_plan_kernel<256>, dim3(1), dim3(256), 0, stream, p)
-                              : launch_pdl(decode_plan_kernel<1024>, dim3(1), dim3(1024), 0, stream, p);
+    // a planned call reads the list an earlier pa_decode_plan left in the workspace
+    if (!c.self_plan && !o.planned) {
+        e = launch_plan(p, stream);
         if (e != cudaSuccess) return e;
     }
     if constexpr (std::is_same<T, float>::value) {
@@ -1635,5 +1640,7 @@ cudaError_t decode_launch_count(const DecodeParams& p, const DecodeOptions& o, p
 }
 
 int decode_fused_max_parts() { return kFusedMaxParts; }
+
+cudaError_t launch_decode_plan(const DecodeParams& p, cudaStream_t stream) { return launch_plan(p, stream); }
 
 }  // namespace pa

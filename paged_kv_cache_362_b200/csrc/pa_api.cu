@@ -179,16 +179,20 @@ pa_status pa_decode(void* out, const void* q, const void* key_cache, const void*
                            partition_size, workspace, workspace_bytes, dtype, status, stream, nullptr);
 }
 
-pa_status pa_decode_tuned(void* out, const void* q, const void* key_cache, const void* value_cache,
-                          const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* context_lens,
-                          int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads, int32_t head_dim,
-                          int32_t block_size, int32_t num_blocks, float scale, int32_t max_context_len,
-                          int32_t partition_size, void* workspace, size_t workspace_bytes, pa_dtype dtype,
-                          int32_t* status, pa_stream_t stream, const pa_decode_tuning* tuning) {
+namespace {
+// pa_decode_tuned and pa_decode_planned: validation, parameters, launch
+// (planned: the workspace holds the step's plan, from pa_decode_plan).
+pa_status decode_impl(void* out, const void* q, const void* key_cache, const void* value_cache,
+                      const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* context_lens,
+                      int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                      int32_t num_blocks, float scale, int32_t max_context_len, int32_t partition_size,
+                      void* workspace, size_t workspace_bytes, pa_dtype dtype, int32_t* status, pa_stream_t stream,
+                      const pa_decode_tuning* tuning, bool planned) {
     DecodeOptions opt;
     int equal_split = 0, class_first = 1, stall = 0;
     uint64_t wait_limit = kWaitLimitNs;
     if (!decode_options(tuning, &opt, &equal_split, &class_first, &wait_limit, &stall)) return PA_ERR_INVALID_ARG;
+    opt.planned = planned;
     if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || num_blocks <= 0 ||
         max_blocks_per_seq <= 0 || max_context_len < 0)
         return PA_ERR_INVALID_ARG;
@@ -246,6 +250,77 @@ pa_status pa_decode_tuned(void* out, const void* q, const void* key_cache, const
     const cudaError_t e = launch_decode(p, opt, dtype, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
+}  // namespace
+
+pa_status pa_decode_tuned(void* out, const void* q, const void* key_cache, const void* value_cache,
+                          const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* context_lens,
+                          int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads, int32_t head_dim,
+                          int32_t block_size, int32_t num_blocks, float scale, int32_t max_context_len,
+                          int32_t partition_size, void* workspace, size_t workspace_bytes, pa_dtype dtype,
+                          int32_t* status, pa_stream_t stream, const pa_decode_tuning* tuning) {
+    return decode_impl(out, q, key_cache, value_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs,
+                       num_heads, num_kv_heads, head_dim, block_size, num_blocks, scale, max_context_len,
+                       partition_size, workspace, workspace_bytes, dtype, status, stream, tuning, false);
+}
+
+pa_status pa_decode_planned(void* out, const void* q, const void* key_cache, const void* value_cache,
+                            const int32_t* block_tables, int32_t max_blocks_per_seq, const int32_t* context_lens,
+                            int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads, int32_t head_dim,
+                            int32_t block_size, int32_t num_blocks, float scale, int32_t max_context_len,
+                            int32_t partition_size, void* workspace, size_t workspace_bytes, pa_dtype dtype,
+                            int32_t* status, pa_stream_t stream) {
+    return decode_impl(out, q, key_cache, value_cache, block_tables, max_blocks_per_seq, context_lens, num_seqs,
+                       num_heads, num_kv_heads, head_dim, block_size, num_blocks, scale, max_context_len,
+                       partition_size, workspace, workspace_bytes, dtype, status, stream, nullptr, true);
+}
+
+pa_status pa_decode_plan(const int32_t* context_lens, int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads,
+                         int32_t head_dim, int32_t block_size, int32_t max_blocks_per_seq, int32_t max_context_len,
+                         int32_t partition_size, void* workspace, size_t workspace_bytes, int32_t* status,
+                         pa_stream_t stream) {
+    if (num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 || max_blocks_per_seq <= 0 ||
+        max_context_len < 0)
+        return PA_ERR_INVALID_ARG;
+    if (num_heads % num_kv_heads != 0) return PA_ERR_INVALID_ARG;
+    if (!block_size_supported(block_size) || (head_dim != 64 && head_dim != 128) || num_kv_heads > 255)
+        return PA_ERR_UNSUPPORTED;
+    if (partition_size != 0 &&
+        (partition_size < kChunk || partition_size > kChunk * kMaxPartBlocks || partition_size % kChunk))
+        return PA_ERR_INVALID_ARG;
+    if (num_seqs == 0) return PA_OK;
+    if (!context_lens || !workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u)) return PA_ERR_INVALID_ARG;
+    WsLayout w;
+    if (!ws_layout(num_seqs, num_heads, num_kv_heads, head_dim, max_context_len, partition_size, &w))
+        return PA_ERR_INVALID_ARG;
+    if (workspace_bytes < w.total) return PA_ERR_INVALID_ARG;
+    if (w.max_items > INT32_MAX) return PA_ERR_UNSUPPORTED;
+    // what the planning kernel reads and writes: the lengths, the partition
+    // geometry (default split and order, as pa_decode_planned uses) and the workspace
+    DecodeParams p{};
+    p.context_lens = context_lens;
+    p.status = status;
+    p.num_seqs = num_seqs;
+    p.num_heads = num_heads;
+    p.num_kv_heads = num_kv_heads;
+    p.head_dim = head_dim;
+    p.group = num_heads / num_kv_heads;
+    p.max_blocks_per_seq = max_blocks_per_seq;
+    p.block_size = block_size;
+    p.ctx_cap = (int)std::min<int64_t>(max_context_len, (int64_t)max_blocks_per_seq * block_size);
+    p.part_blocks = w.partition_size / kChunk;
+    p.max_parts = w.max_parts;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    p.hdr = reinterpret_cast<int32_t*>(ws);
+    p.merge_count = reinterpret_cast<int32_t*>(ws + w.off_cnt);
+    p.items = reinterpret_cast<int4*>(ws + w.off_items);
+    p.part_m = reinterpret_cast<float*>(ws + w.off_m);
+    p.part_l = reinterpret_cast<float*>(ws + w.off_l);
+    p.part_o = reinterpret_cast<float*>(ws + w.off_o);
+    p.equal_split = 0;
+    p.class_first = 1;
+    const cudaError_t e = launch_decode_plan(p, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
 
 int32_t pa_decode_launch_count(int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads, int32_t head_dim,
                                int32_t max_context_len, int32_t partition_size, pa_dtype dtype) {
@@ -253,13 +328,15 @@ int32_t pa_decode_launch_count(int32_t num_seqs, int32_t num_heads, int32_t num_
                                         dtype, nullptr);
 }
 
-int32_t pa_decode_launch_count_tuned(int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads, int32_t head_dim,
-                                     int32_t max_context_len, int32_t partition_size, pa_dtype dtype,
-                                     const pa_decode_tuning* tuning) {
+namespace {
+int32_t launch_count(int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads, int32_t head_dim,
+                     int32_t max_context_len, int32_t partition_size, pa_dtype dtype, const pa_decode_tuning* tuning,
+                     bool planned) {
     DecodeOptions opt;
     int equal_split = 0, class_first = 1, stall = 0;
     uint64_t wait_limit = kWaitLimitNs;
     if (!decode_options(tuning, &opt, &equal_split, &class_first, &wait_limit, &stall)) return -1;
+    opt.planned = planned;
     if (num_seqs <= 0 || num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads != 0) return -1;
     if (!valid_dtype(dtype) || (head_dim != 64 && head_dim != 128) || num_kv_heads > 255) return -1;
     WsLayout w;
@@ -275,6 +352,20 @@ int32_t pa_decode_launch_count_tuned(int32_t num_seqs, int32_t num_heads, int32_
     p.max_parts = w.max_parts;
     int n = 0;
     return decode_launch_count(p, opt, dtype, &n) == cudaSuccess ? n : -1;
+}
+}  // namespace
+
+int32_t pa_decode_launch_count_tuned(int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads, int32_t head_dim,
+                                     int32_t max_context_len, int32_t partition_size, pa_dtype dtype,
+                                     const pa_decode_tuning* tuning) {
+    return launch_count(num_seqs, num_heads, num_kv_heads, head_dim, max_context_len, partition_size, dtype, tuning,
+                        false);
+}
+
+int32_t pa_decode_planned_launch_count(int32_t num_seqs, int32_t num_heads, int32_t num_kv_heads, int32_t head_dim,
+                                       int32_t max_context_len, int32_t partition_size, pa_dtype dtype) {
+    return launch_count(num_seqs, num_heads, num_kv_heads, head_dim, max_context_len, partition_size, dtype, nullptr,
+                        true);
 }
 
 pa_status pa_copy_blocks(void* key_cache, void* value_cache, const int64_t* block_pairs, int32_t num_pairs,

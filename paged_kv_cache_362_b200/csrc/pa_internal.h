@@ -61,11 +61,17 @@ constexpr int kCounterSlots = 16384;
 struct DecodeOptions {
     int shape = PA_SHAPE_AUTO;       // pa_decode_shape
     bool force_plan_kernel = false;  // the planning kernel even where attention CTAs could plan
+    bool planned = false;            // the workspace holds this step's plan (pa_decode_plan): none is made
 };
 
 // [plan] + partition kernel + (if sequences span several partitions and the
 // partition kernel does not merge them) reduce.
 cudaError_t launch_decode(const DecodeParams& p, const DecodeOptions& o, pa_dtype dtype, cudaStream_t stream);
+
+// The planning kernel alone: the work list of p's step into p's workspace
+// (pa_decode_plan).  It reads context_lens and writes hdr, items and the
+// zeroed merge counters.
+cudaError_t launch_decode_plan(const DecodeParams& p, cudaStream_t stream);
 
 // Number of kernels launch_decode enqueues for these sizes (p's pointers unused).
 cudaError_t decode_launch_count(const DecodeParams& p, const DecodeOptions& o, pa_dtype dtype, int* launches);

@@ -158,6 +158,60 @@ def test_decode_tuned_validation():
     assert lc(8, 28, 4, 128, 4096, 512, 1, ctypes.byref(pa.tuning(shape=7))) == -1
 
 
+def test_decode_planned_validation():
+    """pa_decode_planned validates exactly as pa_decode does, on the host, before any launch."""
+    import paged_kv_cache_362_b200 as pa
+
+    f = pa._lib.LIB.pa_decode_planned
+
+    def dec_p(**o):
+        a = [o.get("out", FAKE), o.get("q", FAKE), FAKE, FAKE, FAKE, 4, FAKE, o.get("B", 2), o.get("Hq", 4), 2,
+             o.get("D", 64), o.get("bs", 16), 8, ctypes.c_float(o.get("scale", 0.125)), 64, o.get("P", 0),
+             o.get("ws", P(0x100000)), o.get("wsb", 1 << 20), 1, None, None]
+        return f(*a)
+
+    assert dec_p(Hq=5) == pa.PA_ERR_INVALID_ARG
+    assert dec_p(bs=4) == pa.PA_ERR_UNSUPPORTED
+    assert dec_p(D=80) == pa.PA_ERR_UNSUPPORTED
+    assert dec_p(P=24) == pa.PA_ERR_INVALID_ARG
+    assert dec_p(out=P(0)) == pa.PA_ERR_INVALID_ARG
+    assert dec_p(q=P(0x1004)) == pa.PA_ERR_INVALID_ARG
+    assert dec_p(ws=P(0x100010)) == pa.PA_ERR_INVALID_ARG
+    assert dec_p(wsb=16) == pa.PA_ERR_INVALID_ARG
+    assert dec_p(scale=float("nan")) == pa.PA_ERR_INVALID_ARG
+    assert dec_p(B=0) == pa.PA_OK
+    assert pa._lib.LIB.pa_decode_planned_launch_count(8, 28, 5, 128, 4096, 512, 1) == -1   # Hq % Hkv != 0
+    assert pa._lib.LIB.pa_decode_planned_launch_count(8, 28, 4, 80, 4096, 512, 1) == -1    # head_dim
+
+
+def test_decode_plan_validation():
+    """pa_decode_plan checks what it reads (context_lens, sizes, workspace) on the host, before its launch."""
+    import paged_kv_cache_362_b200 as pa
+
+    f = pa._lib.LIB.pa_decode_plan
+
+    def plan(**o):
+        return f(o.get("cl", FAKE), o.get("B", 2), o.get("Hq", 4), o.get("Hkv", 2), o.get("D", 64), o.get("bs", 16),
+                 o.get("MB", 4), o.get("maxctx", 64), o.get("P", 0), o.get("ws", P(0x100000)), o.get("wsb", 1 << 20),
+                 None, None)
+
+    assert plan(Hq=5) == pa.PA_ERR_INVALID_ARG
+    assert plan(B=-1) == pa.PA_ERR_INVALID_ARG
+    assert plan(MB=0) == pa.PA_ERR_INVALID_ARG
+    assert plan(maxctx=-1) == pa.PA_ERR_INVALID_ARG
+    for bs in (4, 24, 64):
+        assert plan(bs=bs) == pa.PA_ERR_UNSUPPORTED
+    assert plan(D=80) == pa.PA_ERR_UNSUPPORTED
+    assert plan(Hkv=256, Hq=256) == pa.PA_ERR_UNSUPPORTED
+    assert plan(P=24) == pa.PA_ERR_INVALID_ARG
+    assert plan(P=1024) == pa.PA_ERR_INVALID_ARG
+    assert plan(cl=P(0)) == pa.PA_ERR_INVALID_ARG
+    assert plan(ws=P(0)) == pa.PA_ERR_INVALID_ARG
+    assert plan(ws=P(0x100010)) == pa.PA_ERR_INVALID_ARG
+    assert plan(wsb=16) == pa.PA_ERR_INVALID_ARG
+    assert plan(B=0, cl=P(0), ws=P(0)) == pa.PA_OK      # nothing to plan: no pointer is read
+
+
 def test_copy_blocks_validation():
     import paged_kv_cache_362_b200 as pa
 

@@ -143,3 +143,67 @@ def test_scheduling_variants_in_subprocess(env):
                  "or long_contexts or bad_block_drops"]
     r = subprocess.run(cmd, cwd=ROOT, env=dict(os.environ, **env), capture_output=True, text=True, timeout=900)
     assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-2000:]
+
+
+# (B, ctx range, P, dtype, D, Hq, Hkv, what the sizes exercise)
+PLANNED = [
+    (250, 1, 256, 64, "f16", 64, 28, 4, "one partition per sequence"),
+    (200, 1, 4000, 512, "bf16", 128, 28, 4, "fused merge of up to 8 partitions"),
+    (40, 1, 9000, 128, "bf16", 128, 28, 4, "many partitions: reduce kernel"),
+    (1000, 1, 256, 64, "f16", 64, 28, 4, "a large batch"),
+    (64, 1, 2000, 0, "bf16", 128, 48, 2, "G = 24: the SIMT kernel"),
+]
+
+
+@pytest.mark.parametrize("case_args", PLANNED, ids=[f"B={c[0]} P={c[3]} G={c[6] // c[7]}" for c in PLANNED])
+def test_plan_once_decode_every_layer(case_args):
+    """pa_decode_plan once, then pa_decode_planned over several layers' pools: each output equals pa_decode's on
+    that pool bit for bit (the same kernels read the same list) and the oracle, and the merge counters end at
+    zero after every call."""
+    import torch
+
+    import paged_kv_cache_362_b200 as pa
+    from parity import to_host
+
+    B, lo, hi, P, dtype, D, Hq, Hkv, what = case_args
+    wl, vh = _problem(B, lo, hi, Hq=Hq, Hkv=Hkv, D=D, dtype=dtype, seed=B + 7)
+    c = wl.cfg
+    case = DeviceCase(wl, vh)
+    d = case.dev
+    ws = pa.make_workspace(wl.num_seqs, c.num_heads, c.num_kv_heads, D, wl.max_context_len, P)
+    ws_ref = pa.make_workspace(wl.num_seqs, c.num_heads, c.num_kv_heads, D, wl.max_context_len, P)
+    # a second layer: the same sequences and tables over other values (exact in the storage type)
+    kc2, vc2 = -d["key_cache"], d["value_cache"].flip(-1).contiguous()
+    layers = [(d["key_cache"], d["value_cache"]), (kc2, vc2), (d["key_cache"], d["value_cache"])]
+    bs = d["key_cache"].shape[2]
+    pa.decode_plan(case.block_tables, case.context_lens, c.num_heads, c.num_kv_heads, D, bs, wl.max_context_len, ws,
+                   partition_size=P, status=case.status)
+    outs = []
+    for k, (kc, vc) in enumerate(layers):
+        out = torch.full_like(d["q"], float("nan"))
+        pa.decode(out, d["q"], kc, vc, case.block_tables, case.context_lens, c.scale, wl.max_context_len, ws,
+                  partition_size=P, status=case.status, planned=True)
+        ref = torch.full_like(d["q"], float("nan"))
+        pa.decode(ref, d["q"], kc, vc, case.block_tables, case.context_lens, c.scale, wl.max_context_len, ws_ref,
+                  partition_size=P, status=case.status)
+        torch.cuda.synchronize()
+        assert int(case.status.item()) == 0
+        assert torch.equal(out.view(torch.int16), ref.view(torch.int16)), f"{what}: layer {k} differs from pa_decode"
+        ncnt = max(COUNTER_SLOTS, B * c.num_kv_heads)
+        assert int(ws[256:256 + 4 * ncnt].view(torch.int32).abs().sum().item()) == 0, "merge counters not at zero"
+        outs.append(out)
+    compare(out_f64(outs[0]), _oracle(wl, vh), dtype, what + ", layer 0")
+    vh2 = dict(vh, key_cache=to_host(kc2, dtype), value_cache=to_host(vc2, dtype))
+    compare(out_f64(outs[1]), _oracle(wl, vh2), dtype, what + ", layer 1")
+
+
+def test_planned_launch_counts():
+    import paged_kv_cache_362_b200 as pa
+
+    # the attention kernel alone, where pa_decode may add a planning kernel
+    assert pa.decode_launch_count(256, 28, 4, 128, 4096, 512, "f16", planned=True) == 1
+    assert pa.decode_launch_count(8192, 32, 8, 64, 64, 16, "f16", planned=True) == 1
+    # attention + reduce
+    assert pa.decode_launch_count(8, 28, 4, 128, 32768, 512, "bf16", planned=True) == 2
+    # fp32 (SIMT path): attention + reduce, against planning kernel + attention + reduce
+    assert pa.decode_launch_count(8, 28, 4, 128, 4096, 512, "f32", planned=True) == 2
