@@ -39,8 +39,8 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "paged decode attention: achieved KV-read HBM GB/s (% of peak), seq/s"
-# Layers of one model step in the layer rotation: the decode's plan (pa_decode_plan) is made once per
-# this many layers, as a serving engine makes it once per step for all layers.  28 is the layer count
+# Layers of one model step in the layer rotation: the decode's plan is made once per this many layers
+# (the first runs pa_decode, the others pa_decode_planned), as a serving engine plans once per step.  28 is the layer count
 # of Qwen2.5-7B, whose attention shape (28 query heads, 4 KV heads, head_dim 128) the workloads use.
 MODEL_LAYERS = 28
 FALLBACK_HBM_GBS = 6650.0
@@ -272,18 +272,10 @@ class DeviceWorkload:
         self.pa.decode(self.out, self.q, self.kcs[layer], self.vcs[layer], self.bt, self.cl, c.scale, self.max_ctx,
                        self.ws, partition_size=self.P, status=self.status, planned=planned)
 
-    def plan(self):
-        """The step's work list into the workspace (pa_decode_plan): shared by every layer's planned decode."""
-        c = self.cfg
-        self.pa.decode_plan(self.bt, self.cl, c.num_heads, c.num_kv_heads, c.head_dim, c.block_size, self.max_ctx,
-                            self.ws, partition_size=self.P, status=self.status)
-
     def layer_decode(self, layer: int):
-        """Decode of model layer ``layer`` (on pool layer mod the pools): the step's first layer makes the plan
-        that every layer of the step decodes with."""
-        if layer % MODEL_LAYERS == 0:
-            self.plan()
-        self.decode(layer % self.layers, planned=True)
+        """Decode of model layer ``layer`` (on pool layer mod the pools): the step's first layer runs pa_decode,
+        which leaves its plan in the workspace, and the step's other layers decode with that plan."""
+        self.decode(layer % self.layers, planned=layer % MODEL_LAYERS != 0)
 
 
 def unique_kv_bytes(wl) -> int:
@@ -392,9 +384,9 @@ def time_steps_layers(w: DeviceWorkload, steps: int, warmup: int):
     and the decode alone (after an untimed append) are timed in two passes.
     As in a serving engine, the decode's work list depends only on the context
     lengths, which the layers of a model step share: the first layer of every
-    MODEL_LAYERS makes it (pa_decode_plan) and every layer decodes with it
-    (pa_decode_planned), so the plan's time is in the timed steps once per
-    model step.  Layer m decodes pool m mod L.
+    MODEL_LAYERS makes it (pa_decode, which leaves it in the workspace) and the
+    others decode with it (pa_decode_planned), so planning is in the timed
+    steps once per model step.  Layer m decodes pool m mod L.
     """
     import torch
 
@@ -836,8 +828,8 @@ def main():
                 "decode_frac_of_peak": round(sw.kv_bytes / (sd * 1e-3) / 1e9 / peak, 4),
                 "decode_kv_gbs_flushed_every_step": round(sw.kv_bytes / (sfd * 1e-3) / 1e9, 1),
                 "kv_bytes": sw.kv_bytes, "seq_per_s": round(sw.wl.num_seqs / (ss * 1e-3), 1),
-                "decode_launches": (f"{sw.planned_launches} per layer + 1 plan per {MODEL_LAYERS} layers"
-                                    if rotation else sw.decode_launches),
+                "decode_launches": (f"{sw.planned_launches} per planned layer, {sw.decode_launches} in the first "
+                                    f"of every {MODEL_LAYERS}" if rotation else sw.decode_launches),
             }
             del sw
             torch.cuda.empty_cache()
@@ -915,18 +907,18 @@ def main():
                        "cuda_graph": ("one graph per step (copy + append + decode, PDL-chained); the decode "
                                       "alone timed as its own graph") if use_graph else False,
                        "step": ("copy_blocks + " if w.has_copy else "") + "reshape_and_cache + decode" + (
-                           f" (pa_decode_planned; the first of every {MODEL_LAYERS} layers, one model step of "
-                           "a 28-layer model, also makes the step's plan, pa_decode_plan)" if rotation
-                           else " (pa_decode)")},
+                           f" (the first of every {MODEL_LAYERS} layers, one model step of a 28-layer model, "
+                           "pa_decode, which leaves the step's plan in the workspace; the others "
+                           "pa_decode_planned)" if rotation else " (pa_decode)")},
             "pct_of_peak": round(100 * value / world / peak, 2),
             "seq_per_s": round(w.wl.num_seqs * world / (ms * 1e-3), 1),
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4), "traffic": profiled_traffic(c.name if c.block_size == 16 else f"{c.name}_bs{c.block_size}"),
                          "algorithmic_bytes": w.kv_bytes,
-                         "kernel": ((f"pa_decode_planned per layer ({w.planned_launches} launch(es): attention "
-                                     f"[+ reduce]), plus pa_decode_plan (1 launch) once per {MODEL_LAYERS} layers "
-                                     f"(a model step): the mean per layer, plan included, over consecutive timed "
-                                     f"steps")
+                         "kernel": ((f"per layer: pa_decode_planned ({w.planned_launches} launch(es): attention "
+                                     f"[+ reduce]), and in the first of every {MODEL_LAYERS} layers (a model step) "
+                                     f"pa_decode ({w.decode_launches} launch(es), planning included): the mean per "
+                                     f"layer over consecutive timed steps")
                                     if rotation else
                                     f"pa_decode call ({w.decode_launches} launch(es): [plan +] attention "
                                     "[+ reduce]), timed together") +
@@ -948,7 +940,8 @@ def main():
             "swap": swap,
             "prefill": prefill_res,
             "gpu_launches": ((w.launches_per_step - w.decode_launches + w.planned_launches) * args.steps
-                             + -(-args.steps // MODEL_LAYERS)) if rotation else w.launches_per_step * args.steps,
+                             + (w.decode_launches - w.planned_launches) * -(-args.steps // MODEL_LAYERS))
+                            if rotation else w.launches_per_step * args.steps,
             "clocks": clk,
             "secondary": secondary,
         }

@@ -185,11 +185,12 @@ int32_t pa_decode_launch_count(int32_t num_seqs, int32_t num_heads, int32_t num_
  * that depends only on context_lens and the sizes (the partitioning of
  * "PagedAttention" digest, "Why the attention kernel works at all"); every
  * layer of a model decodes the same step over its own pools.  pa_decode_plan
- * writes that list into `workspace` (one small kernel); each
- * pa_decode_planned call then decodes without making it.  pa_decode_planned
- * computes exactly what pa_decode computes (the same kernels, the same
- * result bits) provided that:
- *   - the workspace was last planned by pa_decode_plan with this call's
+ * writes that list into `workspace` (one small kernel), and every pa_decode
+ * call leaves the list it worked from there too; each pa_decode_planned call
+ * then decodes without making it.  pa_decode_planned computes exactly what
+ * pa_decode computes (the same kernels, the same result bits) provided that:
+ *   - the workspace was last planned, by pa_decode_plan or by pa_decode (or
+ *     pa_decode_tuned with the default partition split), with this call's
  *     context_lens values, num_seqs, num_heads, num_kv_heads, head_dim,
  *     block_size, max_blocks_per_seq, max_context_len and partition_size;
  *   - the plan is ordered before the call: the same stream (the library's
@@ -197,8 +198,8 @@ int32_t pa_decode_launch_count(int32_t num_seqs, int32_t num_heads, int32_t num_
  *     between streams;
  *   - no call on the workspace has since reported an error (after
  *     PA_ERR_TIMEOUT, zero the workspace and plan again).
- * A plan stays valid for any number of planned calls.  pa_decode (or
- * pa_decode_tuned) on the same workspace may replace it: plan again after one.
+ * A plan stays valid for any number of planned calls; the next pa_decode or
+ * pa_decode_plan on the workspace replaces it.
  *
  * pa_decode_plan's arguments mean what they mean for pa_decode (status and
  * stream too: a length outside [0, min(max_context_len, max_blocks_per_seq *

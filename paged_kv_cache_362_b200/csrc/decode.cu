@@ -574,6 +574,15 @@ __global__ void __launch_bounds__(TcCfg<D, NT, NCW, STAGES>::kThreads, TcCfg<D, 
         __syncthreads();
     }
     griddep_wait();
+    if (p.self_plan) {
+        // The plan stays in the workspace for pa_decode_planned: each CTA writes
+        // its items at their ranks (the planning kernel's list, entry for entry)
+        // and CTA 0 the length.  After the wait: the preceding kernel may be a
+        // planned decode still reading the previous list.
+        const int n_own = s_plan[1], Cn = (int)gridDim.x, cb = (int)blockIdx.x;
+        for (int it = threadIdx.x; it < n_own; it += blockDim.x) p.items[it * Cn + ((it & 1) ? Cn - 1 - cb : cb)] = own[it];
+        if (blockIdx.x == 0 && threadIdx.x == 0) p.hdr[kHdrItems] = s_plan[0];
+    }
 
     if constexpr (NCW == 1) {
         if (warp == NCW + 1) {

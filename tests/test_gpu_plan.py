@@ -155,11 +155,12 @@ PLANNED = [
 ]
 
 
+@pytest.mark.parametrize("planner", ["pa_decode_plan", "pa_decode"])
 @pytest.mark.parametrize("case_args", PLANNED, ids=[f"B={c[0]} P={c[3]} G={c[6] // c[7]}" for c in PLANNED])
-def test_plan_once_decode_every_layer(case_args):
-    """pa_decode_plan once, then pa_decode_planned over several layers' pools: each output equals pa_decode's on
-    that pool bit for bit (the same kernels read the same list) and the oracle, and the merge counters end at
-    zero after every call."""
+def test_plan_once_decode_every_layer(case_args, planner):
+    """A plan made once, by pa_decode_plan or left by a pa_decode call, then pa_decode_planned over several
+    layers' pools: each output equals pa_decode's on that pool bit for bit (the same kernels read the same list)
+    and the oracle, and the merge counters end at zero after every call."""
     import torch
 
     import paged_kv_cache_362_b200 as pa
@@ -176,8 +177,13 @@ def test_plan_once_decode_every_layer(case_args):
     kc2, vc2 = -d["key_cache"], d["value_cache"].flip(-1).contiguous()
     layers = [(d["key_cache"], d["value_cache"]), (kc2, vc2), (d["key_cache"], d["value_cache"])]
     bs = d["key_cache"].shape[2]
-    pa.decode_plan(case.block_tables, case.context_lens, c.num_heads, c.num_kv_heads, D, bs, wl.max_context_len, ws,
-                   partition_size=P, status=case.status)
+    if planner == "pa_decode_plan":
+        pa.decode_plan(case.block_tables, case.context_lens, c.num_heads, c.num_kv_heads, D, bs, wl.max_context_len,
+                       ws, partition_size=P, status=case.status)
+    else:   # a decode of another layer (other values) leaves the plan
+        scratch = torch.empty_like(d["q"])
+        pa.decode(scratch, d["q"], d["key_cache"].flip(-1).contiguous(), -d["value_cache"], case.block_tables,
+                  case.context_lens, c.scale, wl.max_context_len, ws, partition_size=P, status=case.status)
     outs = []
     for k, (kc, vc) in enumerate(layers):
         out = torch.full_like(d["q"], float("nan"))
