@@ -32,8 +32,8 @@
 //        combined over a row's four threads with shuffles.  The warps load Q
 //        into shared memory; per key tile they read S, mask keys past each
 //        row's position (and blocks whose id is out of range), update the
-//        running max and sum, write P back a quarter of the tile at a time;
-//        at the end they scale O by 1/l and store it.  The max used for the
+//        running max and sum, write P back (one tensor-memory store per
+//        part); at the end they scale O by 1/l and store it.  The max used for the
 //        exponentials only moves when the tile max exceeds it by more than 8
 //        (log2 units), so O is rescaled rarely; the sum and O always use the
 //        same reference, which keeps the result exact algebra.
@@ -69,9 +69,9 @@ constexpr int kBlkT = 16;         // tokens per block
 // by more than this (log2 units): p <= 2^8, well inside fp16 and bf16.
 constexpr float kRescaleSlack = 8.f;
 // Waiting warps sleep this long between polls of an mbarrier: the softmax warps
-// and the MMA warp share schedulers, and a tight poll takes the issue slots the
-// warp being waited for needs (1.5% of the kernel's time on the bench workload;
-// suspending in mbarrier.try_wait instead cost 3.5%).
+// and the MMA issuers share schedulers, and a tight poll takes the issue slots
+// the warp being waited for needs (1.5% of the kernel's time on the bench
+// workload; suspending in mbarrier.try_wait instead cost 3.5%).
 constexpr uint32_t kPollNs = 20;
 
 template <int D>
