@@ -155,9 +155,11 @@ size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_heads, int32_t num
  *                       bytes, 256-byte aligned, ZERO-FILLED before its first
  *                       use (cudaMemset).  It holds counters that each call
  *                       leaves at zero for the next, whatever the sizes of the
- *                       next problem; the rest is scratch.  After a call that
- *                       reported PA_ERR_TIMEOUT, zero it again.  Calls that
- *                       share a workspace must not overlap in time.
+ *                       next problem, and the call's plan, which
+ *                       pa_decode_planned may reuse (below); the rest is
+ *                       scratch.  After a call that reported PA_ERR_TIMEOUT,
+ *                       zero it again.  Calls that share a workspace must not
+ *                       overlap in time.
  *
  * The call enqueues pa_decode_launch_count() kernels on `stream`.
  */
