@@ -372,7 +372,7 @@ def time_steps(w: DeviceWorkload, steps: int, warmup: int, flush, use_graph: boo
     return step_ms, dec_ms
 
 
-def time_steps_layers(w: DeviceWorkload, steps: int, warmup: int):
+def time_steps_layers(w: DeviceWorkload, steps: int, warmup: int, plan_every_call: bool = False):
     """Per-step CUDA-event times (ms) of consecutive steps that go to different layers' K/V pools.
 
     A serving engine runs the decode once per layer, each layer on its own
@@ -386,16 +386,18 @@ def time_steps_layers(w: DeviceWorkload, steps: int, warmup: int):
     lengths, which the layers of a model step share: the first layer of every
     MODEL_LAYERS makes it (pa_decode, which leaves it in the workspace) and the
     others decode with it (pa_decode_planned), so planning is in the timed
-    steps once per model step.  Layer m decodes pool m mod L.
+    steps once per model step.  Layer m decodes pool m mod L.  With
+    plan_every_call, every layer runs pa_decode instead (a plan in every call).
     """
     import torch
 
     stream = torch.cuda.current_stream()
     L = MODEL_LAYERS   # graphs per model step; layer m uses pool m mod w.layers
+    layer_decode = (lambda l: w.decode(l % w.layers)) if plan_every_call else w.layer_decode
     for l in range(L):
         for _ in range(2):
             w.pre(l % w.layers)
-            w.layer_decode(l)
+            layer_decode(l)
     torch.cuda.synchronize()
     s = torch.cuda.Stream()
     s.wait_stream(stream)
@@ -405,7 +407,7 @@ def time_steps_layers(w: DeviceWorkload, steps: int, warmup: int):
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=s):
                 w.pre(l % w.layers)
-                w.layer_decode(l)
+                layer_decode(l)
             g_step.append(g)
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=s):
@@ -413,7 +415,7 @@ def time_steps_layers(w: DeviceWorkload, steps: int, warmup: int):
             g_pre.append(g)
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=s):
-                w.layer_decode(l)
+                layer_decode(l)
             g_dec.append(g)
     stream.wait_stream(s)
     torch.cuda.synchronize()
@@ -786,6 +788,13 @@ def main():
     total_bytes = dist_sum(float(w.kv_bytes))
     dec = dist_max(float(np.mean(dec_ms)))
     achieved = w.kv_bytes / (dec * 1e-3) / 1e9
+    # the same rotation with pa_decode in every layer (a plan in every call)
+    every = None
+    if rotation:
+        _, e_dec = time_steps_layers(w, max(200, args.steps // 4), args.warmup, plan_every_call=True)
+        ed = dist_max(float(np.mean(e_dec)))
+        every = {"decode_ms": round(ed, 5), "achieved": round(w.kv_bytes / (ed * 1e-3) / 1e9, 1),
+                 "frac": round(w.kv_bytes / (ed * 1e-3) / 1e9 / peak, 4)}
     # the same steps after an L2 flush each (K/V, tables and the kernels' code all cold)
     f_step, f_dec = time_steps(w, args.steps, args.warmup, flush, use_graph) if rotation else (step_ms, dec_ms)
     f_s, f_d = dist_max(float(np.mean(f_step))), dist_max(float(np.mean(f_dec)))
@@ -923,10 +932,12 @@ def main():
                                     f"pa_decode call ({w.decode_launches} launch(es): [plan +] attention "
                                     "[+ reduce]), timed together") +
                                    "; traffic = DRAM bytes of the attention kernel from profiles/traffic.json; "
+                                   "plan_in_every_call is the same rotation with pa_decode in every layer; "
                                    "flushed_every_step and after_write_only_flush time pa_decode (a plan in "
                                    "every call)",
                          "peak_kind": peak_kind,
                          "flushed_every_step": flushed,
+                         "plan_in_every_call": every,
                          "after_write_only_flush": {"decode_ms": round(wo, 5),
                                                     "achieved": round(w.kv_bytes / (wo * 1e-3) / 1e9, 1),
                                                     "frac": round(w.kv_bytes / (wo * 1e-3) / 1e9 / peak, 4)}},
