@@ -184,9 +184,9 @@ int32_t pa_decode_launch_count(int32_t num_seqs, int32_t num_heads, int32_t num_
  * per step, and one planned decode per model layer.
  *
  * The work of a decode step is a list of (sequence, partition, KV head) items
- * that depends only on context_lens and the sizes (the partitioning of
- * "PagedAttention" digest, "Why the attention kernel works at all"); every
- * layer of a model decodes the same step over its own pools.  pa_decode_plan
+ * (long contexts are split into partitions that run in parallel, see
+ * pa_decode) that depends only on context_lens and the sizes; every layer of
+ * a model decodes the same step over its own pools.  pa_decode_plan
  * writes that list into `workspace` (one small kernel), and every pa_decode
  * call leaves the list it worked from there too; each pa_decode_planned call
  * then decodes without making it.  pa_decode_planned computes exactly what
